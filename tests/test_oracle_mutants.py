@@ -1,0 +1,115 @@
+"""Planted mistakes: each mutant replaces one oracle function with a plausible wrong version
+(a transposed operand, a dropped term, a wrong sign or rounding or tie rule) and checks that at
+least one of the oracle's pins fails.  Mistakes are planted in the oracle only, on the CPU."""
+import contextlib
+
+import numpy as np
+import pytest
+
+from oracle import spatten_ref as R
+
+import test_oracle_attention as TA
+import test_oracle_cascade as TC
+import test_oracle_quant_topk as TQ
+
+
+@contextlib.contextmanager
+def patched(name, fn):
+    old = getattr(R, name)
+    setattr(R, name, fn)
+    try:
+        yield
+    finally:
+        setattr(R, name, old)
+
+
+def _col_softmax(S):
+    m = S.max(axis=0, keepdims=True)
+    E = np.exp(S - m)
+    ell = E.sum(axis=0, keepdims=True)
+    return E / ell, ell[0]
+
+
+def _no_scale_dense(Q, K, V, sm_scale):
+    P, _ = R.attention_probs(np.asarray(Q) @ np.asarray(K).T)
+    return P @ V, P
+
+
+def _trunc_split(q):
+    q = np.asarray(q, np.int64)
+    msb = np.trunc(q / 16).astype(np.int64)
+    return msb.astype(np.int8), (q - 16 * msb).astype(np.uint8)
+
+
+def _swapped_pack(lsb):
+    lsb = np.asarray(lsb, np.uint8)
+    return (lsb[..., 1::2] | (lsb[..., 0::2] << 4)).astype(np.uint8)
+
+
+def _scale_2048(x32):
+    x = np.asarray(x32, np.float32)
+    amax = np.float32(np.max(np.abs(x)))
+    return np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(2048))
+
+
+def _topk_high_index_ties(scores, k):
+    s = np.asarray(scores, np.float64)
+    n = len(s)
+    order = np.lexsort((-np.arange(n), -s))
+    return np.sort(order[:k])
+
+
+def _rowsum_importance(P):
+    return np.asarray(P, np.float64).sum(axis=1)
+
+
+def _signed_head_importance(O):
+    return float(np.asarray(O, np.float64).sum())
+
+
+_orig_prog = R.progressive_attention
+
+
+def _prog_le(Q, kq, vq, theta, sm_scale, flags_override=None):
+    r = _orig_prog(Q, kq, vq, theta, sm_scale, flags_override)
+    if flags_override is None:
+        fl = r["pmax_msb"] <= theta
+        if not np.array_equal(fl, r["flags"]):
+            r = _orig_prog(Q, kq, vq, theta, sm_scale, fl)
+    return r
+
+
+def _prog_full_v_never(Q, kq, vq, theta, sm_scale, flags_override=None):
+    vq2 = dict(vq, lsb=np.zeros_like(vq["lsb"]))     # forgets the V LSBs on refetch
+    return _orig_prog(Q, kq, vq2, theta, sm_scale, flags_override)
+
+
+MUTANTS = [
+    ("attention_probs", _col_softmax, [lambda: TA.test_dense_attention_matches_sdpa(5, 7, 8)]),
+    ("dense_attention", _no_scale_dense, [lambda: TA.test_dense_attention_matches_sdpa(5, 7, 8)]),
+    ("split_planes", _trunc_split, [TQ.test_quant_codes_golden]),
+    ("pack_lsb", _swapped_pack, [TQ.test_lsb_pack_golden]),
+    ("quant_scale", _scale_2048, [TQ.test_quant_codes_golden]),
+    ("topk_select", _topk_high_index_ties, [lambda: TQ.test_topk_brute_force_small(0), TQ.test_topk_tie_rules]),
+    ("token_importance_increment", _rowsum_importance, [TC.test_decode_keep_all_full_equals_dense_over_cache]),
+    ("head_importance_increment", _signed_head_importance, [TA.test_head_importance_closed_forms]),
+    ("progressive_attention", _prog_le, [lambda: TA.test_constant_keys_refetch_iff_uniform_prob_below_theta(0.1, False)]),
+    ("progressive_attention", _prog_full_v_never, [TC.test_cascade_keep_all_always_refetch_equals_dense_on_full_codes]),
+]
+
+
+@pytest.mark.parametrize("name,fn,pins", MUTANTS, ids=[f"{m[0]}:{m[1].__name__}" for m in MUTANTS])
+def test_pin_catches_planted_mistake(name, fn, pins):
+    with patched(name, fn):
+        caught = False
+        for pin in pins:
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                caught = True
+        assert caught, f"no pin caught mutant {fn.__name__} of {name}"
+
+
+def test_importance_increment_closed_form_non_square():
+    P = np.array([[0.25, 0.75, 0.0], [0.5, 0.5, 0.0]])
+    np.testing.assert_array_equal(R.token_importance_increment(P), [0.75, 1.25, 0.0])
