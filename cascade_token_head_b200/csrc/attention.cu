@@ -1,0 +1,126 @@
+// spatten_attention_layer: argument checks, workspace layout and kernel choice.
+//
+//   tensor-core kernel (attn_tc.cu)   bf16 queries, quantized K/V, d_h in {64, 128}, many rows
+//   decode kernel (attn_decode.cu)    one query row per (sequence, head), quantized K/V
+//   CUDA-core kernel (attn_simt.cu)   everything else (the float32 configuration)
+// Every kernel writes per-CTA partial importance sums to the workspace; attn_reduce adds them to
+// tok_imp / head_imp in a fixed order.
+#include <cmath>
+#include <cstring>
+
+#include "attention.cuh"
+
+namespace spt {
+namespace {
+
+enum class Path { kSimt, kTc, kDecode };
+
+// returns false when a forced kernel cannot run the problem
+bool choose_path(const spatten_attn_args& a, Path* out) {
+  switch (a.kernel) {
+    case SPATTEN_ATTN_CUDA_CORE: *out = Path::kSimt; return true;
+    case SPATTEN_ATTN_TENSOR_CORE: *out = Path::kTc; return attn_tc_supported(a);
+    case SPATTEN_ATTN_DECODE: *out = Path::kDecode; return attn_decode_supported(a);
+    default: break;
+  }
+  if (attn_decode_supported(a)) *out = Path::kDecode;
+  else if (attn_tc_supported(a)) *out = Path::kTc;
+  else *out = Path::kSimt;
+  return true;
+}
+
+int rows_per_cta(Path p) {
+  switch (p) {
+    case Path::kTc: return kTcRows;
+    case Path::kDecode: return 1;
+    default: return kSimtRows;
+  }
+}
+
+int32_t validate(const spatten_attn_args& a) {
+  if (a.B < 1 || a.H < 1 || a.n_q < 1 || a.n_kv < 1) return SPATTEN_E_ARG;
+  if (a.B > 65535 || a.H > 1024) return SPATTEN_E_ARG;
+  if (a.kernel < SPATTEN_ATTN_AUTO || a.kernel > SPATTEN_ATTN_DECODE) return SPATTEN_E_ARG;
+  if (a.d_h != 64 && a.d_h != 128) return SPATTEN_E_UNSUPPORTED;
+  if (a.H_kept < 1 || a.H_kept > a.H) return SPATTEN_E_ARG;
+  if (!a.head_idx && a.H_kept != a.H) return SPATTEN_E_ARG;
+  if (a.head_idx && a.head_idx_ld != 0 && a.head_idx_ld < a.H_kept) return SPATTEN_E_SHAPE;
+  if (!a.q || !a.o) return SPATTEN_E_ARG;
+  if (a.q_dtype != SPATTEN_F32 && a.q_dtype != SPATTEN_BF16) return SPATTEN_E_ARG;
+  const int64_t hd = static_cast<int64_t>(a.H) * a.d_h;
+  if (a.q_ld_tok < hd || a.o_ld_tok < hd) return SPATTEN_E_SHAPE;
+  if (a.quantized) {
+    if (!a.k_msb || !a.k_lsb || !a.k_scale || !a.v_msb || !a.v_lsb || !a.v_scale) return SPATTEN_E_ARG;
+    if (a.kv_cap < 1) return SPATTEN_E_ARG;
+    if (!a.kv_idx && a.n_kv > a.kv_cap) return SPATTEN_E_SHAPE;
+    if (a.kv_idx && a.kv_idx_ld < a.n_kv) return SPATTEN_E_SHAPE;
+    if (!aligned16(a.k_msb) || !aligned16(a.v_msb) || !aligned16(a.k_lsb) || !aligned16(a.v_lsb))
+      return SPATTEN_E_ALIGN;
+  } else {
+    if (!a.k || !a.v) return SPATTEN_E_ARG;
+    if (a.kv_dtype != SPATTEN_F32 && a.kv_dtype != SPATTEN_BF16) return SPATTEN_E_ARG;
+    if (a.kv_ld_tok < hd) return SPATTEN_E_SHAPE;
+    if (a.kv_idx) return SPATTEN_E_UNSUPPORTED;
+    if (a.n_kv != a.n_q) return SPATTEN_E_SHAPE;   // unquantized K/V share the query rows' layout
+  }
+  if (a.tok_imp && a.tok_imp_ld < (a.tok_imp_map ? 1 : a.n_kv)) return SPATTEN_E_SHAPE;
+  if (a.tok_imp_map && a.tok_imp_map_ld < a.n_kv) return SPATTEN_E_SHAPE;
+  const int esz = a.q_dtype == SPATTEN_BF16 ? 2 : 4;
+  if (!aligned16(a.q) || !aligned16(a.o) || (a.q_ld_tok * esz) % 16 != 0 || (a.o_ld_tok * esz) % 16 != 0)
+    return SPATTEN_E_ALIGN;
+  return SPATTEN_OK;
+}
+
+size_t layout(const spatten_attn_args& a, int rows, void* ws, float** tok, float** head) {
+  const int64_t n_qt = ceil_div(a.n_q, rows);
+  WsCursor c(ws, ~size_t(0));
+  float* t = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * n_qt * a.n_kv);
+  float* h = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * n_qt);
+  if (tok) *tok = t;
+  if (head) *head = h;
+  return c.used;
+}
+
+}  // namespace
+}  // namespace spt
+
+extern "C" size_t spatten_attention_workspace_size(const spatten_attn_args* a) {
+  using namespace spt;
+  Path path;
+  if (!a || validate(*a) != SPATTEN_OK || !choose_path(*a, &path)) return 0;
+  return layout(*a, rows_per_cta(path), nullptr, nullptr, nullptr);
+}
+
+namespace spt {
+int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws_bytes, cudaStream_t st,
+                              cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+  if (!args) return SPATTEN_E_ARG;
+  SPT_TRY(validate(*args));
+  AttnProblem p;
+  std::memcpy(&p.a, args, sizeof(spatten_attn_args));
+  if (!(p.a.sm_scale > 0.0f)) p.a.sm_scale = 1.0f / std::sqrt(static_cast<float>(p.a.d_h));
+  if (p.a.head_idx_ld == 0) p.a.head_idx_ld = p.a.H_kept;
+  Path path;
+  if (!choose_path(p.a, &path)) return SPATTEN_E_UNSUPPORTED;
+  p.qt_rows = rows_per_cta(path);
+  p.n_qt = static_cast<int>(ceil_div(p.a.n_q, p.qt_rows));
+  const size_t need = layout(p.a, p.qt_rows, ws, &p.tok_part, &p.head_part);
+  if (!ws || ws_bytes < need) return SPATTEN_E_WORKSPACE;
+  if (ev_begin) SPT_CUDA(cudaEventRecord(ev_begin, st));
+  int32_t s;
+  switch (path) {
+    case Path::kTc: s = attn_tc_launch(p, st); break;
+    case Path::kDecode: s = attn_decode_launch(p, st); break;
+    default: s = attn_simt_launch(p, st); break;
+  }
+  if (s != SPATTEN_OK) return s;
+  if (ev_end) SPT_CUDA(cudaEventRecord(ev_end, st));
+  if (!p.a.tok_imp && !p.a.head_imp) return SPATTEN_OK;
+  return attn_reduce_launch(p, st);
+}
+}  // namespace spt
+
+extern "C" int32_t spatten_attention_layer(const spatten_attn_args* args, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  return spt::attention_layer_timed(args, ws, ws_bytes, spt::as_stream(stream), nullptr, nullptr);
+}

@@ -1,0 +1,50 @@
+// Internal interface between the attention dispatcher and its kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace spt {
+
+// Resolved attention problem (validated by the dispatcher).
+struct AttnProblem {
+  spatten_attn_args a;       // copy of the caller's arguments, sm_scale resolved
+  int qt_rows;               // query rows per CTA of the chosen kernel
+  int n_qt;                  // query tiles = ceil(n_q / qt_rows)
+  float* tok_part;           // ws [B][H_kept][n_qt][n_kv] per-CTA column sums of P
+  float* head_part;          // ws [B][H_kept][n_qt] per-CTA sum |O|
+};
+
+// Kernels (each returns a status after launching on `st`).
+int32_t attn_simt_launch(const AttnProblem& p, cudaStream_t st);
+int32_t attn_tc_launch(const AttnProblem& p, cudaStream_t st);
+int32_t attn_decode_launch(const AttnProblem& p, cudaStream_t st);
+bool attn_tc_supported(const spatten_attn_args& a);
+bool attn_decode_supported(const spatten_attn_args& a);
+constexpr int kTcRows = 128;      // query rows per CTA of the tensor-core kernel
+constexpr int kSimtRows = 32;     // query rows per CTA of the CUDA-core kernel
+
+// spatten_attention_layer with optional events recorded around the main kernel (not the reduce).
+int32_t attention_layer_timed(const spatten_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t st,
+                              cudaEvent_t ev_begin, cudaEvent_t ev_end);
+
+// Fixed-order reduction of the per-CTA partials into tok_imp / head_imp.
+int32_t attn_reduce_launch(const AttnProblem& p, cudaStream_t st);
+
+// Head slot -> original head id; slots >= H_kept name the pruned heads in ascending order.
+__device__ __forceinline__ int head_of_slot(const spatten_attn_args& a, int b, int slot) {
+  if (!a.head_idx) return slot;
+  const int32_t* hi = a.head_idx + static_cast<int64_t>(b) * a.head_idx_ld;
+  if (slot < a.H_kept) return hi[slot];
+  int want = slot - a.H_kept, seen = 0;
+  for (int h = 0; h < a.H; ++h) {
+    bool kept = false;
+    for (int s = 0; s < a.H_kept; ++s) kept |= (hi[s] == h);
+    if (!kept) {
+      if (seen == want) return h;
+      ++seen;
+    }
+  }
+  return -1;
+}
+
+}  // namespace spt

@@ -1,0 +1,200 @@
+// K1: progressive 12-bit K/V quantization into an int8 MSB plane and a packed 4-bit LSB plane.
+//
+// SpAtten §III.A "Progressive Quantization" stores K/V so that the MSBs can be fetched alone and
+// the LSBs only when a row's attention is too flat; §IV "Quantization Support" splits the fetched
+// bits and concatenates MSBs with LSBs.  Codes: q = clamp(rint(float32(x*gain) / s), +-2047),
+// MSB = q >> 4, LSB = q & 15, s = amax / 2047 per (sequence, head) block.
+//
+// Amax mode: one thread-block cluster per (b, h) block; each CTA reduces the amax of its rows,
+// the cluster exchanges the partial maxima through distributed shared memory, and every CTA then
+// quantizes its rows (a second read that hits L2).  No scratch memory is needed.
+// Fixed-scale mode (decode append): one thread per 8-element chunk, saturations counted.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace spt {
+namespace {
+
+constexpr int kQThreads = 256;
+constexpr float kQMax = 2047.0f;
+
+struct QArgs {
+  const void* x;
+  int B, H, n, d_h;
+  int64_t ld_tok;
+  const float* gain;
+  int64_t ld_gain;
+  const float* scale_in;
+  int8_t* msb;
+  uint8_t* lsb;
+  int cap, row0;
+  float* scale_out;
+  int32_t* sat;
+};
+
+// quantize 8 values with scale s; returns the number of saturated codes
+__device__ __forceinline__ int quant8(const float* v, float s, int8_t* msb_dst, uint8_t* lsb_dst) {
+  int sat = 0;
+  uint32_t m[2] = {0u, 0u};
+  uint32_t l = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float r = rintf(__fdiv_rn(v[i], s));
+    sat += fabsf(r) > kQMax ? 1 : 0;
+    int q = static_cast<int>(fminf(fmaxf(r, -kQMax), kQMax));
+    int hi = q >> 4;          // arithmetic shift: floor(q / 16)
+    int lo = q & 15;
+    m[i >> 2] |= (static_cast<uint32_t>(hi) & 0xFFu) << (8 * (i & 3));
+    l |= static_cast<uint32_t>(lo) << (4 * i);
+  }
+  *reinterpret_cast<uint2*>(msb_dst) = make_uint2(m[0], m[1]);
+  *reinterpret_cast<uint32_t*>(lsb_dst) = l;
+  return sat;
+}
+
+template <typename T>
+__device__ __forceinline__ void load_row_chunk(const QArgs& a, int b, int h, int t, int c, float* v) {
+  const T* x = static_cast<const T*>(a.x) + (static_cast<int64_t>(b) * a.n + t) * a.ld_tok +
+               static_cast<int64_t>(h) * a.d_h + c * 8;
+  load8(x, v);
+  if (a.gain) {
+    float g = a.gain[static_cast<int64_t>(b) * a.ld_gain + t];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= g;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int C = a.d_h / 8;
+  const int rows_per = (a.n + S - 1) / S;
+  const int r0 = min(a.n, rank * rows_per), r1 = min(a.n, r0 + rows_per);
+  const int total = (r1 - r0) * C;
+
+  __shared__ float red[kQThreads / 32];
+  __shared__ float cta_amax;
+
+  float amax = 0.0f;
+  for (int e = threadIdx.x; e < total; e += kQThreads) {
+    float v[8];
+    load_row_chunk<T>(a, b, h, r0 + e / C, e % C, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+    for (int w = 0; w < kQThreads / 32; ++w) m = fmaxf(m, red[w]);
+    cta_amax = m;
+  }
+  cluster.sync();
+  float block_amax = 0.0f;
+  for (int r = 0; r < S; ++r) block_amax = fmaxf(block_amax, *cluster.map_shared_rank(&cta_amax, r));
+  cluster.sync();   // no CTA leaves while a peer may still read its shared memory
+
+  const float s = block_amax == 0.0f ? 1.0f : __fdiv_rn(block_amax, kQMax);
+  if (rank == 0 && threadIdx.x == 0) a.scale_out[bh] = s;
+
+  for (int e = threadIdx.x; e < total; e += kQThreads) {
+    const int t = r0 + e / C, c = e % C;
+    float v[8];
+    load_row_chunk<T>(a, b, h, t, c, v);
+    const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
+    quant8(v, s, a.msb + row * a.d_h + c * 8, a.lsb + row * (a.d_h / 2) + c * 4);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
+  const int C = a.d_h / 8;
+  const int64_t total = static_cast<int64_t>(a.B) * a.H * a.n * C;
+  int sat = 0;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(kQThreads) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * kQThreads) {
+    const int c = static_cast<int>(e % C);
+    const int64_t r = e / C;                     // (b*H + h)*n + t
+    const int t = static_cast<int>(r % a.n);
+    const int bh = static_cast<int>(r / a.n);
+    const int b = bh / a.H, h = bh % a.H;
+    float v[8];
+    load_row_chunk<T>(a, b, h, t, c, v);
+    const float s = a.scale_in[bh];
+    const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
+    sat += quant8(v, s, a.msb + row * a.d_h + c * 8, a.lsb + row * (a.d_h / 2) + c * 4);
+  }
+  sat = warp_sum_int(sat);
+  if (a.sat && (threadIdx.x & 31) == 0 && sat) atomicAdd(a.sat, sat);
+}
+
+}  // namespace
+
+int32_t quantize_launch(const QArgs& a, int dtype, cudaStream_t st) {
+  if (a.scale_in) {
+    const int64_t chunks = static_cast<int64_t>(a.B) * a.H * a.n * (a.d_h / 8);
+    int grid = static_cast<int>(std::min<int64_t>(ceil_div(chunks, kQThreads), 8LL * sm_count()));
+    if (dtype == SPATTEN_BF16)
+      quantize_fixed_kernel<__nv_bfloat16><<<grid, kQThreads, 0, st>>>(a);
+    else
+      quantize_fixed_kernel<float><<<grid, kQThreads, 0, st>>>(a);
+    return launch_status();
+  }
+  const int blocks = a.B * a.H;
+  // enough CTAs to fill the GPU twice; at most 8 per block (portable cluster size)
+  int S = static_cast<int>(ceil_div(2LL * sm_count(), blocks));
+  S = std::max(1, std::min(S, 8));
+  S = std::min<int>(S, std::max(1, a.n / 16));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, blocks, 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = dtype == SPATTEN_BF16
+                      ? cudaLaunchKernelEx(&cfg, quantize_amax_kernel<__nv_bfloat16>, a)
+                      : cudaLaunchKernelEx(&cfg, quantize_amax_kernel<float>, a);
+  if (e != cudaSuccess) {
+    record_cuda_error(e);
+    return SPATTEN_E_CUDA;
+  }
+  return launch_status();
+}
+
+}  // namespace spt
+
+extern "C" int32_t spatten_quantize_kv(const void* x, int32_t dtype, int32_t B, int32_t H,
+                                       int32_t n, int32_t d_h, int64_t ld_tok,
+                                       const float* row_gain, int64_t ld_gain,
+                                       const float* scale_in, int8_t* msb, uint8_t* lsb,
+                                       int32_t cap, int32_t row0, float* scale_out,
+                                       int32_t* sat_count, void* stream) {
+  using namespace spt;
+  if (!x || !msb || !lsb) return SPATTEN_E_ARG;
+  if (dtype != SPATTEN_F32 && dtype != SPATTEN_BF16) return SPATTEN_E_ARG;
+  if (B < 1 || H < 1 || n < 1 || d_h < 8 || (d_h % 8) != 0) return SPATTEN_E_ARG;
+  if (!scale_in && !scale_out) return SPATTEN_E_ARG;
+  if (row0 < 0 || cap < 1 || static_cast<int64_t>(row0) + n > cap) return SPATTEN_E_SHAPE;
+  if (ld_tok < static_cast<int64_t>(H) * d_h) return SPATTEN_E_SHAPE;
+  if (row_gain && ld_gain < n) return SPATTEN_E_SHAPE;
+  const int esz = dtype == SPATTEN_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld_tok * esz) % 16 != 0 || (static_cast<int64_t>(d_h) * esz) % 16 != 0)
+    return SPATTEN_E_ALIGN;
+  if (!aligned16(msb) || !aligned16(lsb)) return SPATTEN_E_ALIGN;
+  QArgs a{x, B, H, n, d_h, ld_tok, row_gain, ld_gain, scale_in, msb, lsb, cap, row0, scale_out,
+          sat_count};
+  return quantize_launch(a, dtype, as_stream(stream));
+}

@@ -249,7 +249,8 @@ def cascade_prefill(X, w_qkv, w_o, H: int, d_h: int, token_keep, head_keep, quan
     k_{l+1} tokens of S_l by I_b and the top H_{l+1} heads by J_b.  Pruned rows of X stay frozen.
 
     Returns dict(X (full [B,T,D], frozen rows kept), x_final [B, k_{L-1}, D], kept [L][B] arrays,
-    heads [L][B] arrays, I [B,T], J [B,H], refetch [L], O [L][B] per-layer outputs).
+    heads [L][B] arrays, I [B,T], J [B,H], refetch [L], O [L][B] per-layer outputs, I_sel/J_sel
+    [L-1] copies of I and J at each selection).
     """
     X = np.array(X, np.float64)
     B, T, D = X.shape
@@ -261,7 +262,7 @@ def cascade_prefill(X, w_qkv, w_o, H: int, d_h: int, token_keep, head_keep, quan
     J = np.zeros((B, H))
     kept = [np.arange(T) for _ in range(B)]
     heads = [np.arange(H) for _ in range(B)]
-    kept_log, heads_log, O_log, refetch = [], [], [], []
+    kept_log, heads_log, O_log, refetch, I_sel, J_sel = [], [], [], [], [], []
     for l in range(L):
         assert all(len(s) == token_keep[l] for s in kept)
         assert all(len(hs) == head_keep[l] for hs in heads)
@@ -283,6 +284,8 @@ def cascade_prefill(X, w_qkv, w_o, H: int, d_h: int, token_keep, head_keep, quan
         O_log.append(O_l)
         refetch.append(rf)
         if l < L - 1:
+            I_sel.append(I.copy())
+            J_sel.append(J.copy())
             for b in range(B):
                 sel = topk_select(I[b, kept[b]], token_keep[l + 1])
                 kept[b] = kept[b][sel]
@@ -290,7 +293,7 @@ def cascade_prefill(X, w_qkv, w_o, H: int, d_h: int, token_keep, head_keep, quan
                 heads[b] = heads[b][hsel]
     x_final = np.stack([X[b, kept[b]] for b in range(B)])
     return dict(X=X, x_final=x_final, kept=kept_log, heads=heads_log, I=I, J=J,
-                refetch=refetch, O=O_log)
+                refetch=refetch, O=O_log, I_sel=I_sel, J_sel=J_sel)
 
 
 # ---------------------------------------------------------------------------------------------

@@ -1,0 +1,72 @@
+"""Helpers shared by the GPU parity tests: device buffers, the library handle, oracle comparisons.
+
+Inputs are seeded draws cast to the device dtype on the host (torch CPU), then copied to the
+GPU; the oracle receives the same cast values.  Nothing here computes what the method computes.
+"""
+import numpy as np
+import torch
+
+from oracle import spatten_ref as R
+
+BF = torch.bfloat16
+
+
+def lib():
+    from cascade_token_head_b200 import build
+    build.build()
+    from cascade_token_head_b200 import spatten
+    return spatten
+
+
+def to_dev(a, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dtype).cuda()
+
+
+def host_cast(a, dtype):
+    """The float64 values a device tensor of `dtype` holds after a host cast of `a`."""
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dtype).to(torch.float64).numpy()
+
+
+def ws(nbytes):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device="cuda")
+
+
+def rms(a):
+    return float(np.sqrt(np.mean(np.square(np.asarray(a, np.float64))))) + 1e-30
+
+
+def assert_close_rms(got, ref, frac, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.max(np.abs(got - ref)) if got.size else 0.0
+    bound = frac * rms(ref)
+    assert err <= bound, f"{what}: max |err| {err:.3e} > {frac} x RMS = {bound:.3e}"
+    return err / rms(ref)
+
+
+def planes_to_host(msb, lsb):
+    return msb.cpu().numpy(), lsb.cpu().numpy()
+
+
+def oracle_quantize_blocks(x32, gain32=None):
+    """Oracle quantization of every (b, h) block of x32 [B, H, n, d] (float32 values).
+    Returns msb [B,H,n,d] int8, packed lsb [B,H,n,d/2] uint8, scale [B,H] float32."""
+    B, H, n, d = x32.shape
+    msb = np.empty((B, H, n, d), np.int8)
+    lsb = np.empty((B, H, n, d // 2), np.uint8)
+    sc = np.empty((B, H), np.float32)
+    for b in range(B):
+        for h in range(H):
+            blk = x32[b, h]
+            if gain32 is not None:
+                blk = blk * gain32[b][:, None]
+            r = R.quantize_head(blk)
+            msb[b, h], lsb[b, h], sc[b, h] = r["msb"], R.pack_lsb(r["lsb"]), r["scale"]
+    return msb, lsb, sc
+
+
+def split_heads(x, H, d, which):
+    """[B, n, 3*H*d] -> [B, H, n, d] slice of q (0), k (1) or v (2)."""
+    B, n, _ = x.shape
+    s = x[:, :, which * H * d:(which + 1) * H * d]
+    return np.ascontiguousarray(s.reshape(B, n, H, d).transpose(0, 2, 1, 3))

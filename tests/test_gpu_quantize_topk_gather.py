@@ -1,0 +1,212 @@
+"""GPU parity of K1 (quantize), K4 (top-k) and K5 (gather) against the oracle: bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+from cascade_token_head_b200 import synth
+from oracle import spatten_ref as R
+
+from gpu_helpers import BF, host_cast, lib, oracle_quantize_blocks, split_heads, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------------------------------------
+# K1 quantize
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,B,H,n,d,gain", [
+    (BF, 2, 3, 1, 64, False), (BF, 2, 3, 7, 64, True), (BF, 3, 4, 517, 64, True), (BF, 1, 2, 300, 128, False),
+    (torch.float32, 2, 2, 129, 64, False), (BF, 1, 2, 5000, 128, True)])
+def test_quantize_bit_exact(cuda, dtype, B, H, n, d, gain):
+    S = lib()
+    g = synth.rng_for(n * 7 + d)
+    raw = g.standard_normal((B, n, 3 * H * d)) * 3.0
+    x = to_dev(raw, dtype)
+    gains = None
+    if gain:
+        gains = np.ones((B, n), np.float32)
+        gains[:, g.choice(n, size=max(1, n // 20), replace=False)] = 4.0
+    esz = 2 if dtype == BF else 4
+    msb = torch.zeros((B, H, n, d), dtype=torch.int8, device="cuda")
+    lsb = torch.zeros((B, H, n, d // 2), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(B * H, dtype=torch.float32, device="cuda")
+    gdev = to_dev(gains) if gain else None
+    S.quantize_kv(x.data_ptr() + H * d * esz, B, H, n, d, 3 * H * d, msb, lsb, n, 0, scale_out=sc,
+                  row_gain=gdev, ld_gain=n, dtype=S.dtype_code(x))
+    torch.cuda.synchronize()
+    k32 = split_heads(host_cast(raw, dtype), H, d, 1).astype(np.float32)
+    m_ref, l_ref, s_ref = oracle_quantize_blocks(k32, gains)
+    np.testing.assert_array_equal(sc.cpu().numpy().reshape(B, H), s_ref)
+    np.testing.assert_array_equal(msb.cpu().numpy(), m_ref)
+    np.testing.assert_array_equal(lsb.cpu().numpy(), l_ref)
+
+
+def test_quantize_full_size_bert_layer0(cuda):
+    """K of the BERT-base layer-0 projection shape [32, 12, 512, 64], bf16, with boosted rows."""
+    S = lib()
+    w = synth.bert_base_prefill()
+    g = synth.rng_for(1)
+    B, H, n, d = w.B, w.H, w.T, w.d_h
+    raw = g.standard_normal((B, n, 3 * H * d))
+    x = to_dev(raw, BF)
+    gains = np.ones((B, n), np.float32)
+    for b in range(B):
+        gains[b, g.choice(n, 26, replace=False)] = 4.0
+    msb = torch.empty((B, H, n, d), dtype=torch.int8, device="cuda")
+    lsb = torch.empty((B, H, n, d // 2), dtype=torch.uint8, device="cuda")
+    sc = torch.empty(B * H, dtype=torch.float32, device="cuda")
+    S.quantize_kv(x.data_ptr() + H * d * 2, B, H, n, d, 3 * H * d, msb, lsb, n, 0, scale_out=sc,
+                  row_gain=to_dev(gains), ld_gain=n, dtype=S.BF16)
+    torch.cuda.synchronize()
+    k32 = split_heads(host_cast(raw, BF), H, d, 1).astype(np.float32)
+    m_ref, l_ref, s_ref = oracle_quantize_blocks(k32, gains)
+    np.testing.assert_array_equal(sc.cpu().numpy().reshape(B, H), s_ref)
+    np.testing.assert_array_equal(msb.cpu().numpy(), m_ref)
+    np.testing.assert_array_equal(lsb.cpu().numpy(), l_ref)
+
+
+def test_quantize_append_with_scale_saturates(cuda):
+    S = lib()
+    B, H, d, cap = 2, 3, 64, 10
+    g = synth.rng_for(5)
+    raw = g.standard_normal((B, 1, 3 * H * d)) * 2.0
+    x = to_dev(raw, BF)
+    scales = np.full(B * H, 0.001, np.float32)      # small scale: many codes saturate
+    scales[0] = 0.05
+    msb = torch.zeros((B, H, cap, d), dtype=torch.int8, device="cuda")
+    lsb = torch.zeros((B, H, cap, d // 2), dtype=torch.uint8, device="cuda")
+    sat = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.quantize_kv(x.data_ptr() + 2 * H * d * 2, B, H, 1, d, 3 * H * d, msb, lsb, cap, 7, scale_in=to_dev(scales),
+                  sat_count=sat, dtype=S.BF16)
+    torch.cuda.synchronize()
+    v32 = split_heads(host_cast(raw, BF), H, d, 2).astype(np.float32)
+    want_sat = 0
+    for b in range(B):
+        for h in range(H):
+            r = R.quantize_head(v32[b, h], scale=scales[b * H + h])
+            want_sat += r["sat"]
+            np.testing.assert_array_equal(msb[b, h, 7].cpu().numpy(), r["msb"][0])
+            np.testing.assert_array_equal(lsb[b, h, 7].cpu().numpy(), R.pack_lsb(r["lsb"])[0])
+    assert int(sat.item()) == want_sat > 0
+    assert int(msb[:, :, :7].abs().sum().item()) == 0 and int(msb[:, :, 8:].abs().sum().item()) == 0
+
+
+# ------------------------------------------------------------------------------------------------
+# K4 top-k
+# ------------------------------------------------------------------------------------------------
+def _topk_gpu(S, scores_np, k, map_np=None):
+    R_, n = scores_np.shape if map_np is None else map_np.shape
+    sc = to_dev(scores_np)
+    out = torch.full((R_, max(k, 1)), -1, dtype=torch.int32, device="cuda")
+    comp = torch.full((R_, max(k, 1)), -1, dtype=torch.int32, device="cuda") if map_np is not None else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mp = to_dev(map_np, torch.int32) if map_np is not None else None
+    S.topk_select(sc, R_, n, scores_np.shape[1], k, out, max(k, 1), map=mp, ld_map=n if mp is not None else 0,
+                  comp_out=comp, dev_status=st)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()[:, :k], (comp.cpu().numpy()[:, :k] if comp is not None else None), int(st.item())
+
+
+@pytest.mark.parametrize("R_,n,k,kind", [
+    (3, 1, 1, "u"), (3, 1, 0, "u"), (4, 10, 3, "ties"), (5, 100, 100, "u"), (5, 100, 1, "u"),
+    (8, 517, 200, "ties"), (4, 4097, 2048, "zeros"), (6, 20000, 13, "ln"), (2, 70000, 35000, "ties"),
+    (3, 1000, 500, "const")])
+def test_topk_matches_oracle(cuda, R_, n, k, kind):
+    S = lib()
+    g = synth.rng_for(n + k)
+    if kind == "u":
+        x = g.random((R_, n)).astype(np.float32)
+    elif kind == "ln":
+        x = g.lognormal(0, 2, (R_, n)).astype(np.float32)
+    elif kind == "ties":
+        x = (g.integers(0, 5, (R_, n)) * 0.25 - 0.5).astype(np.float32)
+    elif kind == "zeros":
+        x = np.where(g.random((R_, n)) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
+        x[:, ::7] = -1.0
+    else:
+        x = np.full((R_, n), 3.0, np.float32)
+    got, _, st = _topk_gpu(S, x, k)
+    assert st == 0
+    for r in range(R_):
+        np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
+
+
+def test_topk_through_map_with_composition(cuda):
+    S = lib()
+    g = synth.rng_for(11)
+    Rr, T, n, k = 4, 900, 600, 250
+    imp = g.random((Rr, T)).astype(np.float32)
+    imp[:, ::10] = imp[:, 1::10]                    # ties across the gathered list
+    mp = np.stack([np.sort(g.choice(T, n, replace=False)) for _ in range(Rr)]).astype(np.int32)
+    got, comp, st = _topk_gpu(S, imp, k, mp)
+    assert st == 0
+    for r in range(Rr):
+        sel = R.topk_select(imp[r, mp[r]].astype(np.float64), k)
+        np.testing.assert_array_equal(got[r], sel)
+        np.testing.assert_array_equal(comp[r], mp[r][sel])
+
+
+def test_topk_nan_reports_status(cuda):
+    S = lib()
+    x = np.arange(50, dtype=np.float32)[None].repeat(2, 0)
+    x[1, 7] = np.nan
+    _, _, st = _topk_gpu(S, x, 10)
+    assert st == S.E_NONFINITE
+
+
+@pytest.mark.parametrize("N", [1024, 16384, 262144, 1048576])
+@pytest.mark.parametrize("dist", ["uniform", "lognormal"])
+def test_topk_sweep_full_size(cuda, N, dist):
+    """The top-k sweep workload (64 rows, 1 % exact duplicates), k = 10 % and 50 % of N.
+    Every row is checked bit-exact for N <= 256k; at N = 1M, 8 sampled rows are checked against the
+    oracle and every row against the selection properties."""
+    S = lib()
+    x = synth.draw_topk_row_block(64, N, dist, 0.01, seed=N % 9973 + (dist == "lognormal"))
+    rows = range(64) if N <= 262144 else [0, 9, 17, 30, 38, 45, 51, 63]
+    for frac in (0.1, 0.5):
+        k = int(frac * N)
+        got, _, st = _topk_gpu(S, x, k)
+        assert st == 0
+        for r in rows:
+            np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
+        # properties on every row: ascending, k distinct, threshold rule with lower-index ties
+        assert np.all(np.diff(got, axis=1) > 0)
+        for r in range(64):
+            kth = np.partition(x[r], N - k)[N - k]
+            sel_vals = x[r][got[r]]
+            assert np.all(sel_vals >= kth) and np.count_nonzero(x[r] > kth) <= k
+
+
+# ------------------------------------------------------------------------------------------------
+# K5 gather
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("row_bytes,align16", [(4, True), (12, False), (1536, True), (1540, False), (8192, True)])
+def test_gather_rows_and_compose(cuda, row_bytes, align16):
+    S = lib()
+    g = synth.rng_for(row_bytes)
+    Rr, n, k = 5, 300, 123
+    words = row_bytes // 4
+    src = g.integers(-2**31, 2**31 - 1, (Rr, n, words), dtype=np.int64).astype(np.int32)
+    idx = np.stack([np.sort(g.choice(n, k, replace=False)) for _ in range(Rr)]).astype(np.int32)
+    comp_in = g.integers(0, 10**6, (Rr, n)).astype(np.int32)
+    s = to_dev(src, torch.int32)
+    d = torch.zeros((Rr, k, words), dtype=torch.int32, device="cuda")
+    co = torch.zeros((Rr, k), dtype=torch.int32, device="cuda")
+    S.gather_kept(s, n * row_bytes, row_bytes, n, row_bytes, Rr, to_dev(idx, torch.int32), k, k, d, k * row_bytes,
+                  row_bytes, compose_in=to_dev(comp_in, torch.int32), ld_compose=n, compose_out=co)
+    torch.cuda.synchronize()
+    want = np.stack([src[r][idx[r]] for r in range(Rr)])
+    np.testing.assert_array_equal(d.cpu().numpy(), want)
+    np.testing.assert_array_equal(co.cpu().numpy(), np.stack([comp_in[r][idx[r]] for r in range(Rr)]))
+
+
+def test_gather_checked_index_reports(cuda):
+    S = lib()
+    src = to_dev(np.arange(40, dtype=np.int32).reshape(1, 10, 4), torch.int32)
+    idx = to_dev(np.array([[1, 3, 12]], np.int32), torch.int32)
+    d = torch.zeros((1, 3, 4), dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.gather_kept(src, 160, 16, 10, 16, 1, idx, 3, 3, d, 48, 16, check_index=1, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == S.E_INDEX
+    np.testing.assert_array_equal(d.cpu().numpy()[0, :2], np.arange(40).reshape(10, 4)[[1, 3]])
