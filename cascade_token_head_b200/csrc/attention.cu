@@ -65,6 +65,7 @@ int32_t validate(const spatten_attn_args& a) {
   }
   if (a.tok_imp && a.tok_imp_ld < (a.tok_imp_map ? 1 : a.n_kv)) return SPATTEN_E_SHAPE;
   if (a.tok_imp_map && a.tok_imp_map_ld < a.n_kv) return SPATTEN_E_SHAPE;
+  if (a.refetch_flags && a.refetch_flags_ld != 0 && a.refetch_flags_ld < a.n_q) return SPATTEN_E_SHAPE;
   const int esz = a.q_dtype == SPATTEN_BF16 ? 2 : 4;
   if (!aligned16(a.q) || !aligned16(a.o) || (a.q_ld_tok * esz) % 16 != 0 || (a.o_ld_tok * esz) % 16 != 0)
     return SPATTEN_E_ALIGN;
@@ -100,6 +101,7 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
   std::memcpy(&p.a, args, sizeof(spatten_attn_args));
   if (!(p.a.sm_scale > 0.0f)) p.a.sm_scale = 1.0f / std::sqrt(static_cast<float>(p.a.d_h));
   if (p.a.head_idx_ld == 0) p.a.head_idx_ld = p.a.H_kept;
+  if (p.a.refetch_flags_ld == 0) p.a.refetch_flags_ld = p.a.n_q;
   Path path;
   if (!choose_path(p.a, &path)) return SPATTEN_E_UNSUPPORTED;
   p.qt_rows = rows_per_cta(path);

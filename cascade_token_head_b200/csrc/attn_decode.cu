@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
   habs = block_sum(habs);
   if (threadIdx.x == 0) {
     p.head_part[static_cast<int64_t>(b) * a.H_kept + slot] = habs;
-    if (a.refetch_flags) a.refetch_flags[bh * a.n_q] = flag ? 1 : 0;
+    if (a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld] = flag ? 1 : 0;
     if (flag && a.refetch_count) atomicAdd(a.refetch_count, 1);
   }
   (void)any_flag;

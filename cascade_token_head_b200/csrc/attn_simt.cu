@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnProblem p) {
       st_from_float(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + d, acc_o[r][c]);
     }
     if (lane == 0 && a.refetch_flags)
-      a.refetch_flags[(static_cast<int64_t>(b) * a.H + h) * a.n_q + i] = flag[r] ? 1 : 0;
+      a.refetch_flags[(static_cast<int64_t>(b) * a.H + h) * a.refetch_flags_ld + i] = flag[r] ? 1 : 0;
   }
   habs = warp_sum(habs);
   int nflag = 0;

@@ -248,6 +248,7 @@ int32_t run_prefill(const spatten_cascade_cfg& c, const spatten_layer_weights* w
     a.tok_imp_map_ld = T;
     a.head_imp = io.head_imp;
     a.refetch_flags = io.trace_flags ? io.trace_flags + static_cast<int64_t>(l) * B * H * T : nullptr;
+    a.refetch_flags_ld = T;
     a.refetch_count = io.refetch_count + l;
     a.dev_status = io.dev_status;
     SPT_TRY(attention_layer_timed(&a, ws.attn_ws, ws.attn_ws_bytes, st, ev(io, 2 * l), ev(io, 2 * l + 1)));
@@ -336,6 +337,7 @@ int32_t run_decode(const spatten_cascade_cfg& c, const spatten_layer_weights* w,
     a.tok_imp_map_ld = cap;
     a.head_imp = io.head_imp;
     a.refetch_flags = io.trace_flags ? io.trace_flags + static_cast<int64_t>(l) * B * H : nullptr;
+    a.refetch_flags_ld = 1;
     a.refetch_count = io.refetch_count ? io.refetch_count + l : nullptr;
     a.dev_status = io.dev_status;
     SPT_TRY(attention_layer_timed(&a, ws.attn_ws, ws.attn_ws_bytes, st, ev(io, 2 * l), ev(io, 2 * l + 1)));

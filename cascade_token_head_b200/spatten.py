@@ -38,7 +38,8 @@ class attn_args(C.Structure):
                 ("sm_scale", f32), ("refetch_threshold", f32),
                 ("o", vp), ("o_ld_tok", i64), ("zero_pruned_heads", i32),
                 ("tok_imp", vp), ("tok_imp_ld", i64), ("tok_imp_map", vp), ("tok_imp_map_ld", i64),
-                ("head_imp", vp), ("refetch_flags", vp), ("refetch_count", vp), ("dev_status", vp),
+                ("head_imp", vp), ("refetch_flags", vp), ("refetch_flags_ld", i64), ("refetch_count", vp),
+                ("dev_status", vp),
                 ("kernel", i32)]
 
 

@@ -146,7 +146,8 @@ typedef struct spatten_attn_args {
   int64_t tok_imp_map_ld;
   float* head_imp;           /* device [B][H] (+=) or NULL                                   */
 
-  uint8_t* refetch_flags;    /* device [B][H][n_q] (written for kept heads) or NULL          */
+  uint8_t* refetch_flags;    /* device [B][H][refetch_flags_ld] (kept heads written) or NULL  */
+  int64_t refetch_flags_ld;  /* row stride of refetch_flags; 0 = n_q                          */
   int32_t* refetch_count;    /* device int32 (+= number of refetched rows) or NULL           */
   int32_t* dev_status;       /* device int32 or NULL                                         */
   int32_t kernel;            /* spatten_attn_kernel: 0 = choose automatically                */

@@ -44,6 +44,18 @@ def assert_close_rms(got, ref, frac, what=""):
     return err / rms(ref)
 
 
+def assert_close_bf16_out(got, ref, frac, what=""):
+    """A bf16-stored intermediate: max |got - ref| <= frac x RMS(ref) + one bf16 ulp of |ref|
+    (2**-8 |ref|), the representation error of the stored value itself."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    bound = frac * rms(ref) + 2.0 ** -8 * np.abs(ref)
+    excess = np.abs(got - ref) - bound
+    worst = float(excess.max()) if excess.size else -1.0
+    assert worst <= 0, f"{what}: error exceeds {frac} x RMS + 1 bf16 ulp by {worst:.3e}"
+    return float(np.max(np.abs(got - ref)) / rms(ref)) if got.size else 0.0
+
+
 def planes_to_host(msb, lsb):
     return msb.cpu().numpy(), lsb.cpu().numpy()
 

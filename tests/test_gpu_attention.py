@@ -16,7 +16,8 @@ import torch
 from cascade_token_head_b200 import synth
 from oracle import spatten_ref as R
 
-from gpu_helpers import BF, assert_close_rms, host_cast, lib, oracle_quantize_blocks, split_heads, to_dev, ws
+from gpu_helpers import (BF, assert_close_bf16_out, assert_close_rms, host_cast, lib, oracle_quantize_blocks,
+                         split_heads, to_dev, ws)
 
 pytestmark = pytest.mark.gpu
 
@@ -143,7 +144,14 @@ def oracle_layer(raw, gain, B, H, n, d, theta, heads, dtype, got, kv_idx=None, n
 
 def check(got, ref, heads, H, d, tol_o, tol_head, dtype_name):
     B = got["o"].shape[0]
-    assert_close_rms(got["o"], ref["O"], tol_o, f"O ({dtype_name})")
+    kept_cols = [np.concatenate([np.arange(h * d, (h + 1) * d) for h in (range(H) if heads is None else heads[b])])
+                 for b in range(B)]
+    go = np.stack([got["o"][b][:, kept_cols[b]] for b in range(B)])
+    ro = np.stack([ref["O"][b][:, kept_cols[b]] for b in range(B)])
+    if dtype_name == "fp32":
+        assert_close_rms(go, ro, tol_o, "O (fp32)")
+    else:
+        assert_close_bf16_out(go, ro, tol_o, f"O ({dtype_name})")
     # pruned heads are zero-filled
     if heads is not None:
         for b in range(B):
