@@ -76,6 +76,8 @@ lib.spatten_attention_workspace_size.restype = sz
 lib.spatten_attention_workspace_size.argtypes = [C.POINTER(attn_args)]
 lib.spatten_attention_layer.restype = i32
 lib.spatten_attention_layer.argtypes = [C.POINTER(attn_args), vp, sz, vp]
+lib.spatten_attention_layer_noalloc.restype = i32
+lib.spatten_attention_layer_noalloc.argtypes = [C.POINTER(attn_args), vp]
 lib.spatten_topk_workspace_size.restype = sz
 lib.spatten_topk_workspace_size.argtypes = [i32, i32, i32]
 lib.spatten_topk_select.restype = i32
@@ -90,7 +92,8 @@ lib.spatten_cascade_forward.argtypes = [C.POINTER(cascade_cfg), C.POINTER(layer_
 # every extern "C" symbol of include/spatten.h
 EXPORTS = ["spatten_abi_version", "spatten_status_string", "spatten_last_cuda_error",
            "spatten_kernel_launch_count", "spatten_quantize_kv",
-           "spatten_attention_workspace_size", "spatten_attention_layer", "spatten_topk_workspace_size",
+           "spatten_attention_workspace_size", "spatten_attention_layer", "spatten_attention_layer_noalloc",
+           "spatten_topk_workspace_size",
            "spatten_topk_select", "spatten_gather_kept", "spatten_cascade_workspace_size",
            "spatten_cascade_forward"]
 
@@ -149,6 +152,14 @@ def attention_workspace_size(args: attn_args) -> int:
 
 def attention_layer(args: attn_args, ws, ws_bytes: int, stream=None):
     check(lib.spatten_attention_layer(C.byref(args), ptr(ws), ws_bytes, _stream(stream)), "spatten_attention_layer")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20   # SPATTEN_NOALLOC_SCRATCH_BYTES
+
+
+def attention_layer_noalloc(args: attn_args, stream=None):
+    """The attention layer without a caller workspace (library-owned scratch; see spatten.h)."""
+    check(lib.spatten_attention_layer_noalloc(C.byref(args), _stream(stream)), "spatten_attention_layer_noalloc")
 
 
 def topk_workspace_size(R: int, n: int, k: int) -> int:

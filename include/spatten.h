@@ -169,6 +169,30 @@ size_t spatten_attention_workspace_size(const spatten_attn_args* a);
 int32_t spatten_attention_layer(const spatten_attn_args* a, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * spatten_attention_layer_noalloc -- spatten_attention_layer for callers that cannot allocate.
+ * (The paper has no counterpart: this is a deployment convenience of this library.)
+ *
+ * Some callers have no way to allocate device memory at all -- a plugin whose host application
+ * owns every allocation, a real-time loop that must never enter the CUDA allocator, code that is
+ * only handed its input and output buffers -- and so cannot supply the workspace the call above
+ * needs.  This entry point takes the same arguments without (ws, ws_bytes): its scratch lives in
+ * a fixed array of SPATTEN_NOALLOC_SCRATCH_BYTES in device global memory owned by the library,
+ * which every GPU that loads the library holds until the process exits.  It calls no
+ * cudaMalloc/cudaFree and no allocating library routine.
+ *  - Limit: problems whose spatten_attention_workspace_size() exceeds the array are rejected with
+ *    SPATTEN_E_WORKSPACE before anything is launched (use the workspace entry point for them).
+ *  - Set-up: the first call on each device (with that device current) looks up the array's
+ *    device address with cudaGetSymbolAddress and caches it; make that first call before any
+ *    stream capture.
+ *  - Sharing: all calls use the same array, so calls that overlap on the GPU (other streams or
+ *    threads) race on it; serialise them.  Everything a call reads from the array it has written
+ *    itself first, so no clearing is needed between calls.
+ * The caller still passes every input and output buffer in `a`, as for the call above.
+ * --------------------------------------------------------------------------------------------- */
+#define SPATTEN_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+int32_t spatten_attention_layer_noalloc(const spatten_attn_args* a, void* stream);
+
 /* =============================================================================================
  * spatten_topk_select -- per row, the k indices with the largest scores, ranked by (higher
  * score, then lower index), written in ascending order (§II "Cascade pruning": keep the top-k
