@@ -72,13 +72,34 @@ int32_t validate(const spatten_attn_args& a) {
   return SPATTEN_OK;
 }
 
-size_t layout(const spatten_attn_args& a, int rows, void* ws, float** tok, float** head) {
+size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
+  const int rows = rows_per_cta(path);
   const int64_t n_qt = ceil_div(a.n_q, rows);
-  WsCursor c(ws, ~size_t(0));
+  WsCursor c(p ? p->tok_part : nullptr, ~size_t(0));
   float* t = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * n_qt * a.n_kv);
   float* h = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * n_qt);
-  if (tok) *tok = t;
-  if (head) *head = h;
+  int32_t* fl = nullptr;
+  int32_t* fc = nullptr;
+  float* fp = nullptr;
+  float* fh = nullptr;
+  const int64_t n_pair = ceil_div(a.n_q, 256);
+  if (path == Path::kTc) {
+    fl = c.take<int32_t>(static_cast<size_t>(a.B) * a.H_kept * n_pair * 256);
+    fc = c.take<int32_t>(static_cast<size_t>(a.B) * a.H_kept * n_pair);
+    fp = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * 2 * n_pair * a.n_kv);
+    fh = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * 2 * n_pair);
+  }
+  if (p) {
+    p->qt_rows = rows;
+    p->n_qt = static_cast<int>(n_qt);
+    p->tok_part = t;
+    p->head_part = h;
+    p->n_pair = static_cast<int>(n_pair);
+    p->flag_list = fl;
+    p->flag_cnt = fc;
+    p->full_part = fp;
+    p->full_head = fh;
+  }
   return c.used;
 }
 
@@ -89,7 +110,7 @@ extern "C" size_t spatten_attention_workspace_size(const spatten_attn_args* a) {
   using namespace spt;
   Path path;
   if (!a || validate(*a) != SPATTEN_OK || !choose_path(*a, &path)) return 0;
-  return layout(*a, rows_per_cta(path), nullptr, nullptr, nullptr);
+  return layout(*a, path, nullptr);
 }
 
 namespace spt {
@@ -104,9 +125,8 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
   if (p.a.refetch_flags_ld == 0) p.a.refetch_flags_ld = p.a.n_q;
   Path path;
   if (!choose_path(p.a, &path)) return SPATTEN_E_UNSUPPORTED;
-  p.qt_rows = rows_per_cta(path);
-  p.n_qt = static_cast<int>(ceil_div(p.a.n_q, p.qt_rows));
-  const size_t need = layout(p.a, p.qt_rows, ws, &p.tok_part, &p.head_part);
+  p.tok_part = static_cast<float*>(ws);
+  const size_t need = layout(p.a, path, &p);
   if (!ws || ws_bytes < need) return SPATTEN_E_WORKSPACE;
   if (ev_begin) SPT_CUDA(cudaEventRecord(ev_begin, st));
   int32_t s;

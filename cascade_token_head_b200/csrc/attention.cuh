@@ -12,6 +12,13 @@ struct AttnProblem {
   int n_qt;                  // query tiles = ceil(n_q / qt_rows)
   float* tok_part;           // ws [B][H_kept][n_qt][n_kv] per-CTA column sums of P
   float* head_part;          // ws [B][H_kept][n_qt] per-CTA sum |O|
+  // tensor-core path only: query rows flagged for refetch are recomputed at full precision by a
+  // second kernel, in packed 128-row tiles of the flagged rows of each 256-row query pair tile
+  int n_pair;                // ceil(n_q / 256)
+  int32_t* flag_list;        // ws [B][H_kept][n_pair][256] flagged row ids, ascending
+  int32_t* flag_cnt;         // ws [B][H_kept][n_pair] number of flagged rows
+  float* full_part;          // ws [B][H_kept][2*n_pair][n_kv] column sums of the packed tiles
+  float* full_head;          // ws [B][H_kept][2*n_pair] sum |O| of the packed tiles
 };
 
 // Kernels (each returns a status after launching on `st`).

@@ -1,33 +1,39 @@
-// K2: prefill attention with importance on the 5th-generation tensor cores (tcgen05 + TMEM),
-// warp-specialized and pipelined.
+// K2: prefill attention with importance on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
 // SpAtten §II "Attention mechanism" (S = Q K^T scaled, row softmax, P V), §II "Cascade pruning"
 // (token importance = column sums of P; head importance = sum |O|), §IV.E "Progressive
 // Quantization" (MSB pass; rows whose max probability is below the threshold are recomputed with
-// the LSBs).  One CTA = (sequence, kept head, 128 query rows).
+// the LSBs).
 //
-// Exact operands: K and V are 12-bit codes q = 16*MSB + LSB; 16*MSB (8 significant bits) and
-// LSB (0..15) are exact in bf16, so the MMAs see the codes unrounded and the scales multiply the
-// float32 accumulators:
-//   S_msb = s_k * sm * (Q . (16 MSB)^T),   S_full = S_msb + s_k * sm * (Q . LSB^T)
-//   O     = s_v * (P . 16 MSB_v  [+ P . LSB_v for refetched rows])
-// The LSB products land in their own TMEM columns; each softmax thread adds them only for its own
-// row when that row refetches, so no masked operand copies are needed.
+// Exact operands: K and V are 12-bit codes q = 16*MSB + LSB; 16*MSB (8 significant bits) and LSB
+// (0..15) are exact in bf16, so the MMAs see the codes unrounded and the scales multiply the
+// float32 accumulators:  S = s_k*sm*(Q.(16 MSB)^T [+ Q.LSB^T]),  O = s_v*(P.16 MSB_v [+ P.LSB_v]).
 //
-// Roles (256 threads):
-//   warps 0-3  softmax: thread i owns query row i = TMEM lane i (warp w reads lane quadrant w)
-//   warps 4-6  producers: load Q once, dequantize K/V code tiles into 2-stage shared rings
-//   warp 7     MMA issue (lane 0) and TMEM allocation
-// Key tiles hold 16 KB of bf16 codes: 128 keys at d_h = 64, 64 keys at d_h = 128.
-// Passes over the keys (all pipelined through mbarriers; every wait is bounded):
-//   A   S_msb tiles (double-buffered in TMEM) -> online row max / exp-sum -> refetch flags
-//   A'  only if some row is flagged: S and C = Q.LSB^T (single-buffered) -> stats of flagged rows
-//   B   S (+C) -> P = exp(S - m)/ell in float32 -> column sums by a 31-shuffle butterfly
-//       (deterministic) -> P in bf16 to shared memory (double-buffered) -> O += P V (+ O_lsb)
-//       with QK of tile t+1 issued before PV of tile t
-// Operand layouts: UMMA 128-byte swizzle; Q, K, P K-major; V MN-major (plain key rows).
-// TMEM (512 columns): S buffers [0, 2*KT), O [2*KT, 2*KT + d_h), O_lsb after it; in refetch mode
-// S uses buffer 0 and C buffer 1.
+// Two kernels per layer:
+//  MAIN  one CTA = (sequence, kept head, 256 query rows), 384 threads:
+//          warps 0-7   two softmax warpgroups; warpgroup g owns query rows 128g..128g+127 of the
+//                      CTA, thread r of a warpgroup is TMEM lane r of that warpgroup's S and O
+//          warps 8-10  producers: Q once, then K/V MSB tiles dequantized into 2-stage rings
+//          warp 11     MMA issue (lane 0) and TMEM allocation
+//        pass A computes S_msb tile by tile (the two warpgroups' tiles alternate on the tensor
+//        core while the other warpgroup runs its softmax) -> row max / exp-sum -> refetch flags;
+//        the flagged rows of the CTA are written, ascending, to a packed list.  Pass B computes
+//        P = exp(S - m)/ell for the other rows (float32), column sums by a 31-shuffle butterfly
+//        (deterministic), P in bf16 to shared memory, O += P V.  Flagged rows contribute nothing
+//        here.
+//  FULL  one CTA = 128 consecutive entries of the head's flagged rows (the MAIN lists of its pair
+//        tiles concatenated in order; launched only when theta > 0; CTAs past the end exit at
+//        once), 256 threads (4 softmax, 3 producer, 1 MMA warps): the same two passes with
+//        S = Q.(16 MSB)^T + Q.LSB^T and O = P.16 MSB_v + P.LSB_v accumulated in the same TMEM
+//        columns, reading the LSB planes only for heads with flagged rows.
+// Producers: without an index list the raw code rows of a key tile are contiguous, so one thread
+// keeps several tiles in flight with 1-D bulk copies (TMA engine) into a staging ring, and the
+// producer warps convert staged int8 / packed-nibble tiles to swizzled bf16 shared -> shared.
+// Partial column sums (per 128-row tile) and sum |O| go to the workspace; attn_reduce adds them in
+// a fixed order, so reruns are bit-identical.
+// Operand layouts: UMMA 128-byte swizzle; Q, K, P K-major; V MN-major (plain key rows).  Key tiles
+// hold 16 KB of bf16 codes: 128 keys at d_h = 64, 64 keys at d_h = 128.  Every mbarrier wait is
+// bounded: on timeout the CTA reports SPATTEN_E_TIMEOUT, frees its TMEM and returns.
 #include "attention.cuh"
 #include "tc_ptx.cuh"
 
@@ -36,48 +42,10 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 256;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kProducerThreads = 96;
-constexpr int kMmaWarp = 7;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWaitLimit = 1u << 26;   // polls of one mbarrier phase before giving up
 constexpr float kLog2e = 1.4426950408889634f;
-
-template <int DH>
-struct Cfg {
-  static constexpr int KT = DH == 64 ? 128 : 64;            // keys per tile
-  static constexpr uint32_t QB = 128u * DH * 2u;             // Q tile bytes
-  static constexpr uint32_t TB = static_cast<uint32_t>(KT) * DH * 2u;   // K or V tile (16 KB)
-  static constexpr uint32_t PB = 128u * KT * 2u;             // P tile bytes
-  static constexpr uint32_t oQ = 0;
-  static constexpr uint32_t oK = oQ + QB;                    // 2 stages
-  static constexpr uint32_t oKL = oK + 2 * TB;
-  static constexpr uint32_t oV = oKL + 2 * TB;
-  static constexpr uint32_t oVL = oV + 2 * TB;
-  static constexpr uint32_t oP = oVL + 2 * TB;               // 2 buffers
-  static constexpr uint32_t kEnd = oP + 2 * PB;
-  static constexpr uint32_t kSmem = kEnd + 1024u;
-  static constexpr uint32_t tS = 0;                          // TMEM column offsets
-  static constexpr uint32_t tO = 2u * KT;
-  static constexpr uint32_t tO2 = 2u * KT + DH;
-  static constexpr int CH = KT / 32;                         // 32-column chunks per tile
-};
-
-// barrier slots
-enum : int {
-  B_Q = 0,
-  B_KFULL = 1,    // +stage (2)
-  B_KEMPTY = 3,   // +stage
-  B_VFULL = 5,    // +stage
-  B_VEMPTY = 7,   // +stage
-  B_SFULL = 9,    // +buffer
-  B_SFREE = 11,   // +buffer
-  B_PFULL = 13,   // +buffer
-  B_PFREE = 15,   // +buffer
-  B_ODONE = 17,
-  B_COUNT = 18
-};
+constexpr int kProducerThreads = 96;
 
 // byte offset of 16-byte chunk c8 of `row` in a tile whose 64-element column blocks each hold
 // `rows` rows of 128 bytes (128-byte swizzle)
@@ -110,7 +78,9 @@ __device__ __forceinline__ void cvt_u4x16(uint2 raw, uint32_t* out8) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 // bounded wait that also gives up once another role has aborted
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -138,56 +108,620 @@ __device__ __forceinline__ float warp_colsum32(float* v) {
   return v[0];
 }
 
-enum Pass { kPassA = 0, kPassA2 = 1, kPassB = 2 };
+// two column-sum butterflies interleaved (independent chains, twice the ILP)
+__device__ __forceinline__ void warp_colsum32x2(float* v, float* w, float& sv, float& sw) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < off; ++j) {
+      const float send_v = upper ? v[j] : v[j + off];
+      const float keep_v = upper ? v[j + off] : v[j];
+      const float send_w = upper ? w[j] : w[j + off];
+      const float keep_w = upper ? w[j + off] : w[j];
+      v[j] = keep_v + __shfl_xor_sync(0xffffffffu, send_v, off);
+      w[j] = keep_w + __shfl_xor_sync(0xffffffffu, send_w, off);
+    }
+  }
+  sv = v[0];
+  sw = w[0];
+}
+
+// running max / exp-sum update over 64 log2-domain scores (independent partial sums)
+__device__ __forceinline__ void stats64(const float* v, float& m2, float& l) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    mx[k] = v[k];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mx[k] = fmaxf(mx[k], v[k + 8 * j]);
+  }
+  const float mm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  if (mm == -INFINITY) return;
+  const float mn = fmaxf(m2, mm);
+  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int j = 0; j < 64; ++j) s[j & 3] += ex2(v[j] - mn);
+  l = l * ex2(m2 - mn) + ((s[0] + s[1]) + (s[2] + s[3]));
+  m2 = mn;
+}
+
+template <int DH, int KT>
+__device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int64_t plane0, const int32_t* kv_idx,
+                                             const int8_t* msb, const uint8_t* lsb, uint32_t off_hi,
+                                             uint32_t off_lo, int ptid) {
+  constexpr int L16 = DH / 16;
+  for (int e = ptid; e < KT * L16; e += kProducerThreads) {
+    const int r = e / L16, c16 = e % L16;
+    const int key = t * KT + r;
+    uint32_t hi[8], lo[8];
+    if (key < n_kv) {
+      const int64_t prow = plane0 + (kv_idx ? kv_idx[key] : key);
+      cvt16_s8x16(__ldg(reinterpret_cast<const uint4*>(msb + prow * DH) + c16), hi);
+      if (lsb) cvt_u4x16(__ldg(reinterpret_cast<const uint2*>(lsb + prow * (DH / 2)) + c16), lo);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
+    }
+    *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16, KT)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+    if (lsb) {
+      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16, KT)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    }
+  }
+  fence_async_smem();
+}
+
+// same conversion from a staged raw tile in shared memory: MSB rows (DH bytes each) at raw,
+// packed LSB rows (DH/2 bytes) at raw + KT*DH; rows >= valid are zero-filled
+template <int DH, int KT>
+__device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw, bool with_lsb, int valid,
+                                               uint32_t off_hi, uint32_t off_lo, int ptid) {
+  constexpr int L16 = DH / 16;
+  for (int e = ptid; e < KT * L16; e += kProducerThreads) {
+    const int r = e / L16, c16 = e % L16;
+    uint32_t hi[8], lo[8];
+    if (r < valid) {
+      cvt16_s8x16(*reinterpret_cast<const uint4*>(raw + r * DH + c16 * 16), hi);
+      if (with_lsb) cvt_u4x16(*reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8), lo);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
+    }
+    *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16, KT)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+    if (with_lsb) {
+      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16, KT)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    }
+  }
+  fence_async_smem();
+}
+
+// The producers' work as one job stream: jobs 0..T-1 are the K tiles of pass A, then pass B
+// alternates K(t), V(t).  Without an index list the raw code rows of a tile are contiguous, so one
+// loader thread keeps RS tiles in flight with 1-D bulk copies (TMA engine) into a staging ring and
+// all producer threads convert staged tiles shared -> shared; with an index list they load rows
+// directly.  `emit(is_v, t, stage_dst_hi, stage_dst_lo)` gives the destination of the converted
+// tile and performs the ring handshake around `fill`.
+template <int DH, int KT, int RS>
+struct JobStream {
+  static constexpr uint32_t kMsb = KT * DH;
+  uint8_t* smem;
+  uint32_t o_raw, raw_bytes;   // staging ring: RS slots of raw_bytes
+  uint64_t* raw_full;          // [RS]
+  uint64_t* raw_empty;         // [RS], count kProducerThreads
+  const spatten_attn_args* a;
+  int64_t plane0;
+  int n_tiles;
+  bool with_lsb;
+  int ptid;
+  volatile int* abort_flag;
+  uint32_t issued = 0;
+
+  __device__ __forceinline__ int jobs() const { return 3 * n_tiles; }
+  __device__ __forceinline__ void job(int j, bool& is_v, int& t) const {
+    if (j < n_tiles) {
+      is_v = false;
+      t = j;
+    } else {
+      is_v = ((j - n_tiles) & 1) != 0;
+      t = (j - n_tiles) >> 1;
+    }
+  }
+  __device__ __forceinline__ int valid_rows(int t) const { return min(KT, a->n_kv - t * KT); }
+  // loader only: issue jobs up to j + RS - 1
+  __device__ __forceinline__ bool issue_ahead(int j) {
+    while (static_cast<int>(issued) < jobs() && static_cast<int>(issued) < j + RS) {
+      const uint32_t jn = issued;
+      const uint32_t st = jn % RS;
+      if (!wait_bar(&raw_empty[st], ((jn / RS) & 1u) ^ 1u, abort_flag)) return false;
+      bool is_v;
+      int t;
+      job(static_cast<int>(jn), is_v, t);
+      const int rows = valid_rows(t);
+      const int64_t row0 = plane0 + static_cast<int64_t>(t) * KT;
+      const uint32_t mb = static_cast<uint32_t>(rows) * DH, lb = with_lsb ? mb / 2 : 0u;
+      uint8_t* dst = smem + o_raw + st * raw_bytes;
+      mbar_arrive_expect_tx(&raw_full[st], mb + lb);
+      bulk_g2s(dst, (is_v ? a->v_msb : a->k_msb) + row0 * DH, mb, &raw_full[st]);
+      if (with_lsb) bulk_g2s(dst + kMsb, (is_v ? a->v_lsb : a->k_lsb) + row0 * (DH / 2), lb, &raw_full[st]);
+      ++issued;
+    }
+    return true;
+  }
+  // convert job j into (off_hi, off_lo); returns false on abort
+  __device__ __forceinline__ bool convert(int j, uint32_t off_hi, uint32_t off_lo, const int32_t* kv_idx) {
+    bool is_v;
+    int t;
+    job(j, is_v, t);
+    if (kv_idx) {
+      produce_tile<DH, KT>(smem, t, a->n_kv, plane0, kv_idx, is_v ? a->v_msb : a->k_msb,
+                           with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, off_lo, ptid);
+      return true;
+    }
+    const uint32_t st = static_cast<uint32_t>(j) % RS;
+    if (!wait_bar(&raw_full[st], (static_cast<uint32_t>(j) / RS) & 1u, abort_flag)) return false;
+    convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, off_lo, ptid);
+    mbar_arrive(&raw_empty[st]);
+    return true;
+  }
+};
+
+// QK^T into `d` (accumulate onto it when acc != 0), A = Q tile [128 x DH], B = key tile [KT x DH]
+template <int DH, int KT>
+__device__ __forceinline__ void mma_qk(uint32_t d, uint32_t sQ, uint32_t sK, uint32_t acc) {
+  constexpr uint32_t id = idesc_bf16(128, KT, false, false);
+#pragma unroll
+  for (int s = 0; s < DH / 16; ++s) {
+    const uint32_t qoff = (s >> 2) * 16384u + (s & 3) * 32u;
+    const uint32_t koff = (s >> 2) * (KT * 128u) + (s & 3) * 32u;
+    mma_bf16(d, desc_sw128(sQ + qoff, 16, 1024), desc_sw128(sK + koff, 16, 1024), id, (acc || s > 0) ? 1u : 0u);
+  }
+}
+// P V into `d`: A = P tile [128 x KT] K-major, B = V tile [KT keys x DH] MN-major
+template <int DH, int KT>
+__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t sP, uint32_t sV, uint32_t acc) {
+  constexpr uint32_t id = idesc_bf16(128, DH, false, true);
+#pragma unroll
+  for (int s = 0; s < KT / 16; ++s) {
+    const uint32_t poff = (s >> 2) * 16384u + (s & 3) * 32u;
+    mma_bf16(d, desc_sw128(sP + poff, 16, 1024), desc_sw128(sV + s * 2048u, KT * 128u, 1024), id,
+             (acc || s > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void store_o_row(__nv_bfloat16* dst, const float* v, float vs, float& habs) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float x0 = v[2 * j] * vs, x1 = v[2 * j + 1] * vs;
+    habs += fabsf(x0) + fabsf(x1);
+    pk[j] = pack_bf16x2(x0, x1);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+}
+
+// =================================================================================================
+// MAIN kernel
+// =================================================================================================
+template <int DH>
+struct MainCfg {
+  static constexpr int KT = DH == 64 ? 128 : 64;
+  static constexpr int NST = 2;                  // bf16 K and V ring stages
+  static constexpr int RS = 4;                   // raw code tiles in flight (bulk copies)
+  static constexpr uint32_t QB = 128u * DH * 2u;
+  static constexpr uint32_t TB = static_cast<uint32_t>(KT) * DH * 2u;
+  static constexpr uint32_t PB = 128u * KT * 2u;
+  static constexpr uint32_t RAWB = static_cast<uint32_t>(KT) * DH;   // one raw MSB tile
+  static constexpr uint32_t oQ = 0;              // 2 query tiles
+  static constexpr uint32_t oK = 2 * QB;         // NST stages
+  static constexpr uint32_t oV = oK + NST * TB;  // NST stages
+  static constexpr uint32_t oP = oV + NST * TB;  // one P tile per warpgroup
+  static constexpr uint32_t oRaw = oP + 2 * PB;  // RS staging slots
+  static constexpr uint32_t kSmem = oRaw + RS * RAWB + 1024u;
+  static constexpr uint32_t tS = 0;              // + g * KT
+  static constexpr uint32_t tO = 2u * KT;        // + g * DH
+};
+
+enum : int { M_Q = 0, M_KF = 1, M_KE = 3, M_VF = 5, M_VE = 7, M_SF = 9, M_SR = 11, M_PF = 13, M_PE = 15, M_OD = 17,
+             M_RF = 18, M_RE = 22, M_N = 26 };
 
 template <int DH>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnProblem p) {
-  using C = Cfg<DH>;
+__global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
+  using C = MainCfg<DH>;
   constexpr int KT = C::KT;
+  constexpr int NST = C::NST;
   const spatten_attn_args& a = p.a;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bars[B_COUNT];
+  __shared__ uint64_t bars[M_N];
   __shared__ uint32_t tmem_base_s;
-  __shared__ float colred[2][4][KT];
-  __shared__ float hred[4];
+  __shared__ float colred[2][2][4][KT];    // [tile parity][warpgroup][warp][key]
+  __shared__ float hred[2][4];
+  __shared__ uint32_t wcnt[8];
   __shared__ int abort_s;
 
-  const int qt = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const int pair = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i0 = qt * 128;
+  const int i0 = pair * 256;
   const int h = head_of_slot(a, b, slot);
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
 
   if (slot >= a.H_kept) {   // pruned head: zero its output rows (no TMEM, no barrier)
     if (h < 0) return;
-    for (int e = tid; e < 128 * (DH / 8); e += kThreads) {
+    for (int e = tid; e < 256 * (DH / 8); e += 384) {
       const int i = i0 + e / (DH / 8), c8 = e % (DH / 8);
       if (i < a.n_q)
-        *reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok +
-                                  static_cast<int64_t>(h) * DH + c8 * 8) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8) =
+            make_uint4(0, 0, 0, 0);
     }
     return;
   }
 
-  if (warp == kMmaWarp) {
+  if (warp == 11) {
     tmem_alloc(&tmem_base_s, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
     abort_s = 0;
-    mbar_init(&bars[B_Q], kProducerThreads);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[B_KFULL + s], kProducerThreads);
-      mbar_init(&bars[B_VFULL + s], kProducerThreads);
-      mbar_init(&bars[B_KEMPTY + s], 1);
-      mbar_init(&bars[B_VEMPTY + s], 1);
-      mbar_init(&bars[B_SFULL + s], 1);
-      mbar_init(&bars[B_SFREE + s], kSoftmaxThreads);
-      mbar_init(&bars[B_PFULL + s], kSoftmaxThreads);
-      mbar_init(&bars[B_PFREE + s], 1);
+    mbar_init(&bars[M_Q], kProducerThreads);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars[M_KF + s], kProducerThreads);
+      mbar_init(&bars[M_VF + s], kProducerThreads);
+      mbar_init(&bars[M_KE + s], 1);
+      mbar_init(&bars[M_VE + s], 1);
     }
-    mbar_init(&bars[B_ODONE], 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bars[M_SF + g], 1);
+      mbar_init(&bars[M_SR + g], 128);
+      mbar_init(&bars[M_PF + g], 128);
+      mbar_init(&bars[M_PE + g], 1);
+    }
+    mbar_init(&bars[M_OD], 1);
+    for (int s = 0; s < C::RS; ++s) {
+      mbar_init(&bars[M_RF + s], 1);
+      mbar_init(&bars[M_RE + s], kProducerThreads);
+    }
+    fence_mbar_init();
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort_flag = &abort_s;
+
+  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+  const int64_t plane0 = bh * a.kv_cap;
+  const int n_tiles = (a.n_kv + KT - 1) / KT;
+  const int64_t list_base = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_pair + pair);
+  const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
+  bool aborted = false;
+
+  // softmax thread state
+  const int g = warp >> 2;                        // warpgroup
+  const int r = tid & 127;                        // row within the warpgroup's tile
+  const int i = i0 + g * 128 + r;
+  const bool row_ok = warp < 8 && i < a.n_q;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const float c2 = a.k_scale[bh] * a.sm_scale * kLog2e;
+  float m2 = -INFINITY, l = 0.0f;
+  bool flag = false;
+
+  if (warp >= 8 && warp < 11) {
+    // ------------------------------------------------------------------------- producers
+    const int ptid = tid - 256;
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+    for (int e = ptid; e < 256 * (DH / 8); e += kProducerThreads) {
+      const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + rr;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (qi < a.n_q)
+        v = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
+                                                 static_cast<int64_t>(h) * DH) + c8);
+      *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) = v;
+    }
+    fence_async_smem();
+    mbar_arrive(&bars[M_Q]);
+    JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
+                                abort_flag};
+    uint32_t kc = 0, vc = 0;
+    auto run_jobs = [&](int j0, int j1) {
+      for (int j = j0; j < j1; ++j) {
+        if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; return; }
+        bool is_v;
+        int t;
+        js.job(j, is_v, t);
+        uint32_t& cnt = is_v ? vc : kc;
+        const uint32_t st = cnt % NST;
+        if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag)) { aborted = true; return; }
+        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, 0, kv_idx)) { aborted = true; return; }
+        mbar_arrive(&bars[(is_v ? M_VF : M_KF) + st]);
+        ++cnt;
+      }
+    };
+    run_jobs(0, n_tiles);
+    if (__syncthreads_or(aborted)) aborted = true;
+    if (!aborted) run_jobs(n_tiles, 3 * n_tiles);
+  } else if (warp == 11) {
+    // ------------------------------------------------------------------------- MMA issue
+    uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0};
+    const uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
+    auto qk_both = [&](void) -> bool {
+      const uint32_t ks = kc % NST;
+      if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag)) return false;
+      const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
+      if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag)) return false;
+      tc_after_sync();
+      mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
+      mma_commit(&bars[M_SF + 0]);
+      ++sc[0];
+      if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag)) return false;
+      tc_after_sync();
+      mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
+      mma_commit(&bars[M_SF + 1]);
+      ++sc[1];
+      mma_commit(&bars[M_KE + ks]);
+      ++kc;
+      return true;
+    };
+    if (lane == 0) {
+      if (!wait_bar(&bars[M_Q], 0, abort_flag)) aborted = true;
+      for (int t = 0; t < n_tiles && !aborted; ++t)
+        if (!qk_both()) aborted = true;
+    }
+    if (__syncthreads_or(aborted)) aborted = true;
+    if (lane == 0 && !aborted) {
+      if (!qk_both()) aborted = true;
+      for (int t = 0; t < n_tiles && !aborted; ++t) {
+        if (t + 1 < n_tiles && !qk_both()) { aborted = true; break; }
+        const uint32_t vs = vc % NST;
+        if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag)) { aborted = true; break; }
+        const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
+        for (int gg = 0; gg < 2 && !aborted; ++gg) {
+          if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag)) { aborted = true; break; }
+          tc_after_sync();
+          mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
+          mma_commit(&bars[M_PE + gg]);
+          ++pc[gg];
+        }
+        if (aborted) break;
+        mma_commit(&bars[M_VE + vs]);
+        ++vc;
+      }
+      if (!aborted) mma_commit(&bars[M_OD]);
+    }
+  } else {
+    // ------------------------------------------------------------------------- softmax (pass A)
+    uint32_t sc = 0;
+    for (int t = 0; t < n_tiles; ++t) {
+      if (!wait_bar(&bars[M_SF + g], sc & 1u, abort_flag)) { aborted = true; break; }
+      tc_after_sync();
+#pragma unroll 1
+      for (int hh = 0; hh < KT / 64; ++hh) {
+        float v[64];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64, v);
+        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64 + 32, v + 32);
+        tmem_ld_wait();
+        if (hh == KT / 64 - 1) {
+          tc_before_sync();
+          mbar_arrive(&bars[M_SR + g]);
+        }
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
+        stats64(v, m2, l);
+      }
+      ++sc;
+    }
+    flag = !aborted && row_ok && (1.0f / l < a.refetch_threshold);
+    if (__syncthreads_or(aborted)) aborted = true;
+  }
+  // -------------------------------------------------------------------------------------------
+  // flagged rows -> packed list (ascending row ids); counts of the whole CTA
+  // -------------------------------------------------------------------------------------------
+  if (warp < 8) {
+    const unsigned bal = __ballot_sync(0xffffffffu, flag);
+    if (lane == 0) wcnt[warp] = __popc(bal);
+    named_sync(3, 256);
+    uint32_t pos = __popc(bal & ((1u << lane) - 1u)), total = 0;
+    for (int w = 0; w < 8; ++w) {
+      if (w < warp) pos += wcnt[w];
+      total += wcnt[w];
+    }
+    if (flag) p.flag_list[list_base * 256 + pos] = i;
+    if (tid == 0) p.flag_cnt[list_base] = static_cast<int32_t>(total);
+    if (tid == 0 && total && a.refetch_count) atomicAdd(a.refetch_count, static_cast<int>(total));
+  }
+
+  // ------------------------------------------------------------------------- softmax (pass B)
+  if (warp < 8 && !aborted) {
+    uint32_t sc = static_cast<uint32_t>(n_tiles), pc = 0;
+    const float inv_l = 1.0f / l;
+    const bool live = row_ok && !flag;
+    uint8_t* Pt = smem + C::oP + g * C::PB;
+    const int qt128 = pair * 2 + g;
+    const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
+    for (int t = 0; t < n_tiles; ++t) {
+      if (!wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+      if (!wait_bar(&bars[M_SF + g], sc & 1u, abort_flag)) { aborted = true; break; }
+      tc_after_sync();
+#pragma unroll 1
+      for (int hh = 0; hh < KT / 64; ++hh) {
+        float v[32], w[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64, v);
+        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64 + 32, w);
+        tmem_ld_wait();
+        if (hh == KT / 64 - 1) {
+          tc_before_sync();
+          mbar_arrive(&bars[M_SR + g]);
+        }
+        const int kb = t * KT + hh * 64;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          v[j] = (live && kb + j < a.n_kv) ? ex2(v[j] * c2 - m2) * inv_l : 0.0f;
+          w[j] = (live && kb + 32 + j < a.n_kv) ? ex2(w[j] * c2 - m2) * inv_l : 0.0f;
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + q4, 128)) =
+              make_uint4(pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                         pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+          *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + 4 + q4, 128)) =
+              make_uint4(pack_bf16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_bf16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
+                         pack_bf16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_bf16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
+        }
+        float sv, sw;
+        warp_colsum32x2(v, w, sv, sw);
+        colred[t & 1][g][warp & 3][hh * 64 + lane] = sv;
+        colred[t & 1][g][warp & 3][hh * 64 + 32 + lane] = sw;
+      }
+      ++sc;
+      fence_async_smem();
+      mbar_arrive(&bars[M_PF + g]);
+      ++pc;
+      named_sync(1 + g, 128);
+      if (r < KT) {
+        const int key = t * KT + r;
+        if (key < a.n_kv && qt128 < p.n_qt)
+          p.tok_part[part_row + key] = ((colred[t & 1][g][0][r] + colred[t & 1][g][1][r]) + colred[t & 1][g][2][r]) +
+                                       colred[t & 1][g][3][r];
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------------- epilogue
+  float habs = 0.0f;
+  if (warp < 8 && !aborted) {
+    if (!wait_bar(&bars[M_OD], 0, abort_flag)) aborted = true;
+    tc_after_sync();
+    if (!aborted) {
+      const float vs = a.v_scale[bh];
+#pragma unroll 1
+      for (int ch = 0; ch < DH / 32; ++ch) {
+        float v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + C::tO + g * DH + ch * 32, v);
+        tmem_ld_wait();
+        if (row_ok && !flag)
+          store_o_row(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + ch * 32, v,
+                      vs, habs);
+      }
+      if (row_ok && a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld + i] = flag ? 1 : 0;
+    }
+  }
+  if (warp < 8) {
+    habs = warp_sum(habs);
+    if (lane == 0) hred[g][warp & 3] = habs;
+  }
+  if (__syncthreads_or(aborted)) aborted = true;
+  if (tid == 0 || tid == 128) {
+    const int qt128 = pair * 2 + (tid >> 7);
+    if (qt128 < p.n_qt)
+      p.head_part[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128] =
+          ((hred[tid >> 7][0] + hred[tid >> 7][1]) + hred[tid >> 7][2]) + hred[tid >> 7][3];
+  }
+  if (tid == 0 && aborted) report(a.dev_status, SPATTEN_E_TIMEOUT);
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 11) {
+    tc_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// =================================================================================================
+// FULL kernel: packed flagged rows at full precision
+// =================================================================================================
+template <int DH>
+struct FullCfg {
+  static constexpr int KT = DH == 64 ? 128 : 64;
+  static constexpr uint32_t QB = 128u * DH * 2u;
+  static constexpr uint32_t TB = static_cast<uint32_t>(KT) * DH * 2u;
+  static constexpr uint32_t PB = 128u * KT * 2u;
+  static constexpr int RS = 3;                   // raw (MSB + LSB) tiles in flight
+  static constexpr uint32_t RAWB = static_cast<uint32_t>(KT) * DH * 3u / 2u;
+  static constexpr uint32_t oQ = 0;
+  static constexpr uint32_t oK = QB;             // 2 stages of (MSB tile, LSB tile)
+  static constexpr uint32_t oV = oK + 4 * TB;    // 2 stages of (MSB tile, LSB tile)
+  static constexpr uint32_t oP = oV + 4 * TB;    // 1 buffer
+  static constexpr uint32_t oRaw = oP + PB;      // RS staging slots
+  static constexpr uint32_t kSmem = oRaw + RS * RAWB + 1024u;
+  static constexpr uint32_t tS = 0;              // + buffer * KT
+  static constexpr uint32_t tO = 2u * KT;
+};
+
+enum : int { F_Q = 0, F_KF = 1, F_KE = 3, F_VF = 5, F_VE = 7, F_SF = 9, F_SR = 11, F_PF = 13, F_PE = 15, F_OD = 17,
+             F_RF = 18, F_RE = 21, F_N = 24 };
+constexpr int kMaxPairs = 256;   // query rows per head up to 256 * 256
+
+template <int DH>
+__global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
+  using C = FullCfg<DH>;
+  constexpr int KT = C::KT;
+  const spatten_attn_args& a = p.a;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bars[F_N];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ float colred[2][4][KT];
+  __shared__ float hred[4];
+  __shared__ int abort_s;
+  __shared__ int pref[kMaxPairs + 1];
+  __shared__ int rows[128];
+
+  // the flagged rows of the head, concatenated over its 256-row pair tiles in order; this CTA
+  // takes packed rows [128u, 128u + 128)
+  const int u = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t head_lists = (static_cast<int64_t>(b) * a.H_kept + slot) * p.n_pair;
+  if (tid == 0) {
+    int acc = 0;
+    for (int pp = 0; pp < p.n_pair; ++pp) {
+      pref[pp] = acc;
+      acc += p.flag_cnt[head_lists + pp];
+    }
+    pref[p.n_pair] = acc;
+  }
+  __syncthreads();
+  const int rows_here = min(128, pref[p.n_pair] - u * 128);
+  if (rows_here <= 0) return;   // uniform: nothing to recompute in this packed tile
+  if (tid < rows_here) {
+    const int k = u * 128 + tid;
+    int pp = 0;
+    while (pref[pp + 1] <= k) ++pp;
+    rows[tid] = p.flag_list[(head_lists + pp) * 256 + (k - pref[pp])];
+  }
+
+  const int h = head_of_slot(a, b, slot);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+
+  if (warp == 7) {
+    tmem_alloc(&tmem_base_s, kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    abort_s = 0;
+    mbar_init(&bars[F_Q], kProducerThreads);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[F_KF + s], kProducerThreads);
+      mbar_init(&bars[F_VF + s], kProducerThreads);
+      mbar_init(&bars[F_KE + s], 1);
+      mbar_init(&bars[F_VE + s], 1);
+      mbar_init(&bars[F_SF + s], 1);
+      mbar_init(&bars[F_SR + s], 128);
+      mbar_init(&bars[F_PF + s], 128);
+      mbar_init(&bars[F_PE + s], 1);
+    }
+    mbar_init(&bars[F_OD], 1);
+    for (int s = 0; s < C::RS; ++s) {
+      mbar_init(&bars[F_RF + s], 1);
+      mbar_init(&bars[F_RE + s], kProducerThreads);
+    }
     fence_mbar_init();
   }
   tc_before_sync();
@@ -200,339 +734,212 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnProblem p) {
   const int64_t plane0 = bh * a.kv_cap;
   const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
   const int n_tiles = (a.n_kv + KT - 1) / KT;
-  const uint32_t sQ = smem_u32(smem + C::oQ);
-
-  // ---------------------------------------------------------------------------------------------
-  // role state (each role only touches its own)
-  // ---------------------------------------------------------------------------------------------
-  uint32_t kc = 0, vc = 0;          // K / V ring uses (producer and MMA)
-  uint32_t sc[2] = {0, 0};          // S buffer uses (MMA and softmax)
-  uint32_t pc[2] = {0, 0};          // P buffer uses (MMA and softmax)
   bool aborted = false;
 
-  // softmax row state
-  const int row = tid, i = i0 + row;
-  const bool row_ok = tid < 128 && i < a.n_q;
+  const int r = tid;                      // softmax: packed row r
+  const bool row_ok = tid < 128 && r < rows_here;
+  const int i = row_ok ? rows[r] : 0;
+  const bool warp_live = warp < 4 && warp * 32 < rows_here;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const float c2 = a.k_scale[bh] * a.sm_scale * kLog2e;
   float m2 = -INFINITY, l = 0.0f;
-  bool flag = false;
 
-  // ---- producers: dequantize one code tile -----------------------------------------------------
-  auto produce = [&](int t, const int8_t* msb, const uint8_t* lsb, uint32_t off_hi, uint32_t off_lo) {
+  if (warp >= 4 && warp < 7) {
+    // ------------------------------------------------------------------------- producers
     const int ptid = tid - 128;
-    constexpr int L16 = DH / 16;
-    for (int e = ptid; e < KT * L16; e += kProducerThreads) {
-      const int r = e / L16, c16 = e % L16;
-      const int key = t * KT + r;
-      uint32_t hi[8], lo[8];
-      if (key < a.n_kv) {
-        const int64_t prow = plane0 + (kv_idx ? kv_idx[key] : key);
-        cvt16_s8x16(__ldg(reinterpret_cast<const uint4*>(msb + prow * DH) + c16), hi);
-        if (lsb) cvt_u4x16(__ldg(reinterpret_cast<const uint2*>(lsb + prow * (DH / 2)) + c16), lo);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
-      }
-      *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16, KT)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-      if (lsb) {
-        *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16, KT)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-      }
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+    for (int e = ptid; e < 128 * (DH / 8); e += kProducerThreads) {
+      const int rr = e / (DH / 8), c8 = e % (DH / 8);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (rr < rows_here)
+        v = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + rows[rr]) * a.q_ld_tok +
+                                                 static_cast<int64_t>(h) * DH) + c8);
+      *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = v;
     }
     fence_async_smem();
-  };
-
-  auto run_producer = [&](int pass, bool refetch) {
-    for (int t = 0; t < n_tiles && !aborted; ++t) {
+    mbar_arrive(&bars[F_Q]);
+    JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[F_RF], &bars[F_RE], &a, plane0, n_tiles, true, ptid,
+                                abort_flag};
+    uint32_t kc = 0, vc = 0;
+    auto run_jobs = [&](int j0, int j1) {
+      for (int j = j0; j < j1; ++j) {
+        if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; return; }
+        bool is_v;
+        int t;
+        js.job(j, is_v, t);
+        uint32_t& cnt = is_v ? vc : kc;
+        const uint32_t st = cnt & 1u;
+        if (!wait_bar(&bars[(is_v ? F_VE : F_KE) + st], ((cnt >> 1) & 1u) ^ 1u, abort_flag)) { aborted = true; return; }
+        const uint32_t base = (is_v ? C::oV : C::oK) + st * 2 * C::TB;
+        if (!js.convert(j, base, base + C::TB, kv_idx)) { aborted = true; return; }
+        mbar_arrive(&bars[(is_v ? F_VF : F_KF) + st]);
+        ++cnt;
+      }
+    };
+    run_jobs(0, n_tiles);
+    if (__syncthreads_or(aborted)) aborted = true;
+    if (!aborted) run_jobs(n_tiles, 3 * n_tiles);
+  } else if (warp == 7) {
+    // ------------------------------------------------------------------------- MMA issue
+    uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0};
+    const uint32_t sQ = smem_u32(smem + C::oQ);
+    auto qk = [&](int t) -> bool {
       const uint32_t ks = kc & 1u;
-      if (!wait_bar(&bars[B_KEMPTY + ks], ((kc >> 1) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-      produce(t, a.k_msb, refetch ? a.k_lsb : nullptr, C::oK + ks * C::TB, C::oKL + ks * C::TB);
-      mbar_arrive(&bars[B_KFULL + ks]);
+      if (!wait_bar(&bars[F_KF + ks], (kc >> 1) & 1u, abort_flag)) return false;
+      const int sb = t & 1;
+      if (!wait_bar(&bars[F_SR + sb], (sc[sb] & 1u) ^ 1u, abort_flag)) return false;
+      tc_after_sync();
+      const uint32_t sK = smem_u32(smem + C::oK + ks * 2 * C::TB);
+      mma_qk<DH, KT>(tmem + C::tS + sb * KT, sQ, sK, 0);
+      mma_qk<DH, KT>(tmem + C::tS + sb * KT, sQ, sK + C::TB, 1);
+      mma_commit(&bars[F_SF + sb]);
+      mma_commit(&bars[F_KE + ks]);
+      ++sc[sb];
       ++kc;
-      if (pass == kPassB) {
+      return true;
+    };
+    if (lane == 0) {
+      if (!wait_bar(&bars[F_Q], 0, abort_flag)) aborted = true;
+      for (int t = 0; t < n_tiles && !aborted; ++t)
+        if (!qk(t)) aborted = true;
+    }
+    if (__syncthreads_or(aborted)) aborted = true;
+    if (lane == 0 && !aborted) {
+      if (!qk(0)) aborted = true;
+      for (int t = 0; t < n_tiles && !aborted; ++t) {
+        if (t + 1 < n_tiles && !qk(t + 1)) { aborted = true; break; }
+        const int pb = 0;   // single P buffer
+        if (!wait_bar(&bars[F_PF + pb], pc[pb] & 1u, abort_flag)) { aborted = true; break; }
         const uint32_t vs = vc & 1u;
-        if (!wait_bar(&bars[B_VEMPTY + vs], ((vc >> 1) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-        produce(t, a.v_msb, refetch ? a.v_lsb : nullptr, C::oV + vs * C::TB, C::oVL + vs * C::TB);
-        mbar_arrive(&bars[B_VFULL + vs]);
+        if (!wait_bar(&bars[F_VF + vs], (vc >> 1) & 1u, abort_flag)) { aborted = true; break; }
+        tc_after_sync();
+        const uint32_t sP = smem_u32(smem + C::oP + pb * C::PB);
+        const uint32_t sV = smem_u32(smem + C::oV + vs * 2 * C::TB);
+        mma_pv<DH, KT>(tmem + C::tO, sP, sV, t > 0 ? 1u : 0u);
+        mma_pv<DH, KT>(tmem + C::tO, sP, sV + C::TB, 1);
+        mma_commit(&bars[F_PE + pb]);
+        mma_commit(&bars[F_VE + vs]);
+        ++pc[pb];
         ++vc;
       }
+      if (!aborted) mma_commit(&bars[F_OD]);
     }
-  };
-
-  // ---- MMA issue ---------------------------------------------------------------------------------
-  constexpr uint32_t kIdQK = idesc_bf16(128, KT, false, false);
-  constexpr uint32_t kIdPV = idesc_bf16(128, DH, false, true);
-  auto issue_qk = [&](int t, bool refetch) -> bool {
-    const uint32_t ks = kc & 1u;
-    if (!wait_bar(&bars[B_KFULL + ks], (kc >> 1) & 1u, abort_flag)) return false;
-    const int sb = refetch ? 0 : (t & 1);
-    if (!wait_bar(&bars[B_SFREE + sb], (sc[sb] & 1u) ^ 1u, abort_flag)) return false;
-    tc_after_sync();
-    const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB), sKL = smem_u32(smem + C::oKL + ks * C::TB);
-    const uint32_t dS = tmem + C::tS + sb * KT, dC = tmem + C::tS + KT;
-#pragma unroll
-    for (int s = 0; s < DH / 16; ++s) {
-      const uint32_t qoff = (s >> 2) * 16384u + (s & 3) * 32u;
-      const uint32_t koff = (s >> 2) * (KT * 128u) + (s & 3) * 32u;
-      mma_bf16(dS, desc_sw128(sQ + qoff, 16, 1024), desc_sw128(sK + koff, 16, 1024), kIdQK, s > 0);
-    }
-    if (refetch) {
-#pragma unroll
-      for (int s = 0; s < DH / 16; ++s) {
-        const uint32_t qoff = (s >> 2) * 16384u + (s & 3) * 32u;
-        const uint32_t koff = (s >> 2) * (KT * 128u) + (s & 3) * 32u;
-        mma_bf16(dC, desc_sw128(sQ + qoff, 16, 1024), desc_sw128(sKL + koff, 16, 1024), kIdQK, s > 0);
-      }
-    }
-    mma_commit(&bars[B_SFULL + sb]);
-    mma_commit(&bars[B_KEMPTY + ks]);
-    ++sc[sb];
-    ++kc;
-    return true;
-  };
-  auto issue_pv = [&](int t, bool refetch) -> bool {
-    const int pb = t & 1;
-    if (!wait_bar(&bars[B_PFULL + pb], pc[pb] & 1u, abort_flag)) return false;
-    const uint32_t vs = vc & 1u;
-    if (!wait_bar(&bars[B_VFULL + vs], (vc >> 1) & 1u, abort_flag)) return false;
-    tc_after_sync();
-    const uint32_t sP = smem_u32(smem + C::oP + pb * C::PB);
-    const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB), sVL = smem_u32(smem + C::oVL + vs * C::TB);
-#pragma unroll
-    for (int s = 0; s < KT / 16; ++s) {
-      const uint32_t poff = (s >> 2) * 16384u + (s & 3) * 32u;
-      const uint32_t voff = s * 2048u;
-      const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
-      mma_bf16(tmem + C::tO, desc_sw128(sP + poff, 16, 1024), desc_sw128(sV + voff, KT * 128u, 1024), kIdPV, acc);
-      if (refetch)
-        mma_bf16(tmem + C::tO2, desc_sw128(sP + poff, 16, 1024), desc_sw128(sVL + voff, KT * 128u, 1024), kIdPV, acc);
-    }
-    mma_commit(&bars[B_PFREE + pb]);
-    mma_commit(&bars[B_VEMPTY + vs]);
-    ++pc[pb];
-    ++vc;
-    return true;
-  };
-  auto run_mma = [&](int pass, bool refetch) {
-    if (lane != 0) return;
-    if (pass != kPassB) {
-      for (int t = 0; t < n_tiles; ++t)
-        if (!issue_qk(t, refetch)) { aborted = true; return; }
-      return;
-    }
-    if (!issue_qk(0, refetch)) { aborted = true; return; }
+  } else {
+    // ------------------------------------------------------------------------- softmax (pass A)
+    uint32_t sc[2] = {0, 0};
     for (int t = 0; t < n_tiles; ++t) {
-      if (t + 1 < n_tiles && !issue_qk(t + 1, refetch)) { aborted = true; return; }
-      if (!issue_pv(t, refetch)) { aborted = true; return; }
-    }
-    mma_commit(&bars[B_ODONE]);
-  };
-
-  // ---- softmax ------------------------------------------------------------------------------------
-  const float c2 = a.k_scale[bh] * a.sm_scale * kLog2e;   // raw accumulator -> log2-domain score
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  auto run_stats = [&](bool refetch) {   // pass A (refetch = false) or A' (refetch = true)
-    float mx2 = -INFINITY, lx = 0.0f;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int sb = refetch ? 0 : (t & 1);
-      if (!wait_bar(&bars[B_SFULL + sb], sc[sb] & 1u, abort_flag)) { aborted = true; break; }
+      const int sb = t & 1;
+      if (!wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag)) { aborted = true; break; }
       tc_after_sync();
+      if (warp_live) {
 #pragma unroll 1
-      for (int ch = 0; ch < C::CH; ++ch) {
-        float v[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + C::tS + sb * KT + ch * 32, v);
-        if (refetch) {
-          float w[32];
-          tmem_ld32(tmem + lane_base + C::tS + KT + ch * 32, w);
+        for (int hh = 0; hh < KT / 64; ++hh) {
+          float v[64];
+          __syncwarp();
+          tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64, v);
+          tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64 + 32, v + 32);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] += w[j];
-        } else {
-          tmem_ld_wait();
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = (t * KT + ch * 32 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
-          mx = fmaxf(mx, v[j]);
-        }
-        if (mx != -INFINITY) {
-          const float mn = fmaxf(mx2, mx);
-          float add = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) add += ex2(v[j] - mn);
-          lx = lx * ex2(mx2 - mn) + add;
-          mx2 = mn;
+          for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
+          stats64(v, m2, l);
         }
       }
       tc_before_sync();
-      mbar_arrive(&bars[B_SFREE + sb]);
+      mbar_arrive(&bars[F_SR + sb]);
       ++sc[sb];
     }
-    if (!refetch) {
-      m2 = mx2;
-      l = lx;
-    } else if (flag) {
-      m2 = mx2;
-      l = lx;
-    }
-  };
-
-  const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt) * a.n_kv;
-  auto run_probs = [&](bool refetch) {   // pass B
-    const float inv_l = 1.0f / l;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int sb = refetch ? 0 : (t & 1);
-      const int pb = t & 1;
-      if (!wait_bar(&bars[B_PFREE + pb], (pc[pb] & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-      if (!wait_bar(&bars[B_SFULL + sb], sc[sb] & 1u, abort_flag)) { aborted = true; break; }
-      tc_after_sync();
-      uint8_t* Pt = smem + C::oP + pb * C::PB;
+    if (__syncthreads_or(aborted)) aborted = true;
+    // ------------------------------------------------------------------------- softmax (pass B)
+    if (!aborted) {
+      uint32_t pc[2] = {0, 0};
+      const float inv_l = 1.0f / l;
+      const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * 2 * p.n_pair + u) * a.n_kv;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int sb = t & 1;
+        const int pb = 0;   // single P buffer
+        if (!wait_bar(&bars[F_PE + pb], (pc[pb] & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag)) { aborted = true; break; }
+        tc_after_sync();
+        uint8_t* Pt = smem + C::oP + pb * C::PB;
 #pragma unroll 1
-      for (int ch = 0; ch < C::CH; ++ch) {
-        float v[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + C::tS + sb * KT + ch * 32, v);
-        if (refetch) {
-          float w[32];
-          tmem_ld32(tmem + lane_base + C::tS + KT + ch * 32, w);
-          tmem_ld_wait();
-          if (flag) {
+        for (int hh = 0; hh < KT / 64; ++hh) {
+          float v[32], w[32];
+          if (warp_live) {
+            __syncwarp();
+            tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64, v);
+            tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64 + 32, w);
+            tmem_ld_wait();
+            const int kb = t * KT + hh * 64;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += w[j];
+            for (int j = 0; j < 32; ++j) {
+              v[j] = (row_ok && kb + j < a.n_kv) ? ex2(v[j] * c2 - m2) * inv_l : 0.0f;
+              w[j] = (row_ok && kb + 32 + j < a.n_kv) ? ex2(w[j] * c2 - m2) * inv_l : 0.0f;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = w[j] = 0.0f;
           }
-        } else {
-          tmem_ld_wait();
-        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const bool ok = row_ok && (t * KT + ch * 32 + j < a.n_kv);
-          v[j] = ok ? ex2(v[j] * c2 - m2) * inv_l : 0.0f;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + q4, 128)) =
+                make_uint4(pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                           pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+            *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + 4 + q4, 128)) =
+                make_uint4(pack_bf16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_bf16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
+                           pack_bf16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_bf16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
+          }
+          float sv = 0.0f, sw = 0.0f;
+          if (warp_live) warp_colsum32x2(v, w, sv, sw);
+          colred[t & 1][warp][hh * 64 + lane] = sv;
+          colred[t & 1][warp][hh * 64 + 32 + lane] = sw;
         }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t c8 = ch * 4 + q4;
-          *reinterpret_cast<uint4*>(Pt + tile_off(row, c8, 128)) =
-              make_uint4(pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
-                         pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+        tc_before_sync();
+        mbar_arrive(&bars[F_SR + sb]);
+        ++sc[sb];
+        fence_async_smem();
+        mbar_arrive(&bars[F_PF + pb]);
+        ++pc[pb];
+        named_sync(1, 128);
+        if (r < KT) {
+          const int key = t * KT + r;
+          if (key < a.n_kv)
+            p.full_part[part_row + key] = ((colred[t & 1][0][r] + colred[t & 1][1][r]) + colred[t & 1][2][r]) + colred[t & 1][3][r];
         }
-        colred[t & 1][warp][ch * 32 + lane] = warp_colsum32(v);
-      }
-      tc_before_sync();
-      mbar_arrive(&bars[B_SFREE + sb]);
-      ++sc[sb];
-      fence_async_smem();
-      mbar_arrive(&bars[B_PFULL + pb]);
-      ++pc[pb];
-      named_sync_softmax();
-      for (int kk = tid; kk < KT; kk += kSoftmaxThreads) {
-        const int key = t * KT + kk;
-        if (key < a.n_kv)
-          p.tok_part[part_row + key] =
-              ((colred[t & 1][0][kk] + colred[t & 1][1][kk]) + colred[t & 1][2][kk]) + colred[t & 1][3][kk];
       }
     }
-  };
-
-  // ---------------------------------------------------------------------------------------------
-  // producers load Q once
-  // ---------------------------------------------------------------------------------------------
-  if (warp >= 4 && warp < kMmaWarp) {
-    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-    for (int e = tid - 128; e < 128 * (DH / 8); e += kProducerThreads) {
-      const int r = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + r;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (qi < a.n_q)
-        v = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
-                                                 static_cast<int64_t>(h) * DH) + c8);
-      *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(r, c8, 128)) = v;
-    }
-    fence_async_smem();
-    mbar_arrive(&bars[B_Q]);
-  } else if (warp == kMmaWarp && lane == 0) {
-    if (!wait_bar(&bars[B_Q], 0, abort_flag)) aborted = true;
   }
 
-  // ---- pass A ----------------------------------------------------------------------------------
-  if (!aborted) {
-    if (warp < 4) run_stats(false);
-    else if (warp < kMmaWarp) run_producer(kPassA, false);
-    else run_mma(kPassA, false);
-  }
-  if (warp < 4) flag = !aborted && a.quantized && row_ok && (1.0f / l < a.refetch_threshold);
-  const bool any_flag = __syncthreads_or(flag) != 0;
-  if (__syncthreads_or(aborted)) aborted = true;
-
-  // ---- pass A' ---------------------------------------------------------------------------------
-  if (any_flag && !aborted) {
-    if (warp < 4) run_stats(true);
-    else if (warp < kMmaWarp) run_producer(kPassA2, true);
-    else run_mma(kPassA2, true);
-  }
-  if (__syncthreads_or(aborted)) aborted = true;
-
-  // ---- pass B ----------------------------------------------------------------------------------
-  if (!aborted) {
-    if (warp < 4) run_probs(any_flag);
-    else if (warp < kMmaWarp) run_producer(kPassB, any_flag);
-    else run_mma(kPassB, any_flag);
-  }
-
-  // ---- epilogue (softmax warps): O, head importance, flags ----------------------------------------
+  // ------------------------------------------------------------------------- epilogue
   float habs = 0.0f;
   if (warp < 4 && !aborted) {
-    if (!wait_bar(&bars[B_ODONE], 0, abort_flag)) aborted = true;
+    if (!wait_bar(&bars[F_OD], 0, abort_flag)) aborted = true;
     tc_after_sync();
-    if (!aborted) {
+    if (!aborted && warp_live) {
       const float vs = a.v_scale[bh];
 #pragma unroll 1
       for (int ch = 0; ch < DH / 32; ++ch) {
         float v[32];
         __syncwarp();
         tmem_ld32(tmem + lane_base + C::tO + ch * 32, v);
-        if (any_flag) {
-          float w[32];
-          tmem_ld32(tmem + lane_base + C::tO2 + ch * 32, w);
-          tmem_ld_wait();
-          if (flag) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += w[j];
-          }
-        } else {
-          tmem_ld_wait();
-        }
-        if (row_ok) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float x0 = v[2 * j] * vs, x1 = v[2 * j + 1] * vs;
-            habs += fabsf(x0) + fabsf(x1);
-            pk[j] = pack_bf16x2(x0, x1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok +
-                                                static_cast<int64_t>(h) * DH + ch * 32);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-        }
+        tmem_ld_wait();
+        if (row_ok)
+          store_o_row(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + ch * 32, v,
+                      vs, habs);
       }
-      if (row_ok && a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld + i] = flag ? 1 : 0;
     }
   }
   if (warp < 4) {
     habs = warp_sum(habs);
     if (lane == 0) hred[warp] = habs;
   }
-  const int nflag = __syncthreads_count(flag);
   if (__syncthreads_or(aborted)) aborted = true;
-  tc_before_sync();
-  __syncthreads();
   if (tid == 0) {
-    p.head_part[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt] = ((hred[0] + hred[1]) + hred[2]) + hred[3];
-    if (nflag && a.refetch_count) atomicAdd(a.refetch_count, nflag);
+    p.full_head[(static_cast<int64_t>(b) * a.H_kept + slot) * 2 * p.n_pair + u] = ((hred[0] + hred[1]) + hred[2]) + hred[3];
     if (aborted) report(a.dev_status, SPATTEN_E_TIMEOUT);
   }
-  if (warp == kMmaWarp) {
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 7) {
     tc_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -544,19 +951,27 @@ int32_t launch(const AttnProblem& p, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    SPT_CUDA(cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(Cfg<DH>::kSmem)));
+    SPT_CUDA(cudaFuncSetAttribute(attn_main_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(MainCfg<DH>::kSmem)));
+    SPT_CUDA(cudaFuncSetAttribute(attn_full_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(FullCfg<DH>::kSmem)));
     configured[dev] = true;
   }
   const int slots = p.a.H_kept + (p.a.zero_pruned_heads ? p.a.H - p.a.H_kept : 0);
-  attn_tc_kernel<DH><<<dim3(p.n_qt, slots, p.a.B), kThreads, Cfg<DH>::kSmem, st>>>(p);
-  return launch_status();
+  attn_main_kernel<DH><<<dim3(p.n_pair, slots, p.a.B), 384, MainCfg<DH>::kSmem, st>>>(p);
+  SPT_TRY(launch_status());
+  if (p.a.refetch_threshold > 0.0f) {
+    attn_full_kernel<DH><<<dim3(p.n_qt, p.a.H_kept, p.a.B), 256, FullCfg<DH>::kSmem, st>>>(p);
+    SPT_TRY(launch_status());
+  }
+  return SPATTEN_OK;
 }
 
 }  // namespace
 
 bool attn_tc_supported(const spatten_attn_args& a) {
-  return a.quantized && a.q_dtype == SPATTEN_BF16 && (a.d_h == 64 || a.d_h == 128) && a.n_q > 1;
+  return a.quantized && a.q_dtype == SPATTEN_BF16 && (a.d_h == 64 || a.d_h == 128) && a.n_q > 1 &&
+         a.n_q <= 256 * kMaxPairs;
 }
 
 int32_t attn_tc_launch(const AttnProblem& p, cudaStream_t st) {

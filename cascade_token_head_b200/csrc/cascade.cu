@@ -9,6 +9,7 @@
 // (all sizes come from the schedule), so a whole forward can be captured in a CUDA graph.
 #include <cublasLt.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -110,10 +111,27 @@ struct Ws {
   size_t total;
 };
 
-size_t attn_ws_bound(int B, int H, int n_q, int n_kv) {
-  // the largest per-CTA partial layout any attention kernel uses (32-row query tiles)
-  const size_t n_qt = static_cast<size_t>(ceil_div(n_q, kSimtRows));
-  return align_up(static_cast<size_t>(B) * H * n_qt * n_kv * 4, 256) + align_up(static_cast<size_t>(B) * H * n_qt * 4, 256) + 512;
+// the largest workspace any attention kernel asks for at this size (sizes grow with n and the
+// number of kept heads, so layer 0 bounds every layer)
+size_t attn_ws_bound(const spatten_cascade_cfg& c, int n_q, int n_kv) {
+  spatten_attn_args a;
+  std::memset(&a, 0, sizeof(a));
+  void* const dummy = reinterpret_cast<void*>(uintptr_t(256));   // sizing only, never dereferenced
+  a.B = c.B; a.H = c.H; a.n_q = n_q; a.n_kv = n_kv; a.d_h = c.d_h; a.H_kept = c.H;
+  a.q = dummy; a.o = dummy; a.q_dtype = c.dtype;
+  a.q_ld_tok = 3LL * c.H * c.d_h; a.o_ld_tok = static_cast<int64_t>(c.H) * c.d_h;
+  a.quantized = c.quant;
+  a.k_msb = a.v_msb = static_cast<const int8_t*>(dummy);
+  a.k_lsb = a.v_lsb = static_cast<const uint8_t*>(dummy);
+  a.k_scale = a.v_scale = static_cast<const float*>(dummy);
+  a.kv_cap = n_kv;
+  a.k = a.v = dummy; a.kv_dtype = c.dtype; a.kv_ld_tok = a.q_ld_tok;
+  size_t best = 0;
+  for (int kernel = SPATTEN_ATTN_AUTO; kernel <= SPATTEN_ATTN_DECODE; ++kernel) {
+    a.kernel = kernel;
+    best = std::max(best, spatten_attention_workspace_size(&a));
+  }
+  return best + 512;
 }
 
 Ws carve(const spatten_cascade_cfg& c, void* base) {
@@ -142,7 +160,7 @@ Ws carve(const spatten_cascade_cfg& c, void* base) {
   }
   w.sel = cur.take<int32_t>(static_cast<size_t>(c.B) * c.T);
   w.head_sel = cur.take<int32_t>(static_cast<size_t>(c.B) * c.H);
-  w.attn_ws_bytes = dec ? attn_ws_bound(c.B, c.H, 1, c.T) : attn_ws_bound(c.B, c.H, c.T, c.T);
+  w.attn_ws_bytes = dec ? attn_ws_bound(c, 1, c.T) : attn_ws_bound(c, c.T, c.T);
   w.attn_ws = cur.take<char>(w.attn_ws_bytes);
   w.gemm_ws = cur.take<char>(kGemmWs);
   w.total = cur.used;
