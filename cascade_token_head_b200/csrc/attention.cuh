@@ -34,6 +34,13 @@ constexpr int kSimtRows = 32;     // query rows per CTA of the CUDA-core kernel
 int32_t attention_layer_timed(const spatten_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t st,
                               cudaEvent_t ev_begin, cudaEvent_t ev_end);
 
+// K and V of one projection buffer quantized in one launch (quantize.cu)
+int32_t quantize_kv_pair(const void* k, const void* v, int32_t dtype, int32_t B, int32_t H, int32_t n, int32_t d_h,
+                         int64_t ld_tok, const float* k_gain, int64_t ld_gain, const float* k_scale_in,
+                         const float* v_scale_in, int8_t* k_msb, uint8_t* k_lsb, int8_t* v_msb, uint8_t* v_lsb,
+                         int32_t cap, int32_t row0, float* k_scale_out, float* v_scale_out, int32_t* sat_count,
+                         cudaStream_t st);
+
 // Fixed-order reduction of the per-CTA partials into tok_imp / head_imp.
 int32_t attn_reduce_launch(const AttnProblem& p, cudaStream_t st);
 

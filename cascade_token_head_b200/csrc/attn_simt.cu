@@ -292,46 +292,6 @@ int32_t dispatch_types(const AttnProblem& p, cudaStream_t st) {
   return launch_simt<DH, float, float>(p, st);
 }
 
-// ---- fixed-order reduction of the partials ---------------------------------------------------
-__global__ void __launch_bounds__(256) attn_reduce_kernel(AttnProblem p) {
-  const spatten_attn_args& a = p.a;
-  const int b = blockIdx.y;
-  const int nblk_tok = (a.n_kv + 255) / 256;
-  if (static_cast<int>(blockIdx.x) < nblk_tok) {
-    if (!a.tok_imp) return;
-    const int j = blockIdx.x * 256 + threadIdx.x;
-    if (j >= a.n_kv) return;
-    float s = 0.0f;
-    for (int slot = 0; slot < a.H_kept; ++slot) {
-      for (int qt = 0; qt < p.n_qt; ++qt)
-        s += p.tok_part[((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt) * a.n_kv + j];
-      if (p.flag_cnt) {   // packed full-precision tiles of the refetched rows
-        int total = 0;
-        for (int pp = 0; pp < p.n_pair; ++pp) total += p.flag_cnt[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_pair + pp];
-        for (int u = 0; u * 128 < total; ++u)
-          s += p.full_part[((static_cast<int64_t>(b) * a.H_kept + slot) * 2 * p.n_pair + u) * a.n_kv + j];
-      }
-    }
-    const int64_t dst = a.tok_imp_map ? a.tok_imp_map[static_cast<int64_t>(b) * a.tok_imp_map_ld + j] : j;
-    a.tok_imp[static_cast<int64_t>(b) * a.tok_imp_ld + dst] += s;
-  } else {
-    if (!a.head_imp) return;
-    for (int slot = threadIdx.x; slot < a.H_kept; slot += blockDim.x) {
-      float s = 0.0f;
-      for (int qt = 0; qt < p.n_qt; ++qt)
-        s += p.head_part[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt];
-      if (p.flag_cnt) {
-        int total = 0;
-        for (int pp = 0; pp < p.n_pair; ++pp) total += p.flag_cnt[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_pair + pp];
-        for (int u = 0; u * 128 < total; ++u)
-          s += p.full_head[(static_cast<int64_t>(b) * a.H_kept + slot) * 2 * p.n_pair + u];
-      }
-      const int h = a.head_idx ? a.head_idx[static_cast<int64_t>(b) * a.head_idx_ld + slot] : slot;
-      a.head_imp[static_cast<int64_t>(b) * a.H + h] += s;
-    }
-  }
-}
-
 }  // namespace
 
 int32_t attn_simt_launch(const AttnProblem& p, cudaStream_t st) {
@@ -340,10 +300,5 @@ int32_t attn_simt_launch(const AttnProblem& p, cudaStream_t st) {
   return SPATTEN_E_UNSUPPORTED;
 }
 
-int32_t attn_reduce_launch(const AttnProblem& p, cudaStream_t st) {
-  const int nblk = (p.a.n_kv + 255) / 256 + 1;
-  attn_reduce_kernel<<<dim3(nblk, p.a.B), 256, 0, st>>>(p);
-  return launch_status();
-}
 
 }  // namespace spt

@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   }
   if (tid == 0) {
     abort_s = 0;
-    mbar_init(&bars[M_Q], kProducerThreads);
+    mbar_init(&bars[M_Q], 352);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars[M_KF + s], kProducerThreads);
       mbar_init(&bars[M_VF + s], kProducerThreads);
@@ -412,20 +412,33 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   float m2 = -INFINITY, l = 0.0f;
   bool flag = false;
 
-  if (warp >= 8 && warp < 11) {
-    // ------------------------------------------------------------------------- producers
-    const int ptid = tid - 256;
+  if (warp != 11) {
+    // Q tiles: every thread but the MMA warp, all of its loads in flight at once
+    constexpr int NCH = 256 * (DH / 8);
+    constexpr int PER = (NCH + 351) / 352;
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-    for (int e = ptid; e < 256 * (DH / 8); e += kProducerThreads) {
+    uint4 qv[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int e = tid + k * 352;
       const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + rr;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (qi < a.n_q)
-        v = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
-                                                 static_cast<int64_t>(h) * DH) + c8);
-      *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) = v;
+      qv[k] = make_uint4(0, 0, 0, 0);
+      if (e < NCH && qi < a.n_q)
+        qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
+                                                     static_cast<int64_t>(h) * DH) + c8);
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int e = tid + k * 352;
+      const int rr = e / (DH / 8), c8 = e % (DH / 8);
+      if (e < NCH) *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) = qv[k];
     }
     fence_async_smem();
     mbar_arrive(&bars[M_Q]);
+  }
+  if (warp >= 8 && warp < 11) {
+    // ------------------------------------------------------------------------- producers
+    const int ptid = tid - 256;
     JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
                                 abort_flag};
     uint32_t kc = 0, vc = 0;
@@ -706,7 +719,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   }
   if (tid == 0) {
     abort_s = 0;
-    mbar_init(&bars[F_Q], kProducerThreads);
+    mbar_init(&bars[F_Q], 224);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[F_KF + s], kProducerThreads);
       mbar_init(&bars[F_VF + s], kProducerThreads);
@@ -744,20 +757,33 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   const float c2 = a.k_scale[bh] * a.sm_scale * kLog2e;
   float m2 = -INFINITY, l = 0.0f;
 
-  if (warp >= 4 && warp < 7) {
-    // ------------------------------------------------------------------------- producers
-    const int ptid = tid - 128;
+  if (warp != 7) {
+    // gathered Q rows: every thread but the MMA warp, all of its loads in flight at once
+    constexpr int NCH = 128 * (DH / 8);
+    constexpr int PER = (NCH + 223) / 224;
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-    for (int e = ptid; e < 128 * (DH / 8); e += kProducerThreads) {
+    uint4 qv[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int e = tid + k * 224;
       const int rr = e / (DH / 8), c8 = e % (DH / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (rr < rows_here)
-        v = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + rows[rr]) * a.q_ld_tok +
-                                                 static_cast<int64_t>(h) * DH) + c8);
-      *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = v;
+      qv[k] = make_uint4(0, 0, 0, 0);
+      if (e < NCH && rr < rows_here)
+        qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + rows[rr]) * a.q_ld_tok +
+                                                     static_cast<int64_t>(h) * DH) + c8);
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int e = tid + k * 224;
+      const int rr = e / (DH / 8), c8 = e % (DH / 8);
+      if (e < NCH) *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = qv[k];
     }
     fence_async_smem();
     mbar_arrive(&bars[F_Q]);
+  }
+  if (warp >= 4 && warp < 7) {
+    // ------------------------------------------------------------------------- producers
+    const int ptid = tid - 128;
     JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[F_RF], &bars[F_RE], &a, plane0, n_tiles, true, ptid,
                                 abort_flag};
     uint32_t kc = 0, vc = 0;

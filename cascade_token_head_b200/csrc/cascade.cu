@@ -242,10 +242,8 @@ int32_t run_prefill(const spatten_cascade_cfg& c, const spatten_layer_weights* w
     if (c.quant) {
       const char* kp = ws.qkv + HD * es;
       const char* vp = ws.qkv + 2 * HD * es;
-      SPT_TRY(spatten_quantize_kv(kp, c.dtype, B, H, k, dh, 3 * HD, gain ? g_cur : nullptr, k, nullptr, ws.k_msb,
-                                ws.k_lsb, k, 0, ws.k_scale, nullptr, st));
-      SPT_TRY(spatten_quantize_kv(vp, c.dtype, B, H, k, dh, 3 * HD, nullptr, 0, nullptr, ws.v_msb, ws.v_lsb, k, 0,
-                                ws.v_scale, nullptr, st));
+      SPT_TRY(quantize_kv_pair(kp, vp, c.dtype, B, H, k, dh, 3 * HD, gain ? g_cur : nullptr, k, nullptr, nullptr,
+                               ws.k_msb, ws.k_lsb, ws.v_msb, ws.v_lsb, k, 0, ws.k_scale, ws.v_scale, nullptr, st));
       a.quantized = 1;
       a.k_msb = ws.k_msb; a.k_lsb = ws.k_lsb; a.k_scale = ws.k_scale;
       a.v_msb = ws.v_msb; a.v_lsb = ws.v_lsb; a.v_scale = ws.v_scale;
@@ -331,10 +329,9 @@ int32_t run_decode(const spatten_cascade_cfg& c, const spatten_layer_weights* w,
       SPT_CUDA(cudaMemcpyAsync(static_cast<char*>(io.trace_qkv) + static_cast<size_t>(l) * B * 3 * HD * es, ws.qkv,
                                static_cast<size_t>(B) * 3 * HD * es, cudaMemcpyDeviceToDevice, st));
     // append the new token's K and V codes at row n-1 with the prompt-time scales
-    SPT_TRY(spatten_quantize_kv(ws.qkv + HD * es, c.dtype, B, H, 1, dh, 3 * HD, nullptr, 0, cc.k_scale, cc.k_msb,
-                              cc.k_lsb, cap, io.n_old, nullptr, io.sat_count, st));
-    SPT_TRY(spatten_quantize_kv(ws.qkv + 2 * HD * es, c.dtype, B, H, 1, dh, 3 * HD, nullptr, 0, cc.v_scale, cc.v_msb,
-                              cc.v_lsb, cap, io.n_old, nullptr, io.sat_count, st));
+    SPT_TRY(quantize_kv_pair(ws.qkv + HD * es, ws.qkv + 2 * HD * es, c.dtype, B, H, 1, dh, 3 * HD, nullptr, 0,
+                             cc.k_scale, cc.v_scale, cc.k_msb, cc.k_lsb, cc.v_msb, cc.v_lsb, cap, io.n_old, nullptr,
+                             nullptr, io.sat_count, st));
     spatten_attn_args a = base_attn(c);
     a.n_q = 1;
     a.n_kv = k;

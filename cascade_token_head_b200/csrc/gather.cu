@@ -48,9 +48,19 @@ __global__ void __launch_bounds__(kGThreads) gather_rows_kernel(GArgs a) {
   const char* s = a.src + r * a.src_batch + static_cast<int64_t>(i) * a.src_row;
   char* d = a.dst + r * a.dst_batch + static_cast<int64_t>(j) * a.dst_row;
   if (VEC == 16) {
+    // four 16-byte loads in flight per lane before the stores
     const int64_t nv = a.row_bytes / 16;
-    for (int64_t c = lane; c < nv; c += 32)
-      reinterpret_cast<uint4*>(d)[c] = __ldg(reinterpret_cast<const uint4*>(s) + c);
+    const uint4* s4 = reinterpret_cast<const uint4*>(s);
+    uint4* d4 = reinterpret_cast<uint4*>(d);
+    for (int64_t c0 = lane; c0 < nv; c0 += 128) {
+      uint4 r4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < nv) r4[u] = __ldg(s4 + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < nv) d4[c0 + 32 * u] = r4[u];
+    }
   } else {
     const int64_t nv = a.row_bytes / 4;
     for (int64_t c = lane; c < nv; c += 32)

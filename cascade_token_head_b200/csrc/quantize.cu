@@ -5,9 +5,11 @@
 // bits and concatenates MSBs with LSBs.  Codes: q = clamp(rint(float32(x*gain) / s), +-2047),
 // MSB = q >> 4, LSB = q & 15, s = amax / 2047 per (sequence, head) block.
 //
-// Amax mode: one thread-block cluster per (b, h) block; each CTA reduces the amax of its rows,
-// the cluster exchanges the partial maxima through distributed shared memory, and every CTA then
-// quantizes its rows (a second read that hits L2).  No scratch memory is needed.
+// Amax mode: one thread-block cluster per (b, h) block (gridDim.z selects K or V when both are
+// quantized in one launch); each CTA reduces the amax of its rows, the cluster exchanges the
+// partial maxima through distributed shared memory, and every CTA then quantizes its rows.  When
+// a CTA's rows fit in its registers (16 chunks of 8 values per thread) they are read once and
+// kept there; otherwise they are read again (an L2 hit).  No scratch memory is needed.
 // Fixed-scale mode (decode append): one thread per 8-element chunk, saturations counted.
 #include <cooperative_groups.h>
 
@@ -16,24 +18,30 @@
 namespace cg = cooperative_groups;
 
 namespace spt {
-namespace {
 
 constexpr int kQThreads = 256;
+constexpr int kQRegChunks = 16;
 constexpr float kQMax = 2047.0f;
 
-struct QArgs {
+struct QTensor {
   const void* x;
-  int B, H, n, d_h;
-  int64_t ld_tok;
   const float* gain;
-  int64_t ld_gain;
-  const float* scale_in;
   int8_t* msb;
   uint8_t* lsb;
-  int cap, row0;
   float* scale_out;
+  const float* scale_in;
+};
+
+struct QArgs {
+  QTensor t[2];
+  int B, H, n, d_h;
+  int64_t ld_tok;
+  int64_t ld_gain;
+  int cap, row0;
   int32_t* sat;
 };
+
+namespace {
 
 // quantize 8 values with scale s; returns the number of saturated codes
 __device__ __forceinline__ int quant8(const float* v, float s, int8_t* msb_dst, uint8_t* lsb_dst) {
@@ -56,14 +64,25 @@ __device__ __forceinline__ int quant8(const float* v, float s, int8_t* msb_dst, 
 }
 
 template <typename T>
-__device__ __forceinline__ void load_row_chunk(const QArgs& a, int b, int h, int t, int c, float* v) {
-  const T* x = static_cast<const T*>(a.x) + (static_cast<int64_t>(b) * a.n + t) * a.ld_tok +
-               static_cast<int64_t>(h) * a.d_h + c * 8;
-  load8(x, v);
-  if (a.gain) {
-    float g = a.gain[static_cast<int64_t>(b) * a.ld_gain + t];
+__device__ __forceinline__ const T* chunk_ptr(const QArgs& a, const QTensor& q, int b, int h, int t, int c) {
+  return static_cast<const T*>(q.x) + (static_cast<int64_t>(b) * a.n + t) * a.ld_tok + static_cast<int64_t>(h) * a.d_h + c * 8;
+}
+
+__device__ __forceinline__ void apply_gain(const QArgs& a, const QTensor& q, int b, int t, float* v) {
+  if (q.gain) {
+    const float g = q.gain[static_cast<int64_t>(b) * a.ld_gain + t];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] *= g;
+  }
+}
+
+__device__ __forceinline__ void bf16x8_to_float(uint4 u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
   }
 }
 
@@ -72,22 +91,45 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int S = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
+  const QTensor& q = a.t[blockIdx.z];
   const int bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
   const int C = a.d_h / 8;
   const int rows_per = (a.n + S - 1) / S;
   const int r0 = min(a.n, rank * rows_per), r1 = min(a.n, r0 + rows_per);
   const int total = (r1 - r0) * C;
+  const bool in_regs = (sizeof(T) == 2) && total <= kQRegChunks * kQThreads;
 
   __shared__ float red[kQThreads / 32];
   __shared__ float cta_amax;
 
+  uint4 keep[kQRegChunks];
   float amax = 0.0f;
-  for (int e = threadIdx.x; e < total; e += kQThreads) {
-    float v[8];
-    load_row_chunk<T>(a, b, h, r0 + e / C, e % C, v);
+  if (in_regs) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int k = 0; k < kQRegChunks; ++k) {
+      const int e = threadIdx.x + k * kQThreads;
+      if (e < total) keep[k] = __ldg(reinterpret_cast<const uint4*>(chunk_ptr<T>(a, q, b, h, r0 + e / C, e % C)));
+    }
+#pragma unroll
+    for (int k = 0; k < kQRegChunks; ++k) {
+      const int e = threadIdx.x + k * kQThreads;
+      if (e < total) {
+        float v[8];
+        bf16x8_to_float(keep[k], v);
+        apply_gain(a, q, b, r0 + e / C, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
+    }
+  } else {
+    for (int e = threadIdx.x; e < total; e += kQThreads) {
+      float v[8];
+      load8(chunk_ptr<T>(a, q, b, h, r0 + e / C, e % C), v);
+      apply_gain(a, q, b, r0 + e / C, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
   }
   amax = warp_max(amax);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
@@ -103,19 +145,36 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   cluster.sync();   // no CTA leaves while a peer may still read its shared memory
 
   const float s = block_amax == 0.0f ? 1.0f : __fdiv_rn(block_amax, kQMax);
-  if (rank == 0 && threadIdx.x == 0) a.scale_out[bh] = s;
+  if (rank == 0 && threadIdx.x == 0) q.scale_out[bh] = s;
 
-  for (int e = threadIdx.x; e < total; e += kQThreads) {
-    const int t = r0 + e / C, c = e % C;
-    float v[8];
-    load_row_chunk<T>(a, b, h, t, c, v);
-    const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
-    quant8(v, s, a.msb + row * a.d_h + c * 8, a.lsb + row * (a.d_h / 2) + c * 4);
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kQRegChunks; ++k) {
+      const int e = threadIdx.x + k * kQThreads;
+      if (e < total) {
+        const int t = r0 + e / C, c = e % C;
+        float v[8];
+        bf16x8_to_float(keep[k], v);
+        apply_gain(a, q, b, t, v);
+        const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
+        quant8(v, s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+      }
+    }
+  } else {
+    for (int e = threadIdx.x; e < total; e += kQThreads) {
+      const int t = r0 + e / C, c = e % C;
+      float v[8];
+      load8(chunk_ptr<T>(a, q, b, h, t, c), v);
+      apply_gain(a, q, b, t, v);
+      const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
+      quant8(v, s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+    }
   }
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
+  const QTensor& q = a.t[blockIdx.z];
   const int C = a.d_h / 8;
   const int64_t total = static_cast<int64_t>(a.B) * a.H * a.n * C;
   int sat = 0;
@@ -127,10 +186,11 @@ __global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
     const int bh = static_cast<int>(r / a.n);
     const int b = bh / a.H, h = bh % a.H;
     float v[8];
-    load_row_chunk<T>(a, b, h, t, c, v);
-    const float s = a.scale_in[bh];
+    load8(chunk_ptr<T>(a, q, b, h, t, c), v);
+    apply_gain(a, q, b, t, v);
+    const float s = q.scale_in[bh];
     const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
-    sat += quant8(v, s, a.msb + row * a.d_h + c * 8, a.lsb + row * (a.d_h / 2) + c * 4);
+    sat += quant8(v, s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
   }
   sat = warp_sum_int(sat);
   if (a.sat && (threadIdx.x & 31) == 0 && sat) atomicAdd(a.sat, sat);
@@ -138,23 +198,26 @@ __global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
 
 }  // namespace
 
-int32_t quantize_launch(const QArgs& a, int dtype, cudaStream_t st) {
-  if (a.scale_in) {
+// Quantize `ntensors` (1 or 2) tensors of the same shape in one launch.  Either every tensor has
+// scale_in (fixed-scale mode) or none has.
+int32_t quantize_launch(const QArgs& a, int ntensors, int dtype, cudaStream_t st) {
+  if (a.t[0].scale_in) {
     const int64_t chunks = static_cast<int64_t>(a.B) * a.H * a.n * (a.d_h / 8);
     int grid = static_cast<int>(std::min<int64_t>(ceil_div(chunks, kQThreads), 8LL * sm_count()));
+    dim3 g(grid, 1, ntensors);
     if (dtype == SPATTEN_BF16)
-      quantize_fixed_kernel<__nv_bfloat16><<<grid, kQThreads, 0, st>>>(a);
+      quantize_fixed_kernel<__nv_bfloat16><<<g, kQThreads, 0, st>>>(a);
     else
-      quantize_fixed_kernel<float><<<grid, kQThreads, 0, st>>>(a);
+      quantize_fixed_kernel<float><<<g, kQThreads, 0, st>>>(a);
     return launch_status();
   }
   const int blocks = a.B * a.H;
   // enough CTAs to fill the GPU twice; at most 8 per block (portable cluster size)
-  int S = static_cast<int>(ceil_div(2LL * sm_count(), blocks));
+  int S = static_cast<int>(ceil_div(2LL * sm_count(), static_cast<int64_t>(blocks) * ntensors));
   S = std::max(1, std::min(S, 8));
   S = std::min<int>(S, std::max(1, a.n / 16));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, blocks, 1);
+  cfg.gridDim = dim3(S, blocks, ntensors);
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -174,18 +237,13 @@ int32_t quantize_launch(const QArgs& a, int dtype, cudaStream_t st) {
   return launch_status();
 }
 
-}  // namespace spt
-
-extern "C" int32_t spatten_quantize_kv(const void* x, int32_t dtype, int32_t B, int32_t H,
-                                       int32_t n, int32_t d_h, int64_t ld_tok,
-                                       const float* row_gain, int64_t ld_gain,
-                                       const float* scale_in, int8_t* msb, uint8_t* lsb,
-                                       int32_t cap, int32_t row0, float* scale_out,
-                                       int32_t* sat_count, void* stream) {
-  using namespace spt;
+int32_t quantize_check(const void* x, int32_t dtype, int32_t B, int32_t H, int32_t n, int32_t d_h, int64_t ld_tok,
+                       const float* row_gain, int64_t ld_gain, const float* scale_in, const int8_t* msb,
+                       const uint8_t* lsb, int32_t cap, int32_t row0, const float* scale_out) {
   if (!x || !msb || !lsb) return SPATTEN_E_ARG;
   if (dtype != SPATTEN_F32 && dtype != SPATTEN_BF16) return SPATTEN_E_ARG;
   if (B < 1 || H < 1 || n < 1 || d_h < 8 || (d_h % 8) != 0) return SPATTEN_E_ARG;
+  if (B > 65535 / 1 || static_cast<int64_t>(B) * H > 65535) return SPATTEN_E_ARG;
   if (!scale_in && !scale_out) return SPATTEN_E_ARG;
   if (row0 < 0 || cap < 1 || static_cast<int64_t>(row0) + n > cap) return SPATTEN_E_SHAPE;
   if (ld_tok < static_cast<int64_t>(H) * d_h) return SPATTEN_E_SHAPE;
@@ -194,7 +252,39 @@ extern "C" int32_t spatten_quantize_kv(const void* x, int32_t dtype, int32_t B, 
   if (!aligned16(x) || (ld_tok * esz) % 16 != 0 || (static_cast<int64_t>(d_h) * esz) % 16 != 0)
     return SPATTEN_E_ALIGN;
   if (!aligned16(msb) || !aligned16(lsb)) return SPATTEN_E_ALIGN;
-  QArgs a{x, B, H, n, d_h, ld_tok, row_gain, ld_gain, scale_in, msb, lsb, cap, row0, scale_out,
-          sat_count};
-  return quantize_launch(a, dtype, as_stream(stream));
+  return SPATTEN_OK;
+}
+
+// K and V of one projection buffer in one launch (used by the cascade driver)
+int32_t quantize_kv_pair(const void* k, const void* v, int32_t dtype, int32_t B, int32_t H, int32_t n, int32_t d_h,
+                         int64_t ld_tok, const float* k_gain, int64_t ld_gain, const float* k_scale_in,
+                         const float* v_scale_in, int8_t* k_msb, uint8_t* k_lsb, int8_t* v_msb, uint8_t* v_lsb,
+                         int32_t cap, int32_t row0, float* k_scale_out, float* v_scale_out, int32_t* sat_count,
+                         cudaStream_t st) {
+  SPT_TRY(quantize_check(k, dtype, B, H, n, d_h, ld_tok, k_gain, ld_gain, k_scale_in, k_msb, k_lsb, cap, row0,
+                         k_scale_out));
+  SPT_TRY(quantize_check(v, dtype, B, H, n, d_h, ld_tok, nullptr, 0, v_scale_in, v_msb, v_lsb, cap, row0,
+                         v_scale_out));
+  if ((k_scale_in == nullptr) != (v_scale_in == nullptr)) return SPATTEN_E_ARG;
+  QArgs a{};
+  a.t[0] = QTensor{k, k_gain, k_msb, k_lsb, k_scale_out, k_scale_in};
+  a.t[1] = QTensor{v, nullptr, v_msb, v_lsb, v_scale_out, v_scale_in};
+  a.B = B; a.H = H; a.n = n; a.d_h = d_h; a.ld_tok = ld_tok; a.ld_gain = ld_gain; a.cap = cap; a.row0 = row0;
+  a.sat = sat_count;
+  return quantize_launch(a, 2, dtype, st);
+}
+
+}  // namespace spt
+
+extern "C" int32_t spatten_quantize_kv(const void* x, int32_t dtype, int32_t B, int32_t H, int32_t n,
+                                       int32_t d_h, int64_t ld_tok, const float* row_gain, int64_t ld_gain,
+                                       const float* scale_in, int8_t* msb, uint8_t* lsb, int32_t cap,
+                                       int32_t row0, float* scale_out, int32_t* sat_count, void* stream) {
+  using namespace spt;
+  SPT_TRY(quantize_check(x, dtype, B, H, n, d_h, ld_tok, row_gain, ld_gain, scale_in, msb, lsb, cap, row0, scale_out));
+  QArgs a{};
+  a.t[0] = QTensor{x, row_gain, msb, lsb, scale_out, scale_in};
+  a.B = B; a.H = H; a.n = n; a.d_h = d_h; a.ld_tok = ld_tok; a.ld_gain = ld_gain; a.cap = cap; a.row0 = row0;
+  a.sat = sat_count;
+  return quantize_launch(a, 1, dtype, as_stream(stream));
 }

@@ -270,7 +270,7 @@ int32_t topk_launch(const TArgs& a, cudaStream_t st) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = C > 1 ? 1 : 0;   // a one-CTA row needs no cluster (implicit 1x1x1)
   SPT_CUDA(cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a));
   return launch_status();
 }
