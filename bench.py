@@ -218,17 +218,28 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert int(status.item()) == 0, "device status after warm-up"
 
-    # per-step events and per-layer attention-kernel events (recorded by the library)
+    # per-step events and per-layer attention-kernel events (recorded by the library inside the
+    # captured step); the step is captured once into a CUDA graph and replayed K times
     K = args.steps
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    attn_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * L)] for _ in range(K)]
-    for row in attn_ev:      # materialise the CUDA events before handing their handles over
-        for e in row:
-            e.record(stream)
+    attn_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * L)]
+    for e in attn_ev:      # materialise the CUDA events before handing their handles over
+        e.record(stream)
     torch.cuda.synchronize()
     import ctypes as C
-    attn_arrays = [(C.c_void_p * (2 * L))(*[e.cuda_event for e in row]) for row in attn_ev]
+    attn_array = (C.c_void_p * (2 * L))(*[e.cuda_event for e in attn_ev])
+    io.attn_events = C.cast(attn_array, C.POINTER(C.c_void_p))
+    graph = None
+    launches_per_step = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        l0 = S.kernel_launch_count()
+        with torch.cuda.graph(graph):
+            S.cascade_forward(cfg, W, io, ws, ws.numel(), stream=torch.cuda.current_stream())
+        launches_per_step = S.kernel_launch_count() - l0
+        graph.replay()
+        torch.cuda.synchronize()
 
     clocks = ClockSampler(local)
     if world > 1:
@@ -237,20 +248,24 @@ def run_ours(args):
     launches0 = S.kernel_launch_count()
     clocks.start()
     time.sleep(0.3)
+    attn_ms = []
     for i in range(K):
         flush.zero_()
-        io.attn_events = C.cast(attn_arrays[i], C.POINTER(C.c_void_p))
         ev_s[i].record(stream)
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
         ev_e[i].record(stream)
+        torch.cuda.synchronize()   # read this step's attention events before the next replay
+        attn_ms.append(sum(attn_ev[2 * l].elapsed_time(attn_ev[2 * l + 1]) for l in range(L)))
     torch.cuda.synchronize()
     clk = clocks.stop()
-    launches = S.kernel_launch_count() - launches0
-    io.attn_events = None
+    launches = (launches_per_step * K) if graph is not None else S.kernel_launch_count() - launches0
     if world > 1:
         dist.barrier()
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
-    attn_ms = [sum(attn_ev[i][2 * l].elapsed_time(attn_ev[i][2 * l + 1]) for l in range(L)) for i in range(K)]
+    io.attn_events = None
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
@@ -303,7 +318,8 @@ def run_ours(args):
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, random-init weights)",
         "config": {"workload": w.name, "global_batch": B * world, "seq_len": T, "d_model": D, "heads": H,
                    "layers": L, "token_keep": w.token_keep, "head_keep": w.head_keep, "refetch_threshold": w.theta,
-                   "parallelism": f"dp{world} (independent sequences)", "l2": "flushed between timed steps"},
+                   "parallelism": f"dp{world} (independent sequences)", "l2": "flushed between timed steps",
+                   "launch": "CUDA graph of one step" if graph is not None else "direct launches"},
         "roofline": {"kernel": "attention (spatten_attention_layer main kernel, all layers)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None,
@@ -332,6 +348,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step directly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

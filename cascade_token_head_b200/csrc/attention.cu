@@ -128,7 +128,14 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
   p.tok_part = static_cast<float*>(ws);
   const size_t need = layout(p.a, path, &p);
   if (!ws || ws_bytes < need) return SPATTEN_E_WORKSPACE;
-  if (ev_begin) SPT_CUDA(cudaEventRecord(ev_begin, st));
+  // inside a stream capture, external records become timing event nodes of the graph
+  unsigned ev_flags = 0;
+  if (ev_begin || ev_end) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    SPT_CUDA(cudaStreamIsCapturing(st, &cs));
+    if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
+  }
+  if (ev_begin) SPT_CUDA(cudaEventRecordWithFlags(ev_begin, st, ev_flags));
   int32_t s;
   switch (path) {
     case Path::kTc: s = attn_tc_launch(p, st); break;
@@ -136,7 +143,7 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
     default: s = attn_simt_launch(p, st); break;
   }
   if (s != SPATTEN_OK) return s;
-  if (ev_end) SPT_CUDA(cudaEventRecord(ev_end, st));
+  if (ev_end) SPT_CUDA(cudaEventRecordWithFlags(ev_end, st, ev_flags));
   if (!p.a.tok_imp && !p.a.head_imp) return SPATTEN_OK;
   return attn_reduce_launch(p, st);
 }

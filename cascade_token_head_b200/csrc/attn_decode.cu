@@ -2,15 +2,18 @@
 // with progressive quantization and importance.
 //
 // SpAtten §II "Attention-based NLP models": generation handles one new token per iteration
-// against cached K and V (a memory-bound workload, §I "Takeaways"); §IV.E "Progressive
-// Quantization": the LSBs are fetched only when the max probability is below the threshold.
+// against cached K and V (a memory-bound workload); §IV.E "Progressive Quantization": the LSBs
+// are fetched only when the max probability is below the threshold.
 // Per CTA (b, kept head):
 //   1  MSB scores: lanes read 16-byte slices of the int8 MSB rows (d_h/16 lanes per key, rows
 //      reached through kv_idx), s_j = (16 * s_k * sm_scale) * (q . MSB_j); kept in shared memory.
 //   2  row stats m, ell; flag = 1/ell < theta.
 //   3  flagged rows only: read the LSB rows, s_j += s_k * sm_scale * (q . LSB_j); new m, ell.
 //   4  p_j = exp(s_j - m)/ell -> importance partial; O = s_v * sum_j p_j (16*MSB_j [+ LSB_j]).
-// Importance partials are reduced over heads in a fixed order by attn_reduce.
+// Every sweep over the keys issues kUnroll independent index loads and then kUnroll independent
+// 16-byte row loads per lane before using them, so each CTA keeps tens of KB in flight (the sweep
+// is bound by HBM bandwidth, not by load latency).  Importance partials are reduced over heads
+// in a fixed order by attn_reduce.
 #include "attention.cuh"
 
 namespace spt {
@@ -19,6 +22,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxKv = 32768;   // scores kept in shared memory (128 KB)
+constexpr int kUnroll = 4;
 
 __device__ __forceinline__ void unpack16_s8(uint4 u, float* f) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -41,11 +45,11 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
   constexpr int LPK = DH / 16;          // lanes per key row (16 codes per lane)
   constexpr int KPW = 32 / LPK;         // keys per warp per step
   constexpr int KPS = KPW * kWarps;     // keys per CTA step
-  extern __shared__ __align__(16) float s_sc[];   // [n_kv] scores
+  constexpr int KPU = KPS * kUnroll;    // keys per unrolled step
+  extern __shared__ __align__(16) float s_sc[];   // [n_kv] scores, then probabilities
   __shared__ float red[kWarps];
   __shared__ float o_red[kWarps][DH];
   __shared__ float bcast[2];
-  __shared__ int any_flag;
 
   const int slot = blockIdx.x, b = blockIdx.y;
   const int h = head_of_slot(a, b, slot);
@@ -72,25 +76,39 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
   const float c_lsb = ks * a.sm_scale;
   const int n = a.n_kv;
 
+  // rows of the kUnroll keys this lane group handles in the unrolled step starting at j0
+  auto rows_of = [&](int j0, int64_t* rows, int* js) {
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      js[u] = j0 + u * KPS + warp * KPW + grp;
+      rows[u] = js[u] < n ? plane0 + (kv_idx ? __ldg(kv_idx + js[u]) : js[u]) : 0;
+    }
+  };
+
   // ---- 1: MSB scores -------------------------------------------------------------------------
   float mloc = -INFINITY;
-  for (int j0 = 0; j0 < n; j0 += KPS) {
-    const int j = j0 + warp * KPW + grp;
-    float part = 0.0f;
-    if (j < n) {
-      const int64_t row = plane0 + (kv_idx ? kv_idx[j] : j);
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.k_msb + row * DH) + sub);
+  for (int j0 = 0; j0 < n; j0 += KPU) {
+    int64_t rows[kUnroll];
+    int js[kUnroll];
+    rows_of(j0, rows, js);
+    uint4 raw[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      raw[u] = js[u] < n ? __ldg(reinterpret_cast<const uint4*>(a.k_msb + rows[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
       float f[16];
-      unpack16_s8(u, f);
+      unpack16_s8(raw[u], f);
+      float part = 0.0f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) part = fmaf(qf[i], f[i], part);
-    }
 #pragma unroll
-    for (int o2 = 1; o2 < LPK; o2 <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-    if (j < n && sub == 0) {
-      const float s = part * c_msb;
-      s_sc[j] = s;
-      mloc = fmaxf(mloc, s);
+      for (int o2 = 1; o2 < LPK; o2 <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
+      if (js[u] < n && sub == 0) {
+        const float s = part * c_msb;
+        s_sc[js[u]] = s;
+        mloc = fmaxf(mloc, s);
+      }
     }
   }
   auto block_max = [&](float v) {
@@ -127,23 +145,28 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
   // ---- 3: LSB refetch for a flagged row ------------------------------------------------------
   if (flag) {
     mloc = -INFINITY;
-    for (int j0 = 0; j0 < n; j0 += KPS) {
-      const int j = j0 + warp * KPW + grp;
-      float part = 0.0f;
-      if (j < n) {
-        const int64_t row = plane0 + (kv_idx ? kv_idx[j] : j);
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(a.k_lsb + row * (DH / 2)) + sub);
+    for (int j0 = 0; j0 < n; j0 += KPU) {
+      int64_t rows[kUnroll];
+      int js[kUnroll];
+      rows_of(j0, rows, js);
+      uint2 raw[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        raw[u] = js[u] < n ? __ldg(reinterpret_cast<const uint2*>(a.k_lsb + rows[u] * (DH / 2)) + sub) : make_uint2(0, 0);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
         float f[16];
-        unpack16_u4(u, f);
+        unpack16_u4(raw[u], f);
+        float part = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) part = fmaf(qf[i], f[i], part);
-      }
 #pragma unroll
-      for (int o2 = 1; o2 < LPK; o2 <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-      if (j < n && sub == 0) {
-        const float s = s_sc[j] + part * c_lsb;
-        s_sc[j] = s;
-        mloc = fmaxf(mloc, s);
+        for (int o2 = 1; o2 < LPK; o2 <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
+        if (js[u] < n && sub == 0) {
+          const float s = s_sc[js[u]] + part * c_lsb;
+          s_sc[js[u]] = s;
+          mloc = fmaxf(mloc, s);
+        }
       }
     }
     __syncthreads();
@@ -165,22 +188,26 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
-  for (int j0 = 0; j0 < n; j0 += KPS) {
-    const int j = j0 + warp * KPW + grp;
-    if (j < n) {
-      const int64_t row = plane0 + (kv_idx ? kv_idx[j] : j);
-      const float pr = s_sc[j];
-      float f[16];
-      unpack16_s8(__ldg(reinterpret_cast<const uint4*>(a.v_msb + row * DH) + sub), f);
-      if (flag) {
-        float g[16];
-        unpack16_u4(__ldg(reinterpret_cast<const uint2*>(a.v_lsb + row * (DH / 2)) + sub), g);
+  for (int j0 = 0; j0 < n; j0 += KPU) {
+    int64_t rows[kUnroll];
+    int js[kUnroll];
+    rows_of(j0, rows, js);
+    uint4 rm[kUnroll];
+    uint2 rl[kUnroll];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = fmaf(pr, fmaf(16.0f, f[i], g[i]), acc[i]);
-      } else {
+    for (int u = 0; u < kUnroll; ++u) {
+      rm[u] = js[u] < n ? __ldg(reinterpret_cast<const uint4*>(a.v_msb + rows[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+      rl[u] = (flag && js[u] < n) ? __ldg(reinterpret_cast<const uint2*>(a.v_lsb + rows[u] * (DH / 2)) + sub) : make_uint2(0, 0);
+    }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = fmaf(pr, 16.0f * f[i], acc[i]);
-      }
+    for (int u = 0; u < kUnroll; ++u) {
+      if (js[u] >= n) continue;
+      const float pr = s_sc[js[u]];
+      float f[16], g[16];
+      unpack16_s8(rm[u], f);
+      unpack16_u4(rl[u], g);   // zero unless the row refetches
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = fmaf(pr, fmaf(16.0f, f[i], g[i]), acc[i]);
     }
   }
   // reduce over the key groups of the warp (lanes with equal `sub`), then over warps
@@ -207,7 +234,6 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
     if (a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld] = flag ? 1 : 0;
     if (flag && a.refetch_count) atomicAdd(a.refetch_count, 1);
   }
-  (void)any_flag;
 }
 
 template <int DH, typename QT>

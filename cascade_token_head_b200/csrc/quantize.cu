@@ -7,9 +7,9 @@
 //
 // Amax mode: one thread-block cluster per (b, h) block (gridDim.z selects K or V when both are
 // quantized in one launch); each CTA reduces the amax of its rows, the cluster exchanges the
-// partial maxima through distributed shared memory, and every CTA then quantizes its rows.  When
-// a CTA's rows fit in its registers (16 chunks of 8 values per thread) they are read once and
-// kept there; otherwise they are read again (an L2 hit).  No scratch memory is needed.
+// partial maxima through distributed shared memory, and every CTA then quantizes its rows (a
+// second read that hits L2).  Each thread keeps four 16-byte loads in flight.  No scratch memory
+// is needed.
 // Fixed-scale mode (decode append): one thread per 8-element chunk, saturations counted.
 #include <cooperative_groups.h>
 
@@ -20,7 +20,7 @@ namespace cg = cooperative_groups;
 namespace spt {
 
 constexpr int kQThreads = 256;
-constexpr int kQRegChunks = 16;
+constexpr int kQBatch = 4;   // 16-byte chunks in flight per thread
 constexpr float kQMax = 2047.0f;
 
 struct QTensor {
@@ -76,16 +76,6 @@ __device__ __forceinline__ void apply_gain(const QArgs& a, const QTensor& q, int
   }
 }
 
-__device__ __forceinline__ void bf16x8_to_float(uint4 u, float* f) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 t = __bfloat1622float2(h[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -98,37 +88,28 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   const int rows_per = (a.n + S - 1) / S;
   const int r0 = min(a.n, rank * rows_per), r1 = min(a.n, r0 + rows_per);
   const int total = (r1 - r0) * C;
-  const bool in_regs = (sizeof(T) == 2) && total <= kQRegChunks * kQThreads;
 
   __shared__ float red[kQThreads / 32];
   __shared__ float cta_amax;
 
-  uint4 keep[kQRegChunks];
+  // pass 1: amax, kQBatch chunks (8 values each) in flight per thread
   float amax = 0.0f;
-  if (in_regs) {
+#pragma unroll 1
+  for (int e0 = threadIdx.x; e0 < total; e0 += kQBatch * kQThreads) {
+    float v[kQBatch][8];
 #pragma unroll
-    for (int k = 0; k < kQRegChunks; ++k) {
-      const int e = threadIdx.x + k * kQThreads;
-      if (e < total) keep[k] = __ldg(reinterpret_cast<const uint4*>(chunk_ptr<T>(a, q, b, h, r0 + e / C, e % C)));
+    for (int u = 0; u < kQBatch; ++u) {
+      const int e = e0 + u * kQThreads;
+      if (e < total) load8(chunk_ptr<T>(a, q, b, h, r0 + e / C, e % C), v[u]);
     }
 #pragma unroll
-    for (int k = 0; k < kQRegChunks; ++k) {
-      const int e = threadIdx.x + k * kQThreads;
+    for (int u = 0; u < kQBatch; ++u) {
+      const int e = e0 + u * kQThreads;
       if (e < total) {
-        float v[8];
-        bf16x8_to_float(keep[k], v);
-        apply_gain(a, q, b, r0 + e / C, v);
+        apply_gain(a, q, b, r0 + e / C, v[u]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
       }
-    }
-  } else {
-    for (int e = threadIdx.x; e < total; e += kQThreads) {
-      float v[8];
-      load8(chunk_ptr<T>(a, q, b, h, r0 + e / C, e % C), v);
-      apply_gain(a, q, b, r0 + e / C, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
     }
   }
   amax = warp_max(amax);
@@ -147,27 +128,24 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   const float s = block_amax == 0.0f ? 1.0f : __fdiv_rn(block_amax, kQMax);
   if (rank == 0 && threadIdx.x == 0) q.scale_out[bh] = s;
 
-  if (in_regs) {
+  // pass 2: codes (the rows are read again; they are in L2)
+#pragma unroll 1
+  for (int e0 = threadIdx.x; e0 < total; e0 += kQBatch * kQThreads) {
+    float v[kQBatch][8];
 #pragma unroll
-    for (int k = 0; k < kQRegChunks; ++k) {
-      const int e = threadIdx.x + k * kQThreads;
+    for (int u = 0; u < kQBatch; ++u) {
+      const int e = e0 + u * kQThreads;
+      if (e < total) load8(chunk_ptr<T>(a, q, b, h, r0 + e / C, e % C), v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kQBatch; ++u) {
+      const int e = e0 + u * kQThreads;
       if (e < total) {
         const int t = r0 + e / C, c = e % C;
-        float v[8];
-        bf16x8_to_float(keep[k], v);
-        apply_gain(a, q, b, t, v);
+        apply_gain(a, q, b, t, v[u]);
         const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
-        quant8(v, s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+        quant8(v[u], s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
       }
-    }
-  } else {
-    for (int e = threadIdx.x; e < total; e += kQThreads) {
-      const int t = r0 + e / C, c = e % C;
-      float v[8];
-      load8(chunk_ptr<T>(a, q, b, h, t, c), v);
-      apply_gain(a, q, b, t, v);
-      const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
-      quant8(v, s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
     }
   }
 }

@@ -13,7 +13,8 @@
 //   eliminate  warp ballots + popc give each kept key its output slot (a block-wide exclusive
 //              scan in index order), so the output is written in ascending index order.
 // Each CTA keeps up to kResident keys of its chunk in shared memory; the rest (only for rows
-// longer than clusters x kResident) is re-read from L2 in later passes.
+// longer than clusters x kResident) is streamed again from L2 in every pass, eight keys per
+// thread with 16-byte loads, and compacted with block-wide prefix sums of per-thread counts.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -57,6 +58,51 @@ __device__ __forceinline__ uint32_t load_key(const TArgs& a, int r, int j, int* 
   return float_key(f);
 }
 
+// 8 consecutive keys of row r starting at column j (absolute), columns >= lim invalid; two 16-byte
+// loads when the row is read directly and aligned, otherwise element loads
+__device__ __forceinline__ void load8_keys(const TArgs& a, int r, int j, int lim, bool vec, uint32_t* key, bool* ok,
+                                           int* nan_seen) {
+  if (vec && j + 7 < lim) {
+    const float4* p = reinterpret_cast<const float4*>(a.scores + static_cast<int64_t>(r) * a.ld + j);
+    const float4 f0 = __ldg(p), f1 = __ldg(p + 1);
+    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (f[u] != f[u]) *nan_seen = 1;
+      key[u] = float_key(f[u]);
+      ok[u] = true;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      ok[u] = j + u < lim;
+      key[u] = ok[u] ? load_key(a, r, j + u, nan_seen) : 0u;
+    }
+  }
+}
+
+// exclusive prefix sum of one value per thread over the block (all threads must call)
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wt, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) wt[warp] = inc;
+  __syncthreads();
+  uint32_t pre = 0u, tot = 0u;
+  for (int w = 0; w < kTWarps; ++w) {
+    const uint32_t x = wt[w];
+    if (w < warp) pre += x;
+    tot += x;
+  }
+  __syncthreads();
+  total = tot;
+  return pre + inc - v;
+}
+
 __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
@@ -76,20 +122,30 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   }
   if (a.k == 0) return;
 
-  const int chunk = (a.n + C - 1) / C;
+  // chunks start on a multiple of 4 keys so that direct rows can be read with 16-byte loads
+  const int chunk = (((a.n + C - 1) / C) + 3) & ~3;
   const int c0 = min(a.n, rank * chunk), c1 = min(a.n, c0 + chunk);
   const int len = c1 - c0;
   const int resident = min(len, kResident);
+  const bool vec = a.map == nullptr && (a.ld & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
   if (tid == 0) sh.nan_seen = 0;
   __syncthreads();
   int nan_local = 0;
-  for (int j = tid; j < resident; j += kTThreads) keys_s[j] = load_key(a, r, c0 + j, &nan_local);
+  // resident part: 8 keys per thread per step, 16-byte loads when possible
+  for (int base = 0; base < resident; base += 8 * kTThreads) {
+    const int j = base + 8 * tid;
+    uint32_t key[8];
+    bool ok[8];
+    load8_keys(a, r, c0 + j, c0 + resident, vec, key, ok, &nan_local);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (ok[u]) keys_s[j + u] = key[u];
+  }
   if (nan_local) sh.nan_seen = 1;
   __syncthreads();
 
   uint32_t prefix = 0u, mask = 0u;
   uint32_t krem = static_cast<uint32_t>(a.k);
-  uint32_t above_local = 0u;  // keys of this chunk known to be above the final threshold
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     uint32_t* hist = sh.hist[pass & 1];
@@ -100,12 +156,9 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
     }
     __syncthreads();
     uint32_t above_pass = 0u;
-    for (int base = 0; base < len; base += kTThreads) {
-      const int j = base + tid;
+    auto count_key = [&](uint32_t key, bool ok) {
       uint32_t bin = 256u;  // 256 = no histogram update
-      if (j < len) {
-        int dummy = 0;
-        const uint32_t key = j < resident ? keys_s[j] : load_key(a, r, c0 + j, &dummy);
+      if (ok) {
         const uint32_t hi = key & mask;
         if (hi == prefix)
           bin = (key >> shift) & 255u;
@@ -115,6 +168,18 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
       // warp-aggregated update: one shared atomic per distinct digit in the warp
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
       if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+    };
+    for (int base = 0; base < resident; base += kTThreads) {
+      const int j = base + tid;
+      count_key(j < resident ? keys_s[j] : 0u, j < resident);
+    }
+    for (int base = resident; base < len; base += 8 * kTThreads) {   // streamed part (long rows)
+      uint32_t key[8];
+      bool ok[8];
+      int dummy = 0;
+      load8_keys(a, r, c0 + base + 8 * tid, c0 + len, vec, key, ok, &dummy);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) count_key(key[u], ok[u]);
     }
     if (pass == 3) {
       for (int o = 16; o > 0; o >>= 1) above_pass += __shfl_xor_sync(0xffffffffu, above_pass, o);
@@ -160,15 +225,12 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
     }
     __syncthreads();
     const uint32_t d = sh.digit;
-    if (pass == 3) {
+    if (pass == 3 && tid == 0) {
       uint32_t gt = 0u;
       for (int w = 0; w < kTWarps; ++w) gt += sh.warp_a[w];
       for (uint32_t e = d + 1; e < 256u; ++e) gt += hist[e];
-      above_local = gt;
-      if (tid == 0) {
-        sh.n_gt = gt;
-        sh.n_eq = hist[d];
-      }
+      sh.n_gt = gt;
+      sh.n_eq = hist[d];
     }
     krem -= sh.above;
     prefix |= d << shift;
@@ -189,19 +251,14 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   }
   if (tid == 0 && sh.nan_seen) report(a.status, SPATTEN_E_NONFINITE);
   cluster.sync();  // peers' shared memory is no longer read after this point
-  (void)above_local;
 
-  // compaction in index order, kTThreads keys per tile
+  // compaction in index order: resident keys one per thread (ballot scans) ...
   uint32_t run_sel = sel_before, run_eq = eq_before;
-  for (int base = 0; base < len; base += kTThreads) {
+  for (int base = 0; base < resident; base += kTThreads) {
     const int j = base + tid;
-    uint32_t key = 0u;
-    if (j < len) {
-      int dummy = 0;
-      key = j < resident ? keys_s[j] : load_key(a, r, c0 + j, &dummy);
-    }
-    const bool gt = j < len && key > T;
-    const bool eq = j < len && key == T;
+    const uint32_t key = j < resident ? keys_s[j] : 0u;
+    const bool gt = j < resident && key > T;
+    const bool eq = j < resident && key == T;
     const unsigned beq = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) sh.warp_a[warp] = __popc(beq);
     __syncthreads();
@@ -231,11 +288,46 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
     run_eq += eq_tile;
     __syncthreads();
   }
+  // ... then streamed keys eight per thread (block scans of per-thread counts)
+  for (int base = resident; base < len; base += 8 * kTThreads) {
+    const int j = base + 8 * tid;
+    uint32_t key[8];
+    bool ok[8];
+    int dummy = 0;
+    load8_keys(a, r, c0 + j, c0 + len, vec, key, ok, &dummy);
+    uint32_t eqc = 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) eqc += (ok[u] && key[u] == T) ? 1u : 0u;
+    uint32_t eq_tile;
+    uint32_t er = run_eq + block_excl_scan(eqc, sh.warp_a, eq_tile);
+    bool sel[8];
+    uint32_t selc = 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const bool gt = ok[u] && key[u] > T;
+      const bool eq = ok[u] && key[u] == T;
+      sel[u] = gt || (eq && er < need_eq);
+      if (eq) ++er;
+      selc += sel[u] ? 1u : 0u;
+    }
+    uint32_t sel_tile;
+    uint32_t pos = run_sel + block_excl_scan(selc, sh.warp_b, sel_tile);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (sel[u] && pos < static_cast<uint32_t>(a.k)) {
+        a.idx_out[out_base + pos] = c0 + j + u;
+        if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + c0 + j + u];
+      }
+      pos += sel[u] ? 1u : 0u;
+    }
+    run_sel += sel_tile;
+    run_eq += eq_tile;
+  }
 }
 
 int pick_cluster(int n) {
-  // one CTA per 4096 keys, at most 8 (portable cluster size); 16 for very long rows when the
-  // device can schedule such clusters
+  // one CTA per 4096 keys, at most 8 (portable cluster size); the launcher may widen very long
+  // rows to 16 when the device can schedule such clusters
   int C = static_cast<int>(ceil_div(n, 4096));
   return std::max(1, std::min(C, 8));
 }
@@ -249,15 +341,33 @@ size_t topk_workspace_bytes(int R, int n, int k) {
 
 int32_t topk_launch(const TArgs& a, cudaStream_t st) {
   static bool configured[64] = {false};
+  static bool wide_ok[64] = {false};   // 16-CTA clusters can be scheduled on this device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     SPT_CUDA(cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kResident * 4));
+    if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(16, 1, 1);
+      q.blockDim = dim3(kTThreads, 1, 1);
+      q.dynamicSmemBytes = kResident * 4;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 16;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int clusters = 0;
+      wide_ok[dev] = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &q) == cudaSuccess && clusters >= 4;
+    }
+    cudaGetLastError();   // the probe above may leave an error behind
     configured[dev] = true;
   }
-  const int C = pick_cluster(a.n);
-  const int chunk = static_cast<int>(ceil_div(a.n, C));
+  int C = pick_cluster(a.n);
+  if (C == 8 && a.n > 8 * kResident && dev >= 0 && dev < 64 && wide_ok[dev]) C = 16;
+  const int chunk = static_cast<int>((ceil_div(a.n, C) + 3) & ~int64_t(3));
   const size_t smem = static_cast<size_t>(std::min(chunk, kResident)) * 4;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, a.R, 1);
