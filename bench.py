@@ -2,24 +2,34 @@
 """Benchmark of the cascade-pruned attention path (SpAtten-style) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload bert_base_prefill|gpt2m_decode|long_prefill]
 
-A step is one spatten_cascade_forward over the BERT-base-shaped prefill workload: B=32
-sequences of T=512 tokens, d_model 768, 12 heads of 64, 12 layers, token keep 0.9 per layer,
-one head dropped every 3 layers, 12-bit progressive K/V (8-bit MSB + 4-bit LSB planes), refetch
-when a row's max probability < 0.1, 5 % of tokens with K rows x4.  Inputs are seeded synthetic
-draws with random-init weights (bf16), resident in HBM before the timed region.  Metric: tokens/s
-(B*T per step, summed over ranks; weak scaling: each rank runs its own batch, no collective on the
-data path).  L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
+Default (one JSON line): the BERT-base-shaped prefill, with the GPT-2-medium-shaped decode in the
+line's "decode" object.
+* Prefill step: one spatten_cascade_forward over B=32 sequences of T=512 tokens, d_model 768, 12
+  heads of 64, 12 layers, token keep 0.9 per layer, one head dropped every 3 layers, 12-bit
+  progressive K/V (8-bit MSB + 4-bit LSB planes), refetch when a row's max probability < 0.1, 5 %
+  of tokens with K rows x4.  tokens/s = B*T per step.
+* Decode step: one generation of 128 tokens for B=16 sequences after a 1024-token prompt (24
+  layers, 16 heads of 64, d_model 1024), the K/V caches quantized once before timing, the cache
+  pruned by cumulative importance to 50 % by the last layer, refetch below 0.2.  One
+  spatten_cascade_forward per generated token.  tokens/s = B*128 per step.
+* long_prefill: B=1, T=16384, d_model 4096, 32 heads of 128, 4 layers, keep 0.5 per layer.
+Inputs are seeded synthetic draws with random-init weights (bf16), resident in HBM before the timed
+region; each timed step is one CUDA-graph replay; L2 is flushed (a 256 MB write) between timed
+steps, outside the timed events.  Weak scaling: each rank runs its own sequences, no collective
+on the data path; the value sums all ranks over the slowest rank's time.
 
-The JSON line also carries the roofline of the attention kernel (timed live per layer with CUDA
-events recorded around its launches on the launching stream), the end-to-end rate through the C
-ABI with host buffers (H2D of the inputs and D2H of the results inside the timed region), SM
+Each line carries the roofline of the dominant kernel (attention; timed live with CUDA events
+recorded by the library around its launches on the launching stream), the end-to-end rate through
+the C ABI with host buffers (H2D of the inputs and D2H of the results inside the timed region), SM
 clocks sampled during the timed region, and the float64 CPU oracle timed on a bounded sample.
 `--impl reference` times that oracle alone, as the reference arm.
 """
 from __future__ import annotations
 
 import argparse
+import ctypes as C
 import json
 import math
 import os
@@ -33,6 +43,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = {
+    "bert_base_prefill": "pruned-attn tokens/s (BERT-base prefill, cascade token/head pruning, progressive K/V)",
+    "long_prefill": "pruned-attn tokens/s (long-context prefill, cascade token/head pruning, progressive K/V)",
+    "gpt2m_decode": "generated tokens/s (GPT-2-medium decode, cumulative cache pruning, progressive K/V)",
+}
+DATA = "synthetic (seeded N(0,1) activations, random-init weights)"
 
 
 def load_peaks():
@@ -44,10 +60,29 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def prefill_workload(name):
+    from cascade_token_head_b200 import synth
+    return {"bert_base_prefill": synth.bert_base_prefill, "long_prefill": synth.long_prefill}[name]()
+
+
 def attention_flops(w) -> float:
     """Algorithmic attention flops of one prefill step: 4 * k_l^2 * d_h per kept head and sequence
     (Q K^T and P V on the kept tokens)."""
     return float(sum(w.B * w.head_keep[l] * 4.0 * w.token_keep[l] ** 2 * w.d_h for l in range(w.L)))
+
+
+def decode_attention_bytes(w, refetch_rows) -> float:
+    """Algorithmic bytes of the decode attention launches of one generation: per layer and token,
+    the MSB planes of K and V of the kept rows (B*H*k*d_h*2), the packed LSB planes of K and V for
+    every refetched (sequence, head) row (k*d_h), and the kept-row index list (B*k*4).
+    refetch_rows[s][l]: refetched (sequence, head) rows of token s, layer l."""
+    from cascade_token_head_b200.synth import linear_decode_keep
+    total = 0.0
+    for s in range(w.steps):
+        ks = linear_decode_keep(w.T0 + s + 1, w.L)
+        for l in range(w.L):
+            total += w.B * w.H * ks[l] * w.d_h * 2 + refetch_rows[s][l] * ks[l] * w.d_h + w.B * ks[l] * 4
+    return total
 
 
 # ------------------------------------------------------------------------------------------------
@@ -100,37 +135,101 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ------------------------------------------------------------------------------------------------
-# CPU oracle on a bounded sample
-# ------------------------------------------------------------------------------------------------
-def oracle_sample(w, d, seconds: float, max_seqs: int | None = None):
-    """Run the float64 oracle cascade one sequence at a time until `seconds` elapsed (at least one
-    sequence).  Returns (tokens/s, sequences done, wall seconds, threads)."""
-    import numpy as np
-    import torch
-    from oracle import spatten_ref as R
-
-    def cast(a):
-        return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
-
-    wq = [cast(a) for a in d["w_qkv"]]
-    wo = [cast(a) for a in d["w_o"]]
-    done, t0 = 0, time.perf_counter()
-    while True:
-        b = done % w.B
-        X = cast(d["X"][b:b + 1])
-        g = None if d["key_gain"] is None else d["key_gain"][b:b + 1]
-        R.cascade_prefill(X, wq, wo, w.H, w.d_h, w.token_keep, w.head_keep, w.quant, w.theta, key_gain=g)
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or (max_seqs and done >= max_seqs):
-            break
+def blas_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
-        threads = os.cpu_count() or 1
-    return done * w.T / el, done, el, threads
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle on bounded samples
+# ------------------------------------------------------------------------------------------------
+def _bf16_values(a):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
+
+
+def oracle_prefill_sample(w, d, seconds: float, max_units: int | None = None):
+    """BERT-shaped prefill: the float64 oracle cascade one whole sequence at a time until `seconds`
+    elapsed (at least one).  Long-context prefill (one sequence of 16384 tokens is minutes of
+    oracle work): the oracle's layer-0 attention of whole heads (all query rows, in row blocks),
+    extrapolated to the step by the ratio of the step's attention flops to the sample's.
+    Returns (tokens/s, description, threads)."""
+    import numpy as np
+    from oracle import spatten_ref as R
+
+    wq = [_bf16_values(a) for a in d["w_qkv"]]
+    wo = [_bf16_values(a) for a in d["w_o"]]
+    done, t0 = 0, time.perf_counter()
+    if w.T <= 4096:
+        while True:
+            b = done % w.B
+            X = _bf16_values(d["X"][b:b + 1])
+            g = None if d["key_gain"] is None else d["key_gain"][b:b + 1]
+            R.cascade_prefill(X, wq, wo, w.H, w.d_h, w.token_keep, w.head_keep, w.quant, w.theta, key_gain=g)
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or (max_units and done >= max_units):
+                break
+        return done * w.T / el, f"{done} sequence(s) of the workload (T={w.T}, all {w.L} layers), {el:.1f} s", \
+            blas_threads()
+    X = _bf16_values(d["X"][0])
+    qkv = X @ wq[0]
+    HD = w.H * w.d_h
+    sm = 1.0 / math.sqrt(w.d_h)
+    gain = d["key_gain"][0].astype(np.float32)[:, None]
+    t0 = time.perf_counter()
+    while True:
+        h = done % w.H
+        c = slice(h * w.d_h, (h + 1) * w.d_h)
+        kq = R.quantize_head(qkv[:, HD:2 * HD][:, c].astype(np.float32) * gain)
+        vq = R.quantize_head(qkv[:, 2 * HD:][:, c].astype(np.float32))
+        for r0 in range(0, w.T, 1024):
+            R.progressive_attention(qkv[r0:r0 + 1024, c], kq, vq, w.theta, sm)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_units and done >= max_units):
+            break
+    sample_flops = done * 4.0 * w.T * w.T * w.d_h
+    scale = attention_flops(w) / sample_flops
+    return w.T / (el * scale), (f"layer-0 attention of {done} head(s) (all {w.T} rows), {el:.1f} s, "
+                                f"extrapolated x{scale:.1f} by attention flops to one step"), blas_threads()
+
+
+class OracleDecode:
+    """The float64 oracle generating tokens of the decode workload, for the CPU baseline."""
+
+    def __init__(self, w, d):
+        from oracle import spatten_ref as R
+        self.R, self.w = R, w
+        self.wq = [_bf16_values(a) for a in d["w_qkv"]]
+        self.wo = [_bf16_values(a) for a in d["w_o"]]
+        self.caches = R.empty_decode_caches(len(self.wq), w.B, w.H, w.cap, w.d_h)
+        for l, c in enumerate(self.caches):
+            R.quantize_prompt_cache(c, d["k_prompt"][l], d["v_prompt"][l])
+        self.xs = d["x_steps"]
+
+    def generate(self, seconds: float, max_tokens: int | None = None):
+        """Generate tokens (teacher-forced inputs x_t, all sequences) from the prompt until
+        `seconds` elapsed.  Returns (generated tokens/s, tokens per sequence, wall seconds)."""
+        import numpy as np
+        from cascade_token_head_b200.synth import linear_decode_keep
+        w, R = self.w, self.R
+        n_old, I = w.T0, np.zeros((w.B, w.cap))
+        done, t0 = 0, time.perf_counter()
+        L = len(self.wq)
+        while True:
+            R.decode_step(_bf16_values(self.xs[done % w.steps]), self.caches, n_old, I, self.wq, self.wo,
+                          w.H, w.d_h, lambda n: linear_decode_keep(n, L), w.theta)
+            n_old += 1
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or (max_tokens and done >= max_tokens) or n_old >= w.cap:
+                break
+        return done * w.B / el, done, el
 
 
 def run_reference(args):
@@ -138,24 +237,31 @@ def run_reference(args):
     if rank != 0:
         return 0
     from cascade_token_head_b200 import synth
-    w = synth.bert_base_prefill()
-    d = synth.draw_prefill(w)
-    for _ in range(args.warmup):
-        oracle_sample(w, d, 0.0, max_seqs=1)
-    t0 = time.perf_counter()
-    threads = 1
-    for _ in range(args.steps):
-        _, _, _, threads = oracle_sample(w, d, 0.0, max_seqs=1)
-    el = time.perf_counter() - t0
-    value = args.steps * w.T / el
-    line = {"metric": "pruned-attn tokens/s (BERT-base prefill, cascade token/head pruning, progressive K/V)",
-            "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic (seeded N(0,1) activations, random-init weights)",
-            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "replicas"},
-            "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": f"one sequence (T={w.T}, all {w.L} layers) of the workload per step"},
+    if args.workload == "gpt2m_decode":
+        w = synth.gpt2m_decode()
+        o = OracleDecode(w, synth.draw_decode(w))
+        o.generate(0.0, max_tokens=args.warmup)
+        t0 = time.perf_counter()
+        o.generate(0.0, max_tokens=args.steps)
+        el = time.perf_counter() - t0
+        value = args.steps * w.B / el
+        cfg = {"workload": w.name, "global_batch": w.B, "prompt_len": w.T0, "parallelism": "replicas"}
+        sample = f"one generated token of all {w.B} sequences (all {w.L} layers) per step"
+    else:
+        w = prefill_workload(args.workload)
+        d = synth.draw_prefill(w)
+        oracle_prefill_sample(w, d, 0.0, max_units=args.warmup)
+        t0 = time.perf_counter()
+        value, sample, _ = oracle_prefill_sample(w, d, 0.0, max_units=args.steps)
+        el = time.perf_counter() - t0
+        cfg = {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "replicas"}
+        sample = f"per step: {sample}"
+    line = {"metric": METRIC[args.workload], "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": cfg, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -164,27 +270,91 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------------
-def run_ours(args):
+class Ctx:
+    """Device, ranks, stream and the L2 flush buffer shared by the workloads."""
+
+    def __init__(self):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist = torch, dist
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(self.local)
+        self.dev = torch.device("cuda", self.local)
+        if self.world > 1:
+            from datetime import timedelta
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=self.dev)
+        self.stream = torch.cuda.current_stream()
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=self.dev)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        t = self.torch.tensor([v], device=self.dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def events(self, n):
+        """n timing events, materialised on the stream so their handles can be handed over."""
+        ev = [self.torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in ev:
+            e.record(self.stream)
+        return ev
+
+
+def timed_replays(ctx, replay, K, after_each):
+    """K timed replays bracketed by events, an L2 flush before each (outside the events), clocks
+    sampled throughout.  after_each(i) runs after the replay has finished (reads its events)."""
+    torch = ctx.torch
+    ev_s, ev_e = ctx.events(K), ctx.events(K)
+    clocks = ClockSampler(ctx.local)
+    ctx.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K):
+        ctx.flush.zero_()
+        ev_s[i].record(ctx.stream)
+        replay()
+        ev_e[i].record(ctx.stream)
+        torch.cuda.synchronize()
+        after_each(i)
+    clk = clocks.stop()
+    ctx.barrier()
+    total_ms = ctx.max_over_ranks(sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K)))
+    return total_ms, clk
+
+
+def e2e_loop(ctx, body, n):
+    """Device-timed iterations of `body` (host->device copy, forward, device->host copy)."""
+    torch = ctx.torch
+    ms = []
+    for _ in range(n):
+        ctx.flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(ctx.stream)
+        body()
+        b.record(ctx.stream)
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    return ctx.max_over_ranks(sum(ms)), n
+
+
+def prefill_arm(ctx, args, name):
     import numpy as np
-    import torch
-    import torch.distributed as dist
-
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
+    torch = ctx.torch
     from cascade_token_head_b200 import spatten as S
     from cascade_token_head_b200 import synth
 
-    w = synth.bert_base_prefill()
-    w.seed = rank
+    w = prefill_workload(name)
+    w.seed = ctx.rank
     d = synth.draw_prefill(w)
-    bf = torch.bfloat16
+    bf, dev = torch.bfloat16, ctx.dev
     B, T, D, H, L = w.B, w.T, w.D, w.H, w.L
     X_host = torch.from_numpy(d["X"]).to(bf).pin_memory()
     gain_host = torch.from_numpy(d["key_gain"].astype(np.float32)).pin_memory()
@@ -192,8 +362,7 @@ def run_ours(args):
     gain = gain_host.to(dev)
     W = [(torch.from_numpy(d["w_qkv"][l]).to(bf).to(dev), torch.from_numpy(d["w_o"][l]).to(bf).to(dev))
          for l in range(L)]
-    kl = w.token_keep[-1]
-    x_out = torch.empty((B, kl, D), dtype=bf, device=dev)
+    x_out = torch.empty((B, w.token_keep[-1], D), dtype=bf, device=dev)
     kept_tok = torch.empty((L, B, T), dtype=torch.int32, device=dev)
     kept_head = torch.empty((L, B, H), dtype=torch.int32, device=dev)
     tok_imp = torch.empty((B, T), dtype=torch.float32, device=dev)
@@ -207,31 +376,22 @@ def run_ours(args):
     io.kept_tok, io.kept_head = kept_tok.data_ptr(), kept_head.data_ptr()
     io.tok_imp, io.head_imp, io.refetch_count = tok_imp.data_ptr(), head_imp.data_ptr(), refetch.data_ptr()
     io.dev_status = status.data_ptr()
-    stream = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
-        S.cascade_forward(cfg, W, io, ws, ws.numel(), stream=stream)
+        S.cascade_forward(cfg, W, io, ws, ws.numel(), stream=ctx.stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert int(status.item()) == 0, "device status after warm-up"
 
-    # per-step events and per-layer attention-kernel events (recorded by the library inside the
-    # captured step); the step is captured once into a CUDA graph and replayed K times
-    K = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    attn_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * L)]
-    for e in attn_ev:      # materialise the CUDA events before handing their handles over
-        e.record(stream)
+    # the library records event pair (2l, 2l+1) around layer l's attention launches; inside the
+    # captured step they become event-record nodes of the graph
+    attn_ev = ctx.events(2 * L)
     torch.cuda.synchronize()
-    import ctypes as C
     attn_array = (C.c_void_p * (2 * L))(*[e.cuda_event for e in attn_ev])
     io.attn_events = C.cast(attn_array, C.POINTER(C.c_void_p))
-    graph = None
-    launches_per_step = None
+    graph, launches_per_step = None, None
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
         l0 = S.kernel_launch_count()
@@ -240,37 +400,14 @@ def run_ours(args):
         launches_per_step = S.kernel_launch_count() - l0
         graph.replay()
         torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    launches0 = S.kernel_launch_count()
-    clocks.start()
-    time.sleep(0.3)
+    K = args.steps
     attn_ms = []
-    for i in range(K):
-        flush.zero_()
-        ev_s[i].record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            step()
-        ev_e[i].record(stream)
-        torch.cuda.synchronize()   # read this step's attention events before the next replay
-        attn_ms.append(sum(attn_ev[2 * l].elapsed_time(attn_ev[2 * l + 1]) for l in range(L)))
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    launches = (launches_per_step * K) if graph is not None else S.kernel_launch_count() - launches0
-    if world > 1:
-        dist.barrier()
-    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(K)]
+    launches0 = S.kernel_launch_count()
+    total_ms, clk = timed_replays(
+        ctx, graph.replay if graph is not None else step, K,
+        lambda i: attn_ms.append(sum(attn_ev[2 * l].elapsed_time(attn_ev[2 * l + 1]) for l in range(L))))
+    launches = launches_per_step * K if graph is not None else S.kernel_launch_count() - launches0
     io.attn_events = None
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     assert int(status.item()) == 0, "device status after timing"
     refetch_rows = refetch.cpu().tolist()
 
@@ -281,61 +418,152 @@ def run_ours(args):
     imp_host = torch.empty_like(tok_imp, device="cpu").pin_memory()
     h2d = X_host.numel() * X_host.element_size() + gain_host.numel() * 4
     d2h = out_host.numel() * 2 + kept_host.numel() * 4 + imp_host.numel() * 4
-    e2e_ms = []
-    for i in range(max(3, K // 2)):
-        flush.zero_()
-        a = torch.cuda.Event(enable_timing=True)
-        b_ = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+
+    def e2e_body():
         X.copy_(X_host, non_blocking=True)
         gain.copy_(gain_host, non_blocking=True)
         step()
         out_host.copy_(x_out, non_blocking=True)
         kept_host.copy_(kept_tok, non_blocking=True)
         imp_host.copy_(tok_imp, non_blocking=True)
-        b_.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms.append(a.elapsed_time(b_))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
 
+    e2e_total, n_e2e = e2e_loop(ctx, e2e_body, max(3, K // 2))
     tokens_per_step = B * T
-    value = world * tokens_per_step * K / (total_ms / 1e3)
-    e2e_value = world * tokens_per_step * len(e2e_ms) / (e2e_total / 1e3)
     peaks, peak_kind = load_peaks()
     flops = attention_flops(w)
     attn_s = statistics.mean(attn_ms) / 1e3
     achieved = flops / attn_s / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-
     result = {
-        "metric": "pruned-attn tokens/s (BERT-base prefill, cascade token/head pruning, progressive K/V)",
-        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, random-init weights)",
-        "config": {"workload": w.name, "global_batch": B * world, "seq_len": T, "d_model": D, "heads": H,
+        "metric": METRIC[name],
+        "value": ctx.world * tokens_per_step * K / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": ctx.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": w.name, "global_batch": B * ctx.world, "seq_len": T, "d_model": D, "heads": H,
                    "layers": L, "token_keep": w.token_keep, "head_keep": w.head_keep, "refetch_threshold": w.theta,
-                   "parallelism": f"dp{world} (independent sequences)", "l2": "flushed between timed steps",
+                   "parallelism": f"dp{ctx.world} (independent sequences)", "l2": "flushed between timed steps",
                    "launch": "CUDA graph of one step" if graph is not None else "direct launches"},
-        "roofline": {"kernel": "attention (spatten_attention_layer main kernel, all layers)", "bound": "tensor",
+        "roofline": {"kernel": "attention (spatten_attention_layer kernels, all layers)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None,
                      "algorithmic_flops_per_step": flops, "attn_ms_per_step": attn_s * 1e3},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": ctx.world * tokens_per_step * n_e2e / (e2e_total / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "clocks": clk,
         "refetch_rows_per_layer": refetch_rows,
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        v, n, el, threads = oracle_sample(w, d, args.cpu_seconds)
+    if ctx.rank == 0 and not args.no_cpu_baseline:
+        v, sample, threads = oracle_prefill_sample(w, d, args.cpu_seconds)
         result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                  "sample": f"{n} sequence(s) of the workload (T={T}, all {L} layers), {el:.1f} s"}
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
+                                  "sample": sample}
+    return result
+
+
+def decode_arm(ctx, args, steps):
+    torch = ctx.torch
+    from cascade_token_head_b200 import spatten as S
+    from cascade_token_head_b200 import synth
+    from cascade_token_head_b200.decode import DecodeState
+
+    w = synth.gpt2m_decode()
+    w.seed = ctx.rank
+    d = synth.draw_decode(w)
+    st = DecodeState(w, d["w_qkv"], d["w_o"], d["k_prompt"], d["v_prompt"])
+    torch.cuda.synchronize()
+    bf, dev, L = torch.bfloat16, ctx.dev, w.L
+    xs_host = torch.from_numpy(d["x_steps"]).to(bf).pin_memory()          # [steps, B, D]
+    xs = xs_host.to(dev)
+    outs = torch.empty_like(xs)
+    outs_host = torch.empty_like(xs_host).pin_memory()
+    imp_host = torch.empty_like(st.tok_imp, device="cpu").pin_memory()
+    refetch = torch.zeros((w.steps, L), dtype=torch.int32, device=dev)
+    attn_ev = [ctx.events(2 * L) for _ in range(w.steps)]
+    torch.cuda.synchronize()
+    arrays = [(C.c_void_p * (2 * L))(*[e.cuda_event for e in row]) for row in attn_ev]
+
+    def generation(timed_events):
+        st.reset()
+        for s in range(w.steps):
+            st.step(x=xs[s], x_out=outs[s], refetch=refetch[s], events=arrays[s] if timed_events else None,
+                    stream=torch.cuda.current_stream())
+
+    for _ in range(args.warmup):
+        generation(False)
+    torch.cuda.synchronize()
+    assert int(st.status.item()) == 0, "device status after warm-up (decode)"
+    graph = torch.cuda.CUDAGraph()
+    l0 = S.kernel_launch_count()
+    with torch.cuda.graph(graph):
+        generation(True)
+    launches_per_gen = S.kernel_launch_count() - l0
+    graph.replay()
+    torch.cuda.synchronize()
+    attn_ms = []
+    total_ms, clk = timed_replays(
+        ctx, graph.replay, steps,
+        lambda i: attn_ms.append(sum(row[2 * l].elapsed_time(row[2 * l + 1]) for row in attn_ev for l in range(L))))
+    assert int(st.status.item()) == 0, "device status after timing (decode)"
+    refetch_rows = refetch.cpu().tolist()
+
+    def e2e_body():
+        xs.copy_(xs_host, non_blocking=True)
+        generation(False)
+        outs_host.copy_(outs, non_blocking=True)
+        imp_host.copy_(st.tok_imp, non_blocking=True)
+
+    e2e_total, n_e2e = e2e_loop(ctx, e2e_body, 2)
+    tokens = w.B * w.steps
+    peaks, peak_kind = load_peaks()
+    nbytes = decode_attention_bytes(w, refetch_rows)
+    attn_s = statistics.mean(attn_ms) / 1e3
+    achieved = nbytes / attn_s / 1e9
+    peak = float(peaks.get("hbm_gbs"))
+    all_rows = w.B * w.H * w.steps * L
+    result = {
+        "metric": METRIC["gpt2m_decode"],
+        "value": ctx.world * tokens * steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": ctx.world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": total_ms / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": w.name, "global_batch": w.B * ctx.world, "prompt_len": w.T0,
+                   "generated_per_step": w.steps, "d_model": w.D, "heads": w.H, "layers": L,
+                   "keep": "linear to 50 % of the cache rows by the last layer", "refetch_threshold": w.theta,
+                   "parallelism": f"dp{ctx.world} (independent sequences)", "l2": "flushed between timed steps",
+                   "launch": "CUDA graph of one 128-token generation"},
+        "roofline": {"kernel": "decode attention (spatten_attention_layer decode kernel, all layers and tokens)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} HBM copy", "traffic": None,
+                     "algorithmic_bytes_per_step": nbytes, "attn_ms_per_step": attn_s * 1e3},
+        "e2e": {"value": ctx.world * tokens * n_e2e / (e2e_total / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": xs_host.numel() * 2,
+                "d2h_bytes_per_step": outs_host.numel() * 2 + imp_host.numel() * 4},
+        "gpu_launches": int(launches_per_gen * steps),
+        "clocks": clk,
+        "refetched_row_fraction": sum(map(sum, refetch_rows)) / all_rows,
+    }
+    if ctx.rank == 0 and not args.no_cpu_baseline:
+        o = OracleDecode(w, d)
+        v, n, el = o.generate(args.cpu_seconds)
+        result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                  "sample": f"{n} generated token(s) of all {w.B} sequences (all {L} layers), "
+                                            f"{el:.1f} s"}
+    return result
+
+
+def run_ours(args):
+    ctx = Ctx()
+    if args.workload == "gpt2m_decode":
+        result = decode_arm(ctx, args, args.steps)
+    else:
+        result = prefill_arm(ctx, args, args.workload)
+        if args.workload == "bert_base_prefill" and not args.no_decode:
+            dec = decode_arm(ctx, args, max(3, args.steps // 4))
+            result["decode"] = {k: dec[k] for k in ("metric", "value", "unit", "steps", "ms_per_step", "config",
+                                                    "roofline", "e2e", "gpu_launches", "clocks",
+                                                    "refetched_row_fraction", "cpu_baseline") if k in dec}
+    if ctx.world > 1:
+        ctx.dist.destroy_process_group()
+    if ctx.rank == 0:
         print(json.dumps(result), flush=True)
     return 0
 
@@ -346,9 +574,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--workload", choices=list(METRIC), default="bert_base_prefill")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="launch the step directly instead of replaying a CUDA graph")
+    ap.add_argument("--no-decode", action="store_true", help="leave the decode object out of the default line")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the prefill step directly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

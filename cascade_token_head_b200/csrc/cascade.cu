@@ -365,7 +365,7 @@ int32_t run_decode(const spatten_cascade_cfg& c, const spatten_layer_weights* w,
                                sizeof(float) * B * cap, cudaMemcpyDeviceToDevice, st));
     if (l == L - 1) break;
     int32_t* kept_n = io.kept_tok + static_cast<int64_t>(l + 1) * B * cap;
-    SPT_TRY(spatten_topk_select(io.dec_tok_imp, B, k, cap, c.token_keep[l + 1], kept_l, cap, ws.sel, cap, kept_n,
+    SPT_TRY(spatten_topk_select(io.dec_tok_imp, B, k, cap, c.token_keep[l + 1], kept_l, cap, nullptr, cap, kept_n,
                                 nullptr, 0, io.dev_status, st));
   }
   SPT_CUDA(cudaMemcpyAsync(io.x_out, x, static_cast<size_t>(B) * D * es, cudaMemcpyDeviceToDevice, st));

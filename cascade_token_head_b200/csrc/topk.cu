@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   const int64_t out_base = static_cast<int64_t>(r) * a.ld_out;
   if (a.k == a.n) {  // everything is kept: positions 0..n-1
     for (int j = rank * kTThreads + tid; j < a.n; j += C * kTThreads) {
-      a.idx_out[out_base + j] = j;
+      if (a.idx_out) a.idx_out[out_base + j] = j;
       if (a.comp_out) a.comp_out[out_base + j] = a.map[static_cast<int64_t>(r) * a.ld_map + j];
     }
     return;
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
       sel_tile += v;
     }
     if (sel && pos < static_cast<uint32_t>(a.k)) {
-      a.idx_out[out_base + pos] = c0 + j;
+      if (a.idx_out) a.idx_out[out_base + pos] = c0 + j;
       if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + c0 + j];
     }
     run_sel += sel_tile;
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (sel[u] && pos < static_cast<uint32_t>(a.k)) {
-        a.idx_out[out_base + pos] = c0 + j + u;
+        if (a.idx_out) a.idx_out[out_base + pos] = c0 + j + u;
         if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + c0 + j + u];
       }
       pos += sel[u] ? 1u : 0u;
@@ -398,7 +398,7 @@ extern "C" int32_t spatten_topk_select(const float* scores, int32_t R, int32_t n
                                        void* stream) {
   using namespace spt;
   (void)ws;
-  if (!scores || !idx_out) return SPATTEN_E_ARG;
+  if (!scores || (!idx_out && !comp_out)) return SPATTEN_E_ARG;
   if (R < 1 || n < 1 || k < 0 || R > 65535) return SPATTEN_E_ARG;
   if (k > n) return SPATTEN_E_SHAPE;
   if (ld_out < k) return SPATTEN_E_SHAPE;

@@ -202,7 +202,8 @@ int32_t spatten_attention_layer_noalloc(const spatten_attn_args* a, void* stream
  *
  *  scores   device float; row r element j is scores[r*ld + (map ? map[r*ld_map + j] : j)].
  *  map      device int32 [R][ld_map] or NULL: reads scores through an index list (gather fused).
- *  idx_out  device int32 [R][ld_out]: positions j (0 <= j < n) of the selected elements.
+ *  idx_out  device int32 [R][ld_out] or NULL: positions j (0 <= j < n) of the selected
+ *           elements.  May be NULL only when comp_out is given.
  *  comp_out device int32 [R][ld_out] or NULL: map[r][idx_out[r][c]] (index-map composition);
  *           requires map.
  *  Requirements: R >= 1, 1 <= n, 0 <= k <= n, ld >= n when map is NULL, ld_out >= k.

@@ -1,0 +1,138 @@
+"""GPU parity at the long-context prefill size (T = 16384, 32 heads of d_h = 128, D = 4096).
+
+* One layer, one kept head, every output checked: the oracle runs the head's 16384 query rows in
+  blocks (rows are independent), so the full token-importance vector, O and flags are compared.
+* The whole four-layer cascade with traces, checked on sampled rows and heads of every layer:
+  projections, O and refetch flags of sampled (row, head) pairs against the oracle on the device's
+  own layer inputs; per-layer importance increments by the properties that hold at any size (the
+  increment sums to k_l x H_l, vanishes off the kept rows, head increments equal sum |O|); kept
+  token and head sets bit-exact against the oracle's selection on the device's importance; the
+  next layer's rows X_l + O W_o on sampled rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from cascade_token_head_b200 import synth
+from oracle import spatten_ref as R
+
+from cascade_helpers import run_prefill, upload_prefill
+from gpu_helpers import BF, assert_close_bf16_out, host_cast, lib
+from test_gpu_attention import make_layer, run_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def test_attention_long_one_head_every_output(cuda):
+    S = lib()
+    B, H, n, d, theta = 1, 32, 16384, 128, 0.1
+    h = 5
+    raw, gain = make_layer(B, H, n, d, seed=41, boost=328)
+    got = run_layer(S, raw, gain, B, H, n, d, theta, heads=np.array([[h]]))
+    HD = H * d
+    vals = host_cast(raw[0], BF)
+    Q = vals[:, h * d:(h + 1) * d]
+    K = vals[:, HD + h * d:HD + (h + 1) * d].astype(np.float32) * gain[0][:, None]
+    V = vals[:, 2 * HD + h * d:2 * HD + (h + 1) * d].astype(np.float32)
+    kq, vq = R.quantize_head(K), R.quantize_head(V)
+    np.testing.assert_array_equal(got["msbk"][0, h], kq["msb"])
+    np.testing.assert_array_equal(R.unpack_lsb(got["lsbk"][0, h]), kq["lsb"])
+    np.testing.assert_array_equal(got["msbv"][0, h], vq["msb"])
+    sm = 1.0 / math.sqrt(d)
+    O = np.zeros((n, d))
+    tok = np.zeros(n)
+    gf = got["flags"][0, h].astype(bool)
+    near = 0
+    for r0 in range(0, n, 1024):
+        rows = slice(r0, r0 + 1024)
+        r = R.progressive_attention(Q[rows], kq, vq, theta, sm)
+        diff = gf[rows] != r["flags"]
+        if diff.any():
+            assert np.all(np.abs(r["pmax_msb"][diff] - theta) <= 1e-5 * theta), "flag mismatch off a tie"
+            near += int(diff.sum())
+            r = R.progressive_attention(Q[rows], kq, vq, theta, sm, flags_override=gf[rows])
+        O[rows] = r["O"]
+        tok += R.token_importance_increment(r["P"])
+    assert_close_bf16_out(got["o"][0][:, h * d:(h + 1) * d], O, 2e-2, "O (long, one head)")
+    others = np.delete(got["o"][0], np.arange(h * d, (h + 1) * d), axis=1)
+    assert np.all(others == 0)
+    np.testing.assert_allclose(got["tok"][0], tok, rtol=0, atol=2e-5 * tok.max())
+    np.testing.assert_allclose(got["head"][0, h], R.head_importance_increment(O), rtol=2e-3)
+    assert np.all(np.delete(got["head"][0], h) == 0)
+    assert got["count"] == int(gf.sum())
+    print(f"refetched rows {int(gf.sum())}, near-tie flags {near}")
+
+
+def test_cascade_long_full_size_sampled(cuda):
+    S = lib()
+    w = synth.long_prefill()
+    d = synth.draw_prefill(w)
+    bufs = upload_prefill(S, w, d)
+    run_prefill(S, bufs)
+    assert int(bufs["status"].item()) == 0
+    H, dh, T = w.H, w.d_h, w.T
+    HD = H * dh
+    sm = 1.0 / math.sqrt(dh)
+    g = synth.rng_for(1234)
+    kept_tok = bufs["kept_tok"].cpu().numpy()
+    kept_head = bufs["kept_head"].cpu().numpy()
+    ttok = bufs["ttok"].cpu().numpy().astype(np.float64)
+    thead = bufs["thead"].cpu().numpy().astype(np.float64)
+    refetch = bufs["refetch"].cpu().numpy()
+    gain = d["key_gain"][0].astype(np.float32)
+    I_prev = np.zeros(T)
+    J_prev = np.zeros(H)
+    for l in range(w.L):
+        k, Hl = w.token_keep[l], w.head_keep[l]
+        wq = host_cast(d["w_qkv"][l], BF)
+        wo = host_cast(d["w_o"][l], BF)
+        S_l = kept_tok[l, 0, :k].astype(np.int64)
+        heads = kept_head[l, 0, :Hl].astype(np.int64)
+        assert np.all(np.diff(S_l) > 0) and np.all(np.diff(heads) > 0)
+        X_l = bufs["tx"][l, 0, :k].float().cpu().numpy().astype(np.float64)
+        qkv = bufs["tqkv"][l, 0, :k].float().cpu().numpy()          # bf16 values, exact in float32
+        O_dev = bufs["to"][l, 0, :k].float().cpu().numpy()
+        flags = bufs["tflags"][l, 0, :, :k].cpu().numpy().astype(bool)
+        rows = np.sort(g.choice(k, size=48, replace=False))
+        assert_close_bf16_out(qkv[rows], X_l[rows] @ wq, 2e-2, f"qkv layer {l}")
+        for h in g.choice(heads, size=2, replace=False):
+            c = slice(h * dh, (h + 1) * dh)
+            Kh = qkv[:, HD + h * dh:HD + (h + 1) * dh] * gain[S_l][:, None]
+            Vh = qkv[:, 2 * HD + h * dh:2 * HD + (h + 1) * dh]
+            kq, vq = R.quantize_head(Kh), R.quantize_head(Vh)
+            r = R.progressive_attention(qkv[rows, c].astype(np.float64), kq, vq, w.theta, sm)
+            diff = flags[h, rows] != r["flags"]
+            if diff.any():
+                assert np.all(np.abs(r["pmax_msb"][diff] - w.theta) <= 1e-5 * w.theta), "flag off a tie"
+                r = R.progressive_attention(qkv[rows, c].astype(np.float64), kq, vq, w.theta, sm,
+                                            flags_override=flags[h, rows])
+            assert_close_bf16_out(O_dev[rows, c], r["O"], 2e-2, f"O layer {l} head {h}")
+        # importance increments: properties that hold at any size
+        dI = ttok[l, 0] - I_prev
+        assert abs(dI.sum() - k * Hl) <= 1e-4 * k * Hl
+        assert np.all(np.delete(dI, S_l) == 0) and dI.min() >= -1e-3
+        dJ = thead[l, 0] - J_prev
+        for h in range(H):
+            if h in heads:
+                np.testing.assert_allclose(dJ[h], np.abs(O_dev[:, h * dh:(h + 1) * dh]).sum(dtype=np.float64),
+                                           rtol=5e-3)
+            else:
+                assert dJ[h] == 0
+        assert int(refetch[l]) == int(flags[heads].sum())
+        I_prev, J_prev = ttok[l, 0], thead[l, 0]
+        if l == w.L - 1:
+            x_out = bufs["x_out"][0].float().cpu().numpy()
+            assert_close_bf16_out(x_out[rows], X_l[rows] + O_dev[rows].astype(np.float64) @ wo, 2e-2, "final rows")
+            break
+        k2, H2 = w.token_keep[l + 1], w.head_keep[l + 1]
+        S_n = kept_tok[l + 1, 0, :k2].astype(np.int64)
+        np.testing.assert_array_equal(S_n, S_l[R.topk_select(ttok[l, 0][S_l], k2)])
+        H_n = kept_head[l + 1, 0, :H2].astype(np.int64)
+        np.testing.assert_array_equal(H_n, heads[R.topk_select(thead[l, 0][heads], H2)])
+        nxt = np.sort(g.choice(k2, size=48, replace=False))
+        pos = np.searchsorted(S_l, S_n[nxt])
+        X_next = bufs["tx"][l + 1, 0, :k2].float().cpu().numpy()[nxt]
+        assert_close_bf16_out(X_next, X_l[pos] + O_dev[pos].astype(np.float64) @ wo, 2e-2, f"X layer {l + 1}")
+    print("refetch per layer", refetch.tolist())
