@@ -76,13 +76,27 @@ size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
   const int rows = rows_per_cta(path);
   const int64_t n_qt = ceil_div(a.n_q, rows);
   WsCursor c(p ? p->tok_part : nullptr, ~size_t(0));
-  float* t = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * n_qt * a.n_kv);
-  float* h = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * n_qt);
+  // per-CTA partials of the prefill kernels (the decode kernels keep per-item partials instead)
+  const size_t parts = path == Path::kDecode ? 0 : static_cast<size_t>(a.B) * a.H_kept * n_qt;
+  float* t = c.take<float>(parts * a.n_kv);
+  float* h = c.take<float>(parts);
   int32_t* fl = nullptr;
   int32_t* fc = nullptr;
   float* fp = nullptr;
   float* fh = nullptr;
   const int64_t n_pair = ceil_div(a.n_q, 256);
+  int items = 0;
+  float* de = nullptr;
+  float* ds = nullptr;
+  float* dob = nullptr;
+  if (path == Path::kDecode) {
+    const int ir = decode_item_rows(a.d_h);
+    items = static_cast<int>(ceil_div(a.n_kv, ir));
+    const size_t bh = static_cast<size_t>(a.B) * a.H_kept;
+    de = c.take<float>(2 * bh * a.n_kv);
+    ds = c.take<float>(bh * items * 4);
+    dob = c.take<float>(bh * items * 2 * a.d_h);
+  }
   if (path == Path::kTc) {
     fl = c.take<int32_t>(static_cast<size_t>(a.B) * a.H_kept * n_pair * 256);
     fc = c.take<int32_t>(static_cast<size_t>(a.B) * a.H_kept * n_pair);
@@ -99,6 +113,10 @@ size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
     p->flag_cnt = fc;
     p->full_part = fp;
     p->full_head = fh;
+    p->dec_items = items;
+    p->dec_e = de;
+    p->dec_stat = ds;
+    p->dec_o = dob;
   }
   return c.used;
 }
@@ -139,12 +157,12 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
   int32_t s;
   switch (path) {
     case Path::kTc: s = attn_tc_launch(p, st); break;
-    case Path::kDecode: s = attn_decode_launch(p, st); break;
+    case Path::kDecode: s = attn_decode_launch(p, st); break;   // its own combine step reduces
     default: s = attn_simt_launch(p, st); break;
   }
   if (s != SPATTEN_OK) return s;
   if (ev_end) SPT_CUDA(cudaEventRecordWithFlags(ev_end, st, ev_flags));
-  if (!p.a.tok_imp && !p.a.head_imp) return SPATTEN_OK;
+  if (path == Path::kDecode || (!p.a.tok_imp && !p.a.head_imp)) return SPATTEN_OK;
   return attn_reduce_launch(p, st);
 }
 }  // namespace spt

@@ -19,6 +19,12 @@ struct AttnProblem {
   int32_t* flag_cnt;         // ws [B][H_kept][n_pair] number of flagged rows
   float* full_part;          // ws [B][H_kept][2*n_pair][n_kv] column sums of the packed tiles
   float* full_head;          // ws [B][H_kept][2*n_pair] sum |O| of the packed tiles
+  // decode path only: per-item partials of the streaming kernel (an item is a run of
+  // decode_item_rows(d_h) consecutive entries of a row's key list)
+  int dec_items;             // items per (b, kept head) = ceil(n_kv / item rows)
+  float* dec_e;              // ws [2][B][H_kept][n_kv] exp(s - item max): MSB-only, full precision
+  float* dec_stat;           // ws [B][H_kept][dec_items][4] item max and sum, both variants
+  float* dec_o;              // ws [B][H_kept][dec_items][2][d_h] item sum of exp * V, both variants
 };
 
 // Kernels (each returns a status after launching on `st`).
@@ -27,10 +33,12 @@ int32_t attn_tc_launch(const AttnProblem& p, cudaStream_t st);
 int32_t attn_decode_launch(const AttnProblem& p, cudaStream_t st);
 bool attn_tc_supported(const spatten_attn_args& a);
 bool attn_decode_supported(const spatten_attn_args& a);
+int decode_item_rows(int d_h);    // keys per item of the decode kernel
 constexpr int kTcRows = 128;      // query rows per CTA of the tensor-core kernel
 constexpr int kSimtRows = 32;     // query rows per CTA of the CUDA-core kernel
 
-// spatten_attention_layer with optional events recorded around the main kernel (not the reduce).
+// spatten_attention_layer with optional events recorded around the main kernel (not the reduce;
+// on the decode path around both of its kernels).
 int32_t attention_layer_timed(const spatten_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t st,
                               cudaEvent_t ev_begin, cudaEvent_t ev_end);
 

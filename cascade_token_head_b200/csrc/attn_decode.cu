@@ -4,263 +4,420 @@
 // SpAtten §II "Attention-based NLP models": generation handles one new token per iteration
 // against cached K and V (a memory-bound workload); §IV.E "Progressive Quantization": the LSBs
 // are fetched only when the max probability is below the threshold.
-// Per CTA (b, kept head):
-//   1  MSB scores: lanes read 16-byte slices of the int8 MSB rows (d_h/16 lanes per key, rows
-//      reached through kv_idx), s_j = (16 * s_k * sm_scale) * (q . MSB_j); kept in shared memory.
-//   2  row stats m, ell; flag = 1/ell < theta.
-//   3  flagged rows only: read the LSB rows, s_j += s_k * sm_scale * (q . LSB_j); new m, ell.
-//   4  p_j = exp(s_j - m)/ell -> importance partial; O = s_v * sum_j p_j (16*MSB_j [+ LSB_j]).
-// Every sweep over the keys issues kUnroll independent index loads and then kUnroll independent
-// 16-byte row loads per lane before using them, so each CTA keeps tens of KB in flight (the sweep
-// is bound by HBM bandwidth, not by load latency).  Importance partials are reduced over heads
-// in a fixed order by attn_reduce.
+//
+// The work of one row (b, kept head) is cut into items of decode_item_rows(d_h) consecutive
+// entries of its key list, one warp per item, and finished by a per-sequence combine step:
+//
+// items kernel (memory-bound, no block-level barrier): a warp streams the K and V code rows of
+//   its item once -- lane groups of d_h/16 lanes read 16-byte MSB and 8-byte packed LSB slices,
+//   batches of rows in flight together -- and evaluates both precisions the refetch rule can pick:
+//   s1 = s_k * sm_scale * 16 (q . MSB_j)            (MSB pass)
+//   s2 = s_k * sm_scale (q . (16 MSB_j + LSB_j))     (full 12-bit codes)
+//   It writes, per variant, the item's max m, sum ell of exp(s - m), the exponentials
+//   e_j = exp(s_j - m) and the item's sum of e_j times the V codes (MSB_j for the MSB pass, whose
+//   values are 16 MSB_j; 16 MSB_j + LSB_j for full precision).  With theta <= 0 no row can refetch and only the MSB
+//   variant is computed (the LSB planes are not read).
+// combine kernel (one CTA row per sequence): folds the item statistics of every kept head in item
+//   order into the row's (m, ell) for each variant, takes the refetch decision 1/ell_MSB < theta,
+//   and with the chosen variant's factors f_item = exp(m_item - m) / ell forms
+//   p_j = e_j f_item(j)           -> token importance (summed over heads in slot order)
+//   O   = s_v sum_items f_item o_item -> output, sum |O| -> head importance.
+// Both kernels run in fixed orders, so results are bit-reproducible.  Reading the LSB planes with
+// the MSB planes (rather than after the decision) costs up to half of the MSB bytes again for rows
+// that do not refetch, and saves a dependent second pass over the cache for rows that do.
 #include "attention.cuh"
 
 namespace spt {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kMaxKv = 32768;   // scores kept in shared memory (128 KB)
-constexpr int kUnroll = 4;
+constexpr int kDWarps = 4;        // warps (items) per CTA of the items kernel
+constexpr int kCThreads = 256;    // threads per CTA of the combine kernel
 
-__device__ __forceinline__ void unpack16_s8(uint4 u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) f[4 * i + k] = static_cast<float>(static_cast<int8_t>((w[i] >> (8 * k)) & 0xFFu));
-}
-__device__ __forceinline__ void unpack16_u4(uint2 u, float* f) {
-  const uint32_t w[2] = {u.x, u.y};
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) f[8 * i + k] = static_cast<float>((w[i] >> (4 * k)) & 0xFu);
-}
+template <int DH>
+struct DGeom {
+  static constexpr int LPK = DH / 16;        // lanes per key row (16 codes per lane)
+  static constexpr int KPW = 32 / LPK;       // keys per warp step
+  static constexpr int ITEM = 8192 / DH;     // keys per item: 128 (d_h 64), 64 (d_h 128)
+  static constexpr int STEPS = ITEM / KPW;   // warp steps per item
+  static constexpr int BATCH = 8;            // steps whose row loads are in flight together
+};
 
-template <int DH, typename QT>
-__global__ void __launch_bounds__(kThreads) attn_decode_kernel(AttnProblem p) {
-  const spatten_attn_args& a = p.a;
-  constexpr int LPK = DH / 16;          // lanes per key row (16 codes per lane)
-  constexpr int KPW = 32 / LPK;         // keys per warp per step
-  constexpr int KPS = KPW * kWarps;     // keys per CTA step
-  constexpr int KPU = KPS * kUnroll;    // keys per unrolled step
-  extern __shared__ __align__(16) float s_sc[];   // [n_kv] scores, then probabilities
-  __shared__ float red[kWarps];
-  __shared__ float o_red[kWarps][DH];
-  __shared__ float bcast[2];
+// Paired fp32 arithmetic: the sm_100 float2 intrinsics (two lanes per instruction).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-  const int slot = blockIdx.x, b = blockIdx.y;
-  const int h = head_of_slot(a, b, slot);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane % LPK, grp = lane / LPK;
-  QT* o = static_cast<QT*>(a.o);
-  if (slot >= a.H_kept) {
-    if (h >= 0 && threadIdx.x < DH)
-      st_from_float(o + static_cast<int64_t>(b) * a.n_q * a.o_ld_tok + static_cast<int64_t>(h) * DH + threadIdx.x, 0.0f);
-    return;
+// Signed code bytes to floats: each byte, biased to unsigned (x ^ 0x80), is placed in the low
+// mantissa byte of 2^23; subtracting 2^23 + 128 leaves the signed value exactly.  Sixteen codes
+// (one uint4) give eight pairs, element 2i and 2i+1 in pair i.
+__device__ __forceinline__ void msb16(uint4 v, float2* f) {
+  const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u, v.w ^ 0x80808080u};
+  const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = fadd2(make_float2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540)),
+                                 __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7541))), bias);
+    f[2 * i + 1] = fadd2(make_float2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7542)),
+                                     __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7543))), bias);
   }
+}
+// Sixteen packed 4-bit codes (element 2k in bits 8k..8k+3 of the pair of words, element 2k+1 in
+// bits 8k+4..8k+7) as eight pairs.
+__device__ __forceinline__ void lsb16(uint2 v, float2* f) {
+  const float2 bias = make_float2(-8388608.0f, -8388608.0f);
+  const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      f[4 * i + k] = fadd2(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7540 + k)),
+                                       __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7540 + k))), bias);
+  }
+}
+
+template <int DH, typename QT, bool LSB>
+__global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnProblem p) {
+  using G = DGeom<DH>;
+  constexpr int LPK = G::LPK, KPW = G::KPW, ITEM = G::ITEM, STEPS = G::STEPS, BATCH = G::BATCH;
+  constexpr int NV = LSB ? 2 : 1;   // variants: MSB pass [, full precision]
+  const spatten_attn_args& a = p.a;
+  __shared__ float s_sc[kDWarps][NV][ITEM];         // scores, then exponentials
+  __shared__ float s_o[kDWarps][KPW][NV * DH];      // per lane group sums of e * V
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the (kept head, item) pairs of sequence b, numbered head-major, one per warp
+  const int w_id = blockIdx.x * kDWarps + warp;
+  const int slot = w_id / p.dec_items, item = w_id % p.dec_items;
+  if (slot >= a.H_kept) return;   // warps are independent: no block-level barrier follows
+  const int b = blockIdx.y;
+  const int h = head_of_slot(a, b, slot);
+  const int sub = lane % LPK, grp = lane / LPK;
+  const int n = a.n_kv;
+  const int j0 = item * ITEM;
   const int64_t bh = static_cast<int64_t>(b) * a.H + h;
   const int64_t plane0 = bh * a.kv_cap;
+  const int64_t bs = static_cast<int64_t>(b) * a.H_kept + slot;
   const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
 
-  float qf[16];
+  float2 qf[8];
   {
-    const QT* q = static_cast<const QT*>(a.q) + static_cast<int64_t>(b) * a.n_q * a.q_ld_tok + static_cast<int64_t>(h) * DH + sub * 16;
+    const QT* q = static_cast<const QT*>(a.q) + static_cast<int64_t>(b) * a.n_q * a.q_ld_tok +
+                  static_cast<int64_t>(h) * DH + sub * 16;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) qf[i] = ld_as_float(q + i);
+    for (int i = 0; i < 8; ++i) qf[i] = make_float2(ld_as_float(q + 2 * i), ld_as_float(q + 2 * i + 1));
   }
-  const float ks = a.k_scale[bh], vs = a.v_scale[bh];
-  const float c_msb = 16.0f * ks * a.sm_scale;
-  const float c_lsb = ks * a.sm_scale;
-  const int n = a.n_kv;
+  const float ks = a.k_scale[bh];
+  const float c1 = 16.0f * ks * a.sm_scale, c2 = ks * a.sm_scale;
+  auto row_of = [&](int j) -> int64_t { return j < n ? plane0 + (kv_idx ? __ldg(kv_idx + j) : j) : -1; };
 
-  // rows of the kUnroll keys this lane group handles in the unrolled step starting at j0
-  auto rows_of = [&](int j0, int64_t* rows, int* js) {
+  // ---- scores of both variants -----------------------------------------------------------------
+  float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll 1
+  for (int s0 = 0; s0 < STEPS; s0 += BATCH) {
+    int64_t row[BATCH];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      js[u] = j0 + u * KPS + warp * KPW + grp;
-      rows[u] = js[u] < n ? plane0 + (kv_idx ? __ldg(kv_idx + js[u]) : js[u]) : 0;
+    for (int u = 0; u < BATCH; ++u) row[u] = row_of(j0 + (s0 + u) * KPW + grp);
+    uint4 km[BATCH];
+    uint2 kl[BATCH];
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u)
+      km[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.k_msb + row[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+    if (LSB) {
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u)
+        kl[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint2*>(a.k_lsb + row[u] * (DH / 2)) + sub) : make_uint2(0, 0);
     }
-  };
-
-  // ---- 1: MSB scores -------------------------------------------------------------------------
-  float mloc = -INFINITY;
-  for (int j0 = 0; j0 < n; j0 += KPU) {
-    int64_t rows[kUnroll];
-    int js[kUnroll];
-    rows_of(j0, rows, js);
-    uint4 raw[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      raw[u] = js[u] < n ? __ldg(reinterpret_cast<const uint4*>(a.k_msb + rows[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < BATCH; ++u) {
+      // d1 = q . MSB_j; d2 = q . LSB_j; the full-precision dot product is 16 d1 + d2
+      float2 f[8];
+      msb16(km[u], f);
+      float2 a1 = make_float2(0.0f, 0.0f), a2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      float f[16];
-      unpack16_s8(raw[u], f);
-      float part = 0.0f;
+      for (int i = 0; i < 8; ++i) a1 = ffma2(qf[i], f[i], a1);
+      if (LSB) {
+        float2 g[8];
+        lsb16(kl[u], g);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) part = fmaf(qf[i], f[i], part);
-#pragma unroll
-      for (int o2 = 1; o2 < LPK; o2 <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-      if (js[u] < n && sub == 0) {
-        const float s = part * c_msb;
-        s_sc[js[u]] = s;
-        mloc = fmaxf(mloc, s);
+        for (int i = 0; i < 8; ++i) a2 = ffma2(qf[i], g[i], a2);
       }
-    }
-  }
-  auto block_max = [&](float v) {
-    v = warp_max(v);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = red[0];
-      for (int w = 1; w < kWarps; ++w) t = fmaxf(t, red[w]);
-      bcast[0] = t;
-    }
-    __syncthreads();
-    return bcast[0];
-  };
-  auto block_sum = [&](float v) {
-    v = warp_sum(v);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = 0.0f;
-      for (int w = 0; w < kWarps; ++w) t += red[w];
-      bcast[1] = t;
-    }
-    __syncthreads();
-    return bcast[1];
-  };
-  __syncthreads();
-  float m = block_max(mloc);
-  float l = 0.0f;
-  for (int j = threadIdx.x; j < n; j += kThreads) l += expf(s_sc[j] - m);
-  l = block_sum(l);
-  const bool flag = 1.0f / l < a.refetch_threshold;
-
-  // ---- 3: LSB refetch for a flagged row ------------------------------------------------------
-  if (flag) {
-    mloc = -INFINITY;
-    for (int j0 = 0; j0 < n; j0 += KPU) {
-      int64_t rows[kUnroll];
-      int js[kUnroll];
-      rows_of(j0, rows, js);
-      uint2 raw[kUnroll];
+      float d1 = a1.x + a1.y, d2 = a2.x + a2.y;
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        raw[u] = js[u] < n ? __ldg(reinterpret_cast<const uint2*>(a.k_lsb + rows[u] * (DH / 2)) + sub) : make_uint2(0, 0);
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        float f[16];
-        unpack16_u4(raw[u], f);
-        float part = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) part = fmaf(qf[i], f[i], part);
-#pragma unroll
-        for (int o2 = 1; o2 < LPK; o2 <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-        if (js[u] < n && sub == 0) {
-          const float s = s_sc[js[u]] + part * c_lsb;
-          s_sc[js[u]] = s;
-          mloc = fmaxf(mloc, s);
+      for (int o2 = 1; o2 < LPK; o2 <<= 1) {
+        d1 += __shfl_xor_sync(0xffffffffu, d1, o2);
+        if (LSB) d2 += __shfl_xor_sync(0xffffffffu, d2, o2);
+      }
+      if (row[u] >= 0) {
+        const float s1 = d1 * c1, s2 = fmaf(16.0f, d1, d2) * c2;
+        m1 = fmaxf(m1, s1);
+        if (LSB) m2 = fmaxf(m2, s2);
+        if (sub == 0) {
+          s_sc[warp][0][(s0 + u) * KPW + grp] = s1;
+          if (LSB) s_sc[warp][NV - 1][(s0 + u) * KPW + grp] = s2;
         }
       }
     }
-    __syncthreads();
-    m = block_max(mloc);
-    l = 0.0f;
-    for (int j = threadIdx.x; j < n; j += kThreads) l += expf(s_sc[j] - m);
-    l = block_sum(l);
   }
-  const float inv_l = 1.0f / l;
+  m1 = warp_max(m1);
+  if (LSB) m2 = warp_max(m2);
+  __syncwarp();
 
-  // ---- 4: probabilities, importance partial, output ------------------------------------------
-  float* part_row = p.tok_part + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
-  for (int j = threadIdx.x; j < n; j += kThreads) {
-    const float pr = expf(s_sc[j] - m) * inv_l;
-    s_sc[j] = pr;
-    part_row[j] = pr;
-  }
-  __syncthreads();
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
-  for (int j0 = 0; j0 < n; j0 += KPU) {
-    int64_t rows[kUnroll];
-    int js[kUnroll];
-    rows_of(j0, rows, js);
-    uint4 rm[kUnroll];
-    uint2 rl[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      rm[u] = js[u] < n ? __ldg(reinterpret_cast<const uint4*>(a.v_msb + rows[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
-      rl[u] = (flag && js[u] < n) ? __ldg(reinterpret_cast<const uint2*>(a.v_lsb + rows[u] * (DH / 2)) + sub) : make_uint2(0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (js[u] >= n) continue;
-      const float pr = s_sc[js[u]];
-      float f[16], g[16];
-      unpack16_s8(rm[u], f);
-      unpack16_u4(rl[u], g);   // zero unless the row refetches
-#pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = fmaf(pr, fmaf(16.0f, f[i], g[i]), acc[i]);
+  // ---- exponentials, once per key and variant (coalesced stores) --------------------------------
+  const int64_t vstride = static_cast<int64_t>(a.B) * a.H_kept * n;
+  float* e_out = p.dec_e + bs * n;
+  float l1 = 0.0f, l2 = 0.0f;
+  for (int k = lane; k < ITEM; k += 32) {
+    const int j = j0 + k;
+    if (j < n) {
+      const float e1 = expf(s_sc[warp][0][k] - m1);
+      s_sc[warp][0][k] = e1;
+      e_out[j] = e1;
+      l1 += e1;
+      if (LSB) {
+        const float e2 = expf(s_sc[warp][NV - 1][k] - m2);
+        s_sc[warp][NV - 1][k] = e2;
+        e_out[vstride + j] = e2;
+        l2 += e2;
+      }
     }
   }
-  // reduce over the key groups of the warp (lanes with equal `sub`), then over warps
+  l1 = warp_sum(l1);
+  if (LSB) l2 = warp_sum(l2);
+  __syncwarp();
+
+  // ---- sums of e * V codes ----------------------------------------------------------------------
+  float2 o1[8], o2[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < 8; ++i) o1[i] = o2[i] = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+  for (int s0 = 0; s0 < STEPS; s0 += BATCH) {
+    int64_t row[BATCH];
 #pragma unroll
-    for (int o2 = LPK; o2 < 32; o2 <<= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o2);
-  if (grp == 0) {
+    for (int u = 0; u < BATCH; ++u) row[u] = row_of(j0 + (s0 + u) * KPW + grp);
+    uint4 vm[BATCH];
+    uint2 vl[BATCH];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) o_red[warp][sub * 16 + i] = acc[i];
+    for (int u = 0; u < BATCH; ++u)
+      vm[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.v_msb + row[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+    if (LSB) {
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u)
+        vl[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint2*>(a.v_lsb + row[u] * (DH / 2)) + sub) : make_uint2(0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      if (row[u] < 0) continue;
+      const int k = (s0 + u) * KPW + grp;
+      float2 f[8];
+      msb16(vm[u], f);
+      const float e1 = s_sc[warp][0][k];
+      const float2 e1v = make_float2(e1, e1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o1[i] = ffma2(e1v, f[i], o1[i]);
+      if (LSB) {
+        float2 g[8];
+        lsb16(vl[u], g);
+        const float e2 = s_sc[warp][NV - 1][k];
+        const float2 e2v = make_float2(e2, e2), sixteen = make_float2(16.0f, 16.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o2[i] = ffma2(e2v, ffma2(sixteen, f[i], g[i]), o2[i]);
+      }
+    }
   }
-  __syncthreads();
-  float habs = 0.0f;
-  if (threadIdx.x < DH) {
+  // add the lane groups' sums through shared memory, in group order
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    s_o[warp][grp][sub * 16 + 2 * i] = o1[i].x;
+    s_o[warp][grp][sub * 16 + 2 * i + 1] = o1[i].y;
+    if (LSB) {
+      s_o[warp][grp][DH + sub * 16 + 2 * i] = o2[i].x;
+      s_o[warp][grp][DH + sub * 16 + 2 * i + 1] = o2[i].y;
+    }
+  }
+  __syncwarp();
+  float* o_out = p.dec_o + (bs * p.dec_items + item) * 2 * DH;
+  for (int t = lane; t < NV * DH; t += 32) {
     float v = 0.0f;
-    for (int w = 0; w < kWarps; ++w) v += o_red[w][threadIdx.x];
-    v *= vs;
-    habs = fabsf(v);
-    st_from_float(o + static_cast<int64_t>(b) * a.n_q * a.o_ld_tok + static_cast<int64_t>(h) * DH + threadIdx.x, v);
+#pragma unroll
+    for (int g = 0; g < KPW; ++g) v += s_o[warp][g][t];
+    o_out[t] = v;
   }
-  habs = block_sum(habs);
+  if (lane == 0)
+    reinterpret_cast<float4*>(p.dec_stat)[bs * p.dec_items + item] = make_float4(m1, l1, LSB ? m2 : m1, LSB ? l2 : l1);
+}
+
+// Row statistics of one kept head folded by one warp in a fixed order (lane-strided item partials,
+// then a butterfly); returns whether the row refetches, and the chosen variant's (m, 1/ell).
+template <bool LSB>
+__device__ __forceinline__ bool fold_row(const float4* st, int NI, float theta, float* m_out, float* inv_l_out) {
+  const int lane = threadIdx.x & 31;
+  float M1 = -INFINITY, M2 = -INFINITY;
+  for (int i = lane; i < NI; i += 32) {
+    const float4 v = st[i];
+    M1 = fmaxf(M1, v.x);
+    M2 = fmaxf(M2, v.z);
+  }
+  M1 = warp_max(M1);
+  if (LSB) M2 = warp_max(M2);
+  float L1 = 0.0f, L2 = 0.0f;
+  for (int i = lane; i < NI; i += 32) {
+    const float4 v = st[i];
+    L1 += v.y * expf(v.x - M1);
+    if (LSB) L2 += v.w * expf(v.z - M2);
+  }
+  L1 = warp_sum(L1);
+  if (LSB) L2 = warp_sum(L2);
+  const bool full = LSB && (1.0f / L1 < theta);
+  *m_out = full ? M2 : M1;
+  *inv_l_out = 1.0f / (full ? L2 : L1);
+  return full;
+}
+
+constexpr int kCWarps = kCThreads / 32;
+
+template <int DH, typename QT, bool LSB>
+__global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProblem p) {
+  constexpr int ITEM = DGeom<DH>::ITEM;
+  constexpr int IG = kCThreads / DH;                     // item groups of an output block
+  constexpr int TI = (kCThreads + ITEM - 1) / ITEM + 1;  // items a token block can touch
+  const spatten_attn_args& a = p.a;
+  extern __shared__ float sh[];
+  __shared__ float part[IG][DH];
+  __shared__ float red[kCWarps];
+  const int HK = a.H_kept, NI = p.dec_items, n = a.n_kv;
+  const int b = blockIdx.y;
+  const int nblk = (n + kCThreads - 1) / kCThreads;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float4* stats = reinterpret_cast<const float4*>(p.dec_stat) + static_cast<int64_t>(b) * HK * NI;
+
+  if (static_cast<int>(blockIdx.x) < nblk) {
+    // ---- token importance of keys [j0, j0 + kCThreads): p_j summed over kept heads in slot order
+    if (!a.tok_imp) return;
+    const int j0 = blockIdx.x * kCThreads;
+    const int it0 = j0 / ITEM;
+    float* factor = sh;                                   // [HK][TI] factors of items it0 ..
+    int* use_full = reinterpret_cast<int*>(sh + HK * TI); // [HK]
+    for (int slot = warp; slot < HK; slot += kCWarps) {
+      float m, inv_l;
+      const bool full = fold_row<LSB>(stats + static_cast<int64_t>(slot) * NI, NI, a.refetch_threshold, &m, &inv_l);
+      if (lane < TI && it0 + lane < NI) {
+        const float4 v = stats[static_cast<int64_t>(slot) * NI + it0 + lane];
+        factor[slot * TI + lane] = expf((full ? v.z : v.x) - m) * inv_l;
+      }
+      if (lane == 0) use_full[slot] = full ? 1 : 0;
+    }
+    __syncthreads();
+    const int j = j0 + threadIdx.x;
+    if (j >= n) return;
+    const int it = j / ITEM - it0;
+    const int64_t vstride = static_cast<int64_t>(a.B) * HK * n;
+    const float* e = p.dec_e + static_cast<int64_t>(b) * HK * n + j;
+    float t = 0.0f;
+#pragma unroll 4
+    for (int slot = 0; slot < HK; ++slot)
+      t += e[(use_full[slot] ? vstride : 0) + static_cast<int64_t>(slot) * n] * factor[slot * TI + it];
+    const int64_t col = a.tok_imp_map ? a.tok_imp_map[static_cast<int64_t>(b) * a.tok_imp_map_ld + j] : j;
+    a.tok_imp[static_cast<int64_t>(b) * a.tok_imp_ld + col] += t;
+    return;
+  }
+
+  // ---- output block of one head slot: O, sum |O| -> head importance, refetch flag
+  const int slot = static_cast<int>(blockIdx.x) - nblk;
+  const int h = head_of_slot(a, b, slot);
+  QT* o = static_cast<QT*>(a.o) + static_cast<int64_t>(b) * a.n_q * a.o_ld_tok + static_cast<int64_t>(h) * DH;
+  if (slot >= HK) {   // a pruned head: zero-filled output
+    if (h >= 0 && threadIdx.x < DH) st_from_float(o + threadIdx.x, 0.0f);
+    return;
+  }
+  float* factor = sh;   // [NI]
+  __shared__ int s_full;
+  if (warp == 0) {
+    float m, inv_l;
+    const bool full = fold_row<LSB>(stats + static_cast<int64_t>(slot) * NI, NI, a.refetch_threshold, &m, &inv_l);
+    for (int i = lane; i < NI; i += 32) {
+      const float4 v = stats[static_cast<int64_t>(slot) * NI + i];
+      factor[i] = expf((full ? v.z : v.x) - m) * inv_l;
+    }
+    if (lane == 0) s_full = full ? 1 : 0;
+  }
+  __syncthreads();
+  const bool full = s_full != 0;
+  const int dim = threadIdx.x % DH, g = threadIdx.x / DH;
+  {
+    const float* op = p.dec_o + (static_cast<int64_t>(b) * HK + slot) * NI * 2 * DH + (full ? DH : 0) + dim;
+    float v = 0.0f;
+#pragma unroll 4
+    for (int i = g; i < NI; i += IG) v += op[static_cast<int64_t>(i) * 2 * DH] * factor[i];
+    part[g][dim] = v;
+  }
+  __syncthreads();
+  float absv = 0.0f;
+  if (static_cast<int>(threadIdx.x) < DH) {
+    float v = 0.0f;
+#pragma unroll
+    for (int gg = 0; gg < IG; ++gg) v += part[gg][threadIdx.x];
+    // the MSB-pass sums hold e * MSB_j; its dequantized value is s_v * 16 * MSB_j
+    v *= a.v_scale[static_cast<int64_t>(b) * a.H + h] * (full ? 1.0f : 16.0f);
+    st_from_float(o + threadIdx.x, v);
+    absv = fabsf(v);
+  }
+  absv = warp_sum(absv);
+  if (lane == 0) red[warp] = absv;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    p.head_part[static_cast<int64_t>(b) * a.H_kept + slot] = habs;
-    if (a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld] = flag ? 1 : 0;
-    if (flag && a.refetch_count) atomicAdd(a.refetch_count, 1);
+    float hs = 0.0f;
+    for (int w = 0; w < DH / 32; ++w) hs += red[w];
+    const int64_t bhh = static_cast<int64_t>(b) * a.H + h;
+    if (a.head_imp) a.head_imp[bhh] += hs;
+    if (a.refetch_flags) a.refetch_flags[bhh * a.refetch_flags_ld] = full ? 1 : 0;
+    if (full && a.refetch_count) atomicAdd(a.refetch_count, 1);
   }
 }
 
-template <int DH, typename QT>
+// dynamic shared memory of the combine kernel: the larger of a token block's factor table and
+// flags and an output block's factor row
+size_t combine_smem(int d_h, int H_kept, int items) {
+  const int item_rows = d_h == 64 ? DGeom<64>::ITEM : DGeom<128>::ITEM;
+  const int ti = (kCThreads + item_rows - 1) / item_rows + 1;
+  const size_t tok = static_cast<size_t>(H_kept) * (ti + 1) * 4;
+  const size_t out = static_cast<size_t>(items) * 4;
+  return tok > out ? tok : out;
+}
+
+template <int DH, typename QT, bool LSB>
 int32_t launch(const AttnProblem& p, cudaStream_t st) {
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    SPT_CUDA(cudaFuncSetAttribute(attn_decode_kernel<DH, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxKv * 4));
-    configured[dev] = true;
-  }
+  const int items = p.dec_items;
+  const int64_t per_seq = static_cast<int64_t>(items) * p.a.H_kept;
+  attn_decode_items_kernel<DH, QT, LSB>
+      <<<dim3(static_cast<unsigned>(ceil_div(per_seq, kDWarps)), p.a.B), kDWarps * 32, 0, st>>>(p);
+  SPT_TRY(launch_status());
+  const int nblk = static_cast<int>(ceil_div(p.a.n_kv, kCThreads));
   const int slots = p.a.H_kept + (p.a.zero_pruned_heads ? p.a.H - p.a.H_kept : 0);
-  const size_t smem = static_cast<size_t>(p.a.n_kv) * 4;
-  attn_decode_kernel<DH, QT><<<dim3(slots, p.a.B), kThreads, smem, st>>>(p);
+  attn_decode_combine_kernel<DH, QT, LSB>
+      <<<dim3(nblk + slots, p.a.B), kCThreads, combine_smem(DH, p.a.H_kept, items), st>>>(p);
   return launch_status();
+}
+
+template <int DH, typename QT>
+int32_t launch_dh(const AttnProblem& p, cudaStream_t st) {
+  return p.a.refetch_threshold > 0.0f ? launch<DH, QT, true>(p, st) : launch<DH, QT, false>(p, st);
 }
 
 }  // namespace
 
+int decode_item_rows(int d_h) { return d_h == 64 ? DGeom<64>::ITEM : DGeom<128>::ITEM; }
+
 bool attn_decode_supported(const spatten_attn_args& a) {
-  return a.quantized && a.n_q == 1 && a.n_kv <= kMaxKv && (a.d_h == 64 || a.d_h == 128);
+  if (!a.quantized || a.n_q != 1 || (a.d_h != 64 && a.d_h != 128)) return false;
+  // the combine step keeps item factors in shared memory (48 KB without opting in)
+  const int64_t items = ceil_div(a.n_kv, decode_item_rows(a.d_h));
+  return items <= 12 * 1024 && combine_smem(a.d_h, a.H_kept, static_cast<int>(items)) <= 48 * 1024;
 }
 
 int32_t attn_decode_launch(const AttnProblem& p, cudaStream_t st) {
   const bool bf = p.a.q_dtype == SPATTEN_BF16;
-  if (p.a.d_h == 64) return bf ? launch<64, __nv_bfloat16>(p, st) : launch<64, float>(p, st);
-  return bf ? launch<128, __nv_bfloat16>(p, st) : launch<128, float>(p, st);
+  if (p.a.d_h == 64) return bf ? launch_dh<64, __nv_bfloat16>(p, st) : launch_dh<64, float>(p, st);
+  return bf ? launch_dh<128, __nv_bfloat16>(p, st) : launch_dh<128, float>(p, st);
 }
 
 }  // namespace spt

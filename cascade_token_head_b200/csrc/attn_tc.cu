@@ -128,6 +128,25 @@ __device__ __forceinline__ void warp_colsum32x2(float* v, float* w, float& sv, f
   sw = w[0];
 }
 
+// the same update over 64 raw scores of a full chunk: c2 (> 0) carries the softmax scale into the
+// log2 domain, max(c2 v) = c2 max(v), and each exponent is one fused c2 v - m
+__device__ __forceinline__ void stats64_scaled(const float* v, float c2, float& m2, float& l) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    mx[k] = v[k];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mx[k] = fmaxf(mx[k], v[k + 8 * j]);
+  }
+  const float mm = c2 * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  const float mn = fmaxf(m2, mm);
+  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int j = 0; j < 64; ++j) s[j & 3] += ex2(fmaf(v[j], c2, -mn));
+  l = l * ex2(m2 - mn) + ((s[0] + s[1]) + (s[2] + s[3]));
+  m2 = mn;
+}
+
 // running max / exp-sum update over 64 log2-domain scores (independent partial sums)
 __device__ __forceinline__ void stats64(const float* v, float& m2, float& l) {
   float mx[8];
@@ -524,9 +543,13 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
           tc_before_sync();
           mbar_arrive(&bars[M_SR + g]);
         }
+        if (t * KT + hh * 64 + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
+          stats64_scaled(v, c2, m2, l);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
-        stats64(v, m2, l);
+          for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
+          stats64(v, m2, l);
+        }
       }
       ++sc;
     }
@@ -553,8 +576,9 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   // ------------------------------------------------------------------------- softmax (pass B)
   if (warp < 8 && !aborted) {
     uint32_t sc = static_cast<uint32_t>(n_tiles), pc = 0;
-    const float inv_l = 1.0f / l;
     const bool live = row_ok && !flag;
+    // p = 2^(c2 s - m2) / ell = 2^(c2 s - mb); rows that are not stored here get p = 0
+    const float mb = live ? m2 + log2f(l) : INFINITY;
     uint8_t* Pt = smem + C::oP + g * C::PB;
     const int qt128 = pair * 2 + g;
     const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
@@ -574,10 +598,18 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
           mbar_arrive(&bars[M_SR + g]);
         }
         const int kb = t * KT + hh * 64;
+        if (kb + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = (live && kb + j < a.n_kv) ? ex2(v[j] * c2 - m2) * inv_l : 0.0f;
-          w[j] = (live && kb + 32 + j < a.n_kv) ? ex2(w[j] * c2 - m2) * inv_l : 0.0f;
+          for (int j = 0; j < 32; ++j) {
+            v[j] = ex2(fmaf(v[j], c2, -mb));
+            w[j] = ex2(fmaf(w[j], c2, -mb));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            v[j] = kb + j < a.n_kv ? ex2(fmaf(v[j], c2, -mb)) : 0.0f;
+            w[j] = kb + 32 + j < a.n_kv ? ex2(fmaf(w[j], c2, -mb)) : 0.0f;
+          }
         }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -865,9 +897,13 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
           tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64, v);
           tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64 + 32, v + 32);
           tmem_ld_wait();
+          if (t * KT + hh * 64 + 64 <= a.n_kv) {   // a full chunk
+            stats64_scaled(v, c2, m2, l);
+          } else {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
-          stats64(v, m2, l);
+            for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
+            stats64(v, m2, l);
+          }
         }
       }
       tc_before_sync();
@@ -878,7 +914,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     // ------------------------------------------------------------------------- softmax (pass B)
     if (!aborted) {
       uint32_t pc[2] = {0, 0};
-      const float inv_l = 1.0f / l;
+      const float mb = row_ok ? m2 + log2f(l) : INFINITY;   // p = 2^(c2 s - mb)
       const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * 2 * p.n_pair + u) * a.n_kv;
       for (int t = 0; t < n_tiles; ++t) {
         const int sb = t & 1;
@@ -896,10 +932,18 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
             tmem_ld32(tmem + lane_base + C::tS + sb * KT + hh * 64 + 32, w);
             tmem_ld_wait();
             const int kb = t * KT + hh * 64;
+            if (kb + 64 <= a.n_kv) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              v[j] = (row_ok && kb + j < a.n_kv) ? ex2(v[j] * c2 - m2) * inv_l : 0.0f;
-              w[j] = (row_ok && kb + 32 + j < a.n_kv) ? ex2(w[j] * c2 - m2) * inv_l : 0.0f;
+              for (int j = 0; j < 32; ++j) {
+                v[j] = ex2(fmaf(v[j], c2, -mb));
+                w[j] = ex2(fmaf(w[j], c2, -mb));
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                v[j] = kb + j < a.n_kv ? ex2(fmaf(v[j], c2, -mb)) : 0.0f;
+                w[j] = kb + 32 + j < a.n_kv ? ex2(fmaf(w[j], c2, -mb)) : 0.0f;
+              }
             }
           } else {
 #pragma unroll

@@ -43,14 +43,26 @@ struct QArgs {
 
 namespace {
 
-// quantize 8 values with scale s; returns the number of saturated codes
-__device__ __forceinline__ int quant8(const float* v, float s, int8_t* msb_dst, uint8_t* lsb_dst) {
+// rint(float32(v / s)) without a division per element: t = v * (1/s) (reciprocal correctly
+// rounded) lies within 1.5 ulp(t) of the float32 quotient, i.e. within 2^-10 for |t| < 4096, so
+// unless t is within 2^-9 of a half-integer both round to the same integer; those rare near-ties
+// are recomputed with the IEEE division.  |t| >= 4096 saturates either way.
+__device__ __forceinline__ float code_of(float v, float s, float rcp) {
+  const float t = v * rcp;
+  const float r = rintf(t);
+  if (fabsf(t - r) > 0.5f - 0.001953125f && fabsf(t) < 4096.0f) return rintf(__fdiv_rn(v, s));
+  return r;
+}
+
+// quantize 8 values with scale s (rcp = 1/s, correctly rounded); returns the number of saturated
+// codes
+__device__ __forceinline__ int quant8(const float* v, float s, float rcp, int8_t* msb_dst, uint8_t* lsb_dst) {
   int sat = 0;
   uint32_t m[2] = {0u, 0u};
   uint32_t l = 0u;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float r = rintf(__fdiv_rn(v[i], s));
+    const float r = code_of(v[i], s, rcp);
     sat += fabsf(r) > kQMax ? 1 : 0;
     int q = static_cast<int>(fminf(fmaxf(r, -kQMax), kQMax));
     int hi = q >> 4;          // arithmetic shift: floor(q / 16)
@@ -126,6 +138,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   cluster.sync();   // no CTA leaves while a peer may still read its shared memory
 
   const float s = block_amax == 0.0f ? 1.0f : __fdiv_rn(block_amax, kQMax);
+  const float rcp = __frcp_rn(s);
   if (rank == 0 && threadIdx.x == 0) q.scale_out[bh] = s;
 
   // pass 2: codes (the rows are read again; they are in L2)
@@ -144,7 +157,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
         const int t = r0 + e / C, c = e % C;
         apply_gain(a, q, b, t, v[u]);
         const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
-        quant8(v[u], s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+        quant8(v[u], s, rcp, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
       }
     }
   }
@@ -168,7 +181,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
     apply_gain(a, q, b, t, v);
     const float s = q.scale_in[bh];
     const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
-    sat += quant8(v, s, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+    sat += quant8(v, s, __frcp_rn(s), q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
   }
   sat = warp_sum_int(sat);
   if (a.sat && (threadIdx.x & 31) == 0 && sat) atomicAdd(a.sat, sat);

@@ -191,17 +191,22 @@ def test_attention_fp32_unquantized(cuda, n):
 
 
 @pytest.mark.parametrize("kernel", [0, 1])
-@pytest.mark.parametrize("d,theta", [(64, 0.2), (64, 0.0), (128, 0.2)])
-def test_attention_decode_index_listed(cuda, kernel, d, theta):
-    """One query row per (sequence, head) against an index-listed subset of a cache."""
+@pytest.mark.parametrize("d,theta,cap,n_kv,keep", [
+    (64, 0.2, 300, 211, None), (64, 0.0, 300, 211, None), (128, 0.2, 300, 211, None),
+    (64, 0.2, 40, 7, None), (64, 0.2, 2600, 2048, None), (128, 0.05, 2600, 2047, [1, 3]),
+    (64, 0.2, 3000, 2500, None), (128, 0.2, 1300, 1153, [0, 2, 3])])
+def test_attention_decode_index_listed(cuda, kernel, d, theta, cap, n_kv, keep):
+    """One query row per (sequence, head) against an index-listed subset of a cache.  Lists of up
+    to 2048 rows go to the cluster kernel (1..8 CTAs per row), longer ones to the streaming one."""
     S = lib()
-    B, H, cap = 3, 4, 300
-    g = synth.rng_for(d + int(theta * 10))
+    B, H = 3, 4
+    g = synth.rng_for(d + int(theta * 10) + n_kv)
     raw, gain = make_layer(B, H, cap, d, seed=99 + d)
-    kv_idx = np.stack([np.sort(g.choice(cap, 211, replace=False)) for _ in range(B)]).astype(np.int32)
-    got = run_layer(S, raw, gain, B, H, cap, d, theta, kernel=kernel, kv_idx=kv_idx, n_q=1)
-    ref = oracle_layer(raw, gain, B, H, cap, d, theta, None, BF, got, kv_idx=kv_idx, n_q=1)
-    check(got, ref, None, H, d, 2e-2, 1e-2, "decode")
+    kv_idx = np.stack([np.sort(g.choice(cap, n_kv, replace=False)) for _ in range(B)]).astype(np.int32)
+    heads = None if keep is None else np.array([keep] * B, np.int32)
+    got = run_layer(S, raw, gain, B, H, cap, d, theta, heads=heads, kernel=kernel, kv_idx=kv_idx, n_q=1)
+    ref = oracle_layer(raw, gain, B, H, cap, d, theta, heads, BF, got, kv_idx=kv_idx, n_q=1)
+    check(got, ref, heads, H, d, 2e-2, 1e-2, "decode")
     # importance lands only on the listed rows
     for b in range(B):
         mask = np.ones(cap, bool)

@@ -41,6 +41,74 @@ def test_quantize_bit_exact(cuda, dtype, B, H, n, d, gain):
     np.testing.assert_array_equal(lsb.cpu().numpy(), l_ref)
 
 
+def _half_boundary_values(s, count, rng):
+    """float32 values at and a few ulps around (k + 1/2) s for integer k across the code range,
+    plus the float32 neighbours of the exact quotient boundaries."""
+    k = rng.integers(-2047, 2047, size=count)
+    centre = ((k + 0.5) * np.float64(s)).astype(np.float32)
+    steps = rng.integers(-3, 4, size=count)
+    out = centre.copy()
+    for i, st in enumerate(steps):
+        v = centre[i]
+        for _ in range(abs(int(st))):
+            v = np.nextafter(v, np.float32(np.inf) if st > 0 else np.float32(-np.inf))
+        out[i] = v
+    return out
+
+
+@pytest.mark.parametrize("s", [0.0013672, 0.1, 1.0 / 3.0, 7.123e-5])
+def test_quantize_half_integer_boundaries_fixed_scale(cuda, s):
+    """Codes of values crafted at rounding boundaries of x/s (the fast reciprocal path must defer
+    to the IEEE quotient there): bit-exact against the oracle's float32 division."""
+    S = lib()
+    rng = synth.rng_for(int(s * 1e7) % 10007)
+    B, H, n, d, cap = 2, 2, 64, 64, 64
+    s32 = np.float32(s)
+    vals = _half_boundary_values(s32, B * n * H * d, rng).reshape(B, n, H * d)
+    x = to_dev(vals, torch.float32)
+    msb = torch.zeros((B, H, cap, d), dtype=torch.int8, device="cuda")
+    lsb = torch.zeros((B, H, cap, d // 2), dtype=torch.uint8, device="cuda")
+    sat = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scales = to_dev(np.full(B * H, s32, np.float32))
+    S.quantize_kv(x, B, H, n, d, H * d, msb, lsb, cap, 0, scale_in=scales, sat_count=sat, dtype=S.F32)
+    torch.cuda.synchronize()
+    x32 = vals.reshape(B, n, H, d).transpose(0, 2, 1, 3)
+    want_sat = 0
+    for b in range(B):
+        for h in range(H):
+            r = R.quantize_head(np.ascontiguousarray(x32[b, h]), scale=s32)
+            want_sat += r["sat"]
+            np.testing.assert_array_equal(msb[b, h].cpu().numpy(), r["msb"])
+            np.testing.assert_array_equal(lsb[b, h].cpu().numpy(), R.pack_lsb(r["lsb"]))
+    assert int(sat.item()) == want_sat
+
+
+def test_quantize_half_integer_boundaries_amax_scale(cuda):
+    """The same with the scale derived from the block's amax on the device."""
+    S = lib()
+    rng = synth.rng_for(4242)
+    B, H, n, d = 2, 3, 256, 64
+    vals = np.empty((B, n, H * d), np.float32)
+    for b in range(B):
+        for h in range(H):
+            amax = np.float32(rng.uniform(0.5, 9.0))
+            s = np.float32(amax / np.float32(2047.0))
+            blk = _half_boundary_values(s, n * d, rng).reshape(n, d)
+            blk = np.clip(blk, -amax, amax)
+            blk[0, 0] = amax
+            vals[b, :, h * d:(h + 1) * d] = blk
+    x = to_dev(vals, torch.float32)
+    msb = torch.zeros((B, H, n, d), dtype=torch.int8, device="cuda")
+    lsb = torch.zeros((B, H, n, d // 2), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(B * H, dtype=torch.float32, device="cuda")
+    S.quantize_kv(x, B, H, n, d, H * d, msb, lsb, n, 0, scale_out=sc, dtype=S.F32)
+    torch.cuda.synchronize()
+    m_ref, l_ref, s_ref = oracle_quantize_blocks(np.ascontiguousarray(vals.reshape(B, n, H, d).transpose(0, 2, 1, 3)))
+    np.testing.assert_array_equal(sc.cpu().numpy().reshape(B, H), s_ref)
+    np.testing.assert_array_equal(msb.cpu().numpy(), m_ref)
+    np.testing.assert_array_equal(lsb.cpu().numpy(), l_ref)
+
+
 def test_quantize_full_size_bert_layer0(cuda):
     """K of the BERT-base layer-0 projection shape [32, 12, 512, 64], bf16, with boosted rows."""
     S = lib()
