@@ -23,12 +23,19 @@ from . import synth
 
 
 def _time(fn, reps: int) -> float:
+    """Mean device time of one call: `reps` calls captured in a CUDA graph and replayed (host launch
+    overhead excluded; for small kernels it would otherwise be what is timed)."""
     fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for _ in range(reps):
-        fn()
+    g.replay()
     b.record()
     torch.cuda.synchronize()
     return a.elapsed_time(b) / reps
@@ -68,7 +75,7 @@ def attention_case(B, H, n, d, theta, boost, kernel, reps, n_kv=None):
     ms = _time(lambda: S.attention_layer(a, ws, ws.numel()), reps)
     flops = 4.0 * B * H * n * n * d
     return dict(case="attention", B=B, H=H, n=n, d=d, theta=theta, ms=ms, flops=flops,
-                tflops=flops / ms / 1e9, refetch_rows=int(cnt.item()) // (reps + 1))
+                tflops=flops / ms / 1e9, refetch_rows=int(cnt.item()) // (2 * reps + 1))
 
 
 def topk_case(R, n, k, dist, reps):
@@ -132,7 +139,7 @@ def decode_case(B, H, n, d, keep, theta, reps):
     a.refetch_threshold = theta
     ws = torch.empty(S.attention_workspace_size(a), dtype=torch.uint8, device="cuda")
     ms = _time(lambda: S.attention_layer(a, ws, ws.numel()), reps)
-    refetched = int(cnt.item()) / (reps + 1)
+    refetched = int(cnt.item()) / (2 * reps + 1)
     byts = B * H * keep * d * 2.0 + refetched * keep * d + B * keep * 4.0
     return dict(case="decode", B=B, H=H, n=n, keep=keep, d=d, ms=ms, bytes=byts, gbs=byts / ms / 1e6,
                 refetch_frac=refetched / (B * H))

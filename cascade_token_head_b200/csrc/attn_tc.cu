@@ -5,9 +5,13 @@
 // Quantization" (MSB pass; rows whose max probability is below the threshold are recomputed with
 // the LSBs).
 //
-// Exact operands: K and V are 12-bit codes q = 16*MSB + LSB; 16*MSB (8 significant bits) and LSB
-// (0..15) are exact in bf16, so the MMAs see the codes unrounded and the scales multiply the
-// float32 accumulators:  S = s_k*sm*(Q.(16 MSB)^T [+ Q.LSB^T]),  O = s_v*(P.16 MSB_v [+ P.LSB_v]).
+// Exact operands: K and V are 12-bit codes q = 16*MSB + LSB; 16*MSB (in [-2048, 2032]) and LSB
+// (0..15) are exact in fp16, so the MMAs (kind::f16 with fp16 A and B, f32 accumulate) see the
+// codes unrounded and the scales multiply the float32 accumulators:
+//   S = s_k*sm*(Q.(16 MSB)^T [+ Q.LSB^T]),  O = s_v*(P.16 MSB_v [+ P.LSB_v]).
+// The bf16 query tile is converted to fp16 on its way to shared memory (exact for magnitudes in
+// [2^-14, 65504]; smaller ones keep fp16 subnormal precision, larger ones saturate) and P is
+// stored as fp16 (11 significant bits).
 //
 // Two kernels per layer:
 //  MAIN  one CTA = (sequence, kept head, 256 query rows), 384 threads:
@@ -19,7 +23,7 @@
 //        core while the other warpgroup runs its softmax) -> row max / exp-sum -> refetch flags;
 //        the flagged rows of the CTA are written, ascending, to a packed list.  Pass B computes
 //        P = exp(S - m)/ell for the other rows (float32), column sums by a 31-shuffle butterfly
-//        (deterministic), P in bf16 to shared memory, O += P V.  Flagged rows contribute nothing
+//        (deterministic), P in fp16 to shared memory, O += P V.  Flagged rows contribute nothing
 //        here.
 //  FULL  one CTA = 128 consecutive entries of the head's flagged rows (the MAIN lists of its pair
 //        tiles concatenated in order; launched only when theta > 0; CTAs past the end exit at
@@ -28,12 +32,16 @@
 //        columns, reading the LSB planes only for heads with flagged rows.
 // Producers: without an index list the raw code rows of a key tile are contiguous, so one thread
 // keeps several tiles in flight with 1-D bulk copies (TMA engine) into a staging ring, and the
-// producer warps convert staged int8 / packed-nibble tiles to swizzled bf16 shared -> shared.
+// producer warps convert staged int8 / packed-nibble tiles to swizzled fp16 shared -> shared (a
+// byte placed under the fp16 exponent byte 0x64 reads as 1024 + byte; one fp16 FMA or add per pair
+// of codes removes the offset, no int-to-float conversions).
 // Partial column sums (per 128-row tile) and sum |O| go to the workspace; attn_reduce adds them in
 // a fixed order, so reruns are bit-identical.
 // Operand layouts: UMMA 128-byte swizzle; Q, K, P K-major; V MN-major (plain key rows).  Key tiles
-// hold 16 KB of bf16 codes: 128 keys at d_h = 64, 64 keys at d_h = 128.  Every mbarrier wait is
+// hold 16 KB of fp16 codes: 128 keys at d_h = 64, 64 keys at d_h = 128.  Every mbarrier wait is
 // bounded: on timeout the CTA reports SPATTEN_E_TIMEOUT, frees its TMEM and returns.
+#include <cuda_fp16.h>
+
 #include "attention.cuh"
 #include "tc_ptx.cuh"
 
@@ -53,26 +61,47 @@ __device__ __forceinline__ uint32_t tile_off(uint32_t row, uint32_t c8, uint32_t
   return (c8 >> 3) * rows * 128u + sw128_offset(row, c8 & 7u);
 }
 
+// Code tiles enter the tensor cores as fp16, in which every code value is exact (16 MSB lies in
+// [-2048, 2032], LSB in [0, 15]).  Conversion without int-to-float instructions: a code byte u
+// placed under the high byte 0x64 is the fp16 number 1024 + u.
+// sixteen signed MSB codes -> eight fp16 pairs of 16 * MSB: the biased byte u = MSB + 128 gives
+// 1024 + u, and 16 (1024 + u) - 18432 = 16 MSB is exact in one fp16 FMA
 __device__ __forceinline__ void cvt16_s8x16(uint4 raw, uint32_t* out8) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
+  const __half2 mul = __halves2half2(__float2half_rn(16.0f), __float2half_rn(16.0f));
+  const __half2 add = __halves2half2(__float2half_rn(-18432.0f), __float2half_rn(-18432.0f));
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float f0 = 16.0f * static_cast<float>(static_cast<int8_t>(w[i] & 0xFFu));
-    const float f1 = 16.0f * static_cast<float>(static_cast<int8_t>((w[i] >> 8) & 0xFFu));
-    const float f2 = 16.0f * static_cast<float>(static_cast<int8_t>((w[i] >> 16) & 0xFFu));
-    const float f3 = 16.0f * static_cast<float>(static_cast<int8_t>(w[i] >> 24));
-    out8[2 * i] = pack_bf16x2(f0, f1);
-    out8[2 * i + 1] = pack_bf16x2(f2, f3);
+    uint32_t p0 = __byte_perm(w[i], 0x64646464u, 0x5140u), p1 = __byte_perm(w[i], 0x64646464u, 0x5342u);
+    __half2 h0 = __hfma2(*reinterpret_cast<__half2*>(&p0), mul, add);
+    __half2 h1 = __hfma2(*reinterpret_cast<__half2*>(&p1), mul, add);
+    out8[2 * i] = *reinterpret_cast<uint32_t*>(&h0);
+    out8[2 * i + 1] = *reinterpret_cast<uint32_t*>(&h1);
   }
 }
+// sixteen packed LSB codes (element 2k in bits 8k..8k+3, 2k+1 in bits 8k+4..8k+7 of a word) ->
+// eight fp16 pairs
 __device__ __forceinline__ void cvt_u4x16(uint2 raw, uint32_t* out8) {
   const uint32_t w[2] = {raw.x, raw.y};
+  const __half2 off = __halves2half2(__float2half_rn(-1024.0f), __float2half_rn(-1024.0f));
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      out8[4 * i + k] = pack_bf16x2(static_cast<float>((w[i] >> (8 * k)) & 0xFu),
-                                    static_cast<float>((w[i] >> (8 * k + 4)) & 0xFu));
+    for (int k = 0; k < 4; ++k) {
+      uint32_t p = (__byte_perm(lo, hi, static_cast<uint32_t>(k | ((4 + k) << 8))) & 0x00FF00FFu) | 0x64006400u;
+      __half2 h = __hadd2(*reinterpret_cast<__half2*>(&p), off);
+      out8[4 * i + k] = *reinterpret_cast<uint32_t*>(&h);
+    }
+  }
+}
+// eight bf16 values -> four fp16 pairs (the query tile); exact for magnitudes in [2^-14, 65504]
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = pack_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -292,22 +321,22 @@ struct JobStream {
 // QK^T into `d` (accumulate onto it when acc != 0), A = Q tile [128 x DH], B = key tile [KT x DH]
 template <int DH, int KT>
 __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t sQ, uint32_t sK, uint32_t acc) {
-  constexpr uint32_t id = idesc_bf16(128, KT, false, false);
+  constexpr uint32_t id = idesc_f16(128, KT, false, false);
 #pragma unroll
   for (int s = 0; s < DH / 16; ++s) {
     const uint32_t qoff = (s >> 2) * 16384u + (s & 3) * 32u;
     const uint32_t koff = (s >> 2) * (KT * 128u) + (s & 3) * 32u;
-    mma_bf16(d, desc_sw128(sQ + qoff, 16, 1024), desc_sw128(sK + koff, 16, 1024), id, (acc || s > 0) ? 1u : 0u);
+    mma_f16(d, desc_sw128(sQ + qoff, 16, 1024), desc_sw128(sK + koff, 16, 1024), id, (acc || s > 0) ? 1u : 0u);
   }
 }
 // P V into `d`: A = P tile [128 x KT] K-major, B = V tile [KT keys x DH] MN-major
 template <int DH, int KT>
 __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t sP, uint32_t sV, uint32_t acc) {
-  constexpr uint32_t id = idesc_bf16(128, DH, false, true);
+  constexpr uint32_t id = idesc_f16(128, DH, false, true);
 #pragma unroll
   for (int s = 0; s < KT / 16; ++s) {
     const uint32_t poff = (s >> 2) * 16384u + (s & 3) * 32u;
-    mma_bf16(d, desc_sw128(sP + poff, 16, 1024), desc_sw128(sV + s * 2048u, KT * 128u, 1024), id,
+    mma_f16(d, desc_sw128(sP + poff, 16, 1024), desc_sw128(sV + s * 2048u, KT * 128u, 1024), id,
              (acc || s > 0) ? 1u : 0u);
   }
 }
@@ -331,7 +360,7 @@ __device__ __forceinline__ void store_o_row(__nv_bfloat16* dst, const float* v, 
 template <int DH>
 struct MainCfg {
   static constexpr int KT = DH == 64 ? 128 : 64;
-  static constexpr int NST = 2;                  // bf16 K and V ring stages
+  static constexpr int NST = 2;                  // fp16 K and V ring stages
   static constexpr int RS = 4;                   // raw code tiles in flight (bulk copies)
   static constexpr uint32_t QB = 128u * DH * 2u;
   static constexpr uint32_t TB = static_cast<uint32_t>(KT) * DH * 2u;
@@ -450,7 +479,8 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     for (int k = 0; k < PER; ++k) {
       const int e = tid + k * 352;
       const int rr = e / (DH / 8), c8 = e % (DH / 8);
-      if (e < NCH) *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) = qv[k];
+      if (e < NCH)
+        *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) = bf16x8_to_f16x8(qv[k]);
     }
     fence_async_smem();
     mbar_arrive(&bars[M_Q]);
@@ -614,11 +644,11 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + q4, 128)) =
-              make_uint4(pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
-                         pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+              make_uint4(pack_f16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                         pack_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
           *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + 4 + q4, 128)) =
-              make_uint4(pack_bf16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_bf16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
-                         pack_bf16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_bf16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
+              make_uint4(pack_f16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_f16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
+                         pack_f16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_f16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
         }
         float sv, sw;
         warp_colsum32x2(v, w, sv, sw);
@@ -808,7 +838,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     for (int k = 0; k < PER; ++k) {
       const int e = tid + k * 224;
       const int rr = e / (DH / 8), c8 = e % (DH / 8);
-      if (e < NCH) *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = qv[k];
+      if (e < NCH) *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = bf16x8_to_f16x8(qv[k]);
     }
     fence_async_smem();
     mbar_arrive(&bars[F_Q]);
@@ -952,11 +982,11 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + q4, 128)) =
-                make_uint4(pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
-                           pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+                make_uint4(pack_f16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                           pack_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
             *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + 4 + q4, 128)) =
-                make_uint4(pack_bf16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_bf16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
-                           pack_bf16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_bf16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
+                make_uint4(pack_f16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_f16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
+                           pack_f16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_f16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
           }
           float sv = 0.0f, sw = 0.0f;
           if (warp_live) warp_colsum32x2(v, w, sv, sw);

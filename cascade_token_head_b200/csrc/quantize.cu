@@ -46,12 +46,16 @@ namespace {
 // rint(float32(v / s)) without a division per element: t = v * (1/s) (reciprocal correctly
 // rounded) lies within 1.5 ulp(t) of the float32 quotient, i.e. within 2^-10 for |t| < 4096, so
 // unless t is within 2^-9 of a half-integer both round to the same integer; those rare near-ties
-// are recomputed with the IEEE division.  |t| >= 4096 saturates either way.
-__device__ __forceinline__ float code_of(float v, float s, float rcp) {
+// are recomputed with the IEEE division.  The rounding itself is an add of 1.5 * 2^23, which
+// leaves rint(t) (ties to even) in the low mantissa bits; |t| >= 4096 saturates either way and
+// returns +-4096.
+__device__ __forceinline__ int code_of(float v, float s, float rcp) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
   const float t = v * rcp;
-  const float r = rintf(t);
-  if (fabsf(t - r) > 0.5f - 0.001953125f && fabsf(t) < 4096.0f) return rintf(__fdiv_rn(v, s));
-  return r;
+  if (!(fabsf(t) < 4096.0f)) return t > 0.0f ? 4096 : -4096;
+  float tm = t + kMagic;
+  if (fabsf(t - (tm - kMagic)) > 0.5f - 0.001953125f) tm = __fdiv_rn(v, s) + kMagic;
+  return __float_as_int(tm) - 0x4B400000;
 }
 
 // quantize 8 values with scale s (rcp = 1/s, correctly rounded); returns the number of saturated
@@ -62,11 +66,11 @@ __device__ __forceinline__ int quant8(const float* v, float s, float rcp, int8_t
   uint32_t l = 0u;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float r = code_of(v[i], s, rcp);
-    sat += fabsf(r) > kQMax ? 1 : 0;
-    int q = static_cast<int>(fminf(fmaxf(r, -kQMax), kQMax));
-    int hi = q >> 4;          // arithmetic shift: floor(q / 16)
-    int lo = q & 15;
+    int q = code_of(v[i], s, rcp);
+    sat += (q > 2047 || q < -2047) ? 1 : 0;
+    q = min(max(q, -2047), 2047);
+    const int hi = q >> 4;    // arithmetic shift: floor(q / 16)
+    const int lo = q & 15;
     m[i >> 2] |= (static_cast<uint32_t>(hi) & 0xFFu) << (8 * (i & 3));
     l |= static_cast<uint32_t>(lo) << (4 * i);
   }
@@ -203,8 +207,9 @@ int32_t quantize_launch(const QArgs& a, int ntensors, int dtype, cudaStream_t st
     return launch_status();
   }
   const int blocks = a.B * a.H;
-  // enough CTAs to fill the GPU twice; at most 8 per block (portable cluster size)
-  int S = static_cast<int>(ceil_div(2LL * sm_count(), static_cast<int64_t>(blocks) * ntensors));
+  // enough CTAs for eight per SM (every SM then keeps 2048 threads' loads in flight); at most 8
+  // per block (portable cluster size)
+  int S = static_cast<int>(ceil_div(8LL * sm_count(), static_cast<int64_t>(blocks) * ntensors));
   S = std::max(1, std::min(S, 8));
   S = std::min<int>(S, std::max(1, a.n / 16));
   cudaLaunchConfig_t cfg = {};

@@ -46,6 +46,7 @@ struct TShared {
   uint32_t red[256];
   uint32_t warp_a[kTWarps];
   uint32_t warp_b[kTWarps];
+  uint32_t scan[2][kTWarps];
   uint32_t digit, above;
   uint32_t n_gt, n_eq;   // this CTA's counts after the last pass (read by peers)
   int nan_seen;
@@ -81,7 +82,9 @@ __device__ __forceinline__ void load8_keys(const TArgs& a, int r, int j, int lim
   }
 }
 
-// exclusive prefix sum of one value per thread over the block (all threads must call)
+// exclusive prefix sum of one value per thread over the block (all threads must call); wt is a
+// [kTWarps] scratch array that must not be reused before every thread has passed the next block
+// barrier (callers alternate two arrays)
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wt, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t inc = v;
@@ -92,15 +95,18 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wt, ui
   }
   if (lane == 31) wt[warp] = inc;
   __syncthreads();
-  uint32_t pre = 0u, tot = 0u;
-  for (int w = 0; w < kTWarps; ++w) {
-    const uint32_t x = wt[w];
-    if (w < warp) pre += x;
-    tot += x;
+  if (warp == 0) {
+    uint32_t x = lane < kTWarps ? wt[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < kTWarps; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += t;
+    }
+    if (lane < kTWarps) wt[lane] = x;   // inclusive warp prefixes
   }
   __syncthreads();
-  total = tot;
-  return pre + inc - v;
+  total = wt[kTWarps - 1];
+  return (warp > 0 ? wt[warp - 1] : 0u) + inc - v;
 }
 
 __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
@@ -165,13 +171,27 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
         else if (pass == 3 && hi > prefix)
           ++above_pass;
       }
-      // warp-aggregated update: one shared atomic per distinct digit in the warp
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+      // warp-aggregated update: one shared atomic per distinct digit in the warp; after the first
+      // pass most warps hold no key that still matches the prefix and skip it
+      if (pass == 0 || __any_sync(0xffffffffu, bin < 256u)) {
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+      }
     };
-    for (int base = 0; base < resident; base += kTThreads) {
-      const int j = base + tid;
-      count_key(j < resident ? keys_s[j] : 0u, j < resident);
+    for (int base = 0; base < resident; base += 4 * kTThreads) {   // four keys per thread (16-byte reads)
+      const int j = base + 4 * tid;
+      uint4 k4 = make_uint4(0u, 0u, 0u, 0u);
+      if (j + 3 < resident) {
+        k4 = *reinterpret_cast<const uint4*>(keys_s + j);
+      } else {
+        if (j < resident) k4.x = keys_s[j];
+        if (j + 1 < resident) k4.y = keys_s[j + 1];
+        if (j + 2 < resident) k4.z = keys_s[j + 2];
+      }
+      count_key(k4.x, j < resident);
+      count_key(k4.y, j + 1 < resident);
+      count_key(k4.z, j + 2 < resident);
+      count_key(k4.w, j + 3 < resident);
     }
     for (int base = resident; base < len; base += 8 * kTThreads) {   // streamed part (long rows)
       uint32_t key[8];
@@ -252,76 +272,69 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   if (tid == 0 && sh.nan_seen) report(a.status, SPATTEN_E_NONFINITE);
   cluster.sync();  // peers' shared memory is no longer read after this point
 
-  // compaction in index order: resident keys one per thread (ballot scans) ...
+  // compaction in index order, eight consecutive keys per thread per tile: one block scan of the
+  // packed per-thread counts (above T in the low half, equal to T in the high half) places every
+  // thread's keys; equal keys are taken in index order while the row still needs them
   uint32_t run_sel = sel_before, run_eq = eq_before;
-  for (int base = 0; base < resident; base += kTThreads) {
-    const int j = base + tid;
-    const uint32_t key = j < resident ? keys_s[j] : 0u;
-    const bool gt = j < resident && key > T;
-    const bool eq = j < resident && key == T;
-    const unsigned beq = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) sh.warp_a[warp] = __popc(beq);
-    __syncthreads();
-    uint32_t eq_rank = run_eq + __popc(beq & ((1u << lane) - 1u));
-    uint32_t eq_tile = 0u;
-    for (int w = 0; w < kTWarps; ++w) {
-      const uint32_t v = sh.warp_a[w];
-      if (w < warp) eq_rank += v;
-      eq_tile += v;
+  int tile = 0;
+  auto compact8 = [&](int j, const uint32_t* key, const bool* ok) {
+    uint32_t gtc = 0u, eqc = 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      gtc += (ok[u] && key[u] > T) ? 1u : 0u;
+      eqc += (ok[u] && key[u] == T) ? 1u : 0u;
     }
-    const bool sel = gt || (eq && eq_rank < need_eq);
-    const unsigned bsel = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) sh.warp_b[warp] = __popc(bsel);
-    __syncthreads();
-    uint32_t pos = run_sel + __popc(bsel & ((1u << lane) - 1u));
-    uint32_t sel_tile = 0u;
-    for (int w = 0; w < kTWarps; ++w) {
-      const uint32_t v = sh.warp_b[w];
-      if (w < warp) pos += v;
-      sel_tile += v;
+    uint32_t tot;
+    const uint32_t pre = block_excl_scan(gtc | (eqc << 16), sh.scan[tile & 1], tot);
+    ++tile;
+    const uint32_t rem = need_eq > run_eq ? need_eq - run_eq : 0u;   // equal keys still wanted
+    const uint32_t pre_eq = pre >> 16;
+    uint32_t pos = run_sel + (pre & 0xFFFFu) + min(pre_eq, rem);
+    uint32_t er = run_eq + pre_eq;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const bool gt = ok[u] && key[u] > T;
+      const bool eq = ok[u] && key[u] == T;
+      const bool sel = gt || (eq && er < need_eq);
+      er += eq ? 1u : 0u;
+      if (sel) {
+        if (pos < static_cast<uint32_t>(a.k)) {
+          if (a.idx_out) a.idx_out[out_base + pos] = c0 + j + u;
+          if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + c0 + j + u];
+        }
+        ++pos;
+      }
     }
-    if (sel && pos < static_cast<uint32_t>(a.k)) {
-      if (a.idx_out) a.idx_out[out_base + pos] = c0 + j;
-      if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + c0 + j];
+    run_sel += (tot & 0xFFFFu) + min(tot >> 16, rem);
+    run_eq += tot >> 16;
+  };
+  for (int base = 0; base < resident; base += 8 * kTThreads) {
+    const int j = base + 8 * tid;
+    uint32_t key[8];
+    bool ok[8];
+    if (j + 7 < resident) {
+      const uint4 k0 = *reinterpret_cast<const uint4*>(keys_s + j);
+      const uint4 k1 = *reinterpret_cast<const uint4*>(keys_s + j + 4);
+      key[0] = k0.x; key[1] = k0.y; key[2] = k0.z; key[3] = k0.w;
+      key[4] = k1.x; key[5] = k1.y; key[6] = k1.z; key[7] = k1.w;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ok[u] = true;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        ok[u] = j + u < resident;
+        key[u] = ok[u] ? keys_s[j + u] : 0u;
+      }
     }
-    run_sel += sel_tile;
-    run_eq += eq_tile;
-    __syncthreads();
+    compact8(j, key, ok);
   }
-  // ... then streamed keys eight per thread (block scans of per-thread counts)
-  for (int base = resident; base < len; base += 8 * kTThreads) {
+  for (int base = resident; base < len; base += 8 * kTThreads) {   // streamed keys
     const int j = base + 8 * tid;
     uint32_t key[8];
     bool ok[8];
     int dummy = 0;
     load8_keys(a, r, c0 + j, c0 + len, vec, key, ok, &dummy);
-    uint32_t eqc = 0u;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) eqc += (ok[u] && key[u] == T) ? 1u : 0u;
-    uint32_t eq_tile;
-    uint32_t er = run_eq + block_excl_scan(eqc, sh.warp_a, eq_tile);
-    bool sel[8];
-    uint32_t selc = 0u;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const bool gt = ok[u] && key[u] > T;
-      const bool eq = ok[u] && key[u] == T;
-      sel[u] = gt || (eq && er < need_eq);
-      if (eq) ++er;
-      selc += sel[u] ? 1u : 0u;
-    }
-    uint32_t sel_tile;
-    uint32_t pos = run_sel + block_excl_scan(selc, sh.warp_b, sel_tile);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (sel[u] && pos < static_cast<uint32_t>(a.k)) {
-        if (a.idx_out) a.idx_out[out_base + pos] = c0 + j + u;
-        if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + c0 + j + u];
-      }
-      pos += sel[u] ? 1u : 0u;
-    }
-    run_sel += sel_tile;
-    run_eq += eq_tile;
+    compact8(j, key, ok);
   }
 }
 
