@@ -445,7 +445,8 @@ def prefill_arm(ctx, args, name):
                    "launch": "CUDA graph of one step" if graph is not None else "direct launches"},
         "roofline": {"kernel": "attention (spatten_attention_layer kernels, all layers)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None,
+                     "peak_kind": f"{peak_kind} bf16 sustained (the MMAs take fp16 operands: same nominal "
+                                  f"dense rate, ratio 1)", "traffic": None,
                      "algorithmic_flops_per_step": flops, "attn_ms_per_step": attn_s * 1e3},
         "e2e": {"value": ctx.world * tokens_per_step * n_e2e / (e2e_total / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

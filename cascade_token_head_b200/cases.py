@@ -3,6 +3,7 @@
     python -m cascade_token_head_b200.cases attention --B 32 --H 12 --n 512 --d 64 --theta 0.1 --reps 3
     python -m cascade_token_head_b200.cases topk --R 64 --n 1048576 --k 524288 --reps 3
     python -m cascade_token_head_b200.cases decode --B 16 --H 16 --n 1152 --keep 576 --reps 3
+    python -m cascade_token_head_b200.cases decode_step --reps 4
     python -m cascade_token_head_b200.cases quantize --B 32 --H 12 --n 512 --d 64 --reps 3
     python -m cascade_token_head_b200.cases gather --B 32 --n 512 --k 461 --row-bytes 1536 --reps 3
 
@@ -145,9 +146,32 @@ def decode_case(B, H, n, d, keep, theta, reps):
                 refetch_frac=refetched / (B * H))
 
 
+def decode_step_case(reps, steps_done=0):
+    """Generated tokens of the GPT-2-medium decode workload (B=16 after a 1024-token prompt, 24
+    layers): one spatten_cascade_forward per token, after `steps_done` earlier tokens."""
+    from .decode import DecodeState
+    w = synth.gpt2m_decode()
+    d = synth.draw_decode(w, steps=steps_done + 2 * reps + 2)
+    st = DecodeState(w, d["w_qkv"], d["w_o"], d["k_prompt"], d["v_prompt"])
+    xs = torch.from_numpy(d["x_steps"]).to(torch.bfloat16).cuda()
+    for s in range(steps_done):
+        st.step(x=xs[s])
+    torch.cuda.synchronize()
+    n0 = st.n_old
+    # the same `reps` tokens, captured once and replayed: each replay rewinds to n0 first
+    def tokens():
+        st.reset(n0)
+        for s in range(reps):
+            st.step(x=xs[steps_done + s])
+    ms = _time(tokens, 1) / reps
+    assert int(st.status.item()) == 0
+    return dict(case="decode_step", B=w.B, layers=w.L, cache_rows=n0 + 1, ms_per_token=ms,
+                tokens_per_s=w.B / ms * 1e3)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attention", "topk", "gather", "quantize", "decode"])
+    ap.add_argument("case", choices=["attention", "topk", "gather", "quantize", "decode", "decode_step"])
     ap.add_argument("--B", type=int, default=32)
     ap.add_argument("--H", type=int, default=12)
     ap.add_argument("--n", type=int, default=512)
@@ -170,8 +194,10 @@ def main(argv=None):
         r = gather_case(a.B, a.n, a.k, a.row_bytes, a.reps)
     elif a.case == "quantize":
         r = quantize_case(a.B, a.H, a.n, a.d, a.reps)
-    else:
+    elif a.case == "decode":
         r = decode_case(a.B, a.H, a.n, a.d, a.keep, a.theta, a.reps)
+    else:
+        r = decode_step_case(a.reps)
     print(json.dumps(r), flush=True)
 
 

@@ -92,7 +92,8 @@ __device__ __forceinline__ void apply_gain(const QArgs& a, const QTensor& q, int
   }
 }
 
-template <typename T>
+// CT: 16-byte chunks per head row when known at compile time (d_h / 8), 0 otherwise
+template <typename T, int CT>
 __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int S = static_cast<int>(cluster.num_blocks());
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   const QTensor& q = a.t[blockIdx.z];
   const int bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int C = a.d_h / 8;
+  const int C = CT ? CT : a.d_h / 8;
   const int rows_per = (a.n + S - 1) / S;
   const int r0 = min(a.n, rank * rows_per), r1 = min(a.n, r0 + rows_per);
   const int total = (r1 - r0) * C;
@@ -167,10 +168,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   }
 }
 
-template <typename T>
+template <typename T, int CT>
 __global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
   const QTensor& q = a.t[blockIdx.z];
-  const int C = a.d_h / 8;
+  const int C = CT ? CT : a.d_h / 8;
   const int64_t total = static_cast<int64_t>(a.B) * a.H * a.n * C;
   int sat = 0;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(kQThreads) + threadIdx.x; e < total;
@@ -200,10 +201,17 @@ int32_t quantize_launch(const QArgs& a, int ntensors, int dtype, cudaStream_t st
     const int64_t chunks = static_cast<int64_t>(a.B) * a.H * a.n * (a.d_h / 8);
     int grid = static_cast<int>(std::min<int64_t>(ceil_div(chunks, kQThreads), 8LL * sm_count()));
     dim3 g(grid, 1, ntensors);
-    if (dtype == SPATTEN_BF16)
-      quantize_fixed_kernel<__nv_bfloat16><<<g, kQThreads, 0, st>>>(a);
-    else
-      quantize_fixed_kernel<float><<<g, kQThreads, 0, st>>>(a);
+    const bool bf = dtype == SPATTEN_BF16;
+    if (a.d_h == 64) {
+      if (bf) quantize_fixed_kernel<__nv_bfloat16, 8><<<g, kQThreads, 0, st>>>(a);
+      else quantize_fixed_kernel<float, 8><<<g, kQThreads, 0, st>>>(a);
+    } else if (a.d_h == 128) {
+      if (bf) quantize_fixed_kernel<__nv_bfloat16, 16><<<g, kQThreads, 0, st>>>(a);
+      else quantize_fixed_kernel<float, 16><<<g, kQThreads, 0, st>>>(a);
+    } else {
+      if (bf) quantize_fixed_kernel<__nv_bfloat16, 0><<<g, kQThreads, 0, st>>>(a);
+      else quantize_fixed_kernel<float, 0><<<g, kQThreads, 0, st>>>(a);
+    }
     return launch_status();
   }
   const int blocks = a.B * a.H;
@@ -223,9 +231,17 @@ int32_t quantize_launch(const QArgs& a, int ntensors, int dtype, cudaStream_t st
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = dtype == SPATTEN_BF16
-                      ? cudaLaunchKernelEx(&cfg, quantize_amax_kernel<__nv_bfloat16>, a)
-                      : cudaLaunchKernelEx(&cfg, quantize_amax_kernel<float>, a);
+  const bool bf = dtype == SPATTEN_BF16;
+  cudaError_t e;
+  if (a.d_h == 64)
+    e = bf ? cudaLaunchKernelEx(&cfg, quantize_amax_kernel<__nv_bfloat16, 8>, a)
+           : cudaLaunchKernelEx(&cfg, quantize_amax_kernel<float, 8>, a);
+  else if (a.d_h == 128)
+    e = bf ? cudaLaunchKernelEx(&cfg, quantize_amax_kernel<__nv_bfloat16, 16>, a)
+           : cudaLaunchKernelEx(&cfg, quantize_amax_kernel<float, 16>, a);
+  else
+    e = bf ? cudaLaunchKernelEx(&cfg, quantize_amax_kernel<__nv_bfloat16, 0>, a)
+           : cudaLaunchKernelEx(&cfg, quantize_amax_kernel<float, 0>, a);
   if (e != cudaSuccess) {
     record_cuda_error(e);
     return SPATTEN_E_CUDA;
