@@ -338,6 +338,155 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Short rows (n <= 8192): the row's keys live in registers, sixteen consecutive keys per thread, one
+// warp per row (n <= 512, four rows per CTA, no block barrier) or one CTA of G warps per row (G = 4
+// up to 2048 keys, 16 up to 8192).  The
+// threshold T (the k-th largest key) is found digit by digit, two bits per round: of the candidates
+// T | j << b (j = 1..3) the largest one with at least k keys at or above it is kept, so after 16
+// rounds T is the largest value with count(key >= T) >= k.  Counting is a compare per key and an
+// integer warp reduction (__reduce_add_sync); no histogram, no atomics.  need_eq = k - count(key > T)
+// keys equal to T are taken in index order; one packed scan places every thread's selected keys.
+// ------------------------------------------------------------------------------------------------
+constexpr int kSKeys = 16;
+
+template <int G>
+__global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs a) {
+  constexpr int RPC = G == 1 ? 4 : 1;   // rows per CTA
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * RPC + (G == 1 ? warp : 0);
+  const int t = G == 1 ? lane : static_cast<int>(threadIdx.x);   // thread within the row
+  __shared__ uint32_t red[2][2][G];    // [round parity][word][warp]
+  __shared__ uint32_t wscan[G];
+  __shared__ int nan_any;
+  if (r >= a.R) return;                // G == 1: the whole warp; G > 1: never (grid = R)
+  const int64_t out_base = static_cast<int64_t>(r) * a.ld_out;
+  if (a.k == 0) return;
+  if (a.k == a.n) {
+    for (int j = t; j < a.n; j += 32 * G) {
+      if (a.idx_out) a.idx_out[out_base + j] = j;
+      if (a.comp_out) a.comp_out[out_base + j] = a.map[static_cast<int64_t>(r) * a.ld_map + j];
+    }
+    return;
+  }
+  if (G > 1 && threadIdx.x == 0) nan_any = 0;
+
+  // keys t*16 .. t*16+15 of the row; missing keys are 0 (below every candidate, which is >= 1)
+  uint32_t key[kSKeys];
+  int nan_local = 0;
+  const int j0 = t * kSKeys;
+  const bool vec = a.map == nullptr && (a.ld & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
+  if (vec && j0 + kSKeys <= a.n) {
+    const float4* p = reinterpret_cast<const float4*>(a.scores + static_cast<int64_t>(r) * a.ld + j0);
+#pragma unroll
+    for (int q = 0; q < kSKeys / 4; ++q) {
+      const float4 f = __ldg(p + q);
+      const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        nan_local |= fv[u] != fv[u];
+        key[4 * q + u] = float_key(fv[u]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < kSKeys; ++u) key[u] = j0 + u < a.n ? load_key(a, r, j0 + u, &nan_local) : 0u;
+  }
+  int round = 0;
+  // counts of keys >= c1, c2, c3 over the row: (c1 | c2 << 16) and c3
+  auto count3 = [&](uint32_t c1, uint32_t c2, uint32_t c3, uint32_t& n1, uint32_t& n2, uint32_t& n3) {
+    uint32_t x = 0u, y = 0u;
+#pragma unroll
+    for (int u = 0; u < kSKeys; ++u) {
+      x += (key[u] >= c1 ? 1u : 0u) + (key[u] >= c2 ? 0x10000u : 0u);
+      y += key[u] >= c3 ? 1u : 0u;
+    }
+    x = __reduce_add_sync(0xffffffffu, x);
+    y = __reduce_add_sync(0xffffffffu, y);
+    if (G > 1) {
+      const int pr = round & 1;
+      if (lane == 0) {
+        red[pr][0][warp] = x;
+        red[pr][1][warp] = y;
+      }
+      __syncthreads();
+      x = 0u;
+      y = 0u;
+#pragma unroll
+      for (int w = 0; w < G; ++w) {
+        x += red[pr][0][w];
+        y += red[pr][1][w];
+      }
+    }
+    ++round;
+    n1 = x & 0xFFFFu;
+    n2 = x >> 16;
+    n3 = y;
+  };
+  const uint32_t k = static_cast<uint32_t>(a.k);
+  uint32_t T = 0u;
+#pragma unroll 1
+  for (int b = 30; b >= 0; b -= 2) {
+    uint32_t n1, n2, n3;
+    count3(T | (1u << b), T | (2u << b), T | (3u << b), n1, n2, n3);
+    T |= static_cast<uint32_t>((n1 >= k) + (n2 >= k) + (n3 >= k)) << b;
+  }
+  uint32_t n_gt, d1, d2;
+  if (T == 0xFFFFFFFFu) {
+    n_gt = 0u;
+  } else {
+    count3(T + 1u, 0xFFFFFFFFu, 0xFFFFFFFFu, n_gt, d1, d2);
+  }
+  const uint32_t need_eq = k - n_gt;
+  if (G > 1) {
+    if (nan_local) nan_any = 1;
+    __syncthreads();
+    nan_local = nan_any;
+  } else {
+    nan_local = __any_sync(0xffffffffu, nan_local);
+  }
+  if (nan_local && t == 0) report(a.status, SPATTEN_E_NONFINITE);
+
+  // ordered compaction: exclusive scan of packed (above T | equal to T << 16) per-thread counts
+  uint32_t gtc = 0u, eqc = 0u;
+#pragma unroll
+  for (int u = 0; u < kSKeys; ++u) {
+    gtc += key[u] > T ? 1u : 0u;
+    eqc += (j0 + u < a.n && key[u] == T) ? 1u : 0u;
+  }
+  const uint32_t v = gtc | (eqc << 16);
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  uint32_t pre = inc - v;
+  if (G > 1) {
+    if (lane == 31) wscan[warp] = inc;
+    __syncthreads();
+    uint32_t before = 0u;
+    for (int w = 0; w < warp; ++w) before += wscan[w];
+    pre += before;
+  }
+  uint32_t pos = (pre & 0xFFFFu) + min(pre >> 16, need_eq);
+  uint32_t er = pre >> 16;
+#pragma unroll
+  for (int u = 0; u < kSKeys; ++u) {
+    const bool gt = key[u] > T;
+    const bool eq = j0 + u < a.n && key[u] == T;
+    const bool sel = gt || (eq && er < need_eq);
+    er += eq ? 1u : 0u;
+    if (sel) {
+      if (pos < k) {
+        if (a.idx_out) a.idx_out[out_base + pos] = j0 + u;
+        if (a.comp_out) a.comp_out[out_base + pos] = a.map[static_cast<int64_t>(r) * a.ld_map + j0 + u];
+      }
+      ++pos;
+    }
+  }
+}
+
 int pick_cluster(int n) {
   // one CTA per 4096 keys, at most 8 (portable cluster size); the launcher may widen very long
   // rows to 16 when the device can schedule such clusters
@@ -377,6 +526,18 @@ int32_t topk_launch(const TArgs& a, cudaStream_t st) {
     }
     cudaGetLastError();   // the probe above may leave an error behind
     configured[dev] = true;
+  }
+  if (a.n <= 32 * kSKeys) {
+    topk_small_kernel<1><<<static_cast<unsigned>(ceil_div(a.R, 4)), 128, 0, st>>>(a);
+    return launch_status();
+  }
+  if (a.n <= 128 * kSKeys) {
+    topk_small_kernel<4><<<a.R, 128, 0, st>>>(a);
+    return launch_status();
+  }
+  if (a.n <= 512 * kSKeys) {
+    topk_small_kernel<16><<<a.R, 512, 0, st>>>(a);
+    return launch_status();
   }
   int C = pick_cluster(a.n);
   if (C == 8 && a.n > 8 * kResident && dev >= 0 && dev < 64 && wide_ok[dev]) C = 16;

@@ -178,7 +178,12 @@ def _topk_gpu(S, scores_np, k, map_np=None):
 @pytest.mark.parametrize("R_,n,k,kind", [
     (3, 1, 1, "u"), (3, 1, 0, "u"), (4, 10, 3, "ties"), (5, 100, 100, "u"), (5, 100, 1, "u"),
     (8, 517, 200, "ties"), (4, 4097, 2048, "zeros"), (6, 20000, 13, "ln"), (2, 70000, 35000, "ties"),
-    (3, 1000, 500, "const")])
+    (3, 1000, 500, "const"),
+    # row-length boundaries of the short-row kernels (warp per row <= 512, 4 warps <= 2048,
+    # 16 warps <= 8192, clusters beyond), odd row counts, mixed signs, k = 1 and k = n - 1
+    (7, 512, 461, "neg"), (5, 513, 1, "neg"), (6, 2048, 2047, "ties"), (3, 2049, 1024, "neg"),
+    (2, 8192, 4096, "u"), (2, 8193, 819, "neg"), (9, 12, 11, "neg"), (1, 1153, 1131, "const"),
+    (13, 160, 144, "ties")])
 def test_topk_matches_oracle(cuda, R_, n, k, kind):
     S = lib()
     g = synth.rng_for(n + k)
@@ -188,6 +193,9 @@ def test_topk_matches_oracle(cuda, R_, n, k, kind):
         x = g.lognormal(0, 2, (R_, n)).astype(np.float32)
     elif kind == "ties":
         x = (g.integers(0, 5, (R_, n)) * 0.25 - 0.5).astype(np.float32)
+    elif kind == "neg":
+        x = g.standard_normal((R_, n)).astype(np.float32)
+        x[:, ::11] = x[:, 3:4]   # exact duplicates across the sign boundary
     elif kind == "zeros":
         x = np.where(g.random((R_, n)) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
         x[:, ::7] = -1.0
