@@ -121,6 +121,24 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
+// The AND of `ok` over the 128 threads of a softmax warpgroup (named barrier `id`): after a wait,
+// every thread of the group takes the same branch, so no thread can leave a group barrier or a
+// warp-collective TMEM load short of participants after a timeout.
+__device__ __forceinline__ bool wg_all(bool ok, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n"
+      ".reg .pred p, q;\n"
+      "setp.ne.u32 p, %1, 0;\n"
+      "bar.red.and.pred q, %2, 128, p;\n"
+      "selp.u32 %0, 1, 0, q;\n"
+      "}\n"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
 // column sums over the 32 rows of a warp: afterwards lane l holds the sum of column l
 __device__ __forceinline__ float warp_colsum32(float* v) {
   const int lane = threadIdx.x & 31;
@@ -505,9 +523,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         ++cnt;
       }
     };
-    run_jobs(0, n_tiles);
-    if (__syncthreads_or(aborted)) aborted = true;
-    if (!aborted) run_jobs(n_tiles, 3 * n_tiles);
+    run_jobs(0, 3 * n_tiles);   // pass A keys, then pass B keys and values, without a block barrier
   } else if (warp == 11) {
     // ------------------------------------------------------------------------- MMA issue
     uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0};
@@ -535,8 +551,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       for (int t = 0; t < n_tiles && !aborted; ++t)
         if (!qk_both()) aborted = true;
     }
-    if (__syncthreads_or(aborted)) aborted = true;
-    if (lane == 0 && !aborted) {
+    if (lane == 0 && !aborted) {   // pass B follows at once
       if (!qk_both()) aborted = true;
       for (int t = 0; t < n_tiles && !aborted; ++t) {
         if (t + 1 < n_tiles && !qk_both()) { aborted = true; break; }
@@ -560,7 +575,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     // ------------------------------------------------------------------------- softmax (pass A)
     uint32_t sc = 0;
     for (int t = 0; t < n_tiles; ++t) {
-      if (!wait_bar(&bars[M_SF + g], sc & 1u, abort_flag)) { aborted = true; break; }
+      if (!__all_sync(0xffffffffu, wait_bar(&bars[M_SF + g], sc & 1u, abort_flag))) { aborted = true; break; }
       tc_after_sync();
 #pragma unroll 1
       for (int hh = 0; hh < KT / 64; ++hh) {
@@ -584,7 +599,6 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       ++sc;
     }
     flag = !aborted && row_ok && (1.0f / l < a.refetch_threshold);
-    if (__syncthreads_or(aborted)) aborted = true;
   }
   // -------------------------------------------------------------------------------------------
   // flagged rows -> packed list (ascending row ids); counts of the whole CTA
@@ -604,6 +618,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   }
 
   // ------------------------------------------------------------------------- softmax (pass B)
+  if (warp < 8) aborted = !wg_all(!aborted, 1 + g);   // the warpgroup enters pass B together
   if (warp < 8 && !aborted) {
     uint32_t sc = static_cast<uint32_t>(n_tiles), pc = 0;
     const bool live = row_ok && !flag;
@@ -613,8 +628,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     const int qt128 = pair * 2 + g;
     const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
     for (int t = 0; t < n_tiles; ++t) {
-      if (!wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-      if (!wait_bar(&bars[M_SF + g], sc & 1u, abort_flag)) { aborted = true; break; }
+      if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag), 1 + g)) { aborted = true; break; }
       tc_after_sync();
 #pragma unroll 1
       for (int hh = 0; hh < KT / 64; ++hh) {
@@ -626,6 +640,12 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         if (hh == KT / 64 - 1) {
           tc_before_sync();
           mbar_arrive(&bars[M_SR + g]);
+        }
+        // the previous tile's P V must be done before this tile's P overwrites the buffer; the
+        // score load and the exponentials above and below overlap it
+        if (hh == 0 && !wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag), 1 + g)) {
+          aborted = true;
+          break;
         }
         const int kb = t * KT + hh * 64;
         if (kb + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
@@ -655,6 +675,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         colred[t & 1][g][warp & 3][hh * 64 + lane] = sv;
         colred[t & 1][g][warp & 3][hh * 64 + 32 + lane] = sw;
       }
+      if (aborted) break;   // uniform over the warpgroup
       ++sc;
       fence_async_smem();
       mbar_arrive(&bars[M_PF + g]);
@@ -673,6 +694,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   float habs = 0.0f;
   if (warp < 8 && !aborted) {
     if (!wait_bar(&bars[M_OD], 0, abort_flag)) aborted = true;
+    aborted = __any_sync(0xffffffffu, aborted);   // warp-uniform before the TMEM loads
     tc_after_sync();
     if (!aborted) {
       const float vs = a.v_scale[bh];
@@ -864,9 +886,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
         ++cnt;
       }
     };
-    run_jobs(0, n_tiles);
-    if (__syncthreads_or(aborted)) aborted = true;
-    if (!aborted) run_jobs(n_tiles, 3 * n_tiles);
+    run_jobs(0, 3 * n_tiles);   // pass A keys, then pass B keys and values, without a block barrier
   } else if (warp == 7) {
     // ------------------------------------------------------------------------- MMA issue
     uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0};
@@ -891,8 +911,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       for (int t = 0; t < n_tiles && !aborted; ++t)
         if (!qk(t)) aborted = true;
     }
-    if (__syncthreads_or(aborted)) aborted = true;
-    if (lane == 0 && !aborted) {
+    if (lane == 0 && !aborted) {   // pass B follows at once
       if (!qk(0)) aborted = true;
       for (int t = 0; t < n_tiles && !aborted; ++t) {
         if (t + 1 < n_tiles && !qk(t + 1)) { aborted = true; break; }
@@ -917,7 +936,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     uint32_t sc[2] = {0, 0};
     for (int t = 0; t < n_tiles; ++t) {
       const int sb = t & 1;
-      if (!wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag)) { aborted = true; break; }
+      if (!__all_sync(0xffffffffu, wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag))) { aborted = true; break; }
       tc_after_sync();
       if (warp_live) {
 #pragma unroll 1
@@ -940,7 +959,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       mbar_arrive(&bars[F_SR + sb]);
       ++sc[sb];
     }
-    if (__syncthreads_or(aborted)) aborted = true;
+    aborted = !wg_all(!aborted, 1);   // the warpgroup enters pass B together
     // ------------------------------------------------------------------------- softmax (pass B)
     if (!aborted) {
       uint32_t pc[2] = {0, 0};
@@ -949,8 +968,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       for (int t = 0; t < n_tiles; ++t) {
         const int sb = t & 1;
         const int pb = 0;   // single P buffer
-        if (!wait_bar(&bars[F_PE + pb], (pc[pb] & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-        if (!wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag)) { aborted = true; break; }
+        if (!wg_all(wait_bar(&bars[F_PE + pb], (pc[pb] & 1u) ^ 1u, abort_flag), 1)) { aborted = true; break; }
+        if (!wg_all(wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag), 1)) { aborted = true; break; }
         tc_after_sync();
         uint8_t* Pt = smem + C::oP + pb * C::PB;
 #pragma unroll 1
@@ -1013,6 +1032,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   float habs = 0.0f;
   if (warp < 4 && !aborted) {
     if (!wait_bar(&bars[F_OD], 0, abort_flag)) aborted = true;
+    aborted = __any_sync(0xffffffffu, aborted);   // warp-uniform before the TMEM loads
     tc_after_sync();
     if (!aborted && warp_live) {
       const float vs = a.v_scale[bh];
