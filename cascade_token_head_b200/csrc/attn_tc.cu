@@ -14,10 +14,14 @@
 // stored as fp16 (11 significant bits).
 //
 // Two kernels per layer:
-//  MAIN  one CTA = (sequence, kept head, 256 query rows), 384 threads:
+//  MAIN  persistent: one CTA per SM walks the work items (sequence, kept head, 256 query rows) with
+//        a stride of the grid; TMEM, barriers and all ring counters live across items, so the
+//        producers load the next item's query tile and first key tiles, and the MMA warp issues its
+//        first score MMAs, while the softmax warps finish the current item.  384 threads:
 //          warps 0-7   two softmax warpgroups; warpgroup g owns query rows 128g..128g+127 of the
 //                      CTA, thread r of a warpgroup is TMEM lane r of that warpgroup's S and O
-//          warps 8-10  producers: Q once, then K/V MSB tiles dequantized into 2-stage rings
+//          warps 8-10  producers: the item's query tile, then K/V MSB tiles converted into
+//                      2-stage rings
 //          warp 11     MMA issue (lane 0) and TMEM allocation
 //        pass A computes S_msb tile by tile (the two warpgroups' tiles alternate on the tensor
 //        core while the other warpgroup runs its softmax) -> row max / exp-sum -> refetch flags;
@@ -139,23 +143,8 @@ __device__ __forceinline__ bool wg_all(bool ok, int id) {
   return r != 0;
 }
 
-// column sums over the 32 rows of a warp: afterwards lane l holds the sum of column l
-__device__ __forceinline__ float warp_colsum32(float* v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int j = 0; j < off; ++j) {
-      const float send = upper ? v[j] : v[j + off];
-      const float keep = upper ? v[j + off] : v[j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-  return v[0];
-}
-
-// two column-sum butterflies interleaved (independent chains, twice the ILP)
+// column sums over the 32 rows of a warp for two 32-column arrays: afterwards lane l holds the
+// sums of column l of each (two independent butterfly chains, twice the ILP)
 __device__ __forceinline__ void warp_colsum32x2(float* v, float* w, float& sv, float& sw) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -285,7 +274,8 @@ struct JobStream {
   bool with_lsb;
   int ptid;
   volatile int* abort_flag;
-  uint32_t issued = 0;
+  uint32_t g0 = 0;       // global index of this stream's job 0 in the staging ring's sequence
+  uint32_t issued = 0;   // jobs of this stream issued so far (loader)
 
   __device__ __forceinline__ int jobs() const { return 3 * n_tiles; }
   __device__ __forceinline__ void job(int j, bool& is_v, int& t) const {
@@ -302,8 +292,9 @@ struct JobStream {
   __device__ __forceinline__ bool issue_ahead(int j) {
     while (static_cast<int>(issued) < jobs() && static_cast<int>(issued) < j + RS) {
       const uint32_t jn = issued;
-      const uint32_t st = jn % RS;
-      if (!wait_bar(&raw_empty[st], ((jn / RS) & 1u) ^ 1u, abort_flag)) return false;
+      const uint32_t gj = g0 + jn;
+      const uint32_t st = gj % RS;
+      if (!wait_bar(&raw_empty[st], ((gj / RS) & 1u) ^ 1u, abort_flag)) return false;
       bool is_v;
       int t;
       job(static_cast<int>(jn), is_v, t);
@@ -328,8 +319,9 @@ struct JobStream {
                            with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, off_lo, ptid);
       return true;
     }
-    const uint32_t st = static_cast<uint32_t>(j) % RS;
-    if (!wait_bar(&raw_full[st], (static_cast<uint32_t>(j) / RS) & 1u, abort_flag)) return false;
+    const uint32_t gj = g0 + static_cast<uint32_t>(j);
+    const uint32_t st = gj % RS;
+    if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag)) return false;
     convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, off_lo, ptid);
     mbar_arrive(&raw_empty[st]);
     return true;
@@ -394,9 +386,29 @@ struct MainCfg {
   static constexpr uint32_t tO = 2u * KT;        // + g * DH
 };
 
-enum : int { M_Q = 0, M_KF = 1, M_KE = 3, M_VF = 5, M_VE = 7, M_SF = 9, M_SR = 11, M_PF = 13, M_PE = 15, M_OD = 17,
-             M_RF = 18, M_RE = 22, M_N = 26 };
+enum : int { M_QF = 0, M_QE = 1, M_OE = 2, M_KF = 3, M_KE = 5, M_VF = 7, M_VE = 9, M_SF = 11, M_SR = 13, M_PF = 15,
+             M_PE = 17, M_OD = 19, M_RF = 20, M_RE = 24, M_N = 28 };
 
+// AND of `ok` over the 256 softmax threads of a CTA (named barrier 3)
+__device__ __forceinline__ bool softmax_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n"
+      ".reg .pred p, q;\n"
+      "setp.ne.u32 p, %1, 0;\n"
+      "bar.red.and.pred q, 3, 256, p;\n"
+      "selp.u32 %0, 1, 0, q;\n"
+      "}\n"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
+
+// Persistent: one CTA per SM walks the work items (sequence, kept head, 256-row pair) with a
+// stride of gridDim.x; TMEM, barriers and every ring counter live across items, so the producers
+// load the next item's query tile and first key tiles, and the MMA warp issues its first score
+// MMAs, while the softmax warps finish the previous item.
 template <int DH>
 __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   using C = MainCfg<DH>;
@@ -412,22 +424,10 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   __shared__ uint32_t wcnt[8];
   __shared__ int abort_s;
 
-  const int pair = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i0 = pair * 256;
-  const int h = head_of_slot(a, b, slot);
+  const int n_items = p.n_pair * a.H_kept * a.B;
+  const int n_tiles = (a.n_kv + KT - 1) / KT;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
-
-  if (slot >= a.H_kept) {   // pruned head: zero its output rows (no TMEM, no barrier)
-    if (h < 0) return;
-    for (int e = tid; e < 256 * (DH / 8); e += 384) {
-      const int i = i0 + e / (DH / 8), c8 = e % (DH / 8);
-      if (i < a.n_q)
-        *reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8) =
-            make_uint4(0, 0, 0, 0);
-    }
-    return;
-  }
 
   if (warp == 11) {
     tmem_alloc(&tmem_base_s, kTmemCols);
@@ -435,7 +435,9 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   }
   if (tid == 0) {
     abort_s = 0;
-    mbar_init(&bars[M_Q], 352);
+    mbar_init(&bars[M_QF], kProducerThreads);
+    mbar_init(&bars[M_QE], 1);
+    mbar_init(&bars[M_OE], 256);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars[M_KF + s], kProducerThreads);
       mbar_init(&bars[M_VF + s], kProducerThreads);
@@ -460,274 +462,314 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   tc_after_sync();
   const uint32_t tmem = tmem_base_s;
   volatile int* abort_flag = &abort_s;
-
-  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
-  const int64_t plane0 = bh * a.kv_cap;
-  const int n_tiles = (a.n_kv + KT - 1) / KT;
-  const int64_t list_base = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_pair + pair);
-  const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
   bool aborted = false;
 
-  // softmax thread state
-  const int g = warp >> 2;                        // warpgroup
-  const int r = tid & 127;                        // row within the warpgroup's tile
-  const int i = i0 + g * 128 + r;
-  const bool row_ok = warp < 8 && i < a.n_q;
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const float c2 = a.k_scale[bh] * a.sm_scale * kLog2e;
-  float m2 = -INFINITY, l = 0.0f;
-  bool flag = false;
+  // item -> (sequence, kept head slot, pair)
+  auto item_coords = [&](int it, int& b, int& slot, int& pair) {
+    pair = it % p.n_pair;
+    const int bs = it / p.n_pair;
+    slot = bs % a.H_kept;
+    b = bs / a.H_kept;
+  };
 
-  if (warp != 11) {
-    // Q tiles: every thread but the MMA warp, all of its loads in flight at once
-    constexpr int NCH = 256 * (DH / 8);
-    constexpr int PER = (NCH + 351) / 352;
-    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-    uint4 qv[PER];
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
-      const int e = tid + k * 352;
-      const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + rr;
-      qv[k] = make_uint4(0, 0, 0, 0);
-      if (e < NCH && qi < a.n_q)
-        qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
-                                                     static_cast<int64_t>(h) * DH) + c8);
-    }
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
-      const int e = tid + k * 352;
-      const int rr = e / (DH / 8), c8 = e % (DH / 8);
-      if (e < NCH)
-        *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) = bf16x8_to_f16x8(qv[k]);
-    }
-    fence_async_smem();
-    mbar_arrive(&bars[M_Q]);
-  }
   if (warp >= 8 && warp < 11) {
     // ------------------------------------------------------------------------- producers
     const int ptid = tid - 256;
-    JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
-                                abort_flag};
-    uint32_t kc = 0, vc = 0;
-    auto run_jobs = [&](int j0, int j1) {
-      for (int j = j0; j < j1; ++j) {
-        if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; return; }
+    uint32_t kc = 0, vc = 0, gjob = 0, qc = 0;
+    for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++qc) {
+      int b, slot, pair;
+      item_coords(it, b, slot, pair);
+      const int h = head_of_slot(a, b, slot);
+      const int64_t plane0 = (static_cast<int64_t>(b) * a.H + h) * a.kv_cap;
+      const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
+      JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
+                                  abort_flag, gjob};
+      // the first raw key tiles start before the query tile (both in flight together)
+      if (!kv_idx && ptid == 0 && !js.issue_ahead(0)) { aborted = true; break; }
+      // query tile of the item once the previous item's score MMAs have read the buffer
+      if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+      {
+        constexpr int NCH = 256 * (DH / 8);
+        constexpr int BATCH = 8;
+        const int i0 = pair * 256;
+        const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+        for (int e0 = ptid; e0 < NCH; e0 += BATCH * kProducerThreads) {
+          uint4 qv[BATCH];
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) {
+            const int e = e0 + k * kProducerThreads;
+            const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + rr;
+            qv[k] = make_uint4(0, 0, 0, 0);
+            if (e < NCH && qi < a.n_q)
+              qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
+                                                           static_cast<int64_t>(h) * DH) + c8);
+          }
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) {
+            const int e = e0 + k * kProducerThreads;
+            const int rr = e / (DH / 8), c8 = e % (DH / 8);
+            if (e < NCH)
+              *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) =
+                  bf16x8_to_f16x8(qv[k]);
+          }
+        }
+        fence_async_smem();
+        mbar_arrive(&bars[M_QF]);
+      }
+      // pass A keys, then pass B keys and values
+      for (int j = 0; j < 3 * n_tiles; ++j) {
+        if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; break; }
         bool is_v;
         int t;
         js.job(j, is_v, t);
         uint32_t& cnt = is_v ? vc : kc;
         const uint32_t st = cnt % NST;
-        if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag)) { aborted = true; return; }
-        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, 0, kv_idx)) { aborted = true; return; }
+        if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, 0, kv_idx)) { aborted = true; break; }
         mbar_arrive(&bars[(is_v ? M_VF : M_KF) + st]);
         ++cnt;
       }
-    };
-    run_jobs(0, 3 * n_tiles);   // pass A keys, then pass B keys and values, without a block barrier
+      gjob += 3 * n_tiles;
+    }
   } else if (warp == 11) {
     // ------------------------------------------------------------------------- MMA issue
-    uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0};
-    const uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
-    auto qk_both = [&](void) -> bool {
-      const uint32_t ks = kc % NST;
-      if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag)) return false;
-      const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
-      if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag)) return false;
-      tc_after_sync();
-      mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
-      mma_commit(&bars[M_SF + 0]);
-      ++sc[0];
-      if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag)) return false;
-      tc_after_sync();
-      mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
-      mma_commit(&bars[M_SF + 1]);
-      ++sc[1];
-      mma_commit(&bars[M_KE + ks]);
-      ++kc;
-      return true;
-    };
     if (lane == 0) {
-      if (!wait_bar(&bars[M_Q], 0, abort_flag)) aborted = true;
-      for (int t = 0; t < n_tiles && !aborted; ++t)
-        if (!qk_both()) aborted = true;
-    }
-    if (lane == 0 && !aborted) {   // pass B follows at once
-      if (!qk_both()) aborted = true;
-      for (int t = 0; t < n_tiles && !aborted; ++t) {
-        if (t + 1 < n_tiles && !qk_both()) { aborted = true; break; }
-        const uint32_t vs = vc % NST;
-        if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag)) { aborted = true; break; }
-        const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
-        for (int gg = 0; gg < 2 && !aborted; ++gg) {
-          if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag)) { aborted = true; break; }
-          tc_after_sync();
-          mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
-          mma_commit(&bars[M_PE + gg]);
-          ++pc[gg];
-        }
+      uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0}, ic = 0;
+      const uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
+      auto qk_both = [&](void) -> bool {
+        const uint32_t ks = kc % NST;
+        if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag)) return false;
+        const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
+        if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag)) return false;
+        tc_after_sync();
+        mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
+        mma_commit(&bars[M_SF + 0]);
+        ++sc[0];
+        if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag)) return false;
+        tc_after_sync();
+        mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
+        mma_commit(&bars[M_SF + 1]);
+        ++sc[1];
+        mma_commit(&bars[M_KE + ks]);
+        ++kc;
+        return true;
+      };
+      for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++ic) {
+        if (!wait_bar(&bars[M_QF], ic & 1u, abort_flag)) { aborted = true; break; }
+        for (int t = 0; t < n_tiles && !aborted; ++t)   // pass A
+          if (!qk_both()) aborted = true;
         if (aborted) break;
-        mma_commit(&bars[M_VE + vs]);
-        ++vc;
+        if (!qk_both()) { aborted = true; break; }       // pass B, tile 0
+        if (n_tiles == 1) mma_commit(&bars[M_QE]);      // the item's last read of Q is issued
+        // the previous item's O must have been read before this item's first P V overwrites it
+        if (!wait_bar(&bars[M_OE], (ic & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+        for (int t = 0; t < n_tiles && !aborted; ++t) {
+          if (t + 1 < n_tiles) {
+            if (!qk_both()) { aborted = true; break; }
+            if (t + 2 == n_tiles) mma_commit(&bars[M_QE]);
+          }
+          const uint32_t vs = vc % NST;
+          if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag)) { aborted = true; break; }
+          const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
+          for (int gg = 0; gg < 2 && !aborted; ++gg) {
+            if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag)) { aborted = true; break; }
+            tc_after_sync();
+            mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
+            mma_commit(&bars[M_PE + gg]);
+            ++pc[gg];
+          }
+          if (aborted) break;
+          mma_commit(&bars[M_VE + vs]);
+          ++vc;
+        }
+        if (!aborted) mma_commit(&bars[M_OD]);
       }
-      if (!aborted) mma_commit(&bars[M_OD]);
     }
   } else {
-    // ------------------------------------------------------------------------- softmax (pass A)
-    uint32_t sc = 0;
-    for (int t = 0; t < n_tiles; ++t) {
-      if (!__all_sync(0xffffffffu, wait_bar(&bars[M_SF + g], sc & 1u, abort_flag))) { aborted = true; break; }
-      tc_after_sync();
-#pragma unroll 1
-      for (int hh = 0; hh < KT / 64; ++hh) {
-        float v[64];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64, v);
-        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64 + 32, v + 32);
-        tmem_ld_wait();
-        if (hh == KT / 64 - 1) {
-          tc_before_sync();
-          mbar_arrive(&bars[M_SR + g]);
-        }
-        if (t * KT + hh * 64 + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
-          stats64_scaled(v, c2, m2, l);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
-          stats64(v, m2, l);
-        }
-      }
-      ++sc;
-    }
-    flag = !aborted && row_ok && (1.0f / l < a.refetch_threshold);
-  }
-  // -------------------------------------------------------------------------------------------
-  // flagged rows -> packed list (ascending row ids); counts of the whole CTA
-  // -------------------------------------------------------------------------------------------
-  if (warp < 8) {
-    const unsigned bal = __ballot_sync(0xffffffffu, flag);
-    if (lane == 0) wcnt[warp] = __popc(bal);
-    named_sync(3, 256);
-    uint32_t pos = __popc(bal & ((1u << lane) - 1u)), total = 0;
-    for (int w = 0; w < 8; ++w) {
-      if (w < warp) pos += wcnt[w];
-      total += wcnt[w];
-    }
-    if (flag) p.flag_list[list_base * 256 + pos] = i;
-    if (tid == 0) p.flag_cnt[list_base] = static_cast<int32_t>(total);
-    if (tid == 0 && total && a.refetch_count) atomicAdd(a.refetch_count, static_cast<int>(total));
-  }
+    // ------------------------------------------------------------------------- softmax
+    const int g = warp >> 2;                        // warpgroup
+    const int r = tid & 127;                        // row within the warpgroup's tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t sc = 0, pc = 0, oc = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++oc) {
+      if (!softmax_all(!aborted)) { aborted = true; break; }   // both warpgroups start the item together
+      int b, slot, pair;
+      item_coords(it, b, slot, pair);
+      const int h = head_of_slot(a, b, slot);
+      const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+      const int i = pair * 256 + g * 128 + r;
+      const bool row_ok = i < a.n_q;
+      const float c2 = a.k_scale[bh] * a.sm_scale * kLog2e;
+      const int64_t list_base = (static_cast<int64_t>(b) * a.H_kept + slot) * p.n_pair + pair;
+      float m2 = -INFINITY, l = 0.0f;
 
-  // ------------------------------------------------------------------------- softmax (pass B)
-  if (warp < 8) aborted = !wg_all(!aborted, 1 + g);   // the warpgroup enters pass B together
-  if (warp < 8 && !aborted) {
-    uint32_t sc = static_cast<uint32_t>(n_tiles), pc = 0;
-    const bool live = row_ok && !flag;
-    // p = 2^(c2 s - m2) / ell = 2^(c2 s - mb); rows that are not stored here get p = 0
-    const float mb = live ? m2 + log2f(l) : INFINITY;
-    uint8_t* Pt = smem + C::oP + g * C::PB;
-    const int qt128 = pair * 2 + g;
-    const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
-    for (int t = 0; t < n_tiles; ++t) {
-      if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag), 1 + g)) { aborted = true; break; }
-      tc_after_sync();
+      // ---- pass A: MSB statistics
+      for (int t = 0; t < n_tiles; ++t) {
+        if (!__all_sync(0xffffffffu, wait_bar(&bars[M_SF + g], sc & 1u, abort_flag))) { aborted = true; break; }
+        tc_after_sync();
 #pragma unroll 1
-      for (int hh = 0; hh < KT / 64; ++hh) {
-        float v[32], w[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64, v);
-        tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64 + 32, w);
-        tmem_ld_wait();
-        if (hh == KT / 64 - 1) {
-          tc_before_sync();
-          mbar_arrive(&bars[M_SR + g]);
-        }
-        // the previous tile's P V must be done before this tile's P overwrites the buffer; the
-        // score load and the exponentials above and below overlap it
-        if (hh == 0 && !wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag), 1 + g)) {
-          aborted = true;
-          break;
-        }
-        const int kb = t * KT + hh * 64;
-        if (kb + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            v[j] = ex2(fmaf(v[j], c2, -mb));
-            w[j] = ex2(fmaf(w[j], c2, -mb));
+        for (int hh = 0; hh < KT / 64; ++hh) {
+          float v[64];
+          __syncwarp();
+          tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64, v);
+          tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64 + 32, v + 32);
+          tmem_ld_wait();
+          if (hh == KT / 64 - 1) {
+            tc_before_sync();
+            mbar_arrive(&bars[M_SR + g]);
           }
-        } else {
+          if (t * KT + hh * 64 + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
+            stats64_scaled(v, c2, m2, l);
+          } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            v[j] = kb + j < a.n_kv ? ex2(fmaf(v[j], c2, -mb)) : 0.0f;
-            w[j] = kb + 32 + j < a.n_kv ? ex2(fmaf(w[j], c2, -mb)) : 0.0f;
+            for (int j = 0; j < 64; ++j) v[j] = (t * KT + hh * 64 + j < a.n_kv) ? v[j] * c2 : -INFINITY;
+            stats64(v, m2, l);
           }
         }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + q4, 128)) =
-              make_uint4(pack_f16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
-                         pack_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
-          *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + 4 + q4, 128)) =
-              make_uint4(pack_f16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_f16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
-                         pack_f16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_f16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
-        }
-        float sv, sw;
-        warp_colsum32x2(v, w, sv, sw);
-        colred[t & 1][g][warp & 3][hh * 64 + lane] = sv;
-        colred[t & 1][g][warp & 3][hh * 64 + 32 + lane] = sw;
+        ++sc;
       }
-      if (aborted) break;   // uniform over the warpgroup
-      ++sc;
-      fence_async_smem();
-      mbar_arrive(&bars[M_PF + g]);
-      ++pc;
-      named_sync(1 + g, 128);
-      if (r < KT) {
-        const int key = t * KT + r;
-        if (key < a.n_kv && qt128 < p.n_qt)
-          p.tok_part[part_row + key] = ((colred[t & 1][g][0][r] + colred[t & 1][g][1][r]) + colred[t & 1][g][2][r]) +
-                                       colred[t & 1][g][3][r];
-      }
-    }
-  }
+      const bool flag = !aborted && row_ok && (1.0f / l < a.refetch_threshold);
 
-  // ------------------------------------------------------------------------- epilogue
-  float habs = 0.0f;
-  if (warp < 8 && !aborted) {
-    if (!wait_bar(&bars[M_OD], 0, abort_flag)) aborted = true;
-    aborted = __any_sync(0xffffffffu, aborted);   // warp-uniform before the TMEM loads
-    tc_after_sync();
-    if (!aborted) {
-      const float vs = a.v_scale[bh];
-#pragma unroll 1
-      for (int ch = 0; ch < DH / 32; ++ch) {
-        float v[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + C::tO + g * DH + ch * 32, v);
-        tmem_ld_wait();
-        if (row_ok && !flag)
-          store_o_row(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + ch * 32, v,
-                      vs, habs);
+      // ---- flagged rows -> packed list (ascending row ids); counts of the item
+      const unsigned bal = __ballot_sync(0xffffffffu, flag);
+      if (lane == 0) wcnt[warp] = __popc(bal);
+      if (!softmax_all(!aborted)) { aborted = true; break; }
+      {
+        uint32_t pos = __popc(bal & ((1u << lane) - 1u)), total = 0;
+        for (int w = 0; w < 8; ++w) {
+          if (w < warp) pos += wcnt[w];
+          total += wcnt[w];
+        }
+        if (flag) p.flag_list[list_base * 256 + pos] = i;
+        if (tid == 0) p.flag_cnt[list_base] = static_cast<int32_t>(total);
+        if (tid == 0 && total && a.refetch_count) atomicAdd(a.refetch_count, static_cast<int>(total));
       }
-      if (row_ok && a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld + i] = flag ? 1 : 0;
+
+      // ---- pass B: probabilities of the unflagged rows, column sums, P V
+      {
+        const bool live = row_ok && !flag;
+        // p = 2^(c2 s - m2) / ell = 2^(c2 s - mb); rows that are not stored here get p = 0
+        const float mb = live ? m2 + log2f(l) : INFINITY;
+        uint8_t* Pt = smem + C::oP + g * C::PB;
+        const int qt128 = pair * 2 + g;
+        const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
+        for (int t = 0; t < n_tiles; ++t) {
+          if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag), 1 + g)) { aborted = true; break; }
+          tc_after_sync();
+#pragma unroll 1
+          for (int hh = 0; hh < KT / 64; ++hh) {
+            float v[32], w[32];
+            __syncwarp();
+            tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64, v);
+            tmem_ld32(tmem + lane_base + C::tS + g * KT + hh * 64 + 32, w);
+            tmem_ld_wait();
+            if (hh == KT / 64 - 1) {
+              tc_before_sync();
+              mbar_arrive(&bars[M_SR + g]);
+            }
+            // the previous tile's P V must be done before this tile's P overwrites the buffer; the
+            // score load and the exponentials below overlap it
+            if (hh == 0 && !wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag), 1 + g)) {
+              aborted = true;
+              break;
+            }
+            const int kb = t * KT + hh * 64;
+            if (kb + 64 <= a.n_kv) {   // a full chunk (uniform over the CTA)
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                v[j] = ex2(fmaf(v[j], c2, -mb));
+                w[j] = ex2(fmaf(w[j], c2, -mb));
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                v[j] = kb + j < a.n_kv ? ex2(fmaf(v[j], c2, -mb)) : 0.0f;
+                w[j] = kb + 32 + j < a.n_kv ? ex2(fmaf(w[j], c2, -mb)) : 0.0f;
+              }
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + q4, 128)) =
+                  make_uint4(pack_f16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                             pack_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+              *reinterpret_cast<uint4*>(Pt + tile_off(r, hh * 8 + 4 + q4, 128)) =
+                  make_uint4(pack_f16x2(w[8 * q4 + 0], w[8 * q4 + 1]), pack_f16x2(w[8 * q4 + 2], w[8 * q4 + 3]),
+                             pack_f16x2(w[8 * q4 + 4], w[8 * q4 + 5]), pack_f16x2(w[8 * q4 + 6], w[8 * q4 + 7]));
+            }
+            float sv, sw;
+            warp_colsum32x2(v, w, sv, sw);
+            colred[t & 1][g][warp & 3][hh * 64 + lane] = sv;
+            colred[t & 1][g][warp & 3][hh * 64 + 32 + lane] = sw;
+          }
+          if (aborted) break;   // uniform over the warpgroup
+          ++sc;
+          fence_async_smem();
+          mbar_arrive(&bars[M_PF + g]);
+          ++pc;
+          named_sync(1 + g, 128);
+          if (r < KT) {
+            const int key = t * KT + r;
+            if (key < a.n_kv && qt128 < p.n_qt)
+              p.tok_part[part_row + key] = ((colred[t & 1][g][0][r] + colred[t & 1][g][1][r]) + colred[t & 1][g][2][r]) +
+                                           colred[t & 1][g][3][r];
+          }
+        }
+      }
+
+      // ---- epilogue: O of the unflagged rows, head importance partial, refetch flags
+      float habs = 0.0f;
+      if (!aborted) {
+        if (!wg_all(wait_bar(&bars[M_OD], oc & 1u, abort_flag), 1 + g)) aborted = true;
+      }
+      if (!aborted) {
+        tc_after_sync();
+        float ov[DH];
+#pragma unroll
+        for (int ch = 0; ch < DH / 32; ++ch) tmem_ld32(tmem + lane_base + C::tO + g * DH + ch * 32, ov + ch * 32);
+        tmem_ld_wait();
+        tc_before_sync();
+        mbar_arrive(&bars[M_OE]);   // the next item's P V may overwrite O
+        const float vs = a.v_scale[bh];
+        if (row_ok && !flag) {
+#pragma unroll
+          for (int ch = 0; ch < DH / 32; ++ch)
+            store_o_row(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + ch * 32,
+                        ov + ch * 32, vs, habs);
+        }
+        if (row_ok && a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld + i] = flag ? 1 : 0;
+      }
+      habs = warp_sum(habs);
+      if (lane == 0) hred[g][warp & 3] = habs;
+      if (!softmax_all(!aborted)) { aborted = true; break; }
+      if (tid == 0 || tid == 128) {
+        const int qt128 = pair * 2 + (tid >> 7);
+        if (qt128 < p.n_qt)
+          p.head_part[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128] =
+              ((hred[tid >> 7][0] + hred[tid >> 7][1]) + hred[tid >> 7][2]) + hred[tid >> 7][3];
+      }
     }
   }
-  if (warp < 8) {
-    habs = warp_sum(habs);
-    if (lane == 0) hred[g][warp & 3] = habs;
-  }
-  if (__syncthreads_or(aborted)) aborted = true;
-  if (tid == 0 || tid == 128) {
-    const int qt128 = pair * 2 + (tid >> 7);
-    if (qt128 < p.n_qt)
-      p.head_part[(static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128] =
-          ((hred[tid >> 7][0] + hred[tid >> 7][1]) + hred[tid >> 7][2]) + hred[tid >> 7][3];
-  }
-  if (tid == 0 && aborted) report(a.dev_status, SPATTEN_E_TIMEOUT);
+  if (__syncthreads_or(aborted) && tid == 0) report(a.dev_status, SPATTEN_E_TIMEOUT);
   tc_before_sync();
   __syncthreads();
   if (warp == 11) {
     tc_after_sync();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// zero-filled outputs of the pruned heads (slots H_kept .. H-1): one CTA per (slot, sequence)
+template <int DH>
+__global__ void __launch_bounds__(256) attn_zero_heads_kernel(AttnProblem p) {
+  const spatten_attn_args& a = p.a;
+  const int slot = a.H_kept + blockIdx.x, b = blockIdx.y;
+  const int h = head_of_slot(a, b, slot);
+  if (h < 0) return;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+  for (int e = threadIdx.x; e < a.n_q * (DH / 8); e += blockDim.x) {
+    const int i = e / (DH / 8), c8 = e % (DH / 8);
+    *reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8) =
+        make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -1077,9 +1119,14 @@ int32_t launch(const AttnProblem& p, cudaStream_t st) {
                                   static_cast<int>(FullCfg<DH>::kSmem)));
     configured[dev] = true;
   }
-  const int slots = p.a.H_kept + (p.a.zero_pruned_heads ? p.a.H - p.a.H_kept : 0);
-  attn_main_kernel<DH><<<dim3(p.n_pair, slots, p.a.B), 384, MainCfg<DH>::kSmem, st>>>(p);
+  const int64_t items = static_cast<int64_t>(p.n_pair) * p.a.H_kept * p.a.B;
+  const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
+  attn_main_kernel<DH><<<grid, 384, MainCfg<DH>::kSmem, st>>>(p);
   SPT_TRY(launch_status());
+  if (p.a.zero_pruned_heads && p.a.H_kept < p.a.H) {
+    attn_zero_heads_kernel<DH><<<dim3(p.a.H - p.a.H_kept, p.a.B), 256, 0, st>>>(p);
+    SPT_TRY(launch_status());
+  }
   if (p.a.refetch_threshold > 0.0f) {
     attn_full_kernel<DH><<<dim3(p.n_qt, p.a.H_kept, p.a.B), 256, FullCfg<DH>::kSmem, st>>>(p);
     SPT_TRY(launch_status());
