@@ -82,7 +82,9 @@ def attention_case(B, H, n, d, theta, boost, kernel, reps, n_kv=None):
 def topk_case(R, n, k, dist, reps):
     x = torch.from_numpy(synth.draw_topk_row_block(R, n, dist, 0.01, seed=3)).cuda()
     out = torch.empty((R, max(k, 1)), dtype=torch.int32, device="cuda")
-    ms = _time(lambda: S.topk_select(x, R, n, n, k, out, max(k, 1)), reps)
+    nb = S.topk_workspace_size(R, n, k)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+    ms = _time(lambda: S.topk_select(x, R, n, n, k, out, max(k, 1), ws=ws, ws_bytes=nb), reps)
     byts = R * (4.0 * n + 4.0 * k)
     return dict(case="topk", R=R, n=n, k=k, dist=dist, ms=ms, bytes=byts, gbs=byts / ms / 1e6)
 

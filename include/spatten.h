@@ -207,6 +207,13 @@ int32_t spatten_attention_layer_noalloc(const spatten_attn_args* a, void* stream
  *  comp_out device int32 [R][ld_out] or NULL: map[r][idx_out[r][c]] (index-map composition);
  *           requires map.
  *  Requirements: R >= 1, 1 <= n, 0 <= k <= n, ld >= n when map is NULL, ld_out >= k.
+ *  Workspace (ws, ws_bytes): optional, device memory of spatten_topk_workspace_size(R, n, k)
+ *  bytes (0 for rows shorter than 65,536 keys).  Given it, rows of at least 65,536 keys read
+ *  directly (map NULL, scores 16-byte aligned, ld a multiple of 4) take a two-pass streaming path:
+ *  a 16 K-key sample brackets the k-th key, one pass counts the keys above the bracket and collects
+ *  the bracket's keys, the exact threshold is chosen among them, one pass writes the output; rows
+ *  whose bracket misses fall back to the cluster radix select.  Without it (or with fewer bytes)
+ *  every row takes the cluster radix select.  Results are identical either way.
  * ============================================================================================= */
 size_t spatten_topk_workspace_size(int32_t R, int32_t n, int32_t k);
 int32_t spatten_topk_select(const float* scores, int32_t R, int32_t n, int64_t ld, int32_t k,

@@ -162,15 +162,19 @@ def test_quantize_append_with_scale_saturates(cuda):
 # ------------------------------------------------------------------------------------------------
 # K4 top-k
 # ------------------------------------------------------------------------------------------------
-def _topk_gpu(S, scores_np, k, map_np=None):
+def _topk_gpu(S, scores_np, k, map_np=None, with_ws=True):
+    """with_ws: pass the optional workspace (spatten_topk_workspace_size), which lets long direct
+    rows take the streaming path."""
     R_, n = scores_np.shape if map_np is None else map_np.shape
     sc = to_dev(scores_np)
     out = torch.full((R_, max(k, 1)), -1, dtype=torch.int32, device="cuda")
     comp = torch.full((R_, max(k, 1)), -1, dtype=torch.int32, device="cuda") if map_np is not None else None
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     mp = to_dev(map_np, torch.int32) if map_np is not None else None
+    nb = S.topk_workspace_size(R_, n, k) if with_ws else 0
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
     S.topk_select(sc, R_, n, scores_np.shape[1], k, out, max(k, 1), map=mp, ld_map=n if mp is not None else 0,
-                  comp_out=comp, dev_status=st)
+                  comp_out=comp, ws=ws, ws_bytes=nb, dev_status=st)
     torch.cuda.synchronize()
     return out.cpu().numpy()[:, :k], (comp.cpu().numpy()[:, :k] if comp is not None else None), int(st.item())
 
@@ -251,6 +255,27 @@ def test_topk_sweep_full_size(cuda, N, dist):
             kth = np.partition(x[r], N - k)[N - k]
             sel_vals = x[r][got[r]]
             assert np.all(sel_vals >= kth) and np.count_nonzero(x[r] > kth) <= k
+
+
+@pytest.mark.parametrize("with_ws", [True, False])
+def test_topk_long_rows_bracket_misses_fall_back(cuda, with_ws):
+    """Long rows on the streaming path (with the workspace) where the sample bracket cannot hold the
+    k-th key -- all-equal rows, five distinct values, a row sorted by index -- are redone by the
+    cluster kernel; ordinary rows in the same call stay on the streaming path.  Without the
+    workspace every row takes the cluster kernel.  All rows bit-exact."""
+    S = lib()
+    g = synth.rng_for(77)
+    R_, n = 6, 70001
+    x = g.random((R_, n)).astype(np.float32)
+    x[1] = 2.5                                                     # all equal
+    x[3] = (g.integers(0, 5, n) * 0.5).astype(np.float32)         # five distinct values
+    x[4] = np.linspace(-1.0, 1.0, n, dtype=np.float32)            # sorted by index
+    x[5, ::3] = -x[5, ::3]                                         # mixed signs
+    for k in (1, 7000, 35000, n - 1):
+        got, _, st = _topk_gpu(S, x, k, with_ws=with_ws)
+        assert st == 0
+        for r in range(R_):
+            np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
 
 
 # ------------------------------------------------------------------------------------------------
