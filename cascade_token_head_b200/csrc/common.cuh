@@ -99,11 +99,12 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
-// Order-preserving map float -> uint32 (larger float -> larger key); -0.0 maps like +0.0.
+// Order-preserving map float -> uint32 (larger float -> larger key); -0.0 maps like +0.0 (adding
+// +0.0 turns -0.0 into +0.0 and leaves every other non-NaN value as it is).  Negative values take
+// all bits flipped, the others the sign bit set.
 __device__ __forceinline__ uint32_t float_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const uint32_t u = __float_as_uint(f + 0.0f);
+  return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 
 }  // namespace spt

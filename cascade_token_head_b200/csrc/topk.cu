@@ -490,31 +490,48 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 }
 
 // ------------------------------------------------------------------------------------------------
-// Long rows (n >= kStreamMin, scores read directly, caller workspace given): two streaming passes.
-//  sample   one CTA per row sorts 16 K keys (64 evenly spaced runs of 256) and takes, around the
-//           sample rank of the k-th key (+-4 sigma of the sampling error + 16), a bracket
-//           [e64, e0] cut into 64 sub-bins at sample quantiles e0 >= e1 >= ... >= e64
-//  filter   per chunk of 16 K keys: the count above e0, a histogram of the bracket's keys over the
-//           sub-bins, and the bracket's keys (key, index) appended to the row's candidate buffer
-//  resolve  one CTA per row: the sub-bin holding the k-th key, the exact threshold among that
-//           sub-bin's candidates as the (need)-th largest of (key, ~index) (ties to the lower
-//           index), and every chunk's output offset
+// Long rows (n >= kStreamMin, scores read directly, caller workspace given): two streaming passes
+// over the scores, with two one-CTA-per-row steps on small data between them.
+//  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256), finds by a digit search
+//           the sample keys at the two ends of a rank window around the sample rank of the k-th
+//           key (+-4 sigma of the sampling error + 16), and sorts the few sample keys strictly
+//           inside; 65 edges e0 >= e1 >= ... >= e64 at evenly spaced ranks of the window follow.
+//           The digit search runs first on one key in 16, whose window (widened by its own
+//           sampling error) bounds the few thousand sample keys the exact search then needs
+//  filter   per chunk of 8 K keys: the count above e0, and the keys in [e64, e0] appended as
+//           (key, index) to the row's candidate list
+//  resolve  one CTA per row: a histogram of the candidates over the 64 sub-bins between the
+//           edges, the sub-bin holding the k-th key, the exact threshold among that sub-bin's
+//           candidates as the (need)-th largest (key, ~index) composite (ties to the lower index),
+//           and every chunk's output offset
 //  output   per chunk: key > T, or key = T and index <= T_index, written in index order
-// A row whose k-th key fell outside the bracket, or whose buffers overflowed, is marked and done
-// again by the cluster kernel (only_rows).
+// A row whose k-th key fell outside the window's edges, or whose buffers overflowed, is marked and
+// done again by the cluster kernel (only_rows).
+// Filter and output read a warp's 512 keys as four coalesced 16-byte loads per lane (load q of
+// lane t holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span), so a key's place in index
+// order is (warp, q, lane, element).  They compare floats against the edges and the threshold
+// turned back into floats (the key map is monotone, and -0.0 equals +0.0 on both sides); a NaN
+// fails every ordered comparison, lands in the candidate list and is reported by the resolve step.
 // ------------------------------------------------------------------------------------------------
 constexpr int kStreamMin = 65536;
 constexpr int kSRuns = 64, kSRun = 256, kSamples = kSRuns * kSRun;   // 16 K sample keys per row
 constexpr int kBins = 64;
-constexpr int kChunk = 16384;                                           // keys per filter/output CTA
-constexpr int kCThreads2 = 512;                                         // threads of filter/output
+constexpr int kRThreads = 1024;                                         // sample and resolve CTAs
+constexpr int kFThreads = 512;                                          // filter and output CTAs
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kFKeys = 16;                                              // keys per filter/output lane
+constexpr int kChunk = kFThreads * kFKeys;                              // 8 K keys per filter/output CTA
 constexpr int kBinCap = 8192;                                           // candidates of one sub-bin
+constexpr int kWindow = 1024;                                           // sample keys inside the window
+constexpr int kL1 = 1024;                                               // first-level sample keys
+constexpr int kSList = 4096;                                            // second-level sample keys
+constexpr int kMaxChunks = 8192;
 
 struct StreamWs {
   uint32_t* edges;      // [R][kBins + 1]
-  uint32_t* hist;       // [R][kBins]           (zeroed per call)
-  uint32_t* ccount;     // [R]                   (zeroed per call)
+  uint32_t* ccount;     // [R]        candidates appended (zeroed by the sample kernel)
   uint32_t* chunk_gt;   // [R][nchunk]
+  uint32_t* hist;       // [R][nchunk][kBins]   candidates of each chunk per sub-bin
   uint2* cand;          // [R][cap]  (key, index)
   uint32_t* chunk_off;  // [R][nchunk]
   uint32_t* res;        // [R][4]   valid, T key, T index
@@ -522,60 +539,346 @@ struct StreamWs {
   int cap, nchunk;
 };
 
+// float of a key (the inverse of float_key); the keys of NaNs, which only the window's special
+// ends use, give +-infinity
+__device__ __forceinline__ float key_float(uint32_t k) {
+  if (k > 0xFF800000u) return __int_as_float(0x7F800000);
+  if (k <= 0x007FFFFFu) return __int_as_float(static_cast<int>(0xFF800000u));
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
+__device__ __forceinline__ bool key_is_nan(uint32_t k) { return k > 0xFF800000u || k < 0x007FFFFFu; }
+
 __device__ __forceinline__ int bin_of(uint32_t key, const uint32_t* e) {
-  // number of edges e1..e63 at or above key (edges descending): bin j holds e[j+1] < key <= e[j],
+  // the largest j in [0, 63] with e[j] >= key (edges descending): bin j holds e[j+1] < key <= e[j],
   // the last bin also key == e64
-  int lo = 0, hi = kBins - 1;   // answer in [0, 63]
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (e[mid] >= key) lo = mid;
-    else hi = mid - 1;
-  }
+  int lo = 0;
+#pragma unroll
+  for (int s = kBins / 2; s > 0; s >>= 1)
+    if (e[lo + s] >= key) lo += s;
   return lo;
 }
 
-__global__ void __launch_bounds__(1024) topk_sample_kernel(TArgs a, StreamWs w) {
-  extern __shared__ __align__(16) uint32_t sk[];   // kSamples keys
-  const int r = blockIdx.x, tid = threadIdx.x;
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  for (int e = tid; e < kSamples; e += 1024) {
-    const int run = e / kSRun, o = e % kSRun;
-    const int64_t pos = static_cast<int64_t>(run) * (a.n - kSRun) / (kSRuns - 1) + o;
-    sk[e] = float_key(__ldg(row + pos));
-  }
-  __syncthreads();
-  // bitonic sort, descending
-  for (int size = 2; size <= kSamples; size <<= 1) {
+// bitonic sort of one value per thread over a 1024-thread block, descending (thread t ends with
+// sorted position t); partners closer than a warp exchange by shuffles, the others through
+// `scratch` [1024]; every thread must call it, and scratch is free again after a block barrier
+template <typename V>
+__device__ __forceinline__ V bitonic_desc_1024(V x, V* scratch) {
+  const int tid = threadIdx.x;
+  for (int size = 2; size <= 1024; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < kSamples / 2; i += 1024) {
-        const int lo = 2 * stride * (i / stride) + (i % stride), hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint32_t x = sk[lo], y = sk[hi];
-        if (desc ? (x < y) : (x > y)) {
-          sk[lo] = y;
-          sk[hi] = x;
-        }
+      V y;
+      if (stride >= 32) {
+        __syncthreads();
+        scratch[tid] = x;
+        __syncthreads();
+        y = scratch[tid ^ stride];
+      } else {
+        y = __shfl_xor_sync(0xffffffffu, x, stride);
       }
-      __syncthreads();
+      const bool lower = (tid & stride) == 0, desc = (tid & size) == 0;
+      const bool take_max = lower == desc;
+      x = take_max ? (x > y ? x : y) : (x < y ? x : y);
     }
   }
+  return x;
+}
+
+struct SampleSmem {
+  uint32_t red[2][3][32];
+  uint32_t win[kWindow];
+  uint32_t cnt[32];
+  uint32_t list[kSList];
+  int rank[kBins + 1];
+  int open[2];
+  int l1[2];          // first-level ranks of the outer bounds (< 0 / >= kL1: no bound)
+  uint32_t n_in, n_list;
+};
+
+// ta / tb = the need_a-th / need_b-th largest of the NK keys per thread (block-wide; padding keys
+// are 0 and never counted): the largest T with count(>= T) >= need, two bits per round; counts fit
+// 16 bits (at most 16 K), two per word.  While the two share their high bits one set of three
+// counts serves both.
+template <int NK>
+__device__ __forceinline__ void search2(const uint32_t* key, uint32_t need_a, uint32_t need_b, SampleSmem& sm,
+                                        uint32_t& ta, uint32_t& tb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  ta = 0u;
+  tb = 0u;
+  int rnd = 0;
+#pragma unroll 1
+  for (int b = 30; b >= 0; b -= 2, ++rnd) {
+    const bool same = ta == tb;   // uniform
+    const uint32_t a1 = ta | (1u << b), a2 = ta | (2u << b), a3 = ta | (3u << b);
+    const uint32_t b1 = tb | (1u << b), b2 = tb | (2u << b), b3 = tb | (3u << b);
+    uint32_t x = 0u, y = 0u, z = 0u;
+    if (same) {
+#pragma unroll
+      for (int i = 0; i < NK; ++i) {
+        x += (key[i] >= a1 ? 1u : 0u) + (key[i] >= a2 ? 0x10000u : 0u);
+        y += key[i] >= a3 ? 1u : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NK; ++i) {
+        x += (key[i] >= a1 ? 1u : 0u) + (key[i] >= a2 ? 0x10000u : 0u);
+        y += (key[i] >= a3 ? 1u : 0u) + (key[i] >= b1 ? 0x10000u : 0u);
+        z += (key[i] >= b2 ? 1u : 0u) + (key[i] >= b3 ? 0x10000u : 0u);
+      }
+    }
+    x = __reduce_add_sync(0xffffffffu, x);
+    y = __reduce_add_sync(0xffffffffu, y);
+    z = __reduce_add_sync(0xffffffffu, z);
+    if (lane == 0) {
+      sm.red[rnd & 1][0][warp] = x;
+      sm.red[rnd & 1][1][warp] = y;
+      sm.red[rnd & 1][2][warp] = z;
+    }
+    __syncthreads();
+    x = __reduce_add_sync(0xffffffffu, sm.red[rnd & 1][0][lane]);
+    y = __reduce_add_sync(0xffffffffu, sm.red[rnd & 1][1][lane]);
+    z = __reduce_add_sync(0xffffffffu, sm.red[rnd & 1][2][lane]);
+    const uint32_t n1 = x & 0xFFFFu, n2 = x >> 16, n3 = y & 0xFFFFu;
+    ta |= static_cast<uint32_t>((n1 >= need_a) + (n2 >= need_a) + (n3 >= need_a)) << b;
+    if (same) tb |= static_cast<uint32_t>((n1 >= need_b) + (n2 >= need_b) + (n3 >= need_b)) << b;
+    else tb |= static_cast<uint32_t>(((y >> 16) >= need_b) + ((z & 0xFFFFu) >= need_b) + ((z >> 16) >= need_b)) << b;
+  }
+}
+
+// append the keys with in == true to `list` (warp-aggregated slots; at most cap kept)
+__device__ __forceinline__ void append_keys(bool in, uint32_t key, uint32_t* list, uint32_t* n, uint32_t cap) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t m = __ballot_sync(0xffffffffu, in);
+  if (m) {
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0u;
+    if (lane == leader) base = atomicAdd(n, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    const uint32_t s = base + __popc(m & ((1u << lane) - 1u));
+    if (in && s < cap) list[s] = key;
+  }
+}
+
+// the 65 edges from the NK keys per thread, which hold every sample key ranked in the window;
+// `base` more sample keys lie above all of them
+template <int NK>
+__device__ __forceinline__ void window_edges(const uint32_t* key, uint32_t base, SampleSmem& sm, int r, StreamWs& w) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t need_a = static_cast<uint32_t>(sm.rank[0]) + 1u - base;
+  const uint32_t need_b = static_cast<uint32_t>(sm.rank[kBins]) + 1u - base;
+  uint32_t ta, tb;
+  search2<NK>(key, need_a, need_b, sm, ta, tb);
+  // ge_a = #(key >= ta), gt_b = #(key > tb); the keys strictly between go to the window list
+  uint32_t c = 0u;
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    c += (key[i] >= ta ? 1u : 0u) + (key[i] > tb ? 0x10000u : 0u);
+    append_keys(key[i] > tb && key[i] < ta, key[i], sm.win, &sm.n_in, kWindow);
+  }
+  c = __reduce_add_sync(0xffffffffu, c);
+  if (lane == 0) sm.cnt[warp] = c;
+  __syncthreads();
+  c = __reduce_add_sync(0xffffffffu, sm.cnt[lane]);
+  const int ge_a = static_cast<int>(base + (c & 0xFFFFu)), gt_b = static_cast<int>(base + (c >> 16));
+  // padding below every key strictly inside the window (those exceed its low end)
+  const uint32_t x = bitonic_desc_1024(tid < static_cast<int>(sm.n_in) ? sm.win[tid] : 0u, sm.win);
+  __syncthreads();
+  sm.win[tid] = x;
+  __syncthreads();
   if (tid <= kBins) {
+    // sorted sample position rho holds ta for rho < ge_a (rho >= the rank of ta), tb for
+    // rho >= gt_b (rho <= the rank of tb), else window key rho - ge_a
+    const int rho = sm.rank[tid];
+    uint32_t e;
+    if (tid == 0 && sm.open[0]) e = 0xFFFFFFFFu;
+    else if (tid == kBins && sm.open[1]) e = 0u;
+    else if (rho < ge_a) e = ta;
+    else if (rho >= gt_b) e = tb;
+    else e = sm.win[min(rho - ge_a, kWindow - 1)];
+    w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid] = e;
+  }
+}
+
+__global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamWs w) {
+  constexpr int KPT = kSamples / kRThreads;   // 16 sample keys per thread
+  static_assert(kWindow == kRThreads && kL1 == kRThreads, "one window slot and one first-level key per thread");
+  __shared__ SampleSmem sm;
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  // thread t reads 16 consecutive keys of run t / 16 (runs start on a 16-byte boundary)
+  uint32_t key[KPT];
+  {
+    const int run = tid / (kSRun / KPT);
+    const int64_t pos = ((static_cast<int64_t>(run) * (a.n - kSRun) / (kSRuns - 1)) & ~int64_t(3)) +
+                        (tid % (kSRun / KPT)) * KPT;
+#pragma unroll
+    for (int q = 0; q < KPT / 4; ++q) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + pos) + q);
+      key[4 * q] = float_key(v.x);
+      key[4 * q + 1] = float_key(v.y);
+      key[4 * q + 2] = float_key(v.z);
+      key[4 * q + 3] = float_key(v.w);
+    }
+  }
+  if (tid == 0) {
+    sm.n_in = 0u;
+    sm.n_list = 0u;
+    w.ccount[r] = 0u;
+  }
+  if (tid <= kBins) {
+    // sample ranks of the edges: the window [r_hi, r_lo] around k/n of the sample, cut in 64 steps;
+    // its half-width is at most 4 sqrt(kSamples / 4) + 16 = 272, so at most 544 sample keys lie
+    // strictly between its ends
     const double p = static_cast<double>(a.k) / a.n;
     const double kp = p * kSamples;
     const double delta = 4.0 * sqrt(kSamples * p * (1.0 - p)) + 16.0;
     const double r_hi = kp - delta, r_lo = kp + delta;
     const double rank = r_hi + tid * (r_lo - r_hi) / kBins;
-    const int ri = static_cast<int>(floor(rank));
-    uint32_t e;
-    if (tid == 0 && r_hi < 0.0) e = 0xFFFFFFFFu;
-    else if (tid == kBins && r_lo >= kSamples - 1) e = 0u;
-    else e = sk[min(max(ri, 0), kSamples - 1)];
-    w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid] = e;
+    const int rho = min(max(static_cast<int>(floor(rank)), 0), kSamples - 1);
+    sm.rank[tid] = rho;
+    if (tid == 0) sm.open[0] = r_hi < 0.0;
+    if (tid == kBins) sm.open[1] = r_lo >= kSamples - 1;
+    // first level: one sample key in 16; its keys at the window ends' ranks, moved outwards by 4
+    // sigma of their own rank error (in first-level ranks) + 8, bound a second-level set that holds
+    // the window
+    const int m1 = static_cast<int>(ceil(4.0 * sqrt(kL1 * p * (1.0 - p)) + 8.0));
+    constexpr int kStep = kSamples / kL1;
+    if (tid == 0) sm.l1[0] = rho / kStep - m1;
+    if (tid == kBins) sm.l1[1] = (rho + kStep - 1) / kStep + m1;
+  }
+  __syncthreads();
+  // the first level: each thread's first key, 16 per run
+  uint32_t k1 = key[0];
+  const int l1a = sm.l1[0], l1b = sm.l1[1];
+  uint32_t ca, cb;
+  search2<1>(&k1, static_cast<uint32_t>(max(l1a, 0)) + 1u, static_cast<uint32_t>(min(l1b, kL1 - 1)) + 1u, sm, ca, cb);
+  if (l1a < 0) ca = 0xFFFFFFFFu;
+  if (l1b >= kL1) cb = 0u;
+  // the bound holds if at most rank[0] sample keys exceed ca and at least rank[64] + 1 reach cb
+  uint32_t c = 0u;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) c += (key[i] > ca ? 1u : 0u) + (key[i] >= cb ? 0x10000u : 0u);
+  c = __reduce_add_sync(0xffffffffu, c);
+  if (lane == 0) sm.cnt[warp] = c;
+  __syncthreads();
+  c = __reduce_add_sync(0xffffffffu, sm.cnt[lane]);
+  const uint32_t gt_ca = c & 0xFFFFu, ge_cb = c >> 16;
+  const bool narrow = gt_ca <= static_cast<uint32_t>(sm.rank[0]) && ge_cb >= static_cast<uint32_t>(sm.rank[kBins]) + 1u &&
+                      ge_cb - gt_ca <= static_cast<uint32_t>(kSList);   // uniform
+  if (narrow) {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) append_keys(key[i] >= cb && key[i] <= ca, key[i], sm.list, &sm.n_list, kSList);
+    __syncthreads();
+    constexpr int NL = kSList / kRThreads;
+    uint32_t s[NL];
+    const uint32_t nl = sm.n_list;
+#pragma unroll
+    for (int u = 0; u < NL; ++u) s[u] = tid + u * kRThreads < static_cast<int>(nl) ? sm.list[tid + u * kRThreads] : 0u;
+    window_edges<NL>(s, gt_ca, sm, r, w);
+  } else {
+    window_edges<KPT>(key, 0u, sm, r, w);
   }
 }
 
-// block-wide exclusive scan for 512-thread CTAs (scratch [16])
-__device__ __forceinline__ uint32_t scan512(uint32_t v, uint32_t* wt, uint32_t& total) {
+// the kFKeys scores of one filter/output lane (see the layout note above); FULL: the whole span
+// lies inside the row
+template <bool FULL>
+__device__ __forceinline__ void load_span(const float* row, int jw, int n, float* f) {
+#pragma unroll
+  for (int q = 0; q < kFKeys / 4; ++q) {
+    const int j = jw + 128 * q;
+    if (FULL || j + 3 < n) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
+      f[4 * q] = v.x; f[4 * q + 1] = v.y; f[4 * q + 2] = v.z; f[4 * q + 3] = v.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f[4 * q + u] = j + u < n ? row[j + u] : 0.0f;
+    }
+  }
+}
+
+__device__ __forceinline__ int span_off(int u) { return 128 * (u >> 2) + (u & 3); }
+
+// count above fe0 and the candidate mask (bit u: f[u] in [fe64, fe0], or NaN)
+template <bool FULL>
+__device__ __forceinline__ void filter_span(const float* row, int jw, int n, float fe0, float fe64, uint32_t& gt,
+                                            uint32_t& cm) {
+  float f[kFKeys];
+  load_span<FULL>(row, jw, n, f);
+  gt = 0u;
+  cm = 0u;
+#pragma unroll
+  for (int u = 0; u < kFKeys; ++u) {
+    if (FULL || span_off(u) < n - jw) {
+      gt += f[u] > fe0 ? 1u : 0u;
+      if (!(f[u] < fe64 || f[u] > fe0)) cm |= 1u << u;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, StreamWs w) {
+  __shared__ uint32_t wc[kFWarps], wg[kFWarps], wb[kFWarps];
+  __shared__ uint32_t e_s[kBins + 1], hist[kBins];
+  const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid <= kBins) e_s[tid] = w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid];
+  if (tid < kBins) hist[tid] = 0u;
+  const float fe0 = key_float(w.edges[static_cast<int64_t>(r) * (kBins + 1)]);
+  const float fe64 = key_float(w.edges[static_cast<int64_t>(r) * (kBins + 1) + kBins]);
+  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
+  const int jw = c * kChunk + warp * (32 * kFKeys) + 4 * lane;
+  uint32_t gt, cm;
+  if ((c + 1) * kChunk <= a.n) filter_span<true>(row, jw, a.n, fe0, fe64, gt, cm);
+  else filter_span<false>(row, jw, a.n, fe0, fe64, gt, cm);
+  const uint32_t nc = __popc(cm);
+  uint32_t inc = nc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  if (lane == 31) wc[warp] = inc;
+  if (lane == 0) wg[warp] = gt;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t x = lane < kFWarps ? wc[lane] : 0u;
+    uint32_t xi = x;
+#pragma unroll
+    for (int o = 1; o < kFWarps; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += t;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, xi, kFWarps - 1);
+    const uint32_t g = __reduce_add_sync(0xffffffffu, lane < kFWarps ? wg[lane] : 0u);
+    uint32_t base = 0u;
+    if (lane == 0) {
+      w.chunk_gt[static_cast<int64_t>(r) * w.nchunk + c] = g;
+      if (tot) base = atomicAdd(&w.ccount[r], tot);
+    }
+    base = __shfl_sync(0xffffffffu, base, 0);
+    // a chunk whose candidates would pass the list's end writes none (the row falls back)
+    if (lane < kFWarps) wb[lane] = base + tot <= static_cast<uint32_t>(w.cap) ? base + xi - x : 0xFFFFFFFFu;
+  }
+  __syncthreads();
+  const uint32_t wbase = wb[warp];
+  if (wbase != 0xFFFFFFFFu) {
+    uint2* dst = w.cand + static_cast<int64_t>(r) * w.cap + wbase + (inc - nc);
+    // each candidate's score read again (an L1 hit) rather than held across the barriers
+    uint32_t i = 0u;
+    for (uint32_t mm = cm; mm; mm &= mm - 1u, ++i) {
+      const int u = __ffs(mm) - 1;
+      const int j = jw + 128 * (u >> 2) + (u & 3);
+      const uint32_t key = float_key(row[j]);
+      dst[i] = make_uint2(key, static_cast<uint32_t>(j));
+      atomicAdd(&hist[bin_of(key, e_s)], 1u);
+    }
+  }
+  __syncthreads();
+  if (tid < kBins) w.hist[(static_cast<int64_t>(r) * w.nchunk + c) * kBins + tid] = hist[tid];
+}
+
+// exclusive prefix sum over a 1024-thread block (part: [32] scratch, free again after return)
+__device__ __forceinline__ uint32_t scan1024(uint32_t v, uint32_t* part, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t inc = v;
 #pragma unroll
@@ -583,200 +886,208 @@ __device__ __forceinline__ uint32_t scan512(uint32_t v, uint32_t* wt, uint32_t& 
     const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
     if (lane >= o) inc += t;
   }
-  if (lane == 31) wt[warp] = inc;
+  if (lane == 31) part[warp] = inc;
   __syncthreads();
-  if (warp == 0) {
-    uint32_t x = lane < 16 ? wt[lane] : 0u;
+  const uint32_t p = part[lane];
+  uint32_t pi = p;
 #pragma unroll
-    for (int o = 1; o < 16; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += t;
-    }
-    if (lane < 16) wt[lane] = x;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, pi, o);
+    if (lane >= o) pi += t;
   }
+  total = __shfl_sync(0xffffffffu, pi, 31);
+  const uint32_t before = __shfl_sync(0xffffffffu, pi - p, warp);
   __syncthreads();
-  total = wt[15];
-  const uint32_t pre = (warp > 0 ? wt[warp - 1] : 0u) + inc - v;
-  __syncthreads();   // wt is reused by the caller's next scan
-  return pre;
+  return before + inc - v;
 }
 
-__global__ void __launch_bounds__(kCThreads2) topk_filter_kernel(TArgs a, StreamWs w) {
-  __shared__ uint32_t e[kBins + 1];
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t wt[16];
-  __shared__ uint32_t base_s;
-  const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x;
-  if (tid <= kBins) e[tid] = w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid];
-  if (tid < kBins) hist[tid] = 0u;
-  __syncthreads();
-  const uint32_t e0 = e[0], e64 = e[kBins];
-  const int64_t j0 = static_cast<int64_t>(c) * kChunk;
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  // 32 keys per thread, coalesced: float4 q of thread t covers keys j0 + 4 (q * 512 + t) ..
-  uint32_t key[32];
-  int nan_local = 0;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int64_t j = j0 + 4 * (static_cast<int64_t>(q) * kCThreads2 + tid);
-    float f[4];
-    if (j + 3 < a.n) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
-      f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-    } else {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) f[u] = j + u < a.n ? row[j + u] : 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      nan_local |= f[u] != f[u];
-      key[4 * q + u] = j + u < a.n ? float_key(f[u]) : 0u;   // 0: below every bracket (e64 >= 0 ...)
-    }
-  }
-  uint32_t gt = 0u, nc = 0u;
-#pragma unroll
-  for (int u = 0; u < 32; ++u) {
-    const int64_t j = j0 + 4 * (static_cast<int64_t>(u >> 2) * kCThreads2 + tid) + (u & 3);
-    const bool valid = j < a.n;
-    gt += (valid && key[u] > e0) ? 1u : 0u;
-    const bool cand = valid && key[u] <= e0 && key[u] >= e64;
-    if (cand) {
-      atomicAdd(&hist[bin_of(key[u], e)], 1u);
-      ++nc;
-    }
-  }
-  uint32_t tot_gt, tot_c;
-  scan512(gt, wt, tot_gt);
-  const uint32_t pre = scan512(nc, wt, tot_c);
-  if (tid == 0) {
-    w.chunk_gt[static_cast<int64_t>(r) * w.nchunk + c] = tot_gt;
-    base_s = tot_c ? atomicAdd(&w.ccount[r], tot_c) : 0u;
-  }
-  __syncthreads();
-  if (tid < kBins && hist[tid]) atomicAdd(&w.hist[static_cast<int64_t>(r) * kBins + tid], hist[tid]);
-  if (nan_local) report(a.status, SPATTEN_E_NONFINITE);
-  const uint32_t base = base_s;
-  if (base + tot_c <= static_cast<uint32_t>(w.cap) && nc) {
-    uint2* dst = w.cand + static_cast<int64_t>(r) * w.cap + base + pre;
-    uint32_t m = 0u;
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int64_t j = j0 + 4 * (static_cast<int64_t>(u >> 2) * kCThreads2 + tid) + (u & 3);
-      if (j < a.n && key[u] <= e0 && key[u] >= e64) dst[m++] = make_uint2(key[u], static_cast<uint32_t>(j));
-    }
+__device__ __forceinline__ void stream_fail(StreamWs& w, int r) {
+  if (threadIdx.x == 0) {
+    w.fallback[r] = 1;
+    w.res[static_cast<int64_t>(r) * 4] = 0u;
   }
 }
 
-__global__ void __launch_bounds__(1024) topk_resolve_kernel(TArgs a, StreamWs w) {
+__global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, StreamWs w) {
+  constexpr int BP = 8;   // (key, index) pairs per thread per batch
   extern __shared__ __align__(16) unsigned char rs_smem[];
   uint64_t* bc = reinterpret_cast<uint64_t*>(rs_smem);                   // [kBinCap] sub-bin candidates
   uint32_t* cnt = reinterpret_cast<uint32_t*>(bc + kBinCap);             // [nchunk]
   __shared__ uint32_t e[kBins + 1];
+  __shared__ uint32_t hist[kBins];
   __shared__ uint32_t red[2][2][32];
-  __shared__ uint32_t n_bc, jstar_s, above_s, ok_s;
-  __shared__ uint32_t gt_part[32];
+  __shared__ uint32_t part[32];
+  __shared__ uint32_t n_bc, js_s, above_s;
+  __shared__ uint64_t t_s;
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid <= kBins) e[tid] = w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid];
-  if (tid == 0) n_bc = 0u;
-  // total above the bracket
+  if (tid < kBins) hist[tid] = 0u;
+  if (tid == 0) {
+    n_bc = 0u;
+    js_s = kBins;   // no sub-bin found: the row falls back
+  }
+  const int nchunk = w.nchunk;
   uint32_t g = 0u;
-  for (int c = tid; c < w.nchunk; c += 1024) {
-    const uint32_t x = w.chunk_gt[static_cast<int64_t>(r) * w.nchunk + c];
+  for (int c = tid; c < nchunk; c += kRThreads) {
+    const uint32_t x = w.chunk_gt[static_cast<int64_t>(r) * nchunk + c];
     cnt[c] = x;
     g += x;
   }
   g = __reduce_add_sync(0xffffffffu, g);
-  if (lane == 0) gt_part[warp] = g;
+  if (lane == 0) part[warp] = g;
   __syncthreads();
-  if (tid == 0) {
-    uint32_t total_gt = 0u;
-    for (int i = 0; i < 32; ++i) total_gt += gt_part[i];
-    const uint32_t ncand = w.ccount[r];
-    const uint32_t k = static_cast<uint32_t>(a.k);
-    uint32_t ok = ncand <= static_cast<uint32_t>(w.cap) && total_gt < k && k <= total_gt + ncand;
-    uint32_t acc = total_gt, js = kBins;
-    if (ok) {
-      for (int j = 0; j < kBins; ++j) {
-        const uint32_t hj = w.hist[static_cast<int64_t>(r) * kBins + j];
-        if (acc + hj >= k) { js = j; break; }
-        acc += hj;
-      }
-      if (js == kBins || w.hist[static_cast<int64_t>(r) * kBins + js] > kBinCap) ok = 0u;
-    }
-    jstar_s = js;
-    above_s = acc;
-    ok_s = ok;
-  }
-  __syncthreads();
+  const uint32_t total_gt = __reduce_add_sync(0xffffffffu, part[lane]);
   const uint32_t ncand = w.ccount[r];
-  if (!ok_s) {   // uniform
-    if (tid == 0) {
-      w.fallback[r] = 1;
-      w.res[static_cast<int64_t>(r) * 4] = 0u;
-    }
+  const uint32_t k = static_cast<uint32_t>(a.k);
+  if (!(ncand <= static_cast<uint32_t>(w.cap) && total_gt < k && k <= total_gt + ncand)) {   // uniform
+    stream_fail(w, r);
     return;
   }
-  // the sub-bin's candidates as (key, ~index) composites
-  const int js = static_cast<int>(jstar_s);
-  const uint2* cand = w.cand + static_cast<int64_t>(r) * w.cap;
-  for (uint32_t i = tid; i < ncand; i += 1024) {
-    const uint2 cd = cand[i];
-    if (bin_of(cd.x, e) == js) {
-      const uint32_t slot = atomicAdd(&n_bc, 1u);
-      if (slot < kBinCap) bc[slot] = (static_cast<uint64_t>(cd.x) << 32) | static_cast<uint64_t>(~cd.y);
+  // sub-bin totals from the chunks' histograms (thread: one sub-bin, every 16th chunk)
+  const uint32_t* h = w.hist + static_cast<int64_t>(r) * nchunk * kBins;
+  {
+    const int j = tid & (kBins - 1), cg = tid / kBins;
+    uint32_t s = 0u;
+#pragma unroll 4
+    for (int c = cg; c < nchunk; c += kRThreads / kBins) s += h[static_cast<int64_t>(c) * kBins + j];
+    if (s) atomicAdd(&hist[j], s);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // the first sub-bin whose cumulative count reaches need = k - total_gt (>= 1; the sub-bins
+    // hold all ncand >= need candidates, so exactly one lane finds it)
+    const uint32_t need = k - total_gt;
+    const uint32_t h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
+    uint32_t inc = h0 + h1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    const uint32_t ex = inc - h0 - h1;
+    if (ex < need && ex + h0 >= need) {
+      js_s = 2 * lane;
+      above_s = total_gt + ex;
+    } else if (ex + h0 < need && inc >= need) {
+      js_s = 2 * lane + 1;
+      above_s = total_gt + ex + h0;
     }
   }
+  __syncthreads();
+  const int js = static_cast<int>(js_s);
+  if (js >= kBins || hist[js] > static_cast<uint32_t>(kBinCap)) {   // uniform
+    stream_fail(w, r);
+    return;
+  }
+  // the sub-bin's candidates as (key, ~index) composites: e[js+1] < key <= e[js] (the last sub-bin
+  // also key == e64); the one pass over the candidate list, which also looks for NaNs (they pass
+  // the filter)
+  const uint32_t bin_hi = e[js];
+  const uint64_t bin_lo = js == kBins - 1 ? static_cast<uint64_t>(e[kBins]) : static_cast<uint64_t>(e[js + 1]) + 1u;
+  const uint2* cand = w.cand + static_cast<int64_t>(r) * w.cap;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  bool nan_seen = false;
+  for (uint32_t i0 = 0; i0 < ncand; i0 += BP * kRThreads) {
+    uint2 cd[BP];
+#pragma unroll
+    for (int u = 0; u < BP; ++u) {
+      const uint32_t i = i0 + tid + u * kRThreads;
+      cd[u] = i < ncand ? cand[i] : make_uint2(0x80000000u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < BP; ++u) {
+      nan_seen |= key_is_nan(cd[u].x);
+      const bool hit = i0 + tid + u * kRThreads < ncand && cd[u].x <= bin_hi && cd[u].x >= bin_lo;
+      const uint32_t m = __ballot_sync(0xffffffffu, hit);
+      if (m) {
+        const int leader = __ffs(m) - 1;
+        uint32_t base = 0u;
+        if (lane == leader) base = atomicAdd(&n_bc, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        const uint32_t slot = base + __popc(m & lt_mask);
+        if (hit && slot < kBinCap) bc[slot] = (static_cast<uint64_t>(cd[u].x) << 32) | static_cast<uint64_t>(~cd[u].y);
+      }
+    }
+  }
+  if (nan_seen) report(a.status, SPATTEN_E_NONFINITE);
   __syncthreads();
   const uint32_t m = min(n_bc, static_cast<uint32_t>(kBinCap));
-  const uint32_t need = static_cast<uint32_t>(a.k) - above_s;   // 1 <= need <= m
-  uint64_t v[kBinCap / 1024];
-#pragma unroll
-  for (int u = 0; u < kBinCap / 1024; ++u) {
-    const uint32_t i = tid + u * 1024;
-    v[u] = i < m ? bc[i] : 0ull;   // 0 lies below every candidate composite used as a threshold
-  }
-  // T = the need-th largest composite, two bits per round (the largest T with count(>= T) >= need)
-  uint64_t T = 0ull;
-  int rnd = 0;
-#pragma unroll 1
-  for (int b = 62; b >= 0; b -= 2, ++rnd) {
-    const uint64_t c1 = T | (1ull << b), c2 = T | (2ull << b), c3 = T | (3ull << b);
-    uint32_t x = 0u, y = 0u;
-#pragma unroll
-    for (int u = 0; u < kBinCap / 1024; ++u) {
-      x += (v[u] >= c1 ? 1u : 0u) + (v[u] >= c2 ? 0x10000u : 0u);
-      y += v[u] >= c3 ? 1u : 0u;
-    }
-    x = __reduce_add_sync(0xffffffffu, x);
-    y = __reduce_add_sync(0xffffffffu, y);
-    if (lane == 0) {
-      red[rnd & 1][0][warp] = x;
-      red[rnd & 1][1][warp] = y;
-    }
+  const uint32_t need = k - above_s;   // 1 <= need <= m
+  // T = the need-th largest composite; the selected ones of the sub-bin are counted per chunk
+  uint64_t T;
+  if (m <= static_cast<uint32_t>(kRThreads)) {   // uniform: sort the sub-bin
+    uint64_t x = tid < static_cast<int>(m) ? bc[tid] : 0ull;   // 0: below every composite
+    x = bitonic_desc_1024(x, bc);
+    if (tid == static_cast<int>(need) - 1) t_s = x;
+    const bool s = tid < static_cast<int>(need);
+    const uint32_t chunk = s ? (~static_cast<uint32_t>(x)) / kChunk : 0xFFFFFFFFu;
+    const uint32_t grp = __match_any_sync(0xffffffffu, chunk);
+    if (s && lane == __ffs(grp) - 1) atomicAdd(&cnt[chunk], __popc(grp));
     __syncthreads();
-    x = 0u;
-    y = 0u;
+    T = t_s;
+  } else {
+    // two bits per round (the largest T with count(>= T) >= need)
+    uint64_t v[kBinCap / kRThreads];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      x += red[rnd & 1][0][i];
-      y += red[rnd & 1][1][i];
+    for (int u = 0; u < kBinCap / kRThreads; ++u) {
+      const uint32_t i = tid + u * kRThreads;
+      v[u] = i < m ? bc[i] : 0ull;
     }
-    const uint32_t n1 = x & 0xFFFFu, n2 = x >> 16, n3 = y;
-    T |= static_cast<uint64_t>((n1 >= need) + (n2 >= need) + (n3 >= need)) << b;
+    const int nv = static_cast<int>((m + kRThreads - 1) / kRThreads);   // live registers (uniform)
+    T = 0ull;
+    int rnd = 0;
+#pragma unroll 1
+    for (int b = 62; b >= 0; b -= 2, ++rnd) {
+      const uint64_t c1 = T | (1ull << b), c2 = T | (2ull << b), c3 = T | (3ull << b);
+      uint32_t x = 0u, y = 0u;
+#pragma unroll
+      for (int u = 0; u < kBinCap / kRThreads; ++u) {
+        if (u < nv) {
+          x += (v[u] >= c1 ? 1u : 0u) + (v[u] >= c2 ? 0x10000u : 0u);
+          y += v[u] >= c3 ? 1u : 0u;
+        }
+      }
+      x = __reduce_add_sync(0xffffffffu, x);
+      y = __reduce_add_sync(0xffffffffu, y);
+      if (lane == 0) {
+        red[rnd & 1][0][warp] = x;
+        red[rnd & 1][1][warp] = y;
+      }
+      __syncthreads();
+      x = __reduce_add_sync(0xffffffffu, red[rnd & 1][0][lane]);
+      y = __reduce_add_sync(0xffffffffu, red[rnd & 1][1][lane]);
+      T |= static_cast<uint64_t>(((x & 0xFFFFu) >= need) + ((x >> 16) >= need) + (y >= need)) << b;
+    }
+#pragma unroll
+    for (int u = 0; u < kBinCap / kRThreads; ++u) {
+      const bool s = u < nv && v[u] >= T && v[u] != 0ull;
+      const uint32_t chunk = s ? (~static_cast<uint32_t>(v[u])) / kChunk : 0xFFFFFFFFu;
+      const uint32_t grp = __match_any_sync(0xffffffffu, chunk);
+      if (s && lane == __ffs(grp) - 1) atomicAdd(&cnt[chunk], __popc(grp));
+    }
   }
   const uint32_t t_key = static_cast<uint32_t>(T >> 32), t_idx = ~static_cast<uint32_t>(T);
-  // chunk offsets: above the bracket plus the selected candidates of each chunk
-  for (uint32_t i = tid; i < ncand; i += 1024) {
-    const uint2 cd = cand[i];
-    if (cd.x > t_key || (cd.x == t_key && cd.y <= t_idx)) atomicAdd(&cnt[cd.y / kChunk], 1u);
+  // chunk counts: above the window, plus the candidates of the sub-bins before js (all above T),
+  // plus the sub-bin's selected candidates (above); warp w takes chunks w, w + 32, ...
+  for (int c = warp; c < nchunk; c += kRThreads / 32) {
+    const uint32_t* hc = h + static_cast<int64_t>(c) * kBins;
+    uint32_t s = (lane < js ? hc[lane] : 0u) + (lane + 32 < js ? hc[lane + 32] : 0u);
+    s = __reduce_add_sync(0xffffffffu, s);
+    if (lane == 0 && s) atomicAdd(&cnt[c], s);
   }
   __syncthreads();
+  // chunk offsets: exclusive prefix sums of the counts (each thread a run of consecutive chunks)
+  const int per = (nchunk + kRThreads - 1) / kRThreads;
+  const int c0 = min(tid * per, nchunk), c1 = min(c0 + per, nchunk);
+  uint32_t s = 0u;
+  for (int c = c0; c < c1; ++c) s += cnt[c];
+  uint32_t total;
+  uint32_t acc = scan1024(s, part, total);
+  for (int c = c0; c < c1; ++c) {
+    w.chunk_off[static_cast<int64_t>(r) * nchunk + c] = acc;
+    acc += cnt[c];
+  }
   if (tid == 0) {
-    uint32_t acc = 0u;
-    for (int c = 0; c < w.nchunk; ++c) {
-      w.chunk_off[static_cast<int64_t>(r) * w.nchunk + c] = acc;
-      acc += cnt[c];
-    }
     uint32_t* rr = w.res + static_cast<int64_t>(r) * 4;
     rr[0] = 1u;
     rr[1] = t_key;
@@ -785,43 +1096,57 @@ __global__ void __launch_bounds__(1024) topk_resolve_kernel(TArgs a, StreamWs w)
   }
 }
 
-__global__ void __launch_bounds__(kCThreads2) topk_output_kernel(TArgs a, StreamWs w) {
-  __shared__ uint32_t wt[16];
-  const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x;
+// selection mask of one output lane: f > T, or f == T and index <= T_index (lim_idx = T_index - jw)
+template <bool FULL>
+__device__ __forceinline__ uint32_t select_span(const float* row, int jw, int n, float tf, int64_t lim_idx) {
+  float f[kFKeys];
+  load_span<FULL>(row, jw, n, f);
+  uint32_t sel = 0u;
+#pragma unroll
+  for (int u = 0; u < kFKeys; ++u) {
+    if (FULL || span_off(u) < n - jw)
+      if (f[u] > tf || (f[u] == tf && span_off(u) <= lim_idx)) sel |= 1u << u;
+  }
+  return sel;
+}
+
+__global__ void __launch_bounds__(kFThreads, 4) topk_output_kernel(TArgs a, StreamWs w) {
+  __shared__ uint32_t wc[kFWarps];
+  const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* rr = w.res + static_cast<int64_t>(r) * 4;
   if (!rr[0]) return;   // uniform: the row is redone by the fallback
-  const uint32_t t_key = rr[1], t_idx = rr[2];
-  // 32 consecutive keys per thread (index order within the thread)
-  const int64_t j0 = static_cast<int64_t>(c) * kChunk + tid * 32;
+  const float tf = key_float(rr[1]);
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  uint32_t sel = 0u;   // bit u: key j0 + u selected
+  const int jw = c * kChunk + warp * (32 * kFKeys) + 4 * lane;
+  const int64_t lim_idx = static_cast<int64_t>(rr[2]) - jw;
+  const uint32_t sel = (c + 1) * kChunk <= a.n ? select_span<true>(row, jw, a.n, tf, lim_idx)
+                                               : select_span<false>(row, jw, a.n, tf, lim_idx);
+  const uint32_t cw = __reduce_add_sync(0xffffffffu, __popc(sel));
+  if (lane == 0) wc[warp] = cw;
+  __syncthreads();
+  uint32_t pos = w.chunk_off[static_cast<int64_t>(r) * w.nchunk + c] +
+                 __reduce_add_sync(0xffffffffu, lane < warp ? wc[lane] : 0u);
+  int32_t* out = a.idx_out + static_cast<int64_t>(r) * a.ld_out;
+  const uint32_t kk = static_cast<uint32_t>(a.k);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int64_t j = j0 + 4 * q;
-    float f[4];
-    if (j + 3 < a.n) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(row + j));
-      f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-    } else {
+  for (int q = 0; q < kFKeys / 4; ++q) {
+    const uint32_t s4 = (sel >> (4 * q)) & 15u;
+    const uint32_t n4 = __popc(s4);
+    uint32_t inc = n4;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) f[u] = j + u < a.n ? row[j + u] : 0.0f;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
     }
+    uint32_t p = pos + inc - n4;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint32_t key = float_key(f[u]);
-      const bool s = j + u < a.n && (key > t_key || (key == t_key && static_cast<uint32_t>(j + u) <= t_idx));
-      sel |= (s ? 1u : 0u) << (4 * q + u);
+      if ((s4 >> u) & 1u) {
+        if (p < kk) out[p] = jw + 128 * q + u;
+        ++p;
+      }
     }
-  }
-  uint32_t total;
-  const uint32_t pre = scan512(__popc(sel), wt, total);
-  uint32_t pos = w.chunk_off[static_cast<int64_t>(r) * w.nchunk + c] + pre;
-  int32_t* out = a.idx_out + static_cast<int64_t>(r) * a.ld_out;
-  while (sel) {
-    const int u = __ffs(sel) - 1;
-    sel &= sel - 1u;
-    if (pos < static_cast<uint32_t>(a.k)) out[pos] = static_cast<int32_t>(j0 + u);
-    ++pos;
+    pos += __shfl_sync(0xffffffffu, inc, 31);
   }
 }
 
@@ -836,10 +1161,10 @@ size_t stream_ws_bytes(int R, int n) {
   const size_t nchunk = (static_cast<size_t>(n) + kChunk - 1) / kChunk;
   size_t b = 0;
   auto take = [&](size_t bytes) { b += (bytes + 255) & ~size_t(255); };
-  take(static_cast<size_t>(R) * kBins * 4);            // hist (zeroed)
-  take(static_cast<size_t>(R) * 4);                    // ccount (zeroed)
+  take(static_cast<size_t>(R) * 4);                    // ccount
   take(static_cast<size_t>(R) * (kBins + 1) * 4);      // edges
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_gt
+  take(static_cast<size_t>(R) * nchunk * kBins * 4);   // hist
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_off
   take(static_cast<size_t>(R) * 16);                   // res
   take(static_cast<size_t>(R) * 4);                    // fallback
@@ -858,7 +1183,7 @@ int pick_cluster(int n) {
 
 bool stream_fits(int R, int n) {
   (void)R;
-  return n >= kStreamMin && (static_cast<int64_t>(n) + kChunk - 1) / kChunk <= 8192;
+  return n >= kStreamMin && (static_cast<int64_t>(n) + kChunk - 1) / kChunk <= kMaxChunks;
 }
 
 size_t topk_workspace_bytes(int R, int n, int k) {
@@ -874,9 +1199,8 @@ int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
   SPT_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return SPATTEN_E_UNSUPPORTED;
   if (!configured[dev]) {
-    SPT_CUDA(cudaFuncSetAttribute(topk_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSamples * 4));
     SPT_CUDA(cudaFuncSetAttribute(topk_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kBinCap * 8 + 8192 * 4));
+                                  kBinCap * 8 + kMaxChunks * 4));
     configured[dev] = true;
   }
   const int R = a.R, n = a.n;
@@ -889,23 +1213,21 @@ int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
     p += (bytes + 255) & ~size_t(255);
     return q;
   };
-  w.hist = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * kBins * 4));
   w.ccount = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * 4));
-  const size_t zero_bytes = static_cast<size_t>(p - static_cast<char*>(ws));
   w.edges = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * (kBins + 1) * 4));
   w.chunk_gt = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
+  w.hist = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * kBins * 4));
   w.chunk_off = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
   w.res = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * 16));
   w.fallback = reinterpret_cast<int32_t*>(take(static_cast<size_t>(R) * 4));
   w.cand = reinterpret_cast<uint2*>(take(static_cast<size_t>(R) * w.cap * 8));
-  SPT_CUDA(cudaMemsetAsync(ws, 0, zero_bytes, st));
-  topk_sample_kernel<<<R, 1024, kSamples * 4, st>>>(a, w);
+  topk_sample_kernel<<<R, kRThreads, 0, st>>>(a, w);
   SPT_TRY(launch_status());
-  topk_filter_kernel<<<dim3(w.nchunk, R), kCThreads2, 0, st>>>(a, w);
+  topk_filter_kernel<<<dim3(w.nchunk, R), kFThreads, 0, st>>>(a, w);
   SPT_TRY(launch_status());
-  topk_resolve_kernel<<<R, 1024, static_cast<size_t>(kBinCap) * 8 + static_cast<size_t>(w.nchunk) * 4, st>>>(a, w);
+  topk_resolve_kernel<<<R, kRThreads, static_cast<size_t>(kBinCap) * 8 + static_cast<size_t>(w.nchunk) * 4, st>>>(a, w);
   SPT_TRY(launch_status());
-  topk_output_kernel<<<dim3(w.nchunk, R), kCThreads2, 0, st>>>(a, w);
+  topk_output_kernel<<<dim3(w.nchunk, R), kFThreads, 0, st>>>(a, w);
   SPT_TRY(launch_status());
   TArgs f = a;   // rows whose bracket missed: the cluster kernel, every other row skipped at once
   f.only_rows = w.fallback;
