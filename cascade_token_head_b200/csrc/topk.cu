@@ -110,14 +110,12 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wt, ui
   return (warp > 0 ? wt[warp - 1] : 0u) + inc - v;
 }
 
-__global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
+// one row for one cluster; every CTA of the cluster calls it with the same row
+__device__ __forceinline__ void cluster_row(const TArgs& a, int r, uint32_t* keys_s, TShared& sh) {
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
-  const int r = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  extern __shared__ __align__(16) uint32_t keys_s[];
-  __shared__ TShared sh;
 
   const int64_t out_base = static_cast<int64_t>(r) * a.ld_out;
   if (a.only_rows && !a.only_rows[r]) return;   // uniform over the cluster: no barrier skipped
@@ -340,6 +338,19 @@ __global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
   }
 }
 
+// row blockIdx.y; LOOP: rows blockIdx.y, blockIdx.y + gridDim.y, ... (each row's last cluster
+// barrier ends every read of a peer's shared memory for that row, so the next row may reuse it)
+template <bool LOOP>
+__global__ void __launch_bounds__(kTThreads) topk_cluster_kernel(TArgs a) {
+  extern __shared__ __align__(16) uint32_t keys_s[];
+  __shared__ TShared sh;
+  if (LOOP) {
+    for (int r = blockIdx.y; r < a.R; r += gridDim.y) cluster_row(a, r, keys_s, sh);
+  } else {
+    cluster_row(a, blockIdx.y, keys_s, sh);
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Short rows (n <= 8192): the row's keys live in registers, sixteen consecutive keys per thread, one
 // warp per row (n <= 512, four rows per CTA, no block barrier) or one CTA of G warps per row (G = 4
@@ -492,24 +503,24 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 // ------------------------------------------------------------------------------------------------
 // Long rows (n >= kStreamMin, scores read directly, caller workspace given): two streaming passes
 // over the scores, with two one-CTA-per-row steps on small data between them.
-//  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256), finds by a digit search
-//           the sample keys at the two ends of a rank window around the sample rank of the k-th
-//           key (+-4 sigma of the sampling error + 16), and sorts the few sample keys strictly
-//           inside; 65 edges e0 >= e1 >= ... >= e64 at evenly spaced ranks of the window follow.
-//           The digit search runs first on one key in 16, whose window (widened by its own
-//           sampling error) bounds the few thousand sample keys the exact search then needs
-//  filter   per chunk of 8 K keys: the count above e0, and the keys in [e64, e0] appended as
-//           (key, index) to the row's candidate list
-//  resolve  one CTA per row: a histogram of the candidates over the 64 sub-bins between the
-//           edges, the sub-bin holding the k-th key, the exact threshold among that sub-bin's
-//           candidates as the (need)-th largest (key, ~index) composite (ties to the lower index),
-//           and every chunk's output offset
+//  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256) and finds by a digit
+//           search the sample keys e0 >= e64 at the two ends of a rank window around the sample
+//           rank of the k-th key (+-4 sigma of the sampling error + 16; an end past the sample is
+//           left open).  The search runs first on
+//           one key in 16, whose window (widened by its own sampling error) bounds the few
+//           thousand sample keys the exact search then needs
+//  filter   per chunk of 8 K keys: the count above e0, the keys in [e64, e0] appended as
+//           (key, index) to the row's candidate list, and their histogram over 64 sub-bins of
+//           equal width in value between e0 and e64
+//  resolve  one CTA per row: the sub-bin holding the k-th key, the exact threshold among that
+//           sub-bin's candidates as the (need)-th largest (key, ~index) composite (ties to the lower
+//           index), and every chunk's output offset
 //  output   per chunk: key > T, or key = T and index <= T_index, written in index order
-// A row whose k-th key fell outside the window's edges, or whose buffers overflowed, is marked and
-// done again by the cluster kernel (only_rows).
+// A row whose k-th key fell outside the window, or whose buffers overflowed, is marked and done
+// again by the cluster kernel (only_rows).
 // Filter and output read a warp's 512 keys as four coalesced 16-byte loads per lane (load q of
 // lane t holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span), so a key's place in index
-// order is (warp, q, lane, element).  They compare floats against the edges and the threshold
+// order is (warp, q, lane, element).  They compare floats against the window ends and the threshold
 // turned back into floats (the key map is monotone, and -0.0 equals +0.0 on both sides); a NaN
 // fails every ordered comparison, lands in the candidate list and is reported by the resolve step.
 // ------------------------------------------------------------------------------------------------
@@ -522,19 +533,20 @@ constexpr int kFWarps = kFThreads / 32;
 constexpr int kFKeys = 16;                                              // keys per filter/output lane
 constexpr int kChunk = kFThreads * kFKeys;                              // 8 K keys per filter/output CTA
 constexpr int kBinCap = 8192;                                           // candidates of one sub-bin
-constexpr int kWindow = 1024;                                           // sample keys inside the window
 constexpr int kL1 = 1024;                                               // first-level sample keys
 constexpr int kSList = 4096;                                            // second-level sample keys
 constexpr int kMaxChunks = 8192;
 
 struct StreamWs {
-  uint32_t* edges;      // [R][kBins + 1]
+  float* ends;          // [R][4]     window ends e0 (top), e64 (bottom) for the tests (+-inf when
+                        //            open), and the sub-bin scale's top and 64 / width (its ends
+                        //            the sample's extreme key in place of an open end)
   uint32_t* ccount;     // [R]        candidates appended (zeroed by the sample kernel)
   uint32_t* chunk_gt;   // [R][nchunk]
   uint32_t* hist;       // [R][nchunk][kBins]   candidates of each chunk per sub-bin
-  uint2* cand;          // [R][cap]  (key, index)
+  uint2* cand;          // [R][cap]  (score bits, index)
   uint32_t* chunk_off;  // [R][nchunk]
-  uint32_t* res;        // [R][4]   valid, T key, T index
+  uint32_t* res;        // [R][4]   valid, T key, T index, keys equal to T split by index
   int32_t* fallback;    // [R]
   int cap, nchunk;
 };
@@ -547,16 +559,23 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
 }
 
-__device__ __forceinline__ bool key_is_nan(uint32_t k) { return k > 0xFF800000u || k < 0x007FFFFFu; }
+// sub-bin of a window value: 64 steps of equal width from the scale's top down to its bottom
+// (clamped at both ends; all in sub-bin 0 when an end is infinite); the same rounded operations on
+// both sides of the candidate list, so the filter and the resolve step agree bit for bit; monotone
+// in the value
+struct BinMap {
+  float top, inv;
+};
 
-__device__ __forceinline__ int bin_of(uint32_t key, const uint32_t* e) {
-  // the largest j in [0, 63] with e[j] >= key (edges descending): bin j holds e[j+1] < key <= e[j],
-  // the last bin also key == e64
-  int lo = 0;
-#pragma unroll
-  for (int s = kBins / 2; s > 0; s >>= 1)
-    if (e[lo + s] >= key) lo += s;
-  return lo;
+__device__ __forceinline__ BinMap bin_map(float fe0, float fe64) {
+  const float span = __fsub_rn(fe0, fe64);
+  const bool ok = fabsf(fe0) <= 3.402823466e38f && fabsf(fe64) <= 3.402823466e38f && span > 0.0f;
+  return {fe0, ok ? __fdiv_rn(static_cast<float>(kBins), span) : 0.0f};
+}
+
+__device__ __forceinline__ int bin_of(float f, const BinMap& m) {
+  const int b = __float2int_rz(__fmul_rn(__fsub_rn(m.top, f), m.inv));
+  return min(max(b, 0), kBins - 1);
 }
 
 // bitonic sort of one value per thread over a 1024-thread block, descending (thread t ends with
@@ -586,13 +605,12 @@ __device__ __forceinline__ V bitonic_desc_1024(V x, V* scratch) {
 
 struct SampleSmem {
   uint32_t red[2][3][32];
-  uint32_t win[kWindow];
   uint32_t cnt[32];
   uint32_t list[kSList];
-  int rank[kBins + 1];
-  int open[2];
+  int rank[2];        // sample ranks of the window's ends
+  int open[2];        // the window's top / bottom end lies past the sample
   int l1[2];          // first-level ranks of the outer bounds (< 0 / >= kL1: no bound)
-  uint32_t n_in, n_list;
+  uint32_t n_list;
 };
 
 // ta / tb = the need_a-th / need_b-th largest of the NK keys per thread (block-wide; padding keys
@@ -659,49 +677,26 @@ __device__ __forceinline__ void append_keys(bool in, uint32_t key, uint32_t* lis
   }
 }
 
-// the 65 edges from the NK keys per thread, which hold every sample key ranked in the window;
+// the window's ends from the NK keys per thread, which hold every sample key ranked in the window;
 // `base` more sample keys lie above all of them
 template <int NK>
-__device__ __forceinline__ void window_edges(const uint32_t* key, uint32_t base, SampleSmem& sm, int r, StreamWs& w) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ void window_ends(const uint32_t* key, uint32_t base, SampleSmem& sm, int r, StreamWs& w) {
   const uint32_t need_a = static_cast<uint32_t>(sm.rank[0]) + 1u - base;
-  const uint32_t need_b = static_cast<uint32_t>(sm.rank[kBins]) + 1u - base;
+  const uint32_t need_b = static_cast<uint32_t>(sm.rank[1]) + 1u - base;
   uint32_t ta, tb;
   search2<NK>(key, need_a, need_b, sm, ta, tb);
-  // ge_a = #(key >= ta), gt_b = #(key > tb); the keys strictly between go to the window list
-  uint32_t c = 0u;
-#pragma unroll
-  for (int i = 0; i < NK; ++i) {
-    c += (key[i] >= ta ? 1u : 0u) + (key[i] > tb ? 0x10000u : 0u);
-    append_keys(key[i] > tb && key[i] < ta, key[i], sm.win, &sm.n_in, kWindow);
-  }
-  c = __reduce_add_sync(0xffffffffu, c);
-  if (lane == 0) sm.cnt[warp] = c;
-  __syncthreads();
-  c = __reduce_add_sync(0xffffffffu, sm.cnt[lane]);
-  const int ge_a = static_cast<int>(base + (c & 0xFFFFu)), gt_b = static_cast<int>(base + (c >> 16));
-  // padding below every key strictly inside the window (those exceed its low end)
-  const uint32_t x = bitonic_desc_1024(tid < static_cast<int>(sm.n_in) ? sm.win[tid] : 0u, sm.win);
-  __syncthreads();
-  sm.win[tid] = x;
-  __syncthreads();
-  if (tid <= kBins) {
-    // sorted sample position rho holds ta for rho < ge_a (rho >= the rank of ta), tb for
-    // rho >= gt_b (rho <= the rank of tb), else window key rho - ge_a
-    const int rho = sm.rank[tid];
-    uint32_t e;
-    if (tid == 0 && sm.open[0]) e = 0xFFFFFFFFu;
-    else if (tid == kBins && sm.open[1]) e = 0u;
-    else if (rho < ge_a) e = ta;
-    else if (rho >= gt_b) e = tb;
-    else e = sm.win[min(rho - ge_a, kWindow - 1)];
-    w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid] = e;
+  if (threadIdx.x == 0) {   // with an open end, ta / tb are the sample's largest / smallest key
+    const BinMap bm = bin_map(key_float(ta), key_float(tb));
+    w.ends[4 * r] = key_float(sm.open[0] ? 0xFFFFFFFFu : ta);
+    w.ends[4 * r + 1] = key_float(sm.open[1] ? 0u : tb);
+    w.ends[4 * r + 2] = bm.top;
+    w.ends[4 * r + 3] = bm.inv;
   }
 }
 
 __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamWs w) {
   constexpr int KPT = kSamples / kRThreads;   // 16 sample keys per thread
-  static_assert(kWindow == kRThreads && kL1 == kRThreads, "one window slot and one first-level key per thread");
+  static_assert(kL1 == kRThreads, "one first-level key per thread");
   __shared__ SampleSmem sm;
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
@@ -721,30 +716,24 @@ __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamW
     }
   }
   if (tid == 0) {
-    sm.n_in = 0u;
     sm.n_list = 0u;
     w.ccount[r] = 0u;
   }
-  if (tid <= kBins) {
-    // sample ranks of the edges: the window [r_hi, r_lo] around k/n of the sample, cut in 64 steps;
-    // its half-width is at most 4 sqrt(kSamples / 4) + 16 = 272, so at most 544 sample keys lie
-    // strictly between its ends
+  if (tid < 2) {
+    // sample ranks of the window's ends [r_hi, r_lo] around k/n of the sample
     const double p = static_cast<double>(a.k) / a.n;
     const double kp = p * kSamples;
     const double delta = 4.0 * sqrt(kSamples * p * (1.0 - p)) + 16.0;
     const double r_hi = kp - delta, r_lo = kp + delta;
-    const double rank = r_hi + tid * (r_lo - r_hi) / kBins;
-    const int rho = min(max(static_cast<int>(floor(rank)), 0), kSamples - 1);
+    const int rho = min(max(static_cast<int>(floor(tid == 0 ? r_hi : r_lo)), 0), kSamples - 1);
     sm.rank[tid] = rho;
-    if (tid == 0) sm.open[0] = r_hi < 0.0;
-    if (tid == kBins) sm.open[1] = r_lo >= kSamples - 1;
+    sm.open[tid] = tid == 0 ? r_hi < 0.0 : r_lo >= kSamples - 1;
     // first level: one sample key in 16; its keys at the window ends' ranks, moved outwards by 4
     // sigma of their own rank error (in first-level ranks) + 8, bound a second-level set that holds
     // the window
     const int m1 = static_cast<int>(ceil(4.0 * sqrt(kL1 * p * (1.0 - p)) + 8.0));
     constexpr int kStep = kSamples / kL1;
-    if (tid == 0) sm.l1[0] = rho / kStep - m1;
-    if (tid == kBins) sm.l1[1] = (rho + kStep - 1) / kStep + m1;
+    sm.l1[tid] = tid == 0 ? rho / kStep - m1 : (rho + kStep - 1) / kStep + m1;
   }
   __syncthreads();
   // the first level: each thread's first key, 16 per run
@@ -754,7 +743,7 @@ __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamW
   search2<1>(&k1, static_cast<uint32_t>(max(l1a, 0)) + 1u, static_cast<uint32_t>(min(l1b, kL1 - 1)) + 1u, sm, ca, cb);
   if (l1a < 0) ca = 0xFFFFFFFFu;
   if (l1b >= kL1) cb = 0u;
-  // the bound holds if at most rank[0] sample keys exceed ca and at least rank[64] + 1 reach cb
+  // the bound holds if at most rank[0] sample keys exceed ca and at least rank[1] + 1 reach cb
   uint32_t c = 0u;
 #pragma unroll
   for (int i = 0; i < KPT; ++i) c += (key[i] > ca ? 1u : 0u) + (key[i] >= cb ? 0x10000u : 0u);
@@ -763,7 +752,7 @@ __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamW
   __syncthreads();
   c = __reduce_add_sync(0xffffffffu, sm.cnt[lane]);
   const uint32_t gt_ca = c & 0xFFFFu, ge_cb = c >> 16;
-  const bool narrow = gt_ca <= static_cast<uint32_t>(sm.rank[0]) && ge_cb >= static_cast<uint32_t>(sm.rank[kBins]) + 1u &&
+  const bool narrow = gt_ca <= static_cast<uint32_t>(sm.rank[0]) && ge_cb >= static_cast<uint32_t>(sm.rank[1]) + 1u &&
                       ge_cb - gt_ca <= static_cast<uint32_t>(kSList);   // uniform
   if (narrow) {
 #pragma unroll
@@ -774,9 +763,9 @@ __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamW
     const uint32_t nl = sm.n_list;
 #pragma unroll
     for (int u = 0; u < NL; ++u) s[u] = tid + u * kRThreads < static_cast<int>(nl) ? sm.list[tid + u * kRThreads] : 0u;
-    window_edges<NL>(s, gt_ca, sm, r, w);
+    window_ends<NL>(s, gt_ca, sm, r, w);
   } else {
-    window_edges<KPT>(key, 0u, sm, r, w);
+    window_ends<KPT>(key, 0u, sm, r, w);
   }
 }
 
@@ -818,12 +807,12 @@ __device__ __forceinline__ void filter_span(const float* row, int jw, int n, flo
 
 __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, StreamWs w) {
   __shared__ uint32_t wc[kFWarps], wg[kFWarps], wb[kFWarps];
-  __shared__ uint32_t e_s[kBins + 1], hist[kBins];
+  __shared__ uint32_t hist[kBins];
   const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid <= kBins) e_s[tid] = w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid];
   if (tid < kBins) hist[tid] = 0u;
-  const float fe0 = key_float(w.edges[static_cast<int64_t>(r) * (kBins + 1)]);
-  const float fe64 = key_float(w.edges[static_cast<int64_t>(r) * (kBins + 1) + kBins]);
+  const float4 en = reinterpret_cast<const float4*>(w.ends)[r];
+  const float fe0 = en.x, fe64 = en.y;
+  const BinMap bm{en.z, en.w};
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   const int jw = c * kChunk + warp * (32 * kFKeys) + 4 * lane;
   uint32_t gt, cm;
@@ -868,9 +857,9 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, Stre
     for (uint32_t mm = cm; mm; mm &= mm - 1u, ++i) {
       const int u = __ffs(mm) - 1;
       const int j = jw + 128 * (u >> 2) + (u & 3);
-      const uint32_t key = float_key(row[j]);
-      dst[i] = make_uint2(key, static_cast<uint32_t>(j));
-      atomicAdd(&hist[bin_of(key, e_s)], 1u);
+      const float f = row[j];
+      dst[i] = make_uint2(__float_as_uint(f), static_cast<uint32_t>(j));
+      atomicAdd(&hist[bin_of(f, bm)], 1u);
     }
   }
   __syncthreads();
@@ -913,14 +902,12 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
   extern __shared__ __align__(16) unsigned char rs_smem[];
   uint64_t* bc = reinterpret_cast<uint64_t*>(rs_smem);                   // [kBinCap] sub-bin candidates
   uint32_t* cnt = reinterpret_cast<uint32_t*>(bc + kBinCap);             // [nchunk]
-  __shared__ uint32_t e[kBins + 1];
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t red[2][2][32];
   __shared__ uint32_t part[32];
   __shared__ uint32_t n_bc, js_s, above_s;
   __shared__ uint64_t t_s;
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid <= kBins) e[tid] = w.edges[static_cast<int64_t>(r) * (kBins + 1) + tid];
   if (tid < kBins) hist[tid] = 0u;
   if (tid == 0) {
     n_bc = 0u;
@@ -979,11 +966,9 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     stream_fail(w, r);
     return;
   }
-  // the sub-bin's candidates as (key, ~index) composites: e[js+1] < key <= e[js] (the last sub-bin
-  // also key == e64); the one pass over the candidate list, which also looks for NaNs (they pass
-  // the filter)
-  const uint32_t bin_hi = e[js];
-  const uint64_t bin_lo = js == kBins - 1 ? static_cast<uint64_t>(e[kBins]) : static_cast<uint64_t>(e[js + 1]) + 1u;
+  // the sub-bin's candidates as (key, ~index) composites; the one pass over the candidate list,
+  // which also looks for NaNs (they pass the filter)
+  const BinMap bm{w.ends[4 * r + 2], w.ends[4 * r + 3]};
   const uint2* cand = w.cand + static_cast<int64_t>(r) * w.cap;
   const uint32_t lt_mask = (1u << lane) - 1u;
   bool nan_seen = false;
@@ -992,12 +977,13 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
 #pragma unroll
     for (int u = 0; u < BP; ++u) {
       const uint32_t i = i0 + tid + u * kRThreads;
-      cd[u] = i < ncand ? cand[i] : make_uint2(0x80000000u, 0u);
+      cd[u] = i < ncand ? cand[i] : make_uint2(0u, 0u);
     }
 #pragma unroll
     for (int u = 0; u < BP; ++u) {
-      nan_seen |= key_is_nan(cd[u].x);
-      const bool hit = i0 + tid + u * kRThreads < ncand && cd[u].x <= bin_hi && cd[u].x >= bin_lo;
+      const float f = __uint_as_float(cd[u].x);
+      nan_seen |= f != f;
+      const bool hit = i0 + tid + u * kRThreads < ncand && bin_of(f, bm) == js;
       const uint32_t m = __ballot_sync(0xffffffffu, hit);
       if (m) {
         const int leader = __ffs(m) - 1;
@@ -1005,7 +991,7 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
         if (lane == leader) base = atomicAdd(&n_bc, __popc(m));
         base = __shfl_sync(0xffffffffu, base, leader);
         const uint32_t slot = base + __popc(m & lt_mask);
-        if (hit && slot < kBinCap) bc[slot] = (static_cast<uint64_t>(cd[u].x) << 32) | static_cast<uint64_t>(~cd[u].y);
+        if (hit && slot < kBinCap) bc[slot] = (static_cast<uint64_t>(float_key(f)) << 32) | static_cast<uint64_t>(~cd[u].y);
       }
     }
   }
@@ -1015,16 +1001,21 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
   const uint32_t need = k - above_s;   // 1 <= need <= m
   // T = the need-th largest composite; the selected ones of the sub-bin are counted per chunk
   uint64_t T;
+  bool split = true;   // without the count below the output takes the exact test
   if (m <= static_cast<uint32_t>(kRThreads)) {   // uniform: sort the sub-bin
     uint64_t x = tid < static_cast<int>(m) ? bc[tid] : 0ull;   // 0: below every composite
     x = bitonic_desc_1024(x, bc);
     if (tid == static_cast<int>(need) - 1) t_s = x;
-    const bool s = tid < static_cast<int>(need);
+    const bool s = tid < static_cast<int>(min(need, m));
     const uint32_t chunk = s ? (~static_cast<uint32_t>(x)) / kChunk : 0xFFFFFFFFu;
     const uint32_t grp = __match_any_sync(0xffffffffu, chunk);
     if (s && lane == __ffs(grp) - 1) atomicAdd(&cnt[chunk], __popc(grp));
     __syncthreads();
     T = t_s;
+    // are the keys equal to T's split by index (some above T, some below)?
+    const bool eq = tid < static_cast<int>(m) && static_cast<uint32_t>(x >> 32) == static_cast<uint32_t>(T >> 32);
+    const int n_eq = __syncthreads_count(eq), n_eq_sel = __syncthreads_count(eq && tid < static_cast<int>(need));
+    split = n_eq_sel < n_eq;
   } else {
     // two bits per round (the largest T with count(>= T) >= need)
     uint64_t v[kBinCap / kRThreads];
@@ -1092,22 +1083,30 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     rr[0] = 1u;
     rr[1] = t_key;
     rr[2] = t_idx;
+    rr[3] = split ? 1u : 0u;
     w.fallback[r] = 0;
   }
 }
 
-// selection mask of one output lane: f > T, or f == T and index <= T_index (lim_idx = T_index - jw)
-template <bool FULL>
-__device__ __forceinline__ uint32_t select_span(const float* row, int jw, int n, float tf, int64_t lim_idx) {
+// The output step reads a warp's 512 keys as 16 columns of 32 consecutive keys (lane t of column
+// c: key 32 c + t of the warp's span), so each column's selection is one ballot and its selected
+// indices go out as one coalesced store in index order.  Selection: f >= T when no key equal to T
+// lies past T_index (EXACT false), else f > T, or f == T and index <= T_index.
+template <bool FULL, bool EXACT>
+__device__ __forceinline__ void select_cols(const float* row, int span, int n, float tf, uint32_t t_idx, uint32_t* m) {
+  const int lane = threadIdx.x & 31;
   float f[kFKeys];
-  load_span<FULL>(row, jw, n, f);
-  uint32_t sel = 0u;
 #pragma unroll
-  for (int u = 0; u < kFKeys; ++u) {
-    if (FULL || span_off(u) < n - jw)
-      if (f[u] > tf || (f[u] == tf && span_off(u) <= lim_idx)) sel |= 1u << u;
+  for (int col = 0; col < kFKeys; ++col) {
+    const int j = span + 32 * col + lane;
+    f[col] = (FULL || j < n) ? __ldg(row + j) : __int_as_float(0x7FFFFFFF);   // NaN: never selected
   }
-  return sel;
+#pragma unroll
+  for (int col = 0; col < kFKeys; ++col) {
+    const uint32_t j = static_cast<uint32_t>(span + 32 * col + lane);
+    const bool sel = EXACT ? (f[col] > tf || (f[col] == tf && j <= t_idx)) : f[col] >= tf;
+    m[col] = __ballot_sync(0xffffffffu, sel);
+  }
 }
 
 __global__ void __launch_bounds__(kFThreads, 4) topk_output_kernel(TArgs a, StreamWs w) {
@@ -1116,37 +1115,40 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_output_kernel(TArgs a, Stre
   const uint32_t* rr = w.res + static_cast<int64_t>(r) * 4;
   if (!rr[0]) return;   // uniform: the row is redone by the fallback
   const float tf = key_float(rr[1]);
+  const uint32_t t_idx = rr[2];
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  const int jw = c * kChunk + warp * (32 * kFKeys) + 4 * lane;
-  const int64_t lim_idx = static_cast<int64_t>(rr[2]) - jw;
-  const uint32_t sel = (c + 1) * kChunk <= a.n ? select_span<true>(row, jw, a.n, tf, lim_idx)
-                                               : select_span<false>(row, jw, a.n, tf, lim_idx);
-  const uint32_t cw = __reduce_add_sync(0xffffffffu, __popc(sel));
+  const int span = c * kChunk + warp * (32 * kFKeys);
+  const bool full = (c + 1) * kChunk <= a.n;
+  uint32_t m[kFKeys];
+  if (rr[3]) {
+    if (full) select_cols<true, true>(row, span, a.n, tf, t_idx, m);
+    else select_cols<false, true>(row, span, a.n, tf, t_idx, m);
+  } else {
+    if (full) select_cols<true, false>(row, span, a.n, tf, t_idx, m);
+    else select_cols<false, false>(row, span, a.n, tf, t_idx, m);
+  }
+  uint32_t cw = 0u;
+#pragma unroll
+  for (int col = 0; col < kFKeys; ++col) cw += __popc(m[col]);
   if (lane == 0) wc[warp] = cw;
   __syncthreads();
   uint32_t pos = w.chunk_off[static_cast<int64_t>(r) * w.nchunk + c] +
                  __reduce_add_sync(0xffffffffu, lane < warp ? wc[lane] : 0u);
   int32_t* out = a.idx_out + static_cast<int64_t>(r) * a.ld_out;
-  const uint32_t kk = static_cast<uint32_t>(a.k);
+  const uint32_t kk = static_cast<uint32_t>(a.k), bit = 1u << lane, lt = bit - 1u;
+  if (pos + cw <= kk) {   // warp-uniform; always, when the counts agree
 #pragma unroll
-  for (int q = 0; q < kFKeys / 4; ++q) {
-    const uint32_t s4 = (sel >> (4 * q)) & 15u;
-    const uint32_t n4 = __popc(s4);
-    uint32_t inc = n4;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += t;
+    for (int col = 0; col < kFKeys; ++col) {
+      if (m[col] & bit) out[pos + __popc(m[col] & lt)] = span + 32 * col + lane;
+      pos += __popc(m[col]);
     }
-    uint32_t p = pos + inc - n4;
+  } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if ((s4 >> u) & 1u) {
-        if (p < kk) out[p] = jw + 128 * q + u;
-        ++p;
-      }
+    for (int col = 0; col < kFKeys; ++col) {
+      const uint32_t p = pos + __popc(m[col] & lt);
+      if ((m[col] & bit) && p < kk) out[p] = span + 32 * col + lane;
+      pos += __popc(m[col]);
     }
-    pos += __shfl_sync(0xffffffffu, inc, 31);
   }
 }
 
@@ -1162,7 +1164,7 @@ size_t stream_ws_bytes(int R, int n) {
   size_t b = 0;
   auto take = [&](size_t bytes) { b += (bytes + 255) & ~size_t(255); };
   take(static_cast<size_t>(R) * 4);                    // ccount
-  take(static_cast<size_t>(R) * (kBins + 1) * 4);      // edges
+  take(static_cast<size_t>(R) * 4 * 4);                // ends (16-byte rows)
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_gt
   take(static_cast<size_t>(R) * nchunk * kBins * 4);   // hist
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_off
@@ -1193,6 +1195,31 @@ size_t topk_workspace_bytes(int R, int n, int k) {
 
 int32_t cluster_launch(const TArgs& a, cudaStream_t st);
 
+// the four steps for rows [r0, r0 + rows)
+int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaStream_t st) {
+  TArgs g = a;
+  g.scores = a.scores + static_cast<int64_t>(r0) * a.ld;
+  g.idx_out = a.idx_out + static_cast<int64_t>(r0) * a.ld_out;
+  g.R = rows;
+  StreamWs v = w;
+  v.ends += static_cast<int64_t>(r0) * 4;
+  v.ccount += r0;
+  v.chunk_gt += static_cast<int64_t>(r0) * w.nchunk;
+  v.hist += static_cast<int64_t>(r0) * w.nchunk * kBins;
+  v.chunk_off += static_cast<int64_t>(r0) * w.nchunk;
+  v.res += static_cast<int64_t>(r0) * 4;
+  v.fallback += r0;
+  v.cand += static_cast<int64_t>(r0) * w.cap;
+  topk_sample_kernel<<<rows, kRThreads, 0, st>>>(g, v);
+  SPT_TRY(launch_status());
+  topk_filter_kernel<<<dim3(w.nchunk, rows), kFThreads, 0, st>>>(g, v);
+  SPT_TRY(launch_status());
+  topk_resolve_kernel<<<rows, kRThreads, static_cast<size_t>(kBinCap) * 8 + static_cast<size_t>(w.nchunk) * 4, st>>>(g, v);
+  SPT_TRY(launch_status());
+  topk_output_kernel<<<dim3(w.nchunk, rows), kFThreads, 0, st>>>(g, v);
+  return launch_status();
+}
+
 int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
   static bool configured[64] = {false};
   int dev = 0;
@@ -1214,21 +1241,14 @@ int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
     return q;
   };
   w.ccount = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * 4));
-  w.edges = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * (kBins + 1) * 4));
+  w.ends = reinterpret_cast<float*>(take(static_cast<size_t>(R) * 4 * 4));
   w.chunk_gt = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
   w.hist = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * kBins * 4));
   w.chunk_off = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
   w.res = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * 16));
   w.fallback = reinterpret_cast<int32_t*>(take(static_cast<size_t>(R) * 4));
   w.cand = reinterpret_cast<uint2*>(take(static_cast<size_t>(R) * w.cap * 8));
-  topk_sample_kernel<<<R, kRThreads, 0, st>>>(a, w);
-  SPT_TRY(launch_status());
-  topk_filter_kernel<<<dim3(w.nchunk, R), kFThreads, 0, st>>>(a, w);
-  SPT_TRY(launch_status());
-  topk_resolve_kernel<<<R, kRThreads, static_cast<size_t>(kBinCap) * 8 + static_cast<size_t>(w.nchunk) * 4, st>>>(a, w);
-  SPT_TRY(launch_status());
-  topk_output_kernel<<<dim3(w.nchunk, R), kFThreads, 0, st>>>(a, w);
-  SPT_TRY(launch_status());
+  SPT_TRY(stream_chain(a, w, 0, R, st));
   TArgs f = a;   // rows whose bracket missed: the cluster kernel, every other row skipped at once
   f.only_rows = w.fallback;
   return cluster_launch(f, st);
@@ -1258,9 +1278,12 @@ int32_t cluster_launch(const TArgs& a, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    SPT_CUDA(cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    SPT_CUDA(cudaFuncSetAttribute(topk_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kResident * 4));
-    if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    SPT_CUDA(cudaFuncSetAttribute(topk_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kResident * 4));
+    if (cudaFuncSetAttribute(topk_cluster_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(topk_cluster_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(16, 1, 1);
       q.blockDim = dim3(kTThreads, 1, 1);
@@ -1273,7 +1296,7 @@ int32_t cluster_launch(const TArgs& a, cudaStream_t st) {
       q.attrs = qa;
       q.numAttrs = 1;
       int clusters = 0;
-      wide_ok[dev] = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &q) == cudaSuccess && clusters >= 4;
+      wide_ok[dev] = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel<false>, &q) == cudaSuccess && clusters >= 4;
     }
     cudaGetLastError();   // the probe above may leave an error behind
     configured[dev] = true;
@@ -1283,7 +1306,9 @@ int32_t cluster_launch(const TArgs& a, cudaStream_t st) {
   const int chunk = static_cast<int>((ceil_div(a.n, C) + 3) & ~int64_t(3));
   const size_t smem = static_cast<size_t>(std::min(chunk, kResident)) * 4;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(C, a.R, 1);
+  // rows left to the fallback (only_rows) are rare: a few clusters loop over all rows and skip the
+  // others, instead of one cluster per row
+  cfg.gridDim = dim3(C, a.only_rows ? std::min(a.R, 8) : a.R, 1);
   cfg.blockDim = dim3(kTThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -1294,7 +1319,8 @@ int32_t cluster_launch(const TArgs& a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = C > 1 ? 1 : 0;   // a one-CTA row needs no cluster (implicit 1x1x1)
-  SPT_CUDA(cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a));
+  if (a.only_rows) SPT_CUDA(cudaLaunchKernelEx(&cfg, topk_cluster_kernel<true>, a));
+  else SPT_CUDA(cudaLaunchKernelEx(&cfg, topk_cluster_kernel<false>, a));
   return launch_status();
 }
 

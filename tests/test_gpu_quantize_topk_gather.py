@@ -226,11 +226,14 @@ def test_topk_through_map_with_composition(cuda):
         np.testing.assert_array_equal(comp[r], mp[r][sel])
 
 
-def test_topk_nan_reports_status(cuda):
+@pytest.mark.parametrize("n,k,pos", [(50, 10, 7), (70001, 7000, 123), (70001, 7000, 69999), (70001, 63000, 5)])
+def test_topk_nan_reports_status(cuda, n, k, pos):
+    """A NaN anywhere in a row gives E_NONFINITE: short rows, and long rows on the streaming path
+    (the NaN passes the filter's window tests and is seen among the candidates)."""
     S = lib()
-    x = np.arange(50, dtype=np.float32)[None].repeat(2, 0)
-    x[1, 7] = np.nan
-    _, _, st = _topk_gpu(S, x, 10)
+    x = synth.rng_for(n + pos).random((2, n)).astype(np.float32)
+    x[1, pos] = np.nan
+    _, _, st = _topk_gpu(S, x, k)
     assert st == S.E_NONFINITE
 
 
@@ -276,6 +279,24 @@ def test_topk_long_rows_bracket_misses_fall_back(cuda, with_ws):
         assert st == 0
         for r in range(R_):
             np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
+
+
+def test_topk_long_rows_tie_group_at_threshold(cuda):
+    """Long rows on the streaming path whose k-th value is shared by eight keys: the selection takes
+    one, three, four or all eight of them, always the lowest indices of the group (the tie rule),
+    so the output step meets both its split-tie and its whole-group test.  Bit-exact."""
+    S = lib()
+    g = synth.rng_for(78)
+    R_, n, k = 4, 131072, 40000
+    x = g.random((R_, n)).astype(np.float32)
+    for r, takes in enumerate((1, 8, 4, 3)):
+        v = np.sort(x[r])[::-1][k - takes]
+        below = np.flatnonzero(x[r] < v)
+        x[r, g.choice(below, size=7, replace=False)] = v       # eight keys now hold v
+    got, _, st = _topk_gpu(S, x, k)
+    assert st == 0
+    for r in range(R_):
+        np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
 
 
 # ------------------------------------------------------------------------------------------------
