@@ -5,11 +5,14 @@
 // bits and concatenates MSBs with LSBs.  Codes: q = clamp(rint(float32(x*gain) / s), +-2047),
 // MSB = q >> 4, LSB = q & 15, s = amax / 2047 per (sequence, head) block.
 //
-// Amax mode: one thread-block cluster per (b, h) block (gridDim.z selects K or V when both are
-// quantized in one launch); each CTA reduces the amax of its rows, the cluster exchanges the
-// partial maxima through distributed shared memory, and every CTA then quantizes its rows (a
-// second read that hits L2).  Each thread keeps four 16-byte loads in flight.  No scratch memory
-// is needed.
+// Amax mode, small blocks (at most 4096 chunks of 8 elements for bf16, 2048 for float32, e.g.
+// 512 rows of 64): one CTA per (b, h) block (gridDim.z selects K or V when both are quantized in
+// one launch) holds the block's raw 16-byte words in registers, reduces the amax and writes the
+// codes from the same registers: one read.
+// Amax mode, larger blocks: one thread-block cluster per (b, h) block; each CTA reduces the amax of
+// its rows, the cluster exchanges the partial maxima through distributed shared memory, and every
+// CTA then quantizes its rows (a second read that hits L2).  Each thread keeps four 16-byte loads
+// in flight.  No scratch memory is needed in either mode.
 // Fixed-scale mode (decode append): one thread per 8-element chunk, saturations counted.
 #include <cooperative_groups.h>
 
@@ -168,6 +171,91 @@ __global__ void __launch_bounds__(kQThreads) quantize_amax_kernel(QArgs a) {
   }
 }
 
+// eight consecutive elements of a head row kept as raw 16-byte words (one for bf16, two for float)
+template <typename T>
+struct Chunk8;
+
+template <>
+struct Chunk8<__nv_bfloat16> {
+  uint4 w;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void get(float* f) const {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {   // bf16 -> float: the 16 bits become the high half of the word
+      f[2 * i] = __uint_as_float(u[i] << 16);
+      f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+  }
+};
+
+template <>
+struct Chunk8<float> {
+  uint4 w0, w1;
+  __device__ __forceinline__ void load(const float* p) {
+    w0 = __ldg(reinterpret_cast<const uint4*>(p));
+    w1 = __ldg(reinterpret_cast<const uint4*>(p + 4));
+  }
+  __device__ __forceinline__ void get(float* f) const {
+    f[0] = __uint_as_float(w0.x); f[1] = __uint_as_float(w0.y); f[2] = __uint_as_float(w0.z); f[3] = __uint_as_float(w0.w);
+    f[4] = __uint_as_float(w1.x); f[5] = __uint_as_float(w1.y); f[6] = __uint_as_float(w1.z); f[7] = __uint_as_float(w1.w);
+  }
+};
+
+constexpr int kQBThreads = 512;
+template <typename T>
+constexpr int block_chunks() { return sizeof(T) == 2 ? 8 : 4; }   // chunks per thread (registers)
+
+// C: chunks per head row (d_h / 8)
+template <typename T, int C>
+__global__ void __launch_bounds__(kQBThreads) quantize_amax_block_kernel(QArgs a) {
+  constexpr int CH = block_chunks<T>();
+  const QTensor& q = a.t[blockIdx.z];
+  const int bh = blockIdx.x;
+  const int b = bh / a.H, h = bh % a.H;
+  const int total = a.n * C;
+  __shared__ float red[kQBThreads / 32];
+  Chunk8<T> ch[CH];
+#pragma unroll
+  for (int u = 0; u < CH; ++u) {
+    const int e = threadIdx.x + u * kQBThreads;
+    if (e < total) ch[u].load(chunk_ptr<T>(a, q, b, h, e / C, e % C));
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int u = 0; u < CH; ++u) {
+    const int e = threadIdx.x + u * kQBThreads;
+    if (e < total) {
+      float v[8];
+      ch[u].get(v);
+      apply_gain(a, q, b, e / C, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  float block_amax = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kQBThreads / 32; ++w) block_amax = fmaxf(block_amax, red[w]);
+  const float s = block_amax == 0.0f ? 1.0f : __fdiv_rn(block_amax, kQMax);
+  const float rcp = __frcp_rn(s);
+  if (threadIdx.x == 0) q.scale_out[bh] = s;
+#pragma unroll
+  for (int u = 0; u < CH; ++u) {
+    const int e = threadIdx.x + u * kQBThreads;
+    if (e < total) {
+      const int t = e / C, c = e % C;
+      float v[8];
+      ch[u].get(v);
+      apply_gain(a, q, b, t, v);
+      const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
+      quant8(v, s, rcp, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+    }
+  }
+}
+
 template <typename T, int CT>
 __global__ void __launch_bounds__(kQThreads) quantize_fixed_kernel(QArgs a) {
   const QTensor& q = a.t[blockIdx.z];
@@ -215,6 +303,20 @@ int32_t quantize_launch(const QArgs& a, int ntensors, int dtype, cudaStream_t st
     return launch_status();
   }
   const int blocks = a.B * a.H;
+  const bool bf = dtype == SPATTEN_BF16;
+  const int64_t chunks = static_cast<int64_t>(a.n) * (a.d_h / 8);
+  if ((a.d_h == 64 || a.d_h == 128) &&
+      chunks <= static_cast<int64_t>(kQBThreads) * (bf ? block_chunks<__nv_bfloat16>() : block_chunks<float>())) {
+    const dim3 g(blocks, 1, ntensors);
+    if (a.d_h == 64) {
+      if (bf) quantize_amax_block_kernel<__nv_bfloat16, 8><<<g, kQBThreads, 0, st>>>(a);
+      else quantize_amax_block_kernel<float, 8><<<g, kQBThreads, 0, st>>>(a);
+    } else {
+      if (bf) quantize_amax_block_kernel<__nv_bfloat16, 16><<<g, kQBThreads, 0, st>>>(a);
+      else quantize_amax_block_kernel<float, 16><<<g, kQBThreads, 0, st>>>(a);
+    }
+    return launch_status();
+  }
   // enough CTAs for eight per SM (every SM then keeps 2048 threads' loads in flight); at most 8
   // per block (portable cluster size)
   int S = static_cast<int>(ceil_div(8LL * sm_count(), static_cast<int64_t>(blocks) * ntensors));
@@ -231,7 +333,6 @@ int32_t quantize_launch(const QArgs& a, int ntensors, int dtype, cudaStream_t st
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const bool bf = dtype == SPATTEN_BF16;
   cudaError_t e;
   if (a.d_h == 64)
     e = bf ? cudaLaunchKernelEx(&cfg, quantize_amax_kernel<__nv_bfloat16, 8>, a)
