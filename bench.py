@@ -345,6 +345,51 @@ def e2e_loop(ctx, body, n):
     return ctx.max_over_ranks(sum(ms)), n
 
 
+def e2e_pipelined(ctx, slots, x_host, gain_host, forward, n):
+    """n consecutive steps, device-timed together (L2 flushed once before): step i's inputs are copied
+    into slot i % 2 on a copy stream while step i - 1 runs, and its outputs are copied out on the
+    same stream while step i + 1 runs.  Returns the total milliseconds (max over ranks)."""
+    torch = ctx.torch
+    copy = torch.cuda.Stream(device=ctx.dev)
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    fwd_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+
+    def copy_in(j, after_fwd):
+        xj, gj = slots[j][0], slots[j][1]
+        with torch.cuda.stream(copy):
+            if after_fwd is not None:
+                copy.wait_event(after_fwd)   # the slot's inputs were read by that step's forward
+            xj.copy_(x_host, non_blocking=True)
+            gj.copy_(gain_host, non_blocking=True)
+            h2d_done[j].record(copy)
+
+    ctx.flush.zero_()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(ctx.stream)
+    copy.wait_stream(ctx.stream)
+    copy_in(0, None)
+    for i in range(n):
+        j = i % 2
+        if i + 1 < n:
+            copy_in((i + 1) % 2, fwd_done[(i + 1) % 2] if i >= 1 else None)
+        ctx.stream.wait_event(h2d_done[j])
+        if i >= 2:
+            ctx.stream.wait_event(d2h_done[j])   # the slot's outputs of step i - 2 have been copied out
+        forward(slots[j][3])
+        fwd_done[j].record(ctx.stream)
+        with torch.cuda.stream(copy):
+            copy.wait_event(fwd_done[j])
+            for dev_t, host_t in zip(slots[j][2], slots[j][4]):
+                host_t.copy_(dev_t, non_blocking=True)
+            d2h_done[j].record(copy)
+    ctx.stream.wait_stream(copy)
+    b.record(ctx.stream)
+    torch.cuda.synchronize()
+    return ctx.max_over_ranks(a.elapsed_time(b))
+
+
 def prefill_arm(ctx, args, name):
     import numpy as np
     torch = ctx.torch
@@ -411,23 +456,41 @@ def prefill_arm(ctx, args, name):
     assert int(status.item()) == 0, "device status after timing"
     refetch_rows = refetch.cpu().tolist()
 
-    # end to end through the C ABI with host buffers: H2D of X and key_gain, forward, D2H of the
-    # final rows, the kept sets and the cumulative importance
-    out_host = torch.empty_like(x_out, device="cpu").pin_memory()
-    kept_host = torch.empty_like(kept_tok, device="cpu").pin_memory()
-    imp_host = torch.empty_like(tok_imp, device="cpu").pin_memory()
+    # end to end through the C ABI with host buffers: every step copies X and key_gain in from pinned
+    # host memory, runs spatten_cascade_forward (direct launches) and copies the final rows, the
+    # kept sets and the cumulative importance out; the copies of neighbouring steps overlap the
+    # forward on a second stream (two sets of device inputs and outputs)
     h2d = X_host.numel() * X_host.element_size() + gain_host.numel() * 4
-    d2h = out_host.numel() * 2 + kept_host.numel() * 4 + imp_host.numel() * 4
-
-    def e2e_body():
-        X.copy_(X_host, non_blocking=True)
-        gain.copy_(gain_host, non_blocking=True)
-        step()
-        out_host.copy_(x_out, non_blocking=True)
-        kept_host.copy_(kept_tok, non_blocking=True)
-        imp_host.copy_(tok_imp, non_blocking=True)
-
-    e2e_total, n_e2e = e2e_loop(ctx, e2e_body, max(3, K // 2))
+    d2h = x_out.numel() * 2 + kept_tok.numel() * 4 + tok_imp.numel() * 4
+    slots = []
+    for j in range(2):
+        xj = X if j == 0 else torch.empty_like(X)
+        gj = gain if j == 0 else torch.empty_like(gain)
+        oj = (x_out, kept_tok, tok_imp) if j == 0 else tuple(torch.empty_like(t) for t in (x_out, kept_tok, tok_imp))
+        ioj = S.cascade_io()
+        ioj.x, ioj.key_gain, ioj.x_out = xj.data_ptr(), gj.data_ptr(), oj[0].data_ptr()
+        ioj.kept_tok, ioj.kept_head = oj[1].data_ptr(), kept_head.data_ptr()
+        ioj.tok_imp, ioj.head_imp, ioj.refetch_count = oj[2].data_ptr(), head_imp.data_ptr(), refetch.data_ptr()
+        ioj.dev_status = status.data_ptr()
+        hosts = tuple(torch.empty_like(t, device="cpu").pin_memory() for t in oj)
+        slots.append((xj, gj, oj, ioj, hosts))
+    n_e2e = max(3, K)
+    e2e_total = e2e_pipelined(ctx, slots, X_host, gain_host,
+                              lambda io_j: S.cascade_forward(cfg, W, io_j, ws, ws.numel(), stream=ctx.stream), n_e2e)
+    assert int(status.item()) == 0, "device status after the end-to-end loop"
+    # the same loop with each slot's forward replayed from a CUDA graph captured from the same call
+    e2e_graph_total = None
+    if graph is not None:
+        slot_graphs = []
+        for slot in slots:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                S.cascade_forward(cfg, W, slot[3], ws, ws.numel(), stream=torch.cuda.current_stream())
+            slot_graphs.append(g)
+        torch.cuda.synchronize()
+        e2e_graph_total = e2e_pipelined(ctx, slots, X_host, gain_host,
+                                        lambda io_j: slot_graphs[0 if io_j is slots[0][3] else 1].replay(), n_e2e)
+        assert int(status.item()) == 0, "device status after the graph end-to-end loop"
     tokens_per_step = B * T
     peaks, peak_kind = load_peaks()
     flops = attention_flops(w)
@@ -449,7 +512,14 @@ def prefill_arm(ctx, args, name):
                                   f"dense rate, ratio 1)", "traffic": None,
                      "algorithmic_flops_per_step": flops, "attn_ms_per_step": attn_s * 1e3},
         "e2e": {"value": ctx.world * tokens_per_step * n_e2e / (e2e_total / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "method": f"{n_e2e} consecutive steps timed together, each a direct spatten_cascade_forward "
+                          f"call; each step's copies in and out on a second stream, overlapping the "
+                          f"neighbouring steps' forward",
+                "graph_value": (ctx.world * tokens_per_step * n_e2e / (e2e_graph_total / 1e3)
+                                if e2e_graph_total else None),
+                "graph_method": "the same loop, each step's forward replayed from a CUDA graph captured from "
+                                "the same call"},
         "gpu_launches": int(launches),
         "clocks": clk,
         "refetch_rows_per_layer": refetch_rows,
