@@ -202,10 +202,19 @@ __device__ __forceinline__ void stats64(const float* v, float& m2, float& l) {
   m2 = mn;
 }
 
+// 16·MSB + LSB, pair by pair: the 12-bit code itself, an integer of magnitude at most 2048, so the
+// fp16 sum is exact and one MMA over the combined tile replaces an MSB and an LSB product
+__device__ __forceinline__ void add_f16x8(uint32_t* hi, const uint32_t* lo) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const __half2 s = __hadd2(*reinterpret_cast<const __half2*>(&hi[q]), *reinterpret_cast<const __half2*>(&lo[q]));
+    hi[q] = *reinterpret_cast<const uint32_t*>(&s);
+  }
+}
+
 template <int DH, int KT>
 __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int64_t plane0, const int32_t* kv_idx,
-                                             const int8_t* msb, const uint8_t* lsb, uint32_t off_hi,
-                                             uint32_t off_lo, int ptid) {
+                                             const int8_t* msb, const uint8_t* lsb, uint32_t off_hi, int ptid) {
   constexpr int L16 = DH / 16;
   for (int e = ptid; e < KT * L16; e += kProducerThreads) {
     const int r = e / L16, c16 = e % L16;
@@ -214,17 +223,16 @@ __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int
     if (key < n_kv) {
       const int64_t prow = plane0 + (kv_idx ? kv_idx[key] : key);
       cvt16_s8x16(__ldg(reinterpret_cast<const uint4*>(msb + prow * DH) + c16), hi);
-      if (lsb) cvt_u4x16(__ldg(reinterpret_cast<const uint2*>(lsb + prow * (DH / 2)) + c16), lo);
+      if (lsb) {
+        cvt_u4x16(__ldg(reinterpret_cast<const uint2*>(lsb + prow * (DH / 2)) + c16), lo);
+        add_f16x8(hi, lo);
+      }
     } else {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
+      for (int q = 0; q < 8; ++q) hi[q] = 0u;
     }
     *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16, KT)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-    if (lsb) {
-      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16, KT)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-    }
   }
   fence_async_smem();
 }
@@ -233,24 +241,23 @@ __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int
 // packed LSB rows (DH/2 bytes) at raw + KT*DH; rows >= valid are zero-filled
 template <int DH, int KT>
 __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw, bool with_lsb, int valid,
-                                               uint32_t off_hi, uint32_t off_lo, int ptid) {
+                                               uint32_t off_hi, int ptid) {
   constexpr int L16 = DH / 16;
   for (int e = ptid; e < KT * L16; e += kProducerThreads) {
     const int r = e / L16, c16 = e % L16;
     uint32_t hi[8], lo[8];
     if (r < valid) {
       cvt16_s8x16(*reinterpret_cast<const uint4*>(raw + r * DH + c16 * 16), hi);
-      if (with_lsb) cvt_u4x16(*reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8), lo);
+      if (with_lsb) {
+        cvt_u4x16(*reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8), lo);
+        add_f16x8(hi, lo);
+      }
     } else {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
+      for (int q = 0; q < 8; ++q) hi[q] = 0u;
     }
     *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16, KT)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(smem + off_hi + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-    if (with_lsb) {
-      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16, KT)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(smem + off_lo + tile_off(r, 2 * c16 + 1, KT)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-    }
   }
   fence_async_smem();
 }
@@ -309,20 +316,21 @@ struct JobStream {
     }
     return true;
   }
-  // convert job j into (off_hi, off_lo); returns false on abort
-  __device__ __forceinline__ bool convert(int j, uint32_t off_hi, uint32_t off_lo, const int32_t* kv_idx) {
+  // convert job j into the fp16 tile at off_hi (16·MSB, or with the LSB plane the combined
+  // 16·MSB + LSB); returns false on abort
+  __device__ __forceinline__ bool convert(int j, uint32_t off_hi, const int32_t* kv_idx) {
     bool is_v;
     int t;
     job(j, is_v, t);
     if (kv_idx) {
       produce_tile<DH, KT>(smem, t, a->n_kv, plane0, kv_idx, is_v ? a->v_msb : a->k_msb,
-                           with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, off_lo, ptid);
+                           with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, ptid);
       return true;
     }
     const uint32_t gj = g0 + static_cast<uint32_t>(j);
     const uint32_t st = gj % RS;
     if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag)) return false;
-    convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, off_lo, ptid);
+    convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid);
     mbar_arrive(&raw_empty[st]);
     return true;
   }
@@ -525,7 +533,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         uint32_t& cnt = is_v ? vc : kc;
         const uint32_t st = cnt % NST;
         if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, 0, kv_idx)) { aborted = true; break; }
+        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, kv_idx)) { aborted = true; break; }
         mbar_arrive(&bars[(is_v ? M_VF : M_KF) + st]);
         ++cnt;
       }
@@ -785,9 +793,9 @@ struct FullCfg {
   static constexpr int RS = 3;                   // raw (MSB + LSB) tiles in flight
   static constexpr uint32_t RAWB = static_cast<uint32_t>(KT) * DH * 3u / 2u;
   static constexpr uint32_t oQ = 0;
-  static constexpr uint32_t oK = QB;             // 2 stages of (MSB tile, LSB tile)
-  static constexpr uint32_t oV = oK + 4 * TB;    // 2 stages of (MSB tile, LSB tile)
-  static constexpr uint32_t oP = oV + 4 * TB;    // 1 buffer
+  static constexpr uint32_t oK = QB;             // 2 stages of one combined (16·MSB + LSB) tile
+  static constexpr uint32_t oV = oK + 2 * TB;    // 2 stages of one combined tile
+  static constexpr uint32_t oP = oV + 2 * TB;    // 1 buffer
   static constexpr uint32_t oRaw = oP + PB;      // RS staging slots
   static constexpr uint32_t kSmem = oRaw + RS * RAWB + 1024u;
   static constexpr uint32_t tS = 0;              // + buffer * KT
@@ -922,8 +930,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
         uint32_t& cnt = is_v ? vc : kc;
         const uint32_t st = cnt & 1u;
         if (!wait_bar(&bars[(is_v ? F_VE : F_KE) + st], ((cnt >> 1) & 1u) ^ 1u, abort_flag)) { aborted = true; return; }
-        const uint32_t base = (is_v ? C::oV : C::oK) + st * 2 * C::TB;
-        if (!js.convert(j, base, base + C::TB, kv_idx)) { aborted = true; return; }
+        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, kv_idx)) { aborted = true; return; }
         mbar_arrive(&bars[(is_v ? F_VF : F_KF) + st]);
         ++cnt;
       }
@@ -939,9 +946,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       const int sb = t & 1;
       if (!wait_bar(&bars[F_SR + sb], (sc[sb] & 1u) ^ 1u, abort_flag)) return false;
       tc_after_sync();
-      const uint32_t sK = smem_u32(smem + C::oK + ks * 2 * C::TB);
-      mma_qk<DH, KT>(tmem + C::tS + sb * KT, sQ, sK, 0);
-      mma_qk<DH, KT>(tmem + C::tS + sb * KT, sQ, sK + C::TB, 1);
+      const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
+      mma_qk<DH, KT>(tmem + C::tS + sb * KT, sQ, sK, 0);   // the combined (16·MSB + LSB) tile
       mma_commit(&bars[F_SF + sb]);
       mma_commit(&bars[F_KE + ks]);
       ++sc[sb];
@@ -963,9 +969,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
         if (!wait_bar(&bars[F_VF + vs], (vc >> 1) & 1u, abort_flag)) { aborted = true; break; }
         tc_after_sync();
         const uint32_t sP = smem_u32(smem + C::oP + pb * C::PB);
-        const uint32_t sV = smem_u32(smem + C::oV + vs * 2 * C::TB);
-        mma_pv<DH, KT>(tmem + C::tO, sP, sV, t > 0 ? 1u : 0u);
-        mma_pv<DH, KT>(tmem + C::tO, sP, sV + C::TB, 1);
+        const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
+        mma_pv<DH, KT>(tmem + C::tO, sP, sV, t > 0 ? 1u : 0u);   // the combined tile
         mma_commit(&bars[F_PE + pb]);
         mma_commit(&bars[F_VE + vs]);
         ++pc[pb];
