@@ -213,7 +213,9 @@ int32_t spatten_attention_layer_noalloc(const spatten_attn_args* a, void* stream
  *  a 16 K-key sample brackets the k-th key, one pass counts the keys above the bracket and collects
  *  the bracket's keys, the exact threshold is chosen among them, one pass writes the output; rows
  *  whose bracket misses fall back to the cluster radix select.  Without it (or with fewer bytes)
- *  every row takes the cluster radix select.  Results are identical either way.
+ *  every row takes the cluster radix select.  Results are identical either way.  The workspace
+ *  holds only this call's intermediates (nothing to clear): later calls on the same stream may
+ *  reuse it, calls that overlap on the GPU need one each.
  * ============================================================================================= */
 size_t spatten_topk_workspace_size(int32_t R, int32_t n, int32_t k);
 int32_t spatten_topk_select(const float* scores, int32_t R, int32_t n, int64_t ld, int32_t k,
