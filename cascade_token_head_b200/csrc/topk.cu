@@ -2,19 +2,22 @@
 //
 // SpAtten §IV.B "Top-k Engine" avoids a full sort: it finds the k-th largest value as a threshold
 // with quick-select, filters the array against it and removes the gaps with a prefix-sum-driven
-// zero eliminator.  The B200 form of the same three steps:
-//   threshold  radix select over the order-preserving 32-bit image of each float: four 8-bit
-//              digit passes, each a shared-memory histogram of the keys that still match the
-//              known high digits; the CTAs of a thread-block cluster (one cluster per row) add
-//              their histograms through distributed shared memory, so every CTA learns the
-//              same digit without a trip through global memory.
-//   filter     a key is kept if it is above the threshold T, or equal to T and among the first
-//              (k - #above) equal keys in index order (ties go to the lower index).
-//   eliminate  warp ballots + popc give each kept key its output slot (a block-wide exclusive
-//              scan in index order), so the output is written in ascending index order.
-// Each CTA keeps up to kResident keys of its chunk in shared memory; the rest (only for rows
-// longer than clusters x kResident) is streamed again from L2 in every pass, eight keys per
-// thread with 16-byte loads, and compacted with block-wide prefix sums of per-thread counts.
+// zero eliminator.  The B200 forms of the same three steps, by row length:
+//   n <= 8192      (topk_small_kernel) the row's order-preserving 32-bit keys live in registers;
+//                  the threshold is a two-bits-per-round digit search with warp reductions; one
+//                  packed block scan places every kept key.
+//   longer rows    (topk_cluster_kernel) radix select over the keys: four 8-bit digit passes, each
+//                  a shared-memory histogram of the keys that still match the known high digits;
+//                  the CTAs of a thread-block cluster (one cluster per row) add their histograms
+//                  through distributed shared memory.  Each CTA keeps up to kResident keys of its
+//                  chunk in shared memory; the rest is streamed again from L2 in every pass.
+//   n >= 65536 with the caller's workspace (sample / filter / resolve / output kernels): a
+//                  sampled rank window around the k-th key, one streaming pass that counts the keys
+//                  above the window and collects the window's keys, an exact select among those
+//                  candidates, one streaming pass that writes the output (see the section below).
+// In every form a key is kept if it is above the threshold T, or equal to T and among the first
+// (k - #above) equal keys in index order (ties go to the lower index), and warp ballots / block
+// scans give each kept key its output slot in ascending index order.
 #include <cooperative_groups.h>
 
 #include "common.cuh"

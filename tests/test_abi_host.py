@@ -78,6 +78,25 @@ def test_topk_argument_errors(S):
     assert L.spatten_topk_select(16, 1, 10, 10, 3, None, 0, 16, 3, 32, None, 0, None, None) == S.E_ARG
 
 
+def test_topk_workspace_size_rules(S):
+    """The optional top-k workspace: none below 64 K keys per row; from there, at least the
+    candidate lists (8 bytes per candidate, max(4096, n/16) candidates per row) plus the per-chunk
+    counters (8 K-key chunks); linear in the row count; k does not matter; rows longer than 8192
+    chunks (64 M keys) take the cluster kernel and need none."""
+    f = S.topk_workspace_size
+    for n in (1, 1000, 65535):
+        assert f(64, n, max(1, n // 2)) == 0
+    for n in (65536, 262144, 1048576, 1 << 22):
+        nchunk = -(-n // 8192)
+        need = 64 * (max(4096, n // 16) * 8 + nchunk * (4 + 4 + 64 * 4))
+        b = f(64, n, n // 2)
+        assert b >= need
+        assert b == f(64, n, 1) == f(64, n, n - 1)
+        assert f(128, n, 7) - b >= need - 256 * 16   # per-row parts (each region rounded to 256 B)
+    assert f(1, 8192 * 8192, 5) > 0
+    assert f(1, 8192 * 8192 + 1, 5) == 0
+
+
 def test_quantize_argument_errors(S):
     L = S.lib
     q = L.spatten_quantize_kv
