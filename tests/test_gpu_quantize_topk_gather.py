@@ -299,6 +299,43 @@ def test_topk_long_rows_tie_group_at_threshold(cuda):
         np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
 
 
+def test_topk_long_rows_special_values_and_strides(cuda):
+    """Long rows (n = 100003: a ragged last chunk) with special values, bit-exact against the
+    oracle for k from 1 to n - 7:
+    - row 0: 50 keys each of +inf and -inf (tie groups at the very top and bottom);
+    - row 1: half the keys zeros of either sign (-0.0 equals +0.0; a tie group of 50 K keys);
+    - row 2: denormals only;
+    - row 3: lognormal.
+    The row stride 100008 keeps the streaming path; the stride 100005 (not a multiple of 4) takes
+    the cluster kernel; the results agree."""
+    S = lib()
+    g = synth.rng_for(79)
+    R_, n = 4, 100003
+    x = g.standard_normal((R_, n)).astype(np.float32)
+    x[0, g.choice(n, 50, replace=False)] = np.inf
+    x[0, g.choice(n, 50, replace=False)] = -np.inf
+    z = g.choice(n, n // 2, replace=False)
+    x[1, z] = np.where(g.random(z.size) < 0.5, -0.0, 0.0).astype(np.float32)
+    x[2] = (g.standard_normal(n) * 1e-39).astype(np.float32)
+    x[3] = g.lognormal(0.0, 2.0, n).astype(np.float32)
+    want = {k: [R.topk_select(x[r].astype(np.float64), k) for r in range(R_)] for k in (1, 3000, n // 2, n - 7)}
+    for ld in (100008, 100005):
+        buf = np.zeros((R_, ld), np.float32)
+        buf[:, :n] = x
+        sc = to_dev(buf)
+        for k, rows in want.items():
+            out = torch.full((R_, k), -1, dtype=torch.int32, device="cuda")
+            st = torch.zeros(1, dtype=torch.int32, device="cuda")
+            nb = S.topk_workspace_size(R_, n, k)
+            ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+            S.topk_select(sc, R_, n, ld, k, out, k, ws=ws, ws_bytes=nb, dev_status=st)
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+            got = out.cpu().numpy()
+            for r in range(R_):
+                np.testing.assert_array_equal(got[r], rows[r], err_msg=f"ld {ld} k {k} row {r}")
+
+
 # ------------------------------------------------------------------------------------------------
 # K5 gather
 # ------------------------------------------------------------------------------------------------
