@@ -270,23 +270,24 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------------
-class Ctx:
-    """Device, ranks, stream and the L2 flush buffer shared by the workloads."""
+class Ranks:
+    """Rank identity (RANK / WORLD_SIZE / LOCAL_RANK from the launcher) and the only collectives the
+    bench takes: a barrier and a max over ranks of a device time.  No collective touches the data
+    path; each rank runs its own sequences (seeded by its rank).  backend "nccl" with a CUDA device
+    on the GPU, "gloo" with the CPU (tests)."""
 
-    def __init__(self):
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: int = 120):
         import torch
         import torch.distributed as dist
         self.torch, self.dist = torch, dist
         self.rank = int(os.environ.get("RANK", "0"))
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(self.local)
-        self.dev = torch.device("cuda", self.local)
+        self.device = device if device is not None else torch.device("cpu")
         if self.world > 1:
             from datetime import timedelta
-            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=self.dev)
-        self.stream = torch.cuda.current_stream()
-        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=self.dev)
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
 
     def barrier(self):
         if self.world > 1:
@@ -295,9 +296,32 @@ class Ctx:
     def max_over_ranks(self, v: float) -> float:
         if self.world == 1:
             return v
-        t = self.torch.tensor([v], device=self.dev)
+        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_total_ms: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank_step per step, and the
+    job takes the slowest rank's time (weak scaling)."""
+    return world * units_per_rank_step * steps / (max_total_ms / 1e3)
+
+
+class Ctx(Ranks):
+    """Device, ranks, stream and the L2 flush buffer shared by the workloads."""
+
+    def __init__(self):
+        import torch
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        super().__init__("nccl", torch.device("cuda", local))
+        self.dev = self.device
+        self.stream = torch.cuda.current_stream()
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=self.dev)
 
     def events(self, n):
         """n timing events, materialised on the stream so their handles can be handed over."""
@@ -499,7 +523,7 @@ def prefill_arm(ctx, args, name):
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     result = {
         "metric": METRIC[name],
-        "value": ctx.world * tokens_per_step * K / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": ctx.world,
+        "value": whole_job_rate(ctx.world, tokens_per_step, K, total_ms), "unit": "tokens/s", "n_gpus": ctx.world,
         "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
         "config": {"workload": w.name, "global_batch": B * ctx.world, "seq_len": T, "d_model": D, "heads": H,
@@ -511,12 +535,12 @@ def prefill_arm(ctx, args, name):
                      "peak_kind": f"{peak_kind} bf16 sustained (the MMAs take fp16 operands: same nominal "
                                   f"dense rate, ratio 1)", "traffic": None,
                      "algorithmic_flops_per_step": flops, "attn_ms_per_step": attn_s * 1e3},
-        "e2e": {"value": ctx.world * tokens_per_step * n_e2e / (e2e_total / 1e3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(ctx.world, tokens_per_step, n_e2e, e2e_total), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "method": f"{n_e2e} consecutive steps timed together, each a direct spatten_cascade_forward "
                           f"call; each step's copies in and out on a second stream, overlapping the "
                           f"neighbouring steps' forward",
-                "graph_value": (ctx.world * tokens_per_step * n_e2e / (e2e_graph_total / 1e3)
+                "graph_value": (whole_job_rate(ctx.world, tokens_per_step, n_e2e, e2e_graph_total)
                                 if e2e_graph_total else None),
                 "graph_method": "the same loop, each step's forward replayed from a CUDA graph captured from "
                                 "the same call"},
@@ -593,7 +617,7 @@ def decode_arm(ctx, args, steps):
     all_rows = w.B * w.H * w.steps * L
     result = {
         "metric": METRIC["gpt2m_decode"],
-        "value": ctx.world * tokens * steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": ctx.world,
+        "value": whole_job_rate(ctx.world, tokens, steps, total_ms), "unit": "tokens/s", "n_gpus": ctx.world,
         "steps": steps, "warmup": args.warmup, "ms_per_step": total_ms / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
         "config": {"workload": w.name, "global_batch": w.B * ctx.world, "prompt_len": w.T0,
@@ -605,7 +629,7 @@ def decode_arm(ctx, args, steps):
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} HBM copy", "traffic": None,
                      "algorithmic_bytes_per_step": nbytes, "attn_ms_per_step": attn_s * 1e3},
-        "e2e": {"value": ctx.world * tokens * n_e2e / (e2e_total / 1e3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(ctx.world, tokens, n_e2e, e2e_total), "unit": "tokens/s",
                 "h2d_bytes_per_step": xs_host.numel() * 2,
                 "d2h_bytes_per_step": outs_host.numel() * 2 + imp_host.numel() * 4},
         "gpu_launches": int(launches_per_gen * steps),
@@ -632,8 +656,7 @@ def run_ours(args):
             result["decode"] = {k: dec[k] for k in ("metric", "value", "unit", "steps", "ms_per_step", "config",
                                                     "roofline", "e2e", "gpu_launches", "clocks",
                                                     "refetched_row_fraction", "cpu_baseline") if k in dec}
-    if ctx.world > 1:
-        ctx.dist.destroy_process_group()
+    ctx.close()
     if ctx.rank == 0:
         print(json.dumps(result), flush=True)
     return 0
