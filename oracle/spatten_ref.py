@@ -11,7 +11,7 @@ below are that page's: §II "Background and Motivation", §II.B "Motivation", §
 Pruning" (printed as "A." after §II.B), §IV "Hardware Architecture", §IV.B "Top-k Engine",
 §IV.E "Query-Key Multiplication Module".
 
-Readings where the page is silent (each is listed with its reason in the design doc):
+Readings where the page is silent:
   * scale is 1/sqrt(d_h) ("scaled Q x K^T", §II);
   * 12-bit symmetric codes, one float32 scale per (sequence, layer, head, tensor) computed as
     amax/2047 in float32; codes are round-half-even of float32(x)/s, clamped to +-2047;
