@@ -130,13 +130,15 @@ def dequant(msb: np.ndarray, lsb: np.ndarray | None, scale) -> np.ndarray:
 # C3  progressive-quantization attention for one head (§IV.E "Progressive Quantization")
 # ---------------------------------------------------------------------------------------------
 def progressive_attention(Q, kq: dict, vq: dict, theta: float, sm_scale: float,
-                          flags_override: np.ndarray | None = None):
+                          flags_override: np.ndarray | None = None, v_keep: int | None = None):
     """MSB pass first; rows whose max probability is below theta refetch the LSBs and recompute
     their scores, probabilities and outputs with the full 12-bit K and V.
 
     ``kq``/``vq`` are quantize_head() results.  ``flags_override`` (bool [n_q]) replaces the
     computed decision; it is used only to compare against a device run row by row after the
-    near-tie rows were checked.  Returns dict(O, P, flags, pmax_msb).
+    near-tie rows were checked.  ``v_keep``: local value pruning of this head (see
+    value_keep_mask) on the final probabilities; None keeps every V vector.
+    Returns dict(O, P, flags, pmax_msb, v_kept).
     """
     Q = np.asarray(Q, np.float64)
     K_msb = dequant(kq["msb"], None, kq["scale"])
@@ -148,16 +150,48 @@ def progressive_attention(Q, kq: dict, vq: dict, theta: float, sm_scale: float,
     if flags_override is not None:
         flags = np.asarray(flags_override, bool)
     P = P_msb.copy()
-    O = P_msb @ V_msb
-    if flags.any():
+    rows = np.nonzero(flags)[0]
+    if rows.size:
         K_full = dequant(kq["msb"], kq["lsb"], kq["scale"])
-        V_full = dequant(vq["msb"], vq["lsb"], vq["scale"])
-        rows = np.nonzero(flags)[0]
         S_full = (Q[rows] @ K_full.T) * sm_scale
         P_full, _ = attention_probs(S_full)
         P[rows] = P_full
-        O[rows] = P_full @ V_full
-    return dict(O=O, P=P, flags=flags, pmax_msb=pmax)
+    mask, kept = value_keep_mask(P, v_keep)
+    Pv = P * mask                      # P itself when every V vector is kept
+    O = Pv @ V_msb
+    if rows.size:
+        V_full = dequant(vq["msb"], vq["lsb"], vq["scale"])
+        O[rows] = Pv[rows] @ V_full
+    return dict(O=O, P=P, flags=flags, pmax_msb=pmax, v_kept=kept)
+
+
+# ---------------------------------------------------------------------------------------------
+# local value pruning (§III.A "Local Value Pruning")
+# ---------------------------------------------------------------------------------------------
+def value_keep_mask(P: np.ndarray, v_keep: int | None):
+    """After the softmax a head drops its low-probability V vectors, for this head only (nothing
+    is removed from other heads or layers).  Reading: a key's probability for the head is its
+    column sum over the head's query rows (its share of the head's attention; one query row in
+    decode); the head keeps the V vectors of the v_keep keys ranked first by (higher column sum,
+    then lower index), the top-k rule; the dropped keys' probabilities are not redistributed.
+    Returns (mask [n_kv] of 0/1 floats, kept indices ascending); v_keep None keeps all."""
+    P = np.asarray(P, np.float64)
+    n = P.shape[1]
+    if v_keep is None:
+        return np.ones(n), np.arange(n)
+    kept = topk_select(P.sum(axis=0), int(v_keep))
+    mask = np.zeros(n)
+    mask[kept] = 1.0
+    return mask, kept
+
+
+def dense_attention_value_pruned(Q, K, V, sm_scale: float, v_keep: int | None):
+    """C1 followed by local value pruning of the head: O = (P * mask) @ V."""
+    O, P = dense_attention(Q, K, V, sm_scale)
+    if v_keep is None:
+        return O, P, np.arange(P.shape[1])
+    mask, kept = value_keep_mask(P, v_keep)
+    return (P * mask) @ np.asarray(V, np.float64), P, kept
 
 
 # ---------------------------------------------------------------------------------------------
@@ -193,9 +227,11 @@ def topk_select(scores: np.ndarray, k: int) -> np.ndarray:
 # one attention layer over the kept tokens / heads of one sequence
 # ---------------------------------------------------------------------------------------------
 def attention_layer_seq(Q, K, V, heads, d_h: int, H: int, quant: bool, theta: float,
-                        sm_scale: float, key_gain=None, flags_override=None):
+                        sm_scale: float, key_gain=None, flags_override=None, v_keep: int | None = None):
     """Q, K, V: [n, H*d_h] projections of the kept rows (all heads).  ``heads``: kept head ids.
-    ``key_gain`` [n]: per-token factor applied to K after projection (boosted keys).
+    ``key_gain`` [n]: per-token factor applied to K after projection (boosted keys).  ``v_keep``:
+    V vectors each head keeps under local value pruning (None: all); token importance uses the
+    full probabilities, head importance the pruned outputs.
 
     Returns dict(O [n, H*d_h] with zeros for pruned heads, tok_inc [n], head_inc [H],
     flags {h: bool[n]}, pmax {h: [n]}, codes {h: (kq, vq)}, refetch (count of refetched rows)).
@@ -219,7 +255,7 @@ def attention_layer_seq(Q, K, V, heads, d_h: int, H: int, quant: bool, theta: fl
             kq = quantize_head(k32)
             vq = quantize_head(v.astype(np.float32))
             fo = None if flags_override is None else flags_override.get(h)
-            r = progressive_attention(q, kq, vq, theta, sm_scale, flags_override=fo)
+            r = progressive_attention(q, kq, vq, theta, sm_scale, flags_override=fo, v_keep=v_keep)
             Oh, P = r["O"], r["P"]
             flags[h], pmaxs[h] = r["flags"], r["pmax_msb"]
             codes[h] = (kq, vq)
@@ -227,7 +263,7 @@ def attention_layer_seq(Q, K, V, heads, d_h: int, H: int, quant: bool, theta: fl
         else:
             if key_gain is not None:
                 k = k * np.asarray(key_gain, np.float64)[:, None]
-            Oh, P = dense_attention(q, k, v, sm_scale)
+            Oh, P, _ = dense_attention_value_pruned(q, k, v, sm_scale, v_keep)
         O[:, sl] = Oh
         tok_inc += token_importance_increment(P)
         head_inc[h] += head_importance_increment(Oh)

@@ -11,6 +11,7 @@ from oracle import spatten_ref as R
 import test_oracle_attention as TA
 import test_oracle_cascade as TC
 import test_oracle_quant_topk as TQ
+import test_oracle_value_pruning as TV
 
 
 @contextlib.contextmanager
@@ -70,18 +71,41 @@ def _signed_head_importance(O):
 _orig_prog = R.progressive_attention
 
 
-def _prog_le(Q, kq, vq, theta, sm_scale, flags_override=None):
-    r = _orig_prog(Q, kq, vq, theta, sm_scale, flags_override)
+def _prog_le(Q, kq, vq, theta, sm_scale, flags_override=None, v_keep=None):
+    r = _orig_prog(Q, kq, vq, theta, sm_scale, flags_override, v_keep)
     if flags_override is None:
         fl = r["pmax_msb"] <= theta
         if not np.array_equal(fl, r["flags"]):
-            r = _orig_prog(Q, kq, vq, theta, sm_scale, fl)
+            r = _orig_prog(Q, kq, vq, theta, sm_scale, fl, v_keep)
     return r
 
 
-def _prog_full_v_never(Q, kq, vq, theta, sm_scale, flags_override=None):
+def _prog_full_v_never(Q, kq, vq, theta, sm_scale, flags_override=None, v_keep=None):
     vq2 = dict(vq, lsb=np.zeros_like(vq["lsb"]))     # forgets the V LSBs on refetch
-    return _orig_prog(Q, kq, vq2, theta, sm_scale, flags_override)
+    return _orig_prog(Q, kq, vq2, theta, sm_scale, flags_override, v_keep)
+
+
+def _vkeep_high_index_ties(P, v_keep):
+    P = np.asarray(P, np.float64)
+    n = P.shape[1]
+    if v_keep is None:
+        return np.ones(n), np.arange(n)
+    col = P.sum(axis=0)
+    kept = np.sort(np.lexsort((-np.arange(n), -col))[:v_keep])   # ties to the higher index
+    mask = np.zeros(n)
+    mask[kept] = 1.0
+    return mask, kept
+
+
+def _vkeep_by_column_max(P, v_keep):
+    P = np.asarray(P, np.float64)
+    n = P.shape[1]
+    if v_keep is None:
+        return np.ones(n), np.arange(n)
+    kept = R.topk_select(P.max(axis=0), v_keep)                  # ranks by the largest probability
+    mask = np.zeros(n)
+    mask[kept] = 1.0
+    return mask, kept
 
 
 MUTANTS = [
@@ -95,6 +119,8 @@ MUTANTS = [
     ("head_importance_increment", _signed_head_importance, [TA.test_head_importance_closed_forms]),
     ("progressive_attention", _prog_le, [lambda: TA.test_constant_keys_refetch_iff_uniform_prob_below_theta(0.1, False)]),
     ("progressive_attention", _prog_full_v_never, [TC.test_cascade_keep_all_always_refetch_equals_dense_on_full_codes]),
+    ("value_keep_mask", _vkeep_high_index_ties, [lambda: TV.test_uniform_attention_closed_form(8, 3)]),
+    ("value_keep_mask", _vkeep_by_column_max, [lambda s=s: TV.test_brute_force_small(s) for s in range(4)]),
 ]
 
 
