@@ -237,27 +237,33 @@ def run_reference(args):
     if rank != 0:
         return 0
     from cascade_token_head_b200 import synth
+    steps = max(1, args.steps)
+    # every step is one bounded unit of the workload: warm-up and timed runs take exactly
+    # args.warmup and `steps` units (no time budget)
     if args.workload == "gpt2m_decode":
         w = synth.gpt2m_decode()
         o = OracleDecode(w, synth.draw_decode(w))
-        o.generate(0.0, max_tokens=args.warmup)
+        if args.warmup > 0:
+            o.generate(math.inf, max_tokens=args.warmup)
         t0 = time.perf_counter()
-        o.generate(0.0, max_tokens=args.steps)
+        _, done, _ = o.generate(math.inf, max_tokens=steps)
         el = time.perf_counter() - t0
-        value = args.steps * w.B / el
+        value = done * w.B / el
         cfg = {"workload": w.name, "global_batch": w.B, "prompt_len": w.T0, "parallelism": "replicas"}
-        sample = f"one generated token of all {w.B} sequences (all {w.L} layers) per step"
+        sample = f"one generated token of all {w.B} sequences (all {w.L} layers) per step, {done} steps"
     else:
         w = prefill_workload(args.workload)
         d = synth.draw_prefill(w)
-        oracle_prefill_sample(w, d, 0.0, max_units=args.warmup)
+        if args.warmup > 0:
+            oracle_prefill_sample(w, d, math.inf, max_units=args.warmup)
         t0 = time.perf_counter()
-        value, sample, _ = oracle_prefill_sample(w, d, 0.0, max_units=args.steps)
+        value, sample, _ = oracle_prefill_sample(w, d, math.inf, max_units=steps)
         el = time.perf_counter() - t0
         cfg = {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "replicas"}
-        sample = f"per step: {sample}"
+        unit = "one sequence" if w.T <= 4096 else "one head's layer-0 attention"
+        sample = f"{unit} per step ({sample})"
     line = {"metric": METRIC[args.workload], "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
             "config": cfg, "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",

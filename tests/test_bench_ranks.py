@@ -69,3 +69,18 @@ def test_single_rank_needs_no_process_group():
         assert r.max_over_ranks(3.5) == 3.5
         r.barrier()
         r.close()
+
+
+def test_reference_arm_times_exactly_the_requested_steps(capsys):
+    """The reference arm (the float64 oracle) times exactly --steps units of the workload, one
+    sequence per step for the BERT-shaped prefill, and reports consistent per-step numbers."""
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.pop("RANK", None)
+    assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "0"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 2
+    assert "2 sequence(s)" in line["cpu_baseline"]["sample"]
+    per_step_s = line["ms_per_step"] / 1e3
+    assert line["value"] == pytest.approx(512 / per_step_s, rel=0.25)   # tokens/s of one sequence per step
+    assert line["e2e"]["value"] == line["value"]
