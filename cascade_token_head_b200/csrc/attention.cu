@@ -169,5 +169,6 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
 
 extern "C" int32_t spatten_attention_layer(const spatten_attn_args* args, void* ws,
                                            size_t ws_bytes, void* stream) {
+  spt::AbiRange nvtx_range("spatten_attention_layer");
   return spt::attention_layer_timed(args, ws, ws_bytes, spt::as_stream(stream), nullptr, nullptr);
 }

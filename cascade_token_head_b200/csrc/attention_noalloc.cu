@@ -50,6 +50,7 @@ int32_t scratch_address(void** out) {
 }  // namespace spt
 
 extern "C" int32_t spatten_attention_layer_noalloc(const spatten_attn_args* a, void* stream) {
+  spt::AbiRange nvtx_range("spatten_attention_layer_noalloc");
   using namespace spt;
   if (!a) return SPATTEN_E_ARG;
   const size_t need = spatten_attention_workspace_size(a);

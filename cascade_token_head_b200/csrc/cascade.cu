@@ -383,6 +383,7 @@ extern "C" size_t spatten_cascade_workspace_size(const spatten_cascade_cfg* cfg)
 
 extern "C" int32_t spatten_cascade_forward(const spatten_cascade_cfg* cfg, const spatten_layer_weights* w,
                                            spatten_cascade_io* io, void* ws, size_t ws_bytes, void* stream) {
+  spt::AbiRange nvtx_range("spatten_cascade_forward");
   using namespace spt;
   if (!cfg || !w || !io) return SPATTEN_E_ARG;
   SPT_TRY(validate_cfg(*cfg));

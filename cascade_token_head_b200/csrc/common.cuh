@@ -3,11 +3,21 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "spatten.h"
 
 namespace spt {
+
+// An NVTX range over one C-ABI call, named after the call: it shows the call's span (host
+// enqueue) in profiler timelines; without a profiler attached the push and pop do nothing.
+struct AbiRange {
+  explicit AbiRange(const char* name) { nvtxRangePushA(name); }
+  ~AbiRange() { nvtxRangePop(); }
+  AbiRange(const AbiRange&) = delete;
+  AbiRange& operator=(const AbiRange&) = delete;
+};
 
 // ----------------------------------------------------------------------------------------------
 // host-side status helpers

@@ -114,6 +114,7 @@ extern "C" int32_t spatten_gather_kept(const void* src, int64_t src_batch, int64
                                        const int32_t* compose_in, int64_t ld_compose,
                                        int32_t* compose_out, int32_t check_index,
                                        int32_t* dev_status, void* stream) {
+  spt::AbiRange nvtx_range("spatten_gather_kept");
   using namespace spt;
   if (R < 1 || k < 0 || n_src < 1) return SPATTEN_E_ARG;
   if (k == 0) return SPATTEN_OK;

@@ -393,6 +393,7 @@ extern "C" int32_t spatten_quantize_kv(const void* x, int32_t dtype, int32_t B, 
                                        int32_t d_h, int64_t ld_tok, const float* row_gain, int64_t ld_gain,
                                        const float* scale_in, int8_t* msb, uint8_t* lsb, int32_t cap,
                                        int32_t row0, float* scale_out, int32_t* sat_count, void* stream) {
+  spt::AbiRange nvtx_range("spatten_quantize_kv");
   using namespace spt;
   SPT_TRY(quantize_check(x, dtype, B, H, n, d_h, ld_tok, row_gain, ld_gain, scale_in, msb, lsb, cap, row0, scale_out));
   QArgs a{};

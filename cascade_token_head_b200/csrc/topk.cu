@@ -1338,6 +1338,7 @@ extern "C" int32_t spatten_topk_select(const float* scores, int32_t R, int32_t n
                                        int32_t* idx_out, int64_t ld_out, int32_t* comp_out,
                                        void* ws, size_t ws_bytes, int32_t* dev_status,
                                        void* stream) {
+  spt::AbiRange nvtx_range("spatten_topk_select");
   using namespace spt;
   if (!scores || (!idx_out && !comp_out)) return SPATTEN_E_ARG;
   if (R < 1 || n < 1 || k < 0 || R > 65535) return SPATTEN_E_ARG;
