@@ -2,6 +2,8 @@
 (a transposed operand, a dropped term, a wrong sign or rounding or tie rule) and checks that at
 least one of the oracle's pins fails.  Mistakes are planted in the oracle only, on the CPU."""
 import contextlib
+import inspect
+import textwrap
 
 import numpy as np
 import pytest
@@ -85,6 +87,61 @@ def _prog_full_v_never(Q, kq, vq, theta, sm_scale, flags_override=None, v_keep=N
     return _orig_prog(Q, kq, vq2, theta, sm_scale, flags_override, v_keep)
 
 
+def source_mutant(fn, old, new):
+    """A copy of oracle function `fn` with one statement of its source replaced: a planted mistake
+    in a function too large to restate by hand.  The copy calls the unpatched oracle helpers."""
+    src = textwrap.dedent(inspect.getsource(fn))
+    assert src.count(old) == 1, old
+    ns = dict(vars(R))
+    exec(compile(src.replace(old, new), f"<mutant of {fn.__name__}>", "exec"), ns)
+    return ns[fn.__name__]
+
+
+_orig_dequant = R.dequant
+_orig_als = R.attention_layer_seq
+
+
+def _codes_half_away(x32, scale):
+    t = np.asarray(x32, np.float32) / np.float32(scale)
+    r = np.sign(t) * np.floor(np.abs(t) + np.float32(0.5))     # ties away from zero
+    return np.clip(r, -R.QMAX, R.QMAX).astype(np.int32), int(np.count_nonzero(np.abs(r) > R.QMAX))
+
+
+def _dequant_no_lsb(msb, lsb, scale):
+    return _orig_dequant(msb, None, scale)                       # the LSB field is never added
+
+
+def _unpack_swapped(packed):
+    p = np.asarray(packed, np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), np.uint8)
+    out[..., 0::2] = p >> 4
+    out[..., 1::2] = p & 0xF
+    return out
+
+
+def _gain_on_values(Q, K, V, heads, d_h, H, quant, theta, sm_scale, key_gain=None, flags_override=None,
+                    v_keep=None):
+    if key_gain is not None:                                     # the boost lands on V, not K
+        V = np.asarray(V, np.float64) * np.asarray(key_gain, np.float64)[:, None]
+    return _orig_als(Q, K, V, heads, d_h, H, quant, theta, sm_scale, None, flags_override, v_keep)
+
+
+def _every_head(Q, K, V, heads, d_h, H, quant, theta, sm_scale, key_gain=None, flags_override=None,
+                v_keep=None):
+    return _orig_als(Q, K, V, range(H), d_h, H, quant, theta, sm_scale, key_gain, flags_override, v_keep)
+
+
+_cascade_reset_importance = source_mutant(R.cascade_prefill, 'I[b, S] += r["tok_inc"]', 'I[b, S] = r["tok_inc"]')
+_cascade_no_residual = source_mutant(R.cascade_prefill, 'X[b, S] = Xk + r["O"] @ w_o[l]', 'X[b, S] = r["O"] @ w_o[l]')
+_decode_fresh_scale = source_mutant(   # the appended K row is quantized with its own amax scale
+    R.decode_step, 'c["k_msb"][b, h, n_old] = kq["msb"][0]',
+    'kq = quantize_head(qkv[b, HD + h * d_h: HD + (h + 1) * d_h][None].astype(np.float32)); '
+    'c["k_msb"][b, h, n_old] = kq["msb"][0]')
+_decode_keep_old_count = source_mutant(R.decode_step, 'ks = keep_fn(n)', 'ks = keep_fn(n_old)')
+_decode_reset_importance = source_mutant(R.decode_step, 'I[b, S] += token_importance_increment(r["P"])',
+                                         'I[b, S] = token_importance_increment(r["P"])')
+
+
 def _vkeep_high_index_ties(P, v_keep):
     P = np.asarray(P, np.float64)
     n = P.shape[1]
@@ -121,6 +178,16 @@ MUTANTS = [
     ("progressive_attention", _prog_full_v_never, [TC.test_cascade_keep_all_always_refetch_equals_dense_on_full_codes]),
     ("value_keep_mask", _vkeep_high_index_ties, [lambda: TV.test_uniform_attention_closed_form(8, 3)]),
     ("value_keep_mask", _vkeep_by_column_max, [lambda s=s: TV.test_brute_force_small(s) for s in range(4)]),
+    ("quantize_codes", _codes_half_away, [TQ.test_quant_rounding_brute_force_near_half_boundaries]),
+    ("dequant", _dequant_no_lsb, [lambda: TQ.test_quant_identity_and_bounds(0)]),
+    ("unpack_lsb", _unpack_swapped, [TQ.test_lsb_pack_golden]),
+    ("attention_layer_seq", _gain_on_values, [TA.test_key_gain_scales_key_rows]),
+    ("attention_layer_seq", _every_head, [TC.test_cascade_pruning_invariants]),
+    ("cascade_prefill", _cascade_reset_importance, [TC.test_cascade_pruning_invariants]),
+    ("cascade_prefill", _cascade_no_residual, [TC.test_cascade_keep_all_unquantized_equals_dense_layers]),
+    ("decode_step", _decode_fresh_scale, [TC.test_decode_keep_all_full_equals_dense_over_cache]),
+    ("decode_step", _decode_keep_old_count, [TC.test_decode_pruning_nested_and_sized]),
+    ("decode_step", _decode_reset_importance, [TC.test_decode_keep_all_full_equals_dense_over_cache]),
 ]
 
 
