@@ -509,23 +509,24 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 //  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256) and finds by a digit
 //           search the sample keys e0 >= e64 at the two ends of a rank window around the sample
 //           rank of the k-th key (+-4 sigma of the sampling error + 16; an end past the sample is
-//           left open).  The search runs first on
-//           one key in 16, whose window (widened by its own sampling error) bounds the few
-//           thousand sample keys the exact search then needs
-//  filter   per chunk of 8 K keys: the count above e0, the keys in [e64, e0] appended as
-//           (key, index) to the row's candidate list, and their histogram over 64 sub-bins of
-//           equal width in value between e0 and e64
+//           left open).  The search runs first on one key in 16, whose own window, widened by its
+//           sampling error, bounds the few thousand sample keys the exact search then needs.  It
+//           also fixes the sub-bin scale: 64 steps of equal width in value between the window's
+//           ends (the sample's extreme key in place of an open end).
+//  filter   per chunk of 8 K keys: the count above e0, the keys in [e64, e0] appended as (score
+//           bits, index) to the row's candidate list, and their histogram over the 64 sub-bins
 //  resolve  one CTA per row: the sub-bin holding the k-th key, the exact threshold among that
 //           sub-bin's candidates as the (need)-th largest (key, ~index) composite (ties to the lower
-//           index), and every chunk's output offset
-//  output   per chunk: key > T, or key = T and index <= T_index, written in index order
+//           index), whether the keys equal to T are split by index, and every chunk's output offset
+//  output   per chunk: key > T, or key = T and index <= T_index (key >= T when the keys equal to T
+//           are all taken), written in index order
 // A row whose k-th key fell outside the window, or whose buffers overflowed, is marked and done
 // again by the cluster kernel (only_rows).
-// Filter and output read a warp's 512 keys as four coalesced 16-byte loads per lane (load q of
-// lane t holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span), so a key's place in index
-// order is (warp, q, lane, element).  They compare floats against the window ends and the threshold
-// turned back into floats (the key map is monotone, and -0.0 equals +0.0 on both sides); a NaN
-// fails every ordered comparison, lands in the candidate list and is reported by the resolve step.
+// The filter reads a warp's 512 keys as four coalesced 16-byte loads per lane (load q of lane t
+// holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span); the output step reads them as 16
+// columns of 32 (see there).  Both compare floats against the window ends and the threshold turned
+// back into floats (the key map is monotone, and -0.0 equals +0.0 on both sides); a NaN fails every
+// ordered comparison, lands in the candidate list and is reported by the resolve step.
 // ------------------------------------------------------------------------------------------------
 constexpr int kStreamMin = 65536;
 constexpr int kSRuns = 64, kSRun = 256, kSamples = kSRuns * kSRun;   // 16 K sample keys per row
