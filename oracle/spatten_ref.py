@@ -337,7 +337,7 @@ def cascade_prefill(X, w_qkv, w_o, H: int, d_h: int, token_keep, head_keep, quan
 #     one new token per iteration against cached K and V)
 # ---------------------------------------------------------------------------------------------
 def decode_step(x, caches, n_old: int, I, w_qkv, w_o, H: int, d_h: int, keep_fn, theta: float,
-                sm_scale: float | None = None, teacher: dict | None = None):
+                sm_scale: float | None = None, teacher: dict | None = None, v_keep_fn=None):
     """One generation step for B sequences.
 
     x [B, D]: this step's input rows.  caches[l]: dict with k_msb, k_lsb, v_msb, v_lsb
@@ -345,7 +345,9 @@ def decode_step(x, caches, n_old: int, I, w_qkv, w_o, H: int, d_h: int, keep_fn,
     new token's K/V codes are appended at row n_old with the prompt-time scale (saturating).
     I [B, cap]: cumulative token importance, mutated in place.  keep_fn(n) -> [k_0..k_{L-1}].
     teacher (optional): {"qkv": [L] arrays [B, 3*H*d_h], "x": [L] arrays [B, D]} replaces the
-    projections and layer inputs with given values (teacher forcing).
+    projections and layer inputs with given values (teacher forcing).  v_keep_fn (optional):
+    v_keep_fn(l, k_l) -> V vectors each head of layer l keeps under local value pruning (its one
+    query row's probabilities rank the keys); None keeps them all.
 
     Per layer l: q,k,v = x_l @ W; append k,v; attend over S_l (S_0 = all n rows); I += P;
     x_{l+1} = x_l + O @ W_o; S_{l+1} = top-k_{l+1}(I restricted to S_l).
@@ -388,7 +390,8 @@ def decode_step(x, caches, n_old: int, I, w_qkv, w_o, H: int, d_h: int, keep_fn,
                 c["v_lsb"][b, h, n_old] = vq["lsb"][0]
                 kblk = dict(msb=c["k_msb"][b, h, S], lsb=c["k_lsb"][b, h, S], scale=c["k_scale"][b, h])
                 vblk = dict(msb=c["v_msb"][b, h, S], lsb=c["v_lsb"][b, h, S], scale=c["v_scale"][b, h])
-                r = progressive_attention(qkv[b, sl][None], kblk, vblk, theta, sm_scale)
+                vk = None if v_keep_fn is None else v_keep_fn(l, len(S))
+                r = progressive_attention(qkv[b, sl][None], kblk, vblk, theta, sm_scale, v_keep=vk)
                 O[b, sl] = r["O"][0]
                 flags[b, h] = r["flags"][0]
                 I[b, S] += token_importance_increment(r["P"])

@@ -96,3 +96,38 @@ def test_progressive_value_pruning_uses_each_row_precision():
         r = R.progressive_attention(Q, kq, vq, theta, 0.5, v_keep=4)
         np.testing.assert_array_equal(r["v_kept"], kept_w)
         np.testing.assert_allclose(r["O"], want, rtol=1e-12, atol=1e-14)
+
+
+def test_decode_step_value_pruning():
+    """Decode (one query row per head): keeping every V vector is the plain step; keeping v of
+    them gives, per layer and head, the probabilities of the v most probable keys times their V
+    rows (checked by hand on the step's own traced projections)."""
+    import math
+    import test_oracle_cascade as TC
+    B, H, d_h, D, T0, L = 2, 2, 8, 16, 20, 2
+    _, w_qkv, w_o, caches0 = TC._decode_setup(B, H, d_h, D, T0, L, seed=3)
+    x = np.random.default_rng(4).standard_normal((B, D))
+    copy = lambda cs: [{k: v.copy() for k, v in c.items()} for c in cs]
+    plain = R.decode_step(x, copy(caches0), T0, np.zeros((B, 24)), w_qkv, w_o, H, d_h, lambda n: [n] * L, 2.0)
+    same = R.decode_step(x, copy(caches0), T0, np.zeros((B, 24)), w_qkv, w_o, H, d_h, lambda n: [n] * L, 2.0,
+                         v_keep_fn=lambda l, k: k)
+    np.testing.assert_array_equal(same["x_out"], plain["x_out"])
+    caches = copy(caches0)
+    v = 5
+    r = R.decode_step(x, caches, T0, np.zeros((B, 24)), w_qkv, w_o, H, d_h, lambda n: [n] * L, 2.0,
+                      v_keep_fn=lambda l, k: v)
+    HD, n = H * d_h, T0 + 1
+    xs = r["xs"]
+    for l in range(L):
+        qkv = xs[l] @ w_qkv[l]
+        c = caches[l]
+        for b in range(B):
+            for h in range(H):
+                K = (16.0 * c["k_msb"][b, h, :n] + c["k_lsb"][b, h, :n]) * float(c["k_scale"][b, h])
+                V = (16.0 * c["v_msb"][b, h, :n] + c["v_lsb"][b, h, :n]) * float(c["v_scale"][b, h])
+                s = (K @ qkv[b, h * d_h:(h + 1) * d_h]) / math.sqrt(d_h)
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                top = sorted(sorted(range(n), key=lambda j: (-p[j], j))[:v])
+                want = sum(p[j] * V[j] for j in top)
+                np.testing.assert_allclose(r["O"][l][b, h * d_h:(h + 1) * d_h], want, rtol=1e-10, atol=1e-12)
