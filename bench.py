@@ -157,7 +157,7 @@ def oracle_prefill_sample(w, d, seconds: float, max_units: int | None = None):
     elapsed (at least one).  Long-context prefill (one sequence of 16384 tokens is minutes of
     oracle work): the oracle's layer-0 attention of whole heads (all query rows, in row blocks),
     extrapolated to the step by the ratio of the step's attention flops to the sample's.
-    Returns (tokens/s, description, threads)."""
+    Returns (tokens/s, description, threads, seconds spent on the sampled units)."""
     import numpy as np
     from oracle import spatten_ref as R
 
@@ -175,28 +175,35 @@ def oracle_prefill_sample(w, d, seconds: float, max_units: int | None = None):
             if el >= seconds or (max_units and done >= max_units):
                 break
         return done * w.T / el, f"{done} sequence(s) of the workload (T={w.T}, all {w.L} layers), {el:.1f} s", \
-            blas_threads()
+            blas_threads(), el
     X = _bf16_values(d["X"][0])
     qkv = X @ wq[0]
     HD = w.H * w.d_h
     sm = 1.0 / math.sqrt(w.d_h)
     gain = d["key_gain"][0].astype(np.float32)[:, None]
+    # units: blocks of 1024 query rows of one head (all keys), heads in turn; a head's K/V are
+    # quantized when its first block is taken
+    n_blk = (w.T + 1023) // 1024
+    cur_h, rows = -1, 0
     t0 = time.perf_counter()
     while True:
-        h = done % w.H
+        h, r0 = (done // n_blk) % w.H, (done % n_blk) * 1024
         c = slice(h * w.d_h, (h + 1) * w.d_h)
-        kq = R.quantize_head(qkv[:, HD:2 * HD][:, c].astype(np.float32) * gain)
-        vq = R.quantize_head(qkv[:, 2 * HD:][:, c].astype(np.float32))
-        for r0 in range(0, w.T, 1024):
-            R.progressive_attention(qkv[r0:r0 + 1024, c], kq, vq, w.theta, sm)
+        if h != cur_h:
+            kq = R.quantize_head(qkv[:, HD:2 * HD][:, c].astype(np.float32) * gain)
+            vq = R.quantize_head(qkv[:, 2 * HD:][:, c].astype(np.float32))
+            cur_h = h
+        R.progressive_attention(qkv[r0:r0 + 1024, c], kq, vq, w.theta, sm)
+        rows += min(1024, w.T - r0)
         done += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_units and done >= max_units):
             break
-    sample_flops = done * 4.0 * w.T * w.T * w.d_h
+    sample_flops = 4.0 * rows * w.T * w.d_h
     scale = attention_flops(w) / sample_flops
-    return w.T / (el * scale), (f"layer-0 attention of {done} head(s) (all {w.T} rows), {el:.1f} s, "
-                                f"extrapolated x{scale:.1f} by attention flops to one step"), blas_threads()
+    return w.T / (el * scale), (f"layer-0 attention of {done} block(s) of up to 1024 query rows of one head "
+                                f"(all {w.T} keys), {el:.1f} s, extrapolated x{scale:.0f} by attention flops "
+                                f"to one step"), blas_threads(), el
 
 
 class OracleDecode:
@@ -256,11 +263,9 @@ def run_reference(args):
         d = synth.draw_prefill(w)
         if args.warmup > 0:
             oracle_prefill_sample(w, d, math.inf, max_units=args.warmup)
-        t0 = time.perf_counter()
-        value, sample, _ = oracle_prefill_sample(w, d, math.inf, max_units=steps)
-        el = time.perf_counter() - t0
+        value, sample, _, el = oracle_prefill_sample(w, d, math.inf, max_units=steps)
         cfg = {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "replicas"}
-        unit = "one sequence" if w.T <= 4096 else "one head's layer-0 attention"
+        unit = "one sequence" if w.T <= 4096 else "one 1024-row block of one head's layer-0 attention"
         sample = f"{unit} per step ({sample})"
     line = {"metric": METRIC[args.workload], "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / steps,
@@ -555,7 +560,7 @@ def prefill_arm(ctx, args, name):
         "refetch_rows_per_layer": refetch_rows,
     }
     if ctx.rank == 0 and not args.no_cpu_baseline:
-        v, sample, threads = oracle_prefill_sample(w, d, args.cpu_seconds)
+        v, sample, threads, _ = oracle_prefill_sample(w, d, args.cpu_seconds)
         result["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                   "sample": sample}
     return result
