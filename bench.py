@@ -656,21 +656,174 @@ def decode_arm(ctx, args, steps):
     return result
 
 
+def graph_of(ctx, call):
+    """A CUDA graph of one call (captured after one direct run), and the library kernels it launches."""
+    from cascade_token_head_b200 import spatten as S
+    torch = ctx.torch
+    call(ctx.stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    l0 = S.kernel_launch_count()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    launches = S.kernel_launch_count() - l0
+    g.replay()
+    torch.cuda.synchronize()
+    return g, launches
+
+
+def hbm_entry(ctx, args, call, nbytes, h2d, d2h, what):
+    """Device time of one call (graph replays, L2 flushed between), its HBM roofline over the
+    algorithmic bytes, and the same call end to end with its host copies (e2e_body)."""
+    torch = ctx.torch
+    g, launches = graph_of(ctx, call)
+    K = max(5, args.steps)
+    for _ in range(3):
+        g.replay()
+    total_ms, clk = timed_replays(ctx, g.replay, K, lambda i: None)
+    t = total_ms / K / 1e3
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("hbm_gbs"))
+    achieved = nbytes / t / 1e9
+    e2e_ms, n = e2e_loop(ctx, lambda: (h2d(), g.replay(), d2h()), 3)
+    return {"us_per_call": t * 1e6, "gpu_launches_per_call": int(launches),
+            "roofline": {"kernel": what, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} HBM copy", "traffic": None,
+                         "algorithmic_bytes_per_call": nbytes},
+            "e2e_ms_per_call": e2e_ms / n, "clocks": clk}
+
+
+def topk_arm(ctx, args):
+    """The top-k sweep's long rows: 64 rows of N in {256k, 1M} keys, k = 10 % and 50 %, uniform and
+    lognormal values with 1 % exact duplicates.  GB/s over the algorithmic bytes 64 (4N + 4k)."""
+    import numpy as np
+    torch = ctx.torch
+    from cascade_token_head_b200 import spatten as S
+    from cascade_token_head_b200 import synth
+    R_, entries = 64, []
+    for N in (262144, 1048576):
+        for dist in ("uniform", "lognormal"):
+            x_np = synth.draw_topk_row_block(R_, N, dist, 0.01, seed=N % 9973 + (dist == "lognormal") + 100 * ctx.rank)
+            x_host = torch.from_numpy(x_np).pin_memory()
+            x = x_host.to(ctx.dev)
+            for frac in (0.1, 0.5):
+                k = int(frac * N)
+                out = torch.empty((R_, k), dtype=torch.int32, device=ctx.dev)
+                out_host = torch.empty((R_, k), dtype=torch.int32).pin_memory()
+                nb = S.topk_workspace_size(R_, N, k)
+                wsb = torch.empty(max(nb, 16), dtype=torch.uint8, device=ctx.dev)
+                call = lambda st, x=x, out=out, k=k, wsb=wsb, nb=nb: S.topk_select(
+                    x, R_, N, N, k, out, k, ws=wsb, ws_bytes=nb, stream=st)
+                e = hbm_entry(ctx, args, call, R_ * (4.0 * N + 4.0 * k),
+                              lambda x=x, x_host=x_host: x.copy_(x_host, non_blocking=True),
+                              lambda out=out, out_host=out_host: out_host.copy_(out, non_blocking=True),
+                              "spatten_topk_select (all of its launches)")
+                n_b = N * R_ * 4
+                e.update(N=N, k=k, dist=dist, value=R_ * (4.0 * N + 4.0 * k) / (e["us_per_call"] / 1e6) / 1e9,
+                         unit="GB/s",
+                         e2e={"value": R_ * (4.0 * N + 4.0 * k) / (e.pop("e2e_ms_per_call") / 1e3) / 1e9,
+                              "unit": "GB/s", "h2d_bytes_per_step": n_b, "d2h_bytes_per_step": R_ * k * 4})
+                if ctx.rank == 0 and not args.no_cpu_baseline:
+                    from oracle import spatten_ref as R
+                    t0, rows = time.perf_counter(), 0
+                    while rows < R_ and (rows == 0 or time.perf_counter() - t0 < 1.0):
+                        R.topk_select(x_np[rows].astype(np.float64), k)
+                        rows += 1
+                    el = time.perf_counter() - t0
+                    e["cpu_baseline"] = {"value": rows * (4.0 * N + 4.0 * k) / el / 1e9, "unit": "GB/s", "cores": 1,
+                                         "kind": "oracle", "sample": f"{rows} row(s) of the 64, {el:.2f} s"}
+                entries.append(e)
+                del out, wsb
+            del x
+    head = next(e for e in entries if e["N"] == 1048576 and e["k"] == 524288 and e["dist"] == "uniform")
+    return {"metric": "top-k select GB/s (64 rows, ascending indices, ties to the lower index)", "unit": "GB/s",
+            "value": head["value"], "config": {"workload": "topk_sweep_long_rows", "rows": R_,
+                                               "l2": "flushed between timed calls"},
+            "roofline": head["roofline"], "entries": entries}
+
+
+def gather_arm(ctx, args):
+    """Kept-row gathers of the two prefill workloads' X (bf16 rows): BERT-base layer 0 -> 1
+    (32 x 461 of 512 rows of 1536 B) and long-context layer 0 -> 1 (8192 of 16384 rows of 8192 B).
+    GB/s over the algorithmic bytes k (2 row_bytes + 4)."""
+    import numpy as np
+    torch = ctx.torch
+    from cascade_token_head_b200 import spatten as S
+    from cascade_token_head_b200 import synth
+    entries = []
+    for name, B, n, D, k in (("bert_base_x_rows", 32, 512, 768, 461), ("long_context_x_rows", 1, 16384, 4096, 8192)):
+        g = synth.rng_for(7 + ctx.rank)
+        src_host = torch.from_numpy(g.standard_normal((B, n, D)).astype(np.float32)).to(torch.bfloat16).pin_memory()
+        idx_np = np.stack([np.sort(g.choice(n, k, replace=False)) for _ in range(B)]).astype(np.int32)
+        src = src_host.to(ctx.dev)
+        idx = torch.from_numpy(idx_np).to(ctx.dev)
+        dst = torch.empty((B, k, D), dtype=torch.bfloat16, device=ctx.dev)
+        dst_host = torch.empty((B, k, D), dtype=torch.bfloat16).pin_memory()
+        rb = D * 2
+        call = lambda st, src=src, idx=idx, dst=dst, B=B, n=n, k=k, rb=rb: S.gather_kept(
+            src, n * rb, rb, n, rb, B, idx, k, k, dst, k * rb, rb, stream=st)
+        nbytes = B * k * (2.0 * rb + 4)
+        e = hbm_entry(ctx, args, call, nbytes, lambda src=src, src_host=src_host: src.copy_(src_host, non_blocking=True),
+                      lambda dst=dst, dst_host=dst_host: dst_host.copy_(dst, non_blocking=True),
+                      "spatten_gather_kept")
+        torch.cuda.synchronize()
+        assert np.array_equal(dst[0].view(torch.int16).cpu().numpy(),
+                              src_host[0].view(torch.int16).numpy()[idx_np[0]]), "gathered rows"
+        e.update(name=name, rows=B * k, row_bytes=rb, value=nbytes / (e["us_per_call"] / 1e6) / 1e9, unit="GB/s",
+                 e2e={"value": nbytes / (e.pop("e2e_ms_per_call") / 1e3) / 1e9, "unit": "GB/s",
+                      "h2d_bytes_per_step": B * n * rb, "d2h_bytes_per_step": B * k * rb})
+        if ctx.rank == 0 and not args.no_cpu_baseline:
+            xs = src_host.view(torch.int16).numpy()
+            t0, reps = time.perf_counter(), 0
+            while reps == 0 or time.perf_counter() - t0 < 0.5:
+                for b in range(B):
+                    np.take(xs[b], idx_np[b], axis=0)
+                reps += 1
+            el = time.perf_counter() - t0
+            e["cpu_baseline"] = {"value": reps * nbytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "numpy take",
+                                 "sample": f"{reps} full gather(s), {el:.2f} s"}
+        entries.append(e)
+        del src, dst
+    head = entries[0]
+    return {"metric": "kept-row gather GB/s", "unit": "GB/s", "value": head["value"],
+            "config": {"workload": "prefill_x_row_gathers", "l2": "flushed between timed calls"},
+            "roofline": head["roofline"], "entries": entries}
+
+
+def sub_line(r, keys=("metric", "value", "unit", "steps", "ms_per_step", "config", "roofline", "e2e", "gpu_launches",
+                      "clocks", "refetched_row_fraction", "refetch_rows_per_layer", "cpu_baseline")):
+    return {k: r[k] for k in keys if k in r}
+
+
 def run_ours(args):
     ctx = Ctx()
     if args.workload == "gpt2m_decode":
         result = decode_arm(ctx, args, args.steps)
     else:
         result = prefill_arm(ctx, args, args.workload)
-        if args.workload == "bert_base_prefill" and not args.no_decode:
-            dec = decode_arm(ctx, args, max(3, args.steps // 4))
-            result["decode"] = {k: dec[k] for k in ("metric", "value", "unit", "steps", "ms_per_step", "config",
-                                                    "roofline", "e2e", "gpu_launches", "clocks",
-                                                    "refetched_row_fraction", "cpu_baseline") if k in dec}
+        if args.workload == "bert_base_prefill" and not args.no_extra:
+            result["decode"] = sub_line(decode_arm(ctx, args, max(3, args.steps // 4)))
+            long_args = argparse.Namespace(**{**vars(args), "steps": max(3, args.steps // 4),
+                                              "cpu_seconds": min(args.cpu_seconds, 8.0)})
+            result["long_prefill"] = sub_line(prefill_arm(ctx, long_args, "long_prefill"))
+            result["topk_sweep"] = topk_arm(ctx, args)
+            result["gather"] = gather_arm(ctx, args)
     ctx.close()
     if ctx.rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def relaunch_with_ranks(args, argv):
+    """`--gpus N` without a launcher: run N local ranks (one per GPU) under torch.distributed.run on
+    127.0.0.1, the way the multi-GPU runs are launched; rank 0 prints the line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def main(argv=None):
@@ -682,10 +835,15 @@ def main(argv=None):
     ap.add_argument("--workload", choices=list(METRIC), default="bert_base_prefill")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="leave the decode object out of the default line")
+    ap.add_argument("--no-extra", "--no-decode", action="store_true",
+                    help="leave the decode, long_prefill, topk_sweep and gather objects out of the default line")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the prefill step directly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_with_ranks(args, sys.argv[1:] if argv is None else list(argv))
+    if "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) != args.gpus:
+        print(f"warning: --gpus {args.gpus} but the launcher started {os.environ['WORLD_SIZE']} ranks", file=sys.stderr)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

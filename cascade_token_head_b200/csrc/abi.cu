@@ -28,16 +28,16 @@ int32_t launch_status() {
 uint64_t launches() { return g_launches.load(std::memory_order_relaxed); }
 
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};   // every thread that fills an entry writes the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int v = 0;
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
       v = 148;
-    cached[dev] = v;
+    cached[dev].store(v, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return v;
 }
 
 }  // namespace spt

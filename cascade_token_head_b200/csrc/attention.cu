@@ -161,9 +161,9 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
     default: s = attn_simt_launch(p, st); break;
   }
   if (s != SPATTEN_OK) return s;
+  if (path != Path::kDecode && (p.a.tok_imp || p.a.head_imp)) SPT_TRY(attn_reduce_launch(p, st));
   if (ev_end) SPT_CUDA(cudaEventRecordWithFlags(ev_end, st, ev_flags));
-  if (path == Path::kDecode || (!p.a.tok_imp && !p.a.head_imp)) return SPATTEN_OK;
-  return attn_reduce_launch(p, st);
+  return SPATTEN_OK;
 }
 }  // namespace spt
 

@@ -37,8 +37,8 @@ int decode_item_rows(int d_h);    // keys per item of the decode kernel
 constexpr int kTcRows = 128;      // query rows per CTA of the tensor-core kernel
 constexpr int kSimtRows = 32;     // query rows per CTA of the CUDA-core kernel
 
-// spatten_attention_layer with optional events recorded around the main kernel (not the reduce;
-// on the decode path around both of its kernels).
+// spatten_attention_layer with optional events recorded around all of its kernels (attention, the
+// pruned-head zero fill, the refetch pass and the importance reduction).
 int32_t attention_layer_timed(const spatten_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t st,
                               cudaEvent_t ev_begin, cudaEvent_t ev_end);
 

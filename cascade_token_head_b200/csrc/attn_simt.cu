@@ -267,14 +267,13 @@ template <int DH, typename QT, typename KVT>
 int32_t launch_simt(const AttnProblem& p, cudaStream_t st) {
   const spatten_attn_args& a = p.a;
   const size_t smem = sizeof(SimtSmem<DH>);
-  static bool configured[64] = {false};
+  static DeviceOnce once;
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  SPT_TRY(once_per_device(once, &dev, [smem](int) -> int32_t {
     SPT_CUDA(cudaFuncSetAttribute(attn_simt_kernel<DH, QT, KVT>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-    configured[dev] = true;
-  }
+    return SPATTEN_OK;
+  }));
   const int slots = a.H_kept + (a.zero_pruned_heads ? a.H - a.H_kept : 0);
   dim3 grid(p.n_qt, slots, a.B);
   attn_simt_kernel<DH, QT, KVT><<<grid, kThreads, smem, st>>>(p);

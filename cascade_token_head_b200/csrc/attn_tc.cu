@@ -1114,16 +1114,15 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
 
 template <int DH>
 int32_t launch(const AttnProblem& p, cudaStream_t st) {
-  static bool configured[64] = {false};
+  static DeviceOnce once;
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  SPT_TRY(once_per_device(once, &dev, [](int) -> int32_t {
     SPT_CUDA(cudaFuncSetAttribute(attn_main_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(MainCfg<DH>::kSmem)));
     SPT_CUDA(cudaFuncSetAttribute(attn_full_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(FullCfg<DH>::kSmem)));
-    configured[dev] = true;
-  }
+    return SPATTEN_OK;
+  }));
   const int64_t items = static_cast<int64_t>(p.n_pair) * p.a.H_kept * p.a.B;
   const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
   attn_main_kernel<DH><<<grid, 384, MainCfg<DH>::kSmem, st>>>(p);

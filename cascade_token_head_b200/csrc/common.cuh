@@ -6,6 +6,9 @@
 #include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "spatten.h"
 
 namespace spt {
@@ -61,6 +64,28 @@ struct WsCursor {
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// First-call set-up (kernel attributes, capability probes) once per device ordinal.  The first
+// caller on a device runs `setup(dev)` under a lock; callers from other host threads wait for it,
+// so no launch can run before its attributes are set.  A set-up that fails is tried again on the
+// next call.  Returns the set-up's status (SPATTEN_OK once it has succeeded) and the device in *dev.
+struct DeviceOnce {
+  std::mutex mu;
+  std::atomic<bool> done[64] = {};
+};
+template <typename F>
+int32_t once_per_device(DeviceOnce& once, int* dev_out, F&& setup) {
+  int dev = 0;
+  SPT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return SPATTEN_E_UNSUPPORTED;
+  *dev_out = dev;
+  if (once.done[dev].load(std::memory_order_acquire)) return SPATTEN_OK;
+  std::lock_guard<std::mutex> lock(once.mu);
+  if (once.done[dev].load(std::memory_order_relaxed)) return SPATTEN_OK;
+  const int32_t s = setup(dev);
+  if (s == SPATTEN_OK) once.done[dev].store(true, std::memory_order_release);
+  return s;
+}
 
 // ----------------------------------------------------------------------------------------------
 // device helpers

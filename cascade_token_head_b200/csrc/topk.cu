@@ -1225,15 +1225,13 @@ int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaSt
 }
 
 int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
-  static bool configured[64] = {false};
+  static DeviceOnce once;
   int dev = 0;
-  SPT_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return SPATTEN_E_UNSUPPORTED;
-  if (!configured[dev]) {
+  SPT_TRY(once_per_device(once, &dev, [](int) -> int32_t {
     SPT_CUDA(cudaFuncSetAttribute(topk_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kBinCap * 8 + kMaxChunks * 4));
-    configured[dev] = true;
-  }
+    return SPATTEN_OK;
+  }));
   const int R = a.R, n = a.n;
   StreamWs w{};
   w.nchunk = static_cast<int>((static_cast<int64_t>(n) + kChunk - 1) / kChunk);
@@ -1277,11 +1275,10 @@ int32_t topk_launch(const TArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) 
 }
 
 int32_t cluster_launch(const TArgs& a, cudaStream_t st) {
-  static bool configured[64] = {false};
+  static DeviceOnce once;
   static bool wide_ok[64] = {false};   // 16-CTA clusters can be scheduled on this device
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  SPT_TRY(once_per_device(once, &dev, [](int dev) -> int32_t {
     SPT_CUDA(cudaFuncSetAttribute(topk_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kResident * 4));
     SPT_CUDA(cudaFuncSetAttribute(topk_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1303,10 +1300,10 @@ int32_t cluster_launch(const TArgs& a, cudaStream_t st) {
       wide_ok[dev] = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel<false>, &q) == cudaSuccess && clusters >= 4;
     }
     cudaGetLastError();   // the probe above may leave an error behind
-    configured[dev] = true;
-  }
+    return SPATTEN_OK;
+  }));
   int C = pick_cluster(a.n);
-  if (C == 8 && a.n > 8 * kResident && dev >= 0 && dev < 64 && wide_ok[dev]) C = 16;
+  if (C == 8 && a.n > 8 * kResident && wide_ok[dev]) C = 16;
   const int chunk = static_cast<int>((ceil_div(a.n, C) + 3) & ~int64_t(3));
   const size_t smem = static_cast<size_t>(std::min(chunk, kResident)) * 4;
   cudaLaunchConfig_t cfg = {};

@@ -308,8 +308,8 @@ typedef struct spatten_cascade_io {
   float* trace_head_imp;     /* [L][B][H]  J after layer l                                     */
   uint8_t* trace_flags;      /* [L][B][H][T] refetch flags of layer l                          */
   /* optional timing hook: host array of 2*L cudaEvent_t (as void*); event 2l is recorded on the
-   * stream right before layer l's attention kernel and event 2l+1 right after it (before the
-   * importance reduction), so callers can time the attention kernel alone.  NULL = off.        */
+   * stream right before layer l's attention kernels and event 2l+1 right after them (after the
+   * importance reduction), so callers can time step a2/a3 of each layer alone.  NULL = off.    */
   void* const* attn_events;
 } spatten_cascade_io;
 

@@ -196,8 +196,10 @@ def test_attention_fp32_unquantized(cuda, n):
     (64, 0.2, 40, 7, None), (64, 0.2, 2600, 2048, None), (128, 0.05, 2600, 2047, [1, 3]),
     (64, 0.2, 3000, 2500, None), (128, 0.2, 1300, 1153, [0, 2, 3])])
 def test_attention_decode_index_listed(cuda, kernel, d, theta, cap, n_kv, keep):
-    """One query row per (sequence, head) against an index-listed subset of a cache.  Lists of up
-    to 2048 rows go to the cluster kernel (1..8 CTAs per row), longer ones to the streaming one."""
+    """One query row per (sequence, head) against an index-listed subset of a cache, through the
+    decode path (the items kernel over runs of the listed keys, then the per-sequence combine) and,
+    with kernel=1, through the float32 CUDA-core kernel on the same inputs.  Lists from 7 to 2500
+    keys, ragged last items, pruned heads."""
     S = lib()
     B, H = 3, 4
     g = synth.rng_for(d + int(theta * 10) + n_kv)

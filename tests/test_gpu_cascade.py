@@ -1,13 +1,15 @@
 """GPU parity of spatten_cascade_forward against the oracle.
 
 * float32 tiny cascade (the full workload size): free-running, binding -- kept sets equal (up to
-  near-ties within 1e-5 of the k-th score, each logged) and final rows within 1e-4 x RMS.
+  near-ties within 1e-5 of the k-th score, each logged) and every final row within 1e-4 x RMS
+  (against the oracle re-run along the device's kept sets when a near-tie changed one).
 * bf16 cascades: layer by layer with the traced device inputs of each layer (teacher forcing, as
-  the correctness statement prescribes).  Every traced value used as an oracle input is itself
-  checked against the oracle first (projection within 2e-2 x RMS, codes bit-exact).  Per layer:
-  O within 2e-2 x RMS; X_{l+1} within 2e-2 x RMS; token/head selection bit-exact against the oracle
-  run on the device's own importance vectors; against the oracle's own importance, kept-set
-  disagreements only at near-ties (1e-5 relative of the k-th score).
+  the correctness statement prescribes).  The traced projections used as oracle inputs are
+  themselves checked against X_l @ W first (bf16 bound below); the oracle quantizes the traced K
+  and V itself (the planes are checked bit-exact in the quantizer tests).  Per layer: O and X_{l+1}
+  are the bf16 roundings of values within 2e-2 x RMS of the oracle; token/head selection is
+  bit-exact against the oracle run on the device's own importance vectors; against the oracle's
+  own importance, kept-set disagreements only at near-ties (1e-5 relative of the k-th score).
 """
 import math
 
@@ -48,6 +50,7 @@ def test_cascade_tiny_fp32_free_running(cuda):
     wq = [host_cast(a, torch.float32) for a in d["w_qkv"]]
     wo = [host_cast(a, torch.float32) for a in d["w_o"]]
     ref = R.cascade_prefill(X32, wq, wo, w.H, w.d_h, w.token_keep, w.head_keep, False, 0.0)
+    same = True
     for l in range(w.L):
         k = w.token_keep[l]
         got = g["kept_tok"][l, 0, :k]
@@ -55,10 +58,36 @@ def test_cascade_tiny_fp32_free_running(cuda):
         if l > 0:
             near_tie_ok(ref["I_sel"][l - 1][0], got.tolist(), want.tolist(), k)
         assert np.all(np.diff(got) > 0)
-    if np.array_equal(g["kept_tok"][-1, 0, :w.token_keep[-1]], ref["kept"][-1][0]):
-        assert_close_rms(g["x_out"], ref["x_final"], 1e-4, "final rows (fp32)")
+        same &= np.array_equal(got, want) and np.array_equal(g["kept_head"][l, 0, :w.head_keep[l]], ref["heads"][l][0])
+    # The binding check runs on every final row.  If a near-tie (logged above) made the device keep
+    # another token, the oracle is re-run along the device's kept sets, so the rows still compare
+    # like for like at 1e-4 x RMS.
+    if not same:
+        print("near-tie changed a kept set: oracle re-run along the device's selections")
+        ref = oracle_along_kept_sets(X32, wq, wo, w, g["kept_tok"][:, 0], g["kept_head"][:, 0])
+    assert_close_rms(g["x_out"][0], ref["x_final"][0], 1e-4, "final rows (fp32)")
     np.testing.assert_allclose(g["tok_imp"], ref["I"], rtol=0, atol=1e-5 * ref["I"].max())
     np.testing.assert_allclose(g["head_imp"], ref["J"], rtol=1e-5)
+
+
+def oracle_along_kept_sets(X, wq, wo, w, kept_tok, kept_head):
+    """The oracle's layer step (projection, attention_layer_seq, importance, residual) for one
+    sequence, with the token and head sets of every layer taken from the device run instead of
+    the oracle's own selection."""
+    X = np.array(X[0], np.float64)
+    HD = w.H * w.d_h
+    I, J = np.zeros(w.T), np.zeros(w.H)
+    for l in range(w.L):
+        S_l = kept_tok[l, :w.token_keep[l]].astype(np.int64)
+        heads = kept_head[l, :w.head_keep[l]].astype(np.int64)
+        qkv = X[S_l] @ wq[l]
+        r = R.attention_layer_seq(qkv[:, :HD], qkv[:, HD:2 * HD], qkv[:, 2 * HD:], heads, w.d_h, w.H, False, 0.0,
+                                  1.0 / math.sqrt(w.d_h))
+        I[S_l] += r["tok_inc"]
+        J += r["head_inc"]
+        X[S_l] = X[S_l] + r["O"] @ wo[l]
+    last = kept_tok[w.L - 1, :w.token_keep[-1]].astype(np.int64)
+    return dict(x_final=X[last][None], I=I[None], J=J[None])
 
 
 def teacher_forced_check(S, w, d, sample_b=None):

@@ -2,12 +2,13 @@
 
 * One layer, one kept head, every output checked: the oracle runs the head's 16384 query rows in
   blocks (rows are independent), so the full token-importance vector, O and flags are compared.
-* The whole four-layer cascade with traces, checked on sampled rows and heads of every layer:
-  projections, O and refetch flags of sampled (row, head) pairs against the oracle on the device's
-  own layer inputs; per-layer importance increments by the properties that hold at any size (the
-  increment sums to k_l x H_l, vanishes off the kept rows, head increments equal sum |O|); kept
-  token and head sets bit-exact against the oracle's selection on the device's importance; the
-  next layer's rows X_l + O W_o on sampled rows.
+* The whole four-layer cascade with traces, on the device's own layer inputs (teacher forcing):
+  the oracle runs every kept head of every layer (a spawn process pool), so the cumulative token
+  importance is compared element by element and the head importance against the oracle's sum |O|;
+  refetch flags of every row agree up to near-ties; kept token sets are bit-exact against the
+  oracle's selection on the device's importance and agree with the oracle's own importance up to
+  near-ties (1e-5 of the k-th score); projections, O and the next layer's rows are checked on
+  sampled rows; the increments also meet the properties that hold at any size.
 """
 import math
 
@@ -20,6 +21,7 @@ from oracle import spatten_ref as R
 
 from cascade_helpers import run_prefill, upload_prefill
 from gpu_helpers import BF, assert_close_bf16_out, host_cast, lib
+from oracle_pool import head_layer_task, spawn_pool
 from test_gpu_attention import make_layer, run_layer
 
 pytestmark = pytest.mark.gpu
@@ -65,7 +67,7 @@ def test_attention_long_one_head_every_output(cuda):
     print(f"refetched rows {int(gf.sum())}, near-tie flags {near}")
 
 
-def test_cascade_long_full_size_sampled(cuda):
+def test_cascade_long_full_size(cuda):
     S = lib()
     w = synth.long_prefill()
     d = synth.draw_prefill(w)
@@ -82,34 +84,56 @@ def test_cascade_long_full_size_sampled(cuda):
     thead = bufs["thead"].cpu().numpy().astype(np.float64)
     refetch = bufs["refetch"].cpu().numpy()
     gain = d["key_gain"][0].astype(np.float32)
-    I_prev = np.zeros(T)
-    J_prev = np.zeros(H)
+    layers = []
     for l in range(w.L):
         k, Hl = w.token_keep[l], w.head_keep[l]
+        layers.append(dict(
+            S_l=kept_tok[l, 0, :k].astype(np.int64), heads=kept_head[l, 0, :Hl].astype(np.int64),
+            X_l=bufs["tx"][l, 0, :k].float().cpu().numpy().astype(np.float64),
+            qkv=bufs["tqkv"][l, 0, :k].float().cpu().numpy(),          # bf16 values, exact in float32
+            O=bufs["to"][l, 0, :k].float().cpu().numpy(),
+            flags=bufs["tflags"][l, 0, :, :k].cpu().numpy().astype(bool)))
+    # the oracle over every kept head of every layer, on the device's own layer inputs
+    tasks = []
+    for l, L_ in enumerate(layers):
+        q = L_["qkv"]
+        for h in L_["heads"]:
+            tasks.append((q[:, h * dh:(h + 1) * dh],
+                           q[:, HD + h * dh:HD + (h + 1) * dh] * gain[L_["S_l"]][:, None],
+                           q[:, 2 * HD + h * dh:2 * HD + (h + 1) * dh], w.theta, sm, L_["flags"][h]))
+    with spawn_pool(16) as pool:
+        results = pool.map(head_layer_task, tasks, chunksize=1)
+    I_ref, J_ref = np.zeros(T), np.zeros(H)
+    I_prev, J_prev = np.zeros(T), np.zeros(H)
+    it = iter(results)
+    stats = dict(near_flags=0, near_tok=0)
+    for l, L_ in enumerate(layers):
+        S_l, heads, X_l, qkv, O_dev, flags = (L_[x] for x in ("S_l", "heads", "X_l", "qkv", "O", "flags"))
+        k, Hl = len(S_l), len(heads)
+        assert np.all(np.diff(S_l) > 0) and np.all(np.diff(heads) > 0)
         wq = host_cast(d["w_qkv"][l], BF)
         wo = host_cast(d["w_o"][l], BF)
-        S_l = kept_tok[l, 0, :k].astype(np.int64)
-        heads = kept_head[l, 0, :Hl].astype(np.int64)
-        assert np.all(np.diff(S_l) > 0) and np.all(np.diff(heads) > 0)
-        X_l = bufs["tx"][l, 0, :k].float().cpu().numpy().astype(np.float64)
-        qkv = bufs["tqkv"][l, 0, :k].float().cpu().numpy()          # bf16 values, exact in float32
-        O_dev = bufs["to"][l, 0, :k].float().cpu().numpy()
-        flags = bufs["tflags"][l, 0, :, :k].cpu().numpy().astype(bool)
         rows = np.sort(g.choice(k, size=48, replace=False))
         assert_close_bf16_out(qkv[rows], X_l[rows] @ wq, 2e-2, f"qkv layer {l}")
+        # O on sampled rows of two sampled heads
         for h in g.choice(heads, size=2, replace=False):
             c = slice(h * dh, (h + 1) * dh)
             Kh = qkv[:, HD + h * dh:HD + (h + 1) * dh] * gain[S_l][:, None]
             Vh = qkv[:, 2 * HD + h * dh:2 * HD + (h + 1) * dh]
             kq, vq = R.quantize_head(Kh), R.quantize_head(Vh)
-            r = R.progressive_attention(qkv[rows, c].astype(np.float64), kq, vq, w.theta, sm)
-            diff = flags[h, rows] != r["flags"]
-            if diff.any():
-                assert np.all(np.abs(r["pmax_msb"][diff] - w.theta) <= 1e-5 * w.theta), "flag off a tie"
-                r = R.progressive_attention(qkv[rows, c].astype(np.float64), kq, vq, w.theta, sm,
-                                            flags_override=flags[h, rows])
+            r = R.progressive_attention(qkv[rows, c].astype(np.float64), kq, vq, w.theta, sm,
+                                        flags_override=flags[h, rows])
             assert_close_bf16_out(O_dev[rows, c], r["O"], 2e-2, f"O layer {l} head {h}")
-        # importance increments: properties that hold at any size
+        # importance of every kept head against the oracle, element by element
+        for h in heads:
+            col, habs, near, off = next(it)
+            assert off == 0, f"refetch flag off a near-tie, layer {l} head {h}"
+            stats["near_flags"] += near
+            I_ref[S_l] += col
+            J_ref[h] += habs
+        np.testing.assert_allclose(ttok[l, 0], I_ref, rtol=0, atol=2e-5 * I_ref.max() + 1e-7)
+        np.testing.assert_allclose(thead[l, 0], J_ref, rtol=2e-2)
+        # properties that hold at any size, on the device's own increments
         dI = ttok[l, 0] - I_prev
         assert abs(dI.sum() - k * Hl) <= 1e-4 * k * Hl
         assert np.all(np.delete(dI, S_l) == 0) and dI.min() >= -1e-3
@@ -128,11 +152,28 @@ def test_cascade_long_full_size_sampled(cuda):
             break
         k2, H2 = w.token_keep[l + 1], w.head_keep[l + 1]
         S_n = kept_tok[l + 1, 0, :k2].astype(np.int64)
+        # bit-exact on the device's importance; against the oracle's own importance only at near-ties
         np.testing.assert_array_equal(S_n, S_l[R.topk_select(ttok[l, 0][S_l], k2)])
+        want = S_l[R.topk_select(I_ref[S_l], k2)]
+        diff = set(S_n.tolist()) ^ set(want.tolist())
+        if diff:
+            kth = np.sort(I_ref[S_l])[::-1][k2 - 1]
+            for t in diff:
+                assert abs(I_ref[t] - kth) <= 1e-5 * abs(kth), f"kept-set disagreement off a near-tie: token {t}"
+            stats["near_tok"] += len(diff)
         H_n = kept_head[l + 1, 0, :H2].astype(np.int64)
         np.testing.assert_array_equal(H_n, heads[R.topk_select(thead[l, 0][heads], H2)])
+        want_h = heads[R.topk_select(J_ref[heads], H2)]
+        assert set(H_n.tolist()) == set(want_h.tolist()) or _heads_near(J_ref, H_n, want_h, H2, heads)
         nxt = np.sort(g.choice(k2, size=48, replace=False))
         pos = np.searchsorted(S_l, S_n[nxt])
         X_next = bufs["tx"][l + 1, 0, :k2].float().cpu().numpy()[nxt]
         assert_close_bf16_out(X_next, X_l[pos] + O_dev[pos].astype(np.float64) @ wo, 2e-2, f"X layer {l + 1}")
-    print("refetch per layer", refetch.tolist())
+    print("refetch per layer", refetch.tolist(), stats)
+
+
+def _heads_near(J_ref, got, want, k, heads):
+    """Head-set disagreements are allowed only where the oracle's head importances tie within 2e-2
+    relative (the tolerance the head importance itself is held to)."""
+    kth = np.sort(J_ref[heads])[::-1][k - 1]
+    return all(abs(J_ref[h] - kth) <= 2e-2 * kth for h in set(got.tolist()) ^ set(want.tolist()))

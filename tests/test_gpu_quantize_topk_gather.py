@@ -241,11 +241,11 @@ def test_topk_nan_reports_status(cuda, n, k, pos):
 @pytest.mark.parametrize("dist", ["uniform", "lognormal"])
 def test_topk_sweep_full_size(cuda, N, dist):
     """The top-k sweep workload (64 rows, 1 % exact duplicates), k = 10 % and 50 % of N.
-    Every row is checked bit-exact for N <= 256k; at N = 1M, 8 sampled rows are checked against the
-    oracle and every row against the selection properties."""
+    Every row is checked bit-exact against the oracle (which also fixes which members of a tie
+    group at the threshold are taken: the lowest indices), plus the selection properties."""
     S = lib()
     x = synth.draw_topk_row_block(64, N, dist, 0.01, seed=N % 9973 + (dist == "lognormal"))
-    rows = range(64) if N <= 262144 else [0, 9, 17, 30, 38, 45, 51, 63]
+    rows = range(64)
     for frac in (0.1, 0.5):
         k = int(frac * N)
         got, _, st = _topk_gpu(S, x, k)
