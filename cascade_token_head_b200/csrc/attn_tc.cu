@@ -47,6 +47,7 @@
 #include <cuda_fp16.h>
 
 #include "attention.cuh"
+#include "exp2_poly.cuh"
 #include "tc_ptx.cuh"
 
 namespace spt {
@@ -58,6 +59,13 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWaitLimit = 1u << 26;   // polls of one mbarrier phase before giving up
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kProducerThreads = 96;
+// Of every four pairs of softmax exponentials in the main kernel, this many are computed by the
+// FMA-pipe polynomial (exp2_poly2) and the rest by the ex2 instruction: the two units then share
+// the work.
+#ifndef SPT_EXP2_POLY_PAIRS
+#define SPT_EXP2_POLY_PAIRS 1
+#endif
+constexpr int kPolyPairs = SPT_EXP2_POLY_PAIRS;
 
 // byte offset of 16-byte chunk c8 of `row` in a tile whose 64-element column blocks each hold
 // `rows` rows of 128 bytes (128-byte swizzle)
@@ -111,6 +119,14 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// 16-byte asynchronous global -> shared copy (no register staging); src_bytes 0 zero-fills
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -123,6 +139,13 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   }
   *abort_flag = 1;
   return false;
+}
+
+// after an abort: wait, with a bound of its own, for a phase that work already in flight (a bulk
+// copy, committed MMAs) will complete, so shared memory and TMEM are not released under it
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 22); ++i)
+    if (mbar_try_wait(bar, parity)) return;
 }
 
 // The AND of `ok` over the 128 threads of a softmax warpgroup (named barrier `id`): after a wait,
@@ -141,6 +164,18 @@ __device__ __forceinline__ bool wg_all(bool ok, int id) {
       : "r"(ok ? 1u : 0u), "r"(id)
       : "memory");
   return r != 0;
+}
+
+// paired float32 arithmetic (two lanes per instruction on sm_100)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// 2^x of a pair: pair `q` of each group of four takes the FMA-pipe polynomial when q < kPolyPairs,
+// else the ex2 instruction (q is a compile-time index, so the choice costs nothing)
+template <int Q>
+__device__ __forceinline__ float2 exp2_pair(float2 x) {
+  if constexpr ((Q & 3) < kPolyPairs) return exp2_poly2(x);
+  else return make_float2(ex2(x.x), ex2(x.y));
 }
 
 // column sums over the 32 rows of a warp for two 32-column arrays: afterwards lane l holds the
@@ -176,10 +211,16 @@ __device__ __forceinline__ void stats64_scaled(const float* v, float c2, float& 
   }
   const float mm = c2 * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
   const float mn = fmaxf(m2, mm);
-  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const float2 c2x2 = make_float2(c2, c2), nmn = make_float2(-mn, -mn);
+  float2 s0 = make_float2(0.0f, 0.0f), s1 = s0;
 #pragma unroll
-  for (int j = 0; j < 64; ++j) s[j & 3] += ex2(fmaf(v[j], c2, -mn));
-  l = l * ex2(m2 - mn) + ((s[0] + s[1]) + (s[2] + s[3]));
+  for (int j = 0; j < 32; j += 4) {
+    s0 = fadd2(s0, exp2_pair<0>(ffma2(make_float2(v[2 * j + 0], v[2 * j + 1]), c2x2, nmn)));
+    s1 = fadd2(s1, exp2_pair<1>(ffma2(make_float2(v[2 * j + 2], v[2 * j + 3]), c2x2, nmn)));
+    s0 = fadd2(s0, exp2_pair<2>(ffma2(make_float2(v[2 * j + 4], v[2 * j + 5]), c2x2, nmn)));
+    s1 = fadd2(s1, exp2_pair<3>(ffma2(make_float2(v[2 * j + 6], v[2 * j + 7]), c2x2, nmn)));
+  }
+  l = l * ex2(m2 - mn) + ((s0.x + s1.x) + (s0.y + s1.y));
   m2 = mn;
 }
 
@@ -243,13 +284,32 @@ template <int DH, int KT>
 __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw, bool with_lsb, int valid,
                                                uint32_t off_hi, int ptid) {
   constexpr int L16 = DH / 16;
-  for (int e = ptid; e < KT * L16; e += kProducerThreads) {
+  constexpr int TOTAL = KT * L16;
+  constexpr int NIT = (TOTAL + kProducerThreads - 1) / kProducerThreads;
+  // every staged read of this thread first (all in flight together), then the conversions
+  uint4 m[NIT];
+  uint2 lb[NIT];
+#pragma unroll
+  for (int i = 0; i < NIT; ++i) {
+    const int e = ptid + i * kProducerThreads;
+    const int r = e / L16, c16 = e % L16;
+    m[i] = make_uint4(0u, 0u, 0u, 0u);
+    lb[i] = make_uint2(0u, 0u);
+    if (e < TOTAL && r < valid) {
+      m[i] = *reinterpret_cast<const uint4*>(raw + r * DH + c16 * 16);
+      if (with_lsb) lb[i] = *reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NIT; ++i) {
+    const int e = ptid + i * kProducerThreads;
+    if (e >= TOTAL) break;
     const int r = e / L16, c16 = e % L16;
     uint32_t hi[8], lo[8];
     if (r < valid) {
-      cvt16_s8x16(*reinterpret_cast<const uint4*>(raw + r * DH + c16 * 16), hi);
+      cvt16_s8x16(m[i], hi);
       if (with_lsb) {
-        cvt_u4x16(*reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8), lo);
+        cvt_u4x16(lb[i], lo);
         add_f16x8(hi, lo);
       }
     } else {
@@ -283,6 +343,7 @@ struct JobStream {
   volatile int* abort_flag;
   uint32_t g0 = 0;       // global index of this stream's job 0 in the staging ring's sequence
   uint32_t issued = 0;   // jobs of this stream issued so far (loader)
+  uint32_t consumed = 0; // jobs of this stream converted so far
 
   __device__ __forceinline__ int jobs() const { return 3 * n_tiles; }
   __device__ __forceinline__ void job(int j, bool& is_v, int& t) const {
@@ -332,6 +393,7 @@ struct JobStream {
     if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag)) return false;
     convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid);
     mbar_arrive(&raw_empty[st]);
+    ++consumed;
     return true;
   }
 };
@@ -359,6 +421,29 @@ __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t sP, uint32_t sV, uin
   }
 }
 
+// S^T = K Q^T into `d`: A = key tile [KT keys x DH] (K-major), B = one warpgroup's query tile
+// [128 rows x DH] (K-major).  TMEM lane = key, column = query row.
+template <int DH, int KT>
+__device__ __forceinline__ void mma_kq(uint32_t d, uint32_t sK, uint32_t sQ) {
+  constexpr uint32_t id = idesc_f16(KT, 128, false, false);
+#pragma unroll
+  for (int s = 0; s < DH / 16; ++s) {
+    const uint32_t koff = (s >> 2) * (KT * 128u) + (s & 3) * 32u;
+    const uint32_t qoff = (s >> 2) * 16384u + (s & 3) * 32u;
+    mma_f16(d, desc_sw128(sK + koff, 16, 1024), desc_sw128(sQ + qoff, 16, 1024), id, s > 0 ? 1u : 0u);
+  }
+}
+// P V into `d` with P stored MN-major (query rows contiguous): A = P tile [128 rows x KT keys] in
+// two 64-row blocks KT*128 bytes apart with 8-key groups 1024 bytes apart; B = V tile MN-major
+template <int DH, int KT>
+__device__ __forceinline__ void mma_pv_mn(uint32_t d, uint32_t sP, uint32_t sV, uint32_t acc) {
+  constexpr uint32_t id = idesc_f16(128, DH, true, true);
+#pragma unroll
+  for (int s = 0; s < KT / 16; ++s)
+    mma_f16(d, desc_sw128(sP + s * 2048u, KT * 128u, 1024), desc_sw128(sV + s * 2048u, KT * 128u, 1024), id,
+            (acc || s > 0) ? 1u : 0u);
+}
+
 __device__ __forceinline__ void store_o_row(__nv_bfloat16* dst, const float* v, float vs, float& habs) {
   uint32_t pk[16];
 #pragma unroll
@@ -377,15 +462,23 @@ __device__ __forceinline__ void store_o_row(__nv_bfloat16* dst, const float* v, 
 // =================================================================================================
 template <int DH>
 struct MainCfg {
+  // d_h = 64: the probability pass runs transposed (S^T = K Q^T, one key per TMEM lane, P written
+  // MN-major); d_h = 128: row orientation with shuffle column sums (its 128-key tiles would not
+  // fit the shared-memory budget)
+  static constexpr bool kT = DH == 64;
   static constexpr int KT = DH == 64 ? 128 : 64;
   static constexpr int NST = 2;                  // fp16 K and V ring stages
-  static constexpr int RS = 4;                   // raw code tiles in flight (bulk copies)
+  // d_h = 64: the next item's query tile is copied into a second buffer while the current item
+  // runs (cp.async, converted in place once the current item's key jobs are done); d_h = 128 has
+  // no room for a second buffer and loads the query tile between items
+  static constexpr int NQ = DH == 64 ? 2 : 1;
+  static constexpr int RS = DH == 64 ? 3 : 4;    // raw code tiles in flight (bulk copies)
   static constexpr uint32_t QB = 128u * DH * 2u;
   static constexpr uint32_t TB = static_cast<uint32_t>(KT) * DH * 2u;
   static constexpr uint32_t PB = 128u * KT * 2u;
   static constexpr uint32_t RAWB = static_cast<uint32_t>(KT) * DH;   // one raw MSB tile
-  static constexpr uint32_t oQ = 0;              // 2 query tiles
-  static constexpr uint32_t oK = 2 * QB;         // NST stages
+  static constexpr uint32_t oQ = 0;              // NQ buffers of 2 query tiles (one per warpgroup)
+  static constexpr uint32_t oK = NQ * 2 * QB;    // NST stages
   static constexpr uint32_t oV = oK + NST * TB;  // NST stages
   static constexpr uint32_t oP = oV + NST * TB;  // one P tile per warpgroup
   static constexpr uint32_t oRaw = oP + 2 * PB;  // RS staging slots
@@ -394,8 +487,8 @@ struct MainCfg {
   static constexpr uint32_t tO = 2u * KT;        // + g * DH
 };
 
-enum : int { M_QF = 0, M_QE = 1, M_OE = 2, M_KF = 3, M_KE = 5, M_VF = 7, M_VE = 9, M_SF = 11, M_SR = 13, M_PF = 15,
-             M_PE = 17, M_OD = 19, M_RF = 20, M_RE = 24, M_N = 28 };
+enum : int { M_QF = 0, M_QE = 2, M_OE = 4, M_KF = 5, M_KE = 7, M_VF = 9, M_VE = 11, M_SF = 13, M_SR = 15, M_PF = 17,
+             M_PE = 19, M_OD = 21, M_RF = 22, M_RE = 26, M_DR = 30, M_N = 31 };   // M_QF, M_QE: one per query buffer
 
 // AND of `ok` over the 256 softmax threads of a CTA (named barrier 3)
 __device__ __forceinline__ bool softmax_all(bool ok) {
@@ -427,7 +520,8 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bars[M_N];
   __shared__ uint32_t tmem_base_s;
-  __shared__ float colred[2][2][4][KT];    // [tile parity][warpgroup][warp][key]
+  __shared__ float colred[C::kT ? 1 : 2][2][4][C::kT ? 1 : KT];    // [tile parity][warpgroup][warp][key]
+  __shared__ __align__(16) float nmb_s[2][128];   // transposed pass: -(m + log2 ell) of each query row
   __shared__ float hred[2][4];
   __shared__ uint32_t wcnt[8];
   __shared__ int abort_s;
@@ -443,8 +537,10 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   }
   if (tid == 0) {
     abort_s = 0;
-    mbar_init(&bars[M_QF], kProducerThreads);
-    mbar_init(&bars[M_QE], 1);
+    for (int qb = 0; qb < C::NQ; ++qb) {
+      mbar_init(&bars[M_QF + qb], kProducerThreads);
+      mbar_init(&bars[M_QE + qb], 1);
+    }
     mbar_init(&bars[M_OE], 256);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars[M_KF + s], kProducerThreads);
@@ -459,6 +555,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       mbar_init(&bars[M_PE + g], 1);
     }
     mbar_init(&bars[M_OD], 1);
+    mbar_init(&bars[M_DR], 1);
     for (int s = 0; s < C::RS; ++s) {
       mbar_init(&bars[M_RF + s], 1);
       mbar_init(&bars[M_RE + s], kProducerThreads);
@@ -484,6 +581,32 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     // ------------------------------------------------------------------------- producers
     const int ptid = tid - 256;
     uint32_t kc = 0, vc = 0, gjob = 0, qc = 0;
+    constexpr int QCH = 256 * (DH / 8);   // 16-byte chunks of one item's query rows
+    // the item's 256 query rows of its head, bf16, into query buffer qb at their swizzled fp16
+    // positions (rows past n_q zero-filled); one commit group
+    auto copy_q_async = [&](int item, uint32_t qbuf) {
+      int b, slot, pair;
+      item_coords(item, b, slot, pair);
+      const int h = head_of_slot(a, b, slot);
+      const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+      for (int e = ptid; e < QCH; e += kProducerThreads) {
+        const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = pair * 256 + rr;
+        const bool ok = qi < a.n_q;
+        const __nv_bfloat16* src =
+            ok ? q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8 : q;
+        cp_async16(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128), src, ok ? 16u : 0u);
+      }
+      cp_async_commit();
+    };
+    // bf16 -> fp16 in place, each thread the chunks it copied
+    auto convert_q_in_place = [&](uint32_t qbuf) {
+      for (int e = ptid; e < QCH; e += kProducerThreads) {
+        const int rr = e / (DH / 8), c8 = e % (DH / 8);
+        uint4* p = reinterpret_cast<uint4*>(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128));
+        *p = bf16x8_to_f16x8(*p);
+      }
+    };
+    uint32_t g_issued = 0, g_consumed = 0;   // staging-ring jobs issued / converted, whole kernel
     for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++qc) {
       int b, slot, pair;
       item_coords(it, b, slot, pair);
@@ -492,11 +615,28 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
       JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
                                   abort_flag, gjob};
+      struct Track {   // records the stream's progress however the item's loop is left
+        JobStream<DH, KT, C::RS>& js;
+        uint32_t &gi, &gc;
+        __device__ ~Track() { gi = js.g0 + js.issued; gc = js.g0 + js.consumed; }
+      } track{js, g_issued, g_consumed};
       // the first raw key tiles start before the query tile (both in flight together)
       if (!kv_idx && ptid == 0 && !js.issue_ahead(0)) { aborted = true; break; }
-      // query tile of the item once the previous item's score MMAs have read the buffer
-      if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
-      {
+      const uint32_t qb = qc % C::NQ;
+      if constexpr (C::NQ == 2) {
+        // this item's query tile was copied (bf16) into buffer qb during the previous item, or just
+        // below for the first item: convert it in place to fp16 (each thread its own chunks)
+        if (qc == 0) {
+          if (!wait_bar(&bars[M_QE + qb], 1u, abort_flag)) { aborted = true; break; }
+          copy_q_async(it, qb);
+        }
+        cp_async_wait_all();
+        convert_q_in_place(qb);
+        fence_async_smem();
+        mbar_arrive(&bars[M_QF + qb]);
+      } else {
+        // query tile of the item once the previous item's score MMAs have read the buffer
+        if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
         constexpr int NCH = 256 * (DH / 8);
         constexpr int BATCH = 8;
         const int i0 = pair * 256;
@@ -526,6 +666,15 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       }
       // pass A keys, then pass B keys and values
       for (int j = 0; j < 3 * n_tiles; ++j) {
+        if constexpr (C::NQ == 2) {
+          // at the first pass-B job the previous item is done with the other query buffer: copy
+          // the next item's query rows into it
+          if (j == n_tiles && it + static_cast<int>(gridDim.x) < n_items) {
+            const uint32_t nb = (qc + 1) % C::NQ;
+            if (!wait_bar(&bars[M_QE + nb], (((qc + 1) / C::NQ) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+            copy_q_async(it + static_cast<int>(gridDim.x), nb);
+          }
+        }
         if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; break; }
         bool is_v;
         int t;
@@ -539,23 +688,30 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       }
       gjob += 3 * n_tiles;
     }
+    cp_async_wait_all();   // no query copy may land after the CTA has left
+    if (aborted && ptid == 0)   // bulk copies already armed complete before shared memory is released
+      for (uint32_t gj = g_consumed; gj < g_issued; ++gj) drain_wait(&bars[M_RF + gj % C::RS], (gj / C::RS) & 1u);
   } else if (warp == 11) {
     // ------------------------------------------------------------------------- MMA issue
     if (lane == 0) {
       uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0}, ic = 0;
-      const uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
-      auto qk_both = [&](void) -> bool {
+      uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
+      // scores of one key tile for both warpgroups: S = Q K^T (pass A, and pass B in row
+      // orientation) or S^T = K Q^T (pass B, transposed)
+      auto qk_both = [&](bool trans) -> bool {
         const uint32_t ks = kc % NST;
         if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag)) return false;
         const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
         if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag)) return false;
         tc_after_sync();
-        mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
+        if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS, sK, sQ0);
+        else mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
         mma_commit(&bars[M_SF + 0]);
         ++sc[0];
         if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag)) return false;
         tc_after_sync();
-        mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
+        if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS + KT, sK, sQ1);
+        else mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
         mma_commit(&bars[M_SF + 1]);
         ++sc[1];
         mma_commit(&bars[M_KE + ks]);
@@ -563,18 +719,21 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         return true;
       };
       for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++ic) {
-        if (!wait_bar(&bars[M_QF], ic & 1u, abort_flag)) { aborted = true; break; }
+        const uint32_t qb = ic % C::NQ;
+        sQ0 = smem_u32(smem + C::oQ + qb * 2 * C::QB);
+        sQ1 = sQ0 + C::QB;
+        if (!wait_bar(&bars[M_QF + qb], (ic / C::NQ) & 1u, abort_flag)) { aborted = true; break; }
         for (int t = 0; t < n_tiles && !aborted; ++t)   // pass A
-          if (!qk_both()) aborted = true;
+          if (!qk_both(false)) aborted = true;
         if (aborted) break;
-        if (!qk_both()) { aborted = true; break; }       // pass B, tile 0
-        if (n_tiles == 1) mma_commit(&bars[M_QE]);      // the item's last read of Q is issued
+        if (!qk_both(true)) { aborted = true; break; }   // pass B, tile 0
+        if (n_tiles == 1) mma_commit(&bars[M_QE + qb]);  // the item's last read of Q is issued
         // the previous item's O must have been read before this item's first P V overwrites it
         if (!wait_bar(&bars[M_OE], (ic & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
         for (int t = 0; t < n_tiles && !aborted; ++t) {
           if (t + 1 < n_tiles) {
-            if (!qk_both()) { aborted = true; break; }
-            if (t + 2 == n_tiles) mma_commit(&bars[M_QE]);
+            if (!qk_both(true)) { aborted = true; break; }
+            if (t + 2 == n_tiles) mma_commit(&bars[M_QE + qb]);
           }
           const uint32_t vs = vc % NST;
           if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag)) { aborted = true; break; }
@@ -582,7 +741,10 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
           for (int gg = 0; gg < 2 && !aborted; ++gg) {
             if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag)) { aborted = true; break; }
             tc_after_sync();
-            mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
+            if constexpr (C::kT)
+              mma_pv_mn<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
+            else
+              mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
             mma_commit(&bars[M_PE + gg]);
             ++pc[gg];
           }
@@ -637,6 +799,8 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         ++sc;
       }
       const bool flag = !aborted && row_ok && (1.0f / l < a.refetch_threshold);
+      // p = 2^(c2 s - m2) / ell = 2^(c2 s + nmb); rows that are not stored here get p = 0
+      if constexpr (C::kT) nmb_s[g][r] = (row_ok && !flag) ? -(m2 + log2f(l)) : -INFINITY;
 
       // ---- flagged rows -> packed list (ascending row ids); counts of the item
       const unsigned bal = __ballot_sync(0xffffffffu, flag);
@@ -654,7 +818,74 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       }
 
       // ---- pass B: probabilities of the unflagged rows, column sums, P V
-      {
+      if constexpr (C::kT) {
+        // transposed: S^T = K Q^T puts one key on each TMEM lane; thread r owns key t*KT + r and
+        // sees the warpgroup's 128 query rows as columns, so its column sum of P is a register
+        // accumulation and it writes its key's column of P (MN-major: rows contiguous)
+        uint8_t* Pt = smem + C::oP + g * C::PB;
+        const int qt128 = pair * 2 + g;
+        const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
+        const float4* nmb4 = reinterpret_cast<const float4*>(&nmb_s[g][0]);
+        const float2 c2x2 = make_float2(c2, c2);
+        const uint32_t kcol = (static_cast<uint32_t>(r) >> 3) * 1024u + (static_cast<uint32_t>(r) & 7u) * 128u;
+        for (int t = 0; t < n_tiles; ++t) {
+          if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag), 1 + g)) { aborted = true; break; }
+          tc_after_sync();
+          const int key = t * KT + r;
+          const bool key_ok = key < a.n_kv;
+          float2 cs0 = make_float2(0.0f, 0.0f), cs1 = cs0;
+          // two halves of 64 query rows: the TMEM columns are released once the second half is
+          // loaded, half a tile before the probabilities are done
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) {
+            float v[64];
+            __syncwarp();
+            tmem_ld32(tmem + lane_base + C::tS + g * KT + hf * 64, v);
+            tmem_ld32(tmem + lane_base + C::tS + g * KT + hf * 64 + 32, v + 32);
+            tmem_ld_wait();
+            if (hf == 1) {
+              tc_before_sync();
+              mbar_arrive(&bars[M_SR + g]);
+              ++sc;
+            } else if (!wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag), 1 + g)) {
+              // the previous tile's P V must be done before this tile's P overwrites the buffer
+              aborted = true;
+              break;
+            }
+            if (key_ok) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {   // query rows 64 hf + 8c .. + 7
+                const float4 na = nmb4[16 * hf + 2 * c], nb = nmb4[16 * hf + 2 * c + 1];
+                float2 e0 = ffma2(make_float2(v[8 * c + 0], v[8 * c + 1]), c2x2, make_float2(na.x, na.y));
+                float2 e1 = ffma2(make_float2(v[8 * c + 2], v[8 * c + 3]), c2x2, make_float2(na.z, na.w));
+                float2 e2 = ffma2(make_float2(v[8 * c + 4], v[8 * c + 5]), c2x2, make_float2(nb.x, nb.y));
+                float2 e3 = ffma2(make_float2(v[8 * c + 6], v[8 * c + 7]), c2x2, make_float2(nb.z, nb.w));
+                e0 = exp2_pair<0>(e0);
+                e1 = exp2_pair<1>(e1);
+                e2 = exp2_pair<2>(e2);
+                e3 = exp2_pair<3>(e3);
+                cs0 = fadd2(cs0, e0);
+                cs1 = fadd2(cs1, e1);
+                cs0 = fadd2(cs0, e2);
+                cs1 = fadd2(cs1, e3);
+                *reinterpret_cast<uint4*>(Pt + hf * (KT * 128u) + kcol + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4)) =
+                    make_uint4(pack_f16x2(e0.x, e0.y), pack_f16x2(e1.x, e1.y), pack_f16x2(e2.x, e2.y),
+                               pack_f16x2(e3.x, e3.y));
+              }
+            } else {   // keys past the end: zero columns (their V rows are zero-filled too)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(Pt + hf * (KT * 128u) + kcol + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          if (aborted) break;   // uniform over the warpgroup
+          fence_async_smem();
+          mbar_arrive(&bars[M_PF + g]);
+          ++pc;
+          if (key < a.n_kv && qt128 < p.n_qt) p.tok_part[part_row + key] = (cs0.x + cs1.x) + (cs0.y + cs1.y);
+        }
+      } else {
         const bool live = row_ok && !flag;
         // p = 2^(c2 s - m2) / ell = 2^(c2 s - mb); rows that are not stored here get p = 0
         const float mb = live ? m2 + log2f(l) : INFINITY;
@@ -757,7 +988,12 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       }
     }
   }
-  if (__syncthreads_or(aborted) && tid == 0) report(a.dev_status, SPATTEN_E_TIMEOUT);
+  const bool any_abort = __syncthreads_or(aborted);
+  if (any_abort && tid == 0) report(a.dev_status, SPATTEN_E_TIMEOUT);
+  if (any_abort && warp == 11 && lane == 0) {   // every MMA already issued completes before TMEM is freed
+    mma_commit(&bars[M_DR]);
+    drain_wait(&bars[M_DR], 0u);
+  }
   tc_before_sync();
   __syncthreads();
   if (warp == 11) {

@@ -78,6 +78,8 @@ lib.spatten_attention_layer.restype = i32
 lib.spatten_attention_layer.argtypes = [C.POINTER(attn_args), vp, sz, vp]
 lib.spatten_attention_layer_noalloc.restype = i32
 lib.spatten_attention_layer_noalloc.argtypes = [C.POINTER(attn_args), vp]
+lib.spatten_selftest_exp2_poly.restype = i32
+lib.spatten_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
 lib.spatten_topk_workspace_size.restype = sz
 lib.spatten_topk_workspace_size.argtypes = [i32, i32, i32]
 lib.spatten_topk_select.restype = i32
@@ -95,7 +97,7 @@ EXPORTS = ["spatten_abi_version", "spatten_status_string", "spatten_last_cuda_er
            "spatten_attention_workspace_size", "spatten_attention_layer", "spatten_attention_layer_noalloc",
            "spatten_topk_workspace_size",
            "spatten_topk_select", "spatten_gather_kept", "spatten_cascade_workspace_size",
-           "spatten_cascade_forward"]
+           "spatten_cascade_forward", "spatten_selftest_exp2_poly"]
 
 
 class SpattenError(RuntimeError):
@@ -177,6 +179,11 @@ def gather_kept(src, src_batch, src_row, n_src, row_bytes, R, idx, ld_idx, k, ds
     check(lib.spatten_gather_kept(ptr(src), src_batch, src_row, n_src, row_bytes, R, ptr(idx), ld_idx, k, ptr(dst),
                                   dst_batch, dst_row, ptr(compose_in), ld_compose, ptr(compose_out), check_index,
                                   ptr(dev_status), _stream(stream)), "spatten_gather_kept")
+
+
+def selftest_exp2_poly(x, y, n, stream=None):
+    """y = 2^x by the attention kernels' FMA-pipe polynomial (diagnostic)."""
+    check(lib.spatten_selftest_exp2_poly(ptr(x), ptr(y), n, _stream(stream)), "spatten_selftest_exp2_poly")
 
 
 def kernel_launch_count() -> int:

@@ -317,6 +317,17 @@ size_t spatten_cascade_workspace_size(const spatten_cascade_cfg* cfg);
 int32_t spatten_cascade_forward(const spatten_cascade_cfg* cfg, const spatten_layer_weights* w,
                                 spatten_cascade_io* io, void* ws, size_t ws_bytes, void* stream);
 
+/* =============================================================================================
+ * Diagnostics
+ *
+ * spatten_selftest_exp2_poly -- y[i] = 2^x[i] by the polynomial the tensor-core attention kernels
+ * use for a share of their softmax exponentials (Cody-Waite reduction to [-1/2, 1/2] and a
+ * degree-5 minimax polynomial; §IV.E "Softmax" only says exponentials are computed).  Defined for
+ * x <= 0, the range of softmax exponents; x < -126 gives 2^-126.  Maximum relative error below
+ * 2^-22.  x, y: device float [n]; asynchronous on `stream`; SPATTEN_E_ARG for NULL or n < 1.
+ * ============================================================================================= */
+int32_t spatten_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

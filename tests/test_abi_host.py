@@ -37,6 +37,13 @@ def test_exports_every_declared_function(S):
     assert S.lib.spatten_abi_version() == 1
 
 
+def test_selftest_exp2_poly_rejects_bad_arguments(S):
+    L = S.lib
+    assert L.spatten_selftest_exp2_poly(None, 16, 4, None) == S.E_ARG
+    assert L.spatten_selftest_exp2_poly(16, None, 4, None) == S.E_ARG
+    assert L.spatten_selftest_exp2_poly(16, 32, 0, None) == S.E_ARG
+
+
 def test_struct_layout_matches_header(S, tmp_path):
     structs = {"spatten_attn_args": S.attn_args, "spatten_cascade_cfg": S.cascade_cfg,
                "spatten_layer_weights": S.layer_weights, "spatten_decode_cache": S.decode_cache,
