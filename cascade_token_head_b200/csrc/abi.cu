@@ -56,6 +56,7 @@ extern "C" const char* spatten_status_string(int32_t s) {
     case SPATTEN_E_TIMEOUT: return "SPATTEN_E_TIMEOUT: bounded device wait gave up";
     case SPATTEN_E_UNSUPPORTED: return "SPATTEN_E_UNSUPPORTED: configuration not implemented";
     case SPATTEN_E_INDEX: return "SPATTEN_E_INDEX: index list entry out of range";
+    case SPATTEN_E_RANGE: return "SPATTEN_E_RANGE: a value outside the range of the kernel's operand type";
     default: return "SPATTEN_E_UNKNOWN";
   }
 }

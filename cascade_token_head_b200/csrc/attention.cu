@@ -41,6 +41,7 @@ int32_t validate(const spatten_attn_args& a) {
   if (a.B < 1 || a.H < 1 || a.n_q < 1 || a.n_kv < 1) return SPATTEN_E_ARG;
   if (a.B > 65535 || a.H > 1024) return SPATTEN_E_ARG;
   if (a.kernel < SPATTEN_ATTN_AUTO || a.kernel > SPATTEN_ATTN_DECODE) return SPATTEN_E_ARG;
+  if (a.v_keep < 0) return SPATTEN_E_ARG;
   if (a.d_h != 64 && a.d_h != 128) return SPATTEN_E_UNSUPPORTED;
   if (a.H_kept < 1 || a.H_kept > a.H) return SPATTEN_E_ARG;
   if (!a.head_idx && a.H_kept != a.H) return SPATTEN_E_ARG;
@@ -103,7 +104,19 @@ size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
     fp = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * 2 * n_pair * a.n_kv);
     fh = c.take<float>(static_cast<size_t>(a.B) * a.H_kept * 2 * n_pair);
   }
+  float* hc = nullptr;
+  int32_t* vs = nullptr;
+  uint8_t* vm = nullptr;
+  if (value_pruning(a)) {
+    const size_t bh = static_cast<size_t>(a.B) * a.H_kept;
+    hc = c.take<float>(bh * a.n_kv);
+    vs = c.take<int32_t>(bh * a.v_keep);
+    if (path != Path::kDecode) vm = c.take<uint8_t>(bh * a.n_kv);
+  }
   if (p) {
+    p->head_col = hc;
+    p->v_sel = vs;
+    p->v_mask = vm;
     p->qt_rows = rows;
     p->n_qt = static_cast<int>(n_qt);
     p->tok_part = t;
@@ -154,14 +167,47 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
     if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
   }
   if (ev_begin) SPT_CUDA(cudaEventRecordWithFlags(ev_begin, st, ev_flags));
-  int32_t s;
-  switch (path) {
-    case Path::kTc: s = attn_tc_launch(p, st); break;
-    case Path::kDecode: s = attn_decode_launch(p, st); break;   // its own combine step reduces
-    default: s = attn_simt_launch(p, st); break;
+  auto run = [&](const AttnProblem& q) -> int32_t {
+    switch (path) {
+      case Path::kTc: return attn_tc_launch(q, st);
+      case Path::kDecode: return attn_decode_launch(q, st);   // its own combine step reduces
+      default: return attn_simt_launch(q, st);
+    }
+  };
+  if (!value_pruning(p.a)) {
+    SPT_TRY(run(p));
+    if (path != Path::kDecode && (p.a.tok_imp || p.a.head_imp)) SPT_TRY(attn_reduce_launch(p, st));
+  } else {
+    // local value pruning: each head's column sums of P select the V vectors it keeps
+    const int32_t R = p.a.B * p.a.H_kept;
+    if (path == Path::kDecode) {
+      // items and combine: token importance and each head's probabilities (p.head_col); the
+      // outputs are left to the pruned-output kernel (p.v_sel set)
+      SPT_TRY(run(p));
+      SPT_TRY(spatten_topk_select(p.head_col, R, p.a.n_kv, p.a.n_kv, p.a.v_keep, nullptr, 0, p.v_sel, p.a.v_keep,
+                                  nullptr, nullptr, 0, p.a.dev_status, st));
+      SPT_TRY(attn_decode_pruned_out_launch(p, st));
+    } else {
+      // run 1: token importance, refetch flags and counts, per-head column sums
+      AttnProblem r1 = p;
+      r1.a.head_imp = nullptr;
+      r1.v_mask = nullptr;
+      SPT_TRY(run(r1));
+      if (r1.a.tok_imp) SPT_TRY(attn_reduce_launch(r1, st));
+      SPT_TRY(attn_head_colsum_launch(r1, st));
+      SPT_TRY(spatten_topk_select(p.head_col, R, p.a.n_kv, p.a.n_kv, p.a.v_keep, nullptr, 0, p.v_sel, p.a.v_keep,
+                                  nullptr, nullptr, 0, p.a.dev_status, st));
+      uint8_t* mask = const_cast<uint8_t*>(p.v_mask);
+      SPT_TRY(attn_value_mask_launch(p, mask, st));
+      // run 2: the same layer with the dropped V vectors masked: outputs and head importance
+      AttnProblem r2 = p;
+      r2.a.tok_imp = nullptr;
+      r2.a.refetch_flags = nullptr;
+      r2.a.refetch_count = nullptr;
+      SPT_TRY(run(r2));
+      if (r2.a.head_imp) SPT_TRY(attn_reduce_launch(r2, st));
+    }
   }
-  if (s != SPATTEN_OK) return s;
-  if (path != Path::kDecode && (p.a.tok_imp || p.a.head_imp)) SPT_TRY(attn_reduce_launch(p, st));
   if (ev_end) SPT_CUDA(cudaEventRecordWithFlags(ev_end, st, ev_flags));
   return SPATTEN_OK;
 }

@@ -25,6 +25,12 @@ struct AttnProblem {
   float* dec_e;              // ws [2][B][H_kept][n_kv] exp(s - item max): MSB-only, full precision
   float* dec_stat;           // ws [B][H_kept][dec_items][4] item max and sum, both variants
   float* dec_o;              // ws [B][H_kept][dec_items][2][d_h] item sum of exp * V, both variants
+  // local value pruning (a.v_keep in [1, n_kv)): each kept head's column sums of P, its kept keys
+  // and (prefill) the V mask of the second run
+  float* head_col = nullptr;        // ws [B][H_kept][n_kv] (decode: written by the combine step)
+  int32_t* v_sel = nullptr;         // ws [B][H_kept][v_keep] kept keys, ascending; decode: set when
+                                    // the combine step leaves the outputs to the pruned-output kernel
+  const uint8_t* v_mask = nullptr;  // ws [B][H_kept][n_kv] 1 = V vector kept (prefill second run)
 };
 
 // Kernels (each returns a status after launching on `st`).
@@ -51,6 +57,13 @@ int32_t quantize_kv_pair(const void* k, const void* v, int32_t dtype, int32_t B,
 
 // Fixed-order reduction of the per-CTA partials into tok_imp / head_imp.
 int32_t attn_reduce_launch(const AttnProblem& p, cudaStream_t st);
+// Local value pruning, prefill: per-head column sums of the partials (same order as the reduction)
+// into p.head_col; the V mask from the kept key lists p.v_sel
+int32_t attn_head_colsum_launch(const AttnProblem& p, cudaStream_t st);
+int32_t attn_value_mask_launch(const AttnProblem& p, uint8_t* mask, cudaStream_t st);
+// Local value pruning, decode: O = sum over the kept keys of P_j v_j, head importance, flags
+int32_t attn_decode_pruned_out_launch(const AttnProblem& p, cudaStream_t st);
+inline bool value_pruning(const spatten_attn_args& a) { return a.v_keep > 0 && a.v_keep < a.n_kv; }
 
 // Head slot -> original head id; slots >= H_kept name the pruned heads in ascending order.
 __device__ __forceinline__ int head_of_slot(const spatten_attn_args& a, int b, int slot) {

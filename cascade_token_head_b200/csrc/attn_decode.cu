@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
 
   if (static_cast<int>(blockIdx.x) < nblk) {
     // ---- token importance of keys [j0, j0 + kCThreads): p_j summed over kept heads in slot order
-    if (!a.tok_imp) return;
+    // (and, under local value pruning, each head's p_j on its own into head_col)
+    if (!a.tok_imp && !p.head_col) return;
     const int j0 = blockIdx.x * kCThreads;
     const int it0 = j0 / ITEM;
     float* factor = sh;                                   // [HK][TI] factors of items it0 ..
@@ -313,13 +314,20 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
     const int64_t vstride = static_cast<int64_t>(a.B) * HK * n;
     const float* e = p.dec_e + static_cast<int64_t>(b) * HK * n + j;
     float t = 0.0f;
+    float* hc = p.head_col ? p.head_col + static_cast<int64_t>(b) * HK * n + j : nullptr;
 #pragma unroll 4
-    for (int slot = 0; slot < HK; ++slot)
-      t += e[(use_full[slot] ? vstride : 0) + static_cast<int64_t>(slot) * n] * factor[slot * TI + it];
-    const int64_t col = a.tok_imp_map ? a.tok_imp_map[static_cast<int64_t>(b) * a.tok_imp_map_ld + j] : j;
-    a.tok_imp[static_cast<int64_t>(b) * a.tok_imp_ld + col] += t;
+    for (int slot = 0; slot < HK; ++slot) {
+      const float pj = e[(use_full[slot] ? vstride : 0) + static_cast<int64_t>(slot) * n] * factor[slot * TI + it];
+      t += pj;
+      if (hc) hc[static_cast<int64_t>(slot) * n] = pj;
+    }
+    if (a.tok_imp) {
+      const int64_t col = a.tok_imp_map ? a.tok_imp_map[static_cast<int64_t>(b) * a.tok_imp_map_ld + j] : j;
+      a.tok_imp[static_cast<int64_t>(b) * a.tok_imp_ld + col] += t;
+    }
     return;
   }
+  if (p.v_sel) return;   // local value pruning: the pruned-output kernel writes the outputs
 
   // ---- output block of one head slot: O, sum |O| -> head importance, refetch flag
   const int slot = static_cast<int>(blockIdx.x) - nblk;
@@ -374,6 +382,76 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
   }
 }
 
+// Local value pruning in decode: one CTA per (kept head slot, sequence) [pruned slots: zero fill].
+// O = s_v * sum over the v_keep kept keys (ascending, p.v_sel) of p_j * code_j, with p_j the head's
+// final probability (p.head_col) and code_j = 16 MSB_j, or 16 MSB_j + LSB_j when the row refetches
+// (the same decision as the combine step); groups of threads take keys g, g + G, ... and their
+// partial sums are added in group order (bit-reproducible).  Then sum |O| -> head importance, the
+// refetch flag and count.
+template <int DH, typename QT, bool LSB>
+__global__ void __launch_bounds__(kCThreads) attn_decode_pruned_out_kernel(AttnProblem p) {
+  constexpr int G = kCThreads / DH;
+  const spatten_attn_args& a = p.a;
+  const int HK = a.H_kept, NI = p.dec_items, n = a.n_kv;
+  const int slot = blockIdx.x, b = blockIdx.y;
+  const int h = head_of_slot(a, b, slot);
+  QT* o = static_cast<QT*>(a.o) + static_cast<int64_t>(b) * a.n_q * a.o_ld_tok + static_cast<int64_t>(h) * DH;
+  if (slot >= HK) {
+    if (h >= 0 && threadIdx.x < DH) st_from_float(o + threadIdx.x, 0.0f);
+    return;
+  }
+  __shared__ float part[G][DH];
+  __shared__ float red[kCWarps];
+  __shared__ int s_full;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float4* stats = reinterpret_cast<const float4*>(p.dec_stat) + (static_cast<int64_t>(b) * HK + slot) * NI;
+  if (warp == 0) {
+    float m, inv_l;
+    const bool full = fold_row<LSB>(stats, NI, a.refetch_threshold, &m, &inv_l);
+    if (lane == 0) s_full = full ? 1 : 0;
+  }
+  __syncthreads();
+  const bool full = s_full != 0;
+  const int dim = threadIdx.x % DH, g = threadIdx.x / DH;
+  const int64_t bh = static_cast<int64_t>(b) * a.H + h;
+  const int64_t plane = bh * a.kv_cap;
+  const int32_t* sel = p.v_sel + (static_cast<int64_t>(b) * HK + slot) * a.v_keep;
+  const float* pj = p.head_col + (static_cast<int64_t>(b) * HK + slot) * n;
+  const int32_t* kvi = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
+  float v = 0.0f;
+  for (int c = g; c < a.v_keep; c += G) {
+    const int j = sel[c];
+    const int64_t row = plane + (kvi ? kvi[j] : j);
+    float code = 16.0f * static_cast<float>(a.v_msb[row * DH + dim]);
+    if (full) {
+      const uint8_t byte = a.v_lsb[row * (DH / 2) + dim / 2];
+      code += static_cast<float>((dim & 1) ? (byte >> 4) : (byte & 15));
+    }
+    v = fmaf(pj[j], code, v);
+  }
+  part[g][dim] = v;
+  __syncthreads();
+  float absv = 0.0f;
+  if (static_cast<int>(threadIdx.x) < DH) {
+    float t = 0.0f;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) t += part[gg][threadIdx.x];
+    t *= a.v_scale[bh];
+    st_from_float(o + threadIdx.x, t);
+    absv = fabsf(t);
+  }
+  absv = warp_sum(absv);
+  if (lane == 0) red[warp] = absv;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float hs = 0.0f;
+    for (int w = 0; w < DH / 32; ++w) hs += red[w];
+    if (a.head_imp) a.head_imp[bh] += hs;
+    if (a.refetch_flags) a.refetch_flags[bh * a.refetch_flags_ld] = full ? 1 : 0;
+    if (full && a.refetch_count) atomicAdd(a.refetch_count, 1);
+  }
+}
+
 // dynamic shared memory of the combine kernel: the larger of a token block's factor table and
 // flags and an output block's factor row
 size_t combine_smem(int d_h, int H_kept, int items) {
@@ -403,6 +481,17 @@ int32_t launch_dh(const AttnProblem& p, cudaStream_t st) {
   return p.a.refetch_threshold > 0.0f ? launch<DH, QT, true>(p, st) : launch<DH, QT, false>(p, st);
 }
 
+template <int DH, typename QT, bool LSB>
+int32_t launch_pruned_out(const AttnProblem& p, cudaStream_t st) {
+  const int slots = p.a.H_kept + (p.a.zero_pruned_heads ? p.a.H - p.a.H_kept : 0);
+  attn_decode_pruned_out_kernel<DH, QT, LSB><<<dim3(slots, p.a.B), kCThreads, 0, st>>>(p);
+  return launch_status();
+}
+template <int DH, typename QT>
+int32_t pruned_out_dh(const AttnProblem& p, cudaStream_t st) {
+  return p.a.refetch_threshold > 0.0f ? launch_pruned_out<DH, QT, true>(p, st) : launch_pruned_out<DH, QT, false>(p, st);
+}
+
 }  // namespace
 
 int decode_item_rows(int d_h) { return d_h == 64 ? DGeom<64>::ITEM : DGeom<128>::ITEM; }
@@ -418,6 +507,12 @@ int32_t attn_decode_launch(const AttnProblem& p, cudaStream_t st) {
   const bool bf = p.a.q_dtype == SPATTEN_BF16;
   if (p.a.d_h == 64) return bf ? launch_dh<64, __nv_bfloat16>(p, st) : launch_dh<64, float>(p, st);
   return bf ? launch_dh<128, __nv_bfloat16>(p, st) : launch_dh<128, float>(p, st);
+}
+
+int32_t attn_decode_pruned_out_launch(const AttnProblem& p, cudaStream_t st) {
+  const bool bf = p.a.q_dtype == SPATTEN_BF16;
+  if (p.a.d_h == 64) return bf ? pruned_out_dh<64, __nv_bfloat16>(p, st) : pruned_out_dh<64, float>(p, st);
+  return bf ? pruned_out_dh<128, __nv_bfloat16>(p, st) : pruned_out_dh<128, float>(p, st);
 }
 
 }  // namespace spt

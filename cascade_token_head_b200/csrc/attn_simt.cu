@@ -38,9 +38,11 @@ __device__ __forceinline__ float ldf(const void* base, int64_t off) {
 }
 
 // load one key tile (rows j0 .. j0+kKeys-1) of K or V into shared memory (hi and optionally lo)
+// keep (V under local value pruning): key j is loaded iff keep[j] != 0; dropped keys read as 0
 template <int DH, typename KVT>
 __device__ void load_tile(const spatten_attn_args& a, int b, int h, int j0, bool is_v, bool want_lo,
-                          float (*hi)[DH + 1], float (*lo)[DH + 1]) {
+                          float (*hi)[DH + 1], float (*lo)[DH + 1], const uint8_t* keep) {
+  if (!is_v) keep = nullptr;
   if (a.quantized) {
     const int8_t* msb = is_v ? a.v_msb : a.k_msb;
     const uint8_t* lsb = is_v ? a.v_lsb : a.k_lsb;
@@ -48,7 +50,7 @@ __device__ void load_tile(const spatten_attn_args& a, int b, int h, int j0, bool
     for (int e = threadIdx.x; e < kKeys * DH; e += kThreads) {
       const int jj = e / DH, d = e % DH, j = j0 + jj;
       float vh = 0.0f, vl = 0.0f;
-      if (j < a.n_kv) {
+      if (j < a.n_kv && (!keep || keep[j])) {
         const int64_t row = a.kv_idx ? a.kv_idx[static_cast<int64_t>(b) * a.kv_idx_ld + j] : j;
         const int64_t base = (static_cast<int64_t>(b) * a.H + h) * a.kv_cap + row;
         vh = s * 16.0f * static_cast<float>(msb[base * DH + d]);
@@ -65,7 +67,7 @@ __device__ void load_tile(const spatten_attn_args& a, int b, int h, int j0, bool
     for (int e = threadIdx.x; e < kKeys * DH; e += kThreads) {
       const int jj = e / DH, d = e % DH, j = j0 + jj;
       float v = 0.0f;
-      if (j < a.n_kv) v = ldf<KVT>(src, (static_cast<int64_t>(b) * a.n_kv + j) * a.kv_ld_tok + static_cast<int64_t>(h) * DH + d);
+      if (j < a.n_kv && (!keep || keep[j])) v = ldf<KVT>(src, (static_cast<int64_t>(b) * a.n_kv + j) * a.kv_ld_tok + static_cast<int64_t>(h) * DH + d);
       hi[jj][d] = v;
     }
   }
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnProblem p) {
   // ---- pass A: MSB / unquantized statistics --------------------------------------------------
   for (int t = 0; t < n_tiles; ++t) {
     __syncthreads();
-    load_tile<DH, KVT>(a, b, h, t * kKeys, false, false, sm.k_hi, sm.k_lo);
+    load_tile<DH, KVT>(a, b, h, t * kKeys, false, false, sm.k_hi, sm.k_lo, nullptr);
     __syncthreads();
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) {
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnProblem p) {
     for (int r = 0; r < kRowsPerWarp; ++r) { mf[r] = -INFINITY; lf[r] = 0.0f; }
     for (int t = 0; t < n_tiles; ++t) {
       __syncthreads();
-      load_tile<DH, KVT>(a, b, h, t * kKeys, false, true, sm.k_hi, sm.k_lo);
+      load_tile<DH, KVT>(a, b, h, t * kKeys, false, true, sm.k_hi, sm.k_lo, nullptr);
       __syncthreads();
 #pragma unroll
       for (int r = 0; r < kRowsPerWarp; ++r) {
@@ -183,10 +185,11 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnProblem p) {
   for (int r = 0; r < kRowsPerWarp; ++r) inv_l[r] = 1.0f / l[r];
 
   const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt) * a.n_kv;
+  const uint8_t* vkeep = p.v_mask ? p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv : nullptr;
   for (int t = 0; t < n_tiles; ++t) {
     __syncthreads();
-    load_tile<DH, KVT>(a, b, h, t * kKeys, false, any_flag, sm.k_hi, sm.k_lo);
-    load_tile<DH, KVT>(a, b, h, t * kKeys, true, any_flag, sm.v_hi, sm.v_lo);
+    load_tile<DH, KVT>(a, b, h, t * kKeys, false, any_flag, sm.k_hi, sm.k_lo, nullptr);
+    load_tile<DH, KVT>(a, b, h, t * kKeys, true, any_flag, sm.v_hi, sm.v_lo, vkeep);
     __syncthreads();
     float col[2] = {0.0f, 0.0f};
 #pragma unroll

@@ -107,6 +107,15 @@ __device__ __forceinline__ void cvt_u4x16(uint2 raw, uint32_t* out8) {
     }
   }
 }
+// true when one of eight bf16 values is out of fp16 range: magnitude 65536 or more (the bf16
+// patterns from 0x4780 up; bf16 has no value in (65504, 65536)), infinity or NaN
+__device__ __forceinline__ bool bf16x8_out_of_f16(uint4 u) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  bool out = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) out |= ((w[i] & 0x7FFFu) >= 0x4780u) || (((w[i] >> 16) & 0x7FFFu) >= 0x4780u);
+  return out;
+}
 // eight bf16 values -> four fp16 pairs (the query tile); exact for magnitudes in [2^-14, 65504]
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -255,13 +264,14 @@ __device__ __forceinline__ void add_f16x8(uint32_t* hi, const uint32_t* lo) {
 
 template <int DH, int KT>
 __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int64_t plane0, const int32_t* kv_idx,
-                                             const int8_t* msb, const uint8_t* lsb, uint32_t off_hi, int ptid) {
+                                             const int8_t* msb, const uint8_t* lsb, uint32_t off_hi, int ptid,
+                                             const uint8_t* keep) {
   constexpr int L16 = DH / 16;
   for (int e = ptid; e < KT * L16; e += kProducerThreads) {
     const int r = e / L16, c16 = e % L16;
     const int key = t * KT + r;
     uint32_t hi[8], lo[8];
-    if (key < n_kv) {
+    if (key < n_kv && (!keep || keep[key])) {
       const int64_t prow = plane0 + (kv_idx ? kv_idx[key] : key);
       cvt16_s8x16(__ldg(reinterpret_cast<const uint4*>(msb + prow * DH) + c16), hi);
       if (lsb) {
@@ -280,9 +290,11 @@ __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int
 
 // same conversion from a staged raw tile in shared memory: MSB rows (DH bytes each) at raw,
 // packed LSB rows (DH/2 bytes) at raw + KT*DH; rows >= valid are zero-filled
+// keep (V tiles under local value pruning): row r of the tile is kept iff keep[r] != 0; dropped
+// rows are zero-filled like the rows past the end
 template <int DH, int KT>
 __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw, bool with_lsb, int valid,
-                                               uint32_t off_hi, int ptid) {
+                                               uint32_t off_hi, int ptid, const uint8_t* keep) {
   constexpr int L16 = DH / 16;
   constexpr int TOTAL = KT * L16;
   constexpr int NIT = (TOTAL + kProducerThreads - 1) / kProducerThreads;
@@ -295,7 +307,7 @@ __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw
     const int r = e / L16, c16 = e % L16;
     m[i] = make_uint4(0u, 0u, 0u, 0u);
     lb[i] = make_uint2(0u, 0u);
-    if (e < TOTAL && r < valid) {
+    if (e < TOTAL && r < valid && (!keep || keep[r])) {
       m[i] = *reinterpret_cast<const uint4*>(raw + r * DH + c16 * 16);
       if (with_lsb) lb[i] = *reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8);
     }
@@ -306,7 +318,7 @@ __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw
     if (e >= TOTAL) break;
     const int r = e / L16, c16 = e % L16;
     uint32_t hi[8], lo[8];
-    if (r < valid) {
+    if (r < valid && (!keep || keep[r])) {
       cvt16_s8x16(m[i], hi);
       if (with_lsb) {
         cvt_u4x16(lb[i], lo);
@@ -344,6 +356,7 @@ struct JobStream {
   uint32_t g0 = 0;       // global index of this stream's job 0 in the staging ring's sequence
   uint32_t issued = 0;   // jobs of this stream issued so far (loader)
   uint32_t consumed = 0; // jobs of this stream converted so far
+  const uint8_t* vmask = nullptr;   // [n_kv] V vectors kept (local value pruning) or NULL
 
   __device__ __forceinline__ int jobs() const { return 3 * n_tiles; }
   __device__ __forceinline__ void job(int j, bool& is_v, int& t) const {
@@ -383,15 +396,17 @@ struct JobStream {
     bool is_v;
     int t;
     job(j, is_v, t);
+    const uint8_t* keep = (is_v && vmask) ? vmask : nullptr;
     if (kv_idx) {
       produce_tile<DH, KT>(smem, t, a->n_kv, plane0, kv_idx, is_v ? a->v_msb : a->k_msb,
-                           with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, ptid);
+                           with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, ptid, keep);
       return true;
     }
     const uint32_t gj = g0 + static_cast<uint32_t>(j);
     const uint32_t st = gj % RS;
     if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag)) return false;
-    convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid);
+    convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
+                           keep ? keep + t * KT : nullptr);
     mbar_arrive(&raw_empty[st]);
     ++consumed;
     return true;
@@ -603,7 +618,9 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       for (int e = ptid; e < QCH; e += kProducerThreads) {
         const int rr = e / (DH / 8), c8 = e % (DH / 8);
         uint4* p = reinterpret_cast<uint4*>(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128));
-        *p = bf16x8_to_f16x8(*p);
+        const uint4 v = *p;
+        if (bf16x8_out_of_f16(v)) report(a.dev_status, SPATTEN_E_RANGE);
+        *p = bf16x8_to_f16x8(v);
       }
     };
     uint32_t g_issued = 0, g_consumed = 0;   // staging-ring jobs issued / converted, whole kernel
@@ -615,6 +632,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
       JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
                                   abort_flag, gjob};
+      if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
       struct Track {   // records the stream's progress however the item's loop is left
         JobStream<DH, KT, C::RS>& js;
         uint32_t &gi, &gc;
@@ -656,9 +674,11 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
           for (int k = 0; k < BATCH; ++k) {
             const int e = e0 + k * kProducerThreads;
             const int rr = e / (DH / 8), c8 = e % (DH / 8);
-            if (e < NCH)
+            if (e < NCH) {
+              if (bf16x8_out_of_f16(qv[k])) report(a.dev_status, SPATTEN_E_RANGE);
               *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) =
                   bf16x8_to_f16x8(qv[k]);
+            }
           }
         }
         fence_async_smem();
@@ -1146,7 +1166,10 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     for (int k = 0; k < PER; ++k) {
       const int e = tid + k * 224;
       const int rr = e / (DH / 8), c8 = e % (DH / 8);
-      if (e < NCH) *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = bf16x8_to_f16x8(qv[k]);
+      if (e < NCH) {
+        if (bf16x8_out_of_f16(qv[k])) report(a.dev_status, SPATTEN_E_RANGE);
+        *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = bf16x8_to_f16x8(qv[k]);
+      }
     }
     fence_async_smem();
     mbar_arrive(&bars[F_Q]);
@@ -1156,6 +1179,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     const int ptid = tid - 128;
     JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[F_RF], &bars[F_RE], &a, plane0, n_tiles, true, ptid,
                                 abort_flag};
+    if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
     uint32_t kc = 0, vc = 0;
     auto run_jobs = [&](int j0, int j1) {
       for (int j = j0; j < j1; ++j) {

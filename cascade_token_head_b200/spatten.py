@@ -18,7 +18,7 @@ if not os.path.exists(LIB_PATH):
 lib = C.CDLL(LIB_PATH)
 
 # ---- enums (spatten.h) --------------------------------------------------------------------------
-OK, E_ARG, E_SHAPE, E_ALIGN, E_WORKSPACE, E_NONFINITE, E_CUDA, E_TIMEOUT, E_UNSUPPORTED, E_INDEX = range(10)
+OK, E_ARG, E_SHAPE, E_ALIGN, E_WORKSPACE, E_NONFINITE, E_CUDA, E_TIMEOUT, E_UNSUPPORTED, E_INDEX, E_RANGE = range(11)
 F32, BF16 = 0, 1
 PREFILL, DECODE_STEP = 0, 1
 ATTN_AUTO, ATTN_CUDA_CORE, ATTN_TENSOR_CORE, ATTN_DECODE = 0, 1, 2, 3
@@ -40,7 +40,7 @@ class attn_args(C.Structure):
                 ("tok_imp", vp), ("tok_imp_ld", i64), ("tok_imp_map", vp), ("tok_imp_map_ld", i64),
                 ("head_imp", vp), ("refetch_flags", vp), ("refetch_flags_ld", i64), ("refetch_count", vp),
                 ("dev_status", vp),
-                ("kernel", i32)]
+                ("kernel", i32), ("v_keep", i32)]
 
 
 class cascade_cfg(C.Structure):

@@ -54,7 +54,12 @@ enum spatten_status {
   SPATTEN_E_CUDA = 6,        /* a CUDA launch or runtime call failed                       */
   SPATTEN_E_TIMEOUT = 7,     /* a bounded device-side wait gave up                         */
   SPATTEN_E_UNSUPPORTED = 8, /* valid but not implemented (e.g. d_h not in {64, 128})      */
-  SPATTEN_E_INDEX = 9        /* (device) an index list entry was outside [0, n)            */
+  SPATTEN_E_INDEX = 9,       /* (device) an index list entry was outside [0, n)            */
+  SPATTEN_E_RANGE = 10       /* (device) a value left the range of the kernel's operand type:
+                                a bf16 query of magnitude 65536 or more (the smallest bf16
+                                value past fp16's 65504), infinite or NaN, given to the
+                                tensor-core kernels, which take fp16 operands; it is stored
+                                saturated to +-65504 and the call's results are unreliable     */
 };
 
 /* ---- element types ------------------------------------------------------------------------ */
@@ -104,6 +109,14 @@ int32_t spatten_quantize_kv(const void* x, int32_t dtype, int32_t B, int32_t H, 
  *   tok_imp[b][map(j)] += sum_{kept h, i} P_ij       (map(j) = tok_imp_map[b][j] or j)
  *   head_imp[b][h]     += sum_{i,d} |O_id|
  * Importance sums are reduced in a fixed order (reruns are bit-identical).
+ *
+ * Local value pruning (§III.A "Local Value Pruning": after the softmax a head discards its
+ * low-probability V vectors, for that head only), when 1 <= v_keep < n_kv: head h keeps the V
+ * vectors of the v_keep keys ranked first by (larger c_hj = sum_i P_ij, the key's column sum of the
+ * head's final probabilities, then lower j); its output becomes O_i = sum_{j kept} P_ij v_j with no
+ * renormalisation, and head_imp uses that output.  The token importance and the refetch decisions
+ * are those of the full probabilities.  The layer then runs its attention twice (once for the
+ * column sums, once with the V mask) and needs the larger workspace the size query reports.
  * ============================================================================================= */
 typedef struct spatten_attn_args {
   int32_t B, H;              /* sequences, heads in the layer (original head count)          */
@@ -151,6 +164,8 @@ typedef struct spatten_attn_args {
   int32_t* refetch_count;    /* device int32 (+= number of refetched rows) or NULL           */
   int32_t* dev_status;       /* device int32 or NULL                                         */
   int32_t kernel;            /* spatten_attn_kernel: 0 = choose automatically                */
+  int32_t v_keep;            /* local value pruning: 0 (or >= n_kv) keeps every V vector;     */
+                             /* else each kept head keeps v_keep of them (see below)          */
 } spatten_attn_args;
 
 /* Kernel choice for spatten_attention_layer.  AUTO picks the tensor-core kernel for bf16

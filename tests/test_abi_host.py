@@ -69,7 +69,7 @@ def test_struct_layout_matches_header(S, tmp_path):
 
 
 def test_status_strings(S):
-    for s in range(10):
+    for s in range(11):
         assert S.lib.spatten_status_string(s).decode().startswith("SPATTEN_")
     assert b"UNKNOWN" in S.lib.spatten_status_string(99)
 
@@ -144,10 +144,15 @@ def test_attention_argument_errors_and_workspace(S):
     assert L.spatten_attention_workspace_size(C.byref(_attn(S))) > 0
     for over, want in [(dict(d_h=96), S.E_UNSUPPORTED), (dict(H_kept=5), S.E_ARG), (dict(H_kept=3), S.E_ARG),
                        (dict(q=0), S.E_ARG), (dict(q_ld_tok=100), S.E_SHAPE), (dict(kv_cap=50), S.E_SHAPE),
-                       (dict(q=(1 << 20) + 8), S.E_ALIGN), (dict(kernel=9), S.E_ARG)]:
+                       (dict(q=(1 << 20) + 8), S.E_ALIGN), (dict(kernel=9), S.E_ARG), (dict(v_keep=-1), S.E_ARG)]:
         assert L.spatten_attention_layer(C.byref(_attn(S, **over)), 1 << 24, 1 << 30, None) == want, over
     # workspace too small
     assert L.spatten_attention_layer(C.byref(_attn(S)), 1 << 24, 16, None) == S.E_WORKSPACE
+    # local value pruning needs room for the per-head column sums, kept lists and V mask; keeping
+    # every key (v_keep >= n_kv) is no pruning and needs nothing more
+    base = L.spatten_attention_workspace_size(C.byref(_attn(S)))
+    assert L.spatten_attention_workspace_size(C.byref(_attn(S, v_keep=50))) >= base + 2 * 4 * 100 * (4 + 1) + 2 * 4 * 50 * 4
+    assert L.spatten_attention_workspace_size(C.byref(_attn(S, v_keep=100))) == base
     # a forced kernel that cannot run the problem
     assert L.spatten_attention_layer(C.byref(_attn(S, kernel=S.ATTN_DECODE)), 1 << 24, 1 << 30, None) == S.E_UNSUPPORTED
 

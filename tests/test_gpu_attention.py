@@ -33,7 +33,7 @@ def make_layer(B, H, n, d, seed, boost=0, dtype=BF, scale=1.0):
 
 
 def run_layer(S, raw, gain, B, H, n, d, theta, heads=None, kernel=0, dtype=BF, kv_idx=None, n_q=None,
-              cap=None, quantized=True):
+              cap=None, quantized=True, v_keep=0):
     """Quantize K/V on the device and run the attention layer.  Returns dict of host arrays."""
     esz = 2 if dtype == BF else 4
     x = to_dev(raw, dtype)
@@ -83,7 +83,7 @@ def run_layer(S, raw, gain, B, H, n, d, theta, heads=None, kernel=0, dtype=BF, k
     if kv_idx is not None:
         a.tok_imp_map, a.tok_imp_map_ld = kvi.data_ptr(), kv_idx.shape[1]
     a.head_imp, a.refetch_flags, a.refetch_count = hed.data_ptr(), flags.data_ptr(), cnt.data_ptr()
-    a.refetch_threshold, a.kernel = theta, kernel
+    a.refetch_threshold, a.kernel, a.v_keep = theta, kernel, v_keep
     w = ws(S.attention_workspace_size(a))
     S.attention_layer(a, w, w.numel())
     torch.cuda.synchronize()
@@ -95,8 +95,10 @@ def run_layer(S, raw, gain, B, H, n, d, theta, heads=None, kernel=0, dtype=BF, k
     return out
 
 
-def oracle_layer(raw, gain, B, H, n, d, theta, heads, dtype, got, kv_idx=None, n_q=None, quantized=True):
-    """Oracle over the same host-cast values; returns O, token/head importance, flags, pmax."""
+def oracle_layer(raw, gain, B, H, n, d, theta, heads, dtype, got, kv_idx=None, n_q=None, quantized=True,
+                 v_keep=None):
+    """Oracle over the same host-cast values; returns O, token/head importance, flags, pmax (and,
+    with v_keep, each head's kept V set and its column sums)."""
     vals = host_cast(raw, dtype)
     Q = split_heads(vals, H, d, 0)
     K = split_heads(vals, H, d, 1).astype(np.float32)
@@ -115,6 +117,7 @@ def oracle_layer(raw, gain, B, H, n, d, theta, heads, dtype, got, kv_idx=None, n
     tok = np.zeros((B, n_kv_cols))
     head = np.zeros((B, H))
     flags = np.zeros((B, H, n_q), bool)
+    kept, colsum = {}, {}
     near = 0
     for b in range(B):
         hs = range(H) if heads is None else heads[b]
@@ -124,22 +127,24 @@ def oracle_layer(raw, gain, B, H, n, d, theta, heads, dtype, got, kv_idx=None, n
             if quantized:
                 kq = dict(msb=mk[b, h, rows], lsb=R.unpack_lsb(lk[b, h, rows]), scale=sk[b, h])
                 vq = dict(msb=mv[b, h, rows], lsb=R.unpack_lsb(lv[b, h, rows]), scale=sv[b, h])
-                r = R.progressive_attention(q, kq, vq, theta, sm)
+                r = R.progressive_attention(q, kq, vq, theta, sm, v_keep=v_keep)
                 gf = got["flags"][b, h].astype(bool)
                 diff = gf != r["flags"]
                 if diff.any():
                     # only near-ties may disagree; then follow the kernel's decision
                     assert np.all(np.abs(r["pmax_msb"][diff] - theta) <= 1e-5 * theta), "flag mismatch off a tie"
                     near += int(diff.sum())
-                    r = R.progressive_attention(q, kq, vq, theta, sm, flags_override=gf)
+                    r = R.progressive_attention(q, kq, vq, theta, sm, flags_override=gf, v_keep=v_keep)
                 Oh, P = r["O"], r["P"]
                 flags[b, h] = r["flags"]
+                kept[b, h] = r["v_kept"]
             else:
-                Oh, P = R.dense_attention(q, K[b, h][rows], V[b, h][rows], sm)
+                Oh, P, kept[b, h] = R.dense_attention_value_pruned(q, K[b, h][rows], V[b, h][rows], sm, v_keep)
+            colsum[b, h] = P.sum(axis=0)
             O[b, :, h * d:(h + 1) * d] = Oh
             tok[b, rows] += R.token_importance_increment(P)
             head[b, h] += R.head_importance_increment(Oh)
-    return dict(O=O, tok=tok, head=head, flags=flags, near=near)
+    return dict(O=O, tok=tok, head=head, flags=flags, near=near, kept=kept, colsum=colsum)
 
 
 def check(got, ref, heads, H, d, tol_o, tol_head, dtype_name):
@@ -225,3 +230,36 @@ def test_attention_deterministic(cuda):
     np.testing.assert_array_equal(a["tok"], b["tok"])
     np.testing.assert_array_equal(a["head"], b["head"])
     np.testing.assert_array_equal(a["o"], b["o"])
+
+
+def test_attention_query_out_of_fp16_range_reports_status(cuda):
+    """The tensor-core kernels take fp16 operands: a bf16 query value past fp16's range is stored
+    saturated, and the call reports SPATTEN_E_RANGE in dev_status (in-range calls report 0)."""
+    S = lib()
+    B, H, n, d = 1, 2, 130, 64
+    for big, want in ((3.0, S.OK), (1.0e5, S.E_RANGE)):
+        raw, gain = make_layer(B, H, n, d, seed=31)
+        raw[0, 77, 5] = big                       # one element of head 0's query row 77
+        x = to_dev(raw, BF)
+        HD = H * d
+        planes = []
+        for t in (1, 2):
+            msb = torch.zeros((B, H, n, d), dtype=torch.int8, device="cuda")
+            lsb = torch.zeros((B, H, n, d // 2), dtype=torch.uint8, device="cuda")
+            sc = torch.zeros(B * H, device="cuda")
+            S.quantize_kv(x.data_ptr() + t * HD * 2, B, H, n, d, 3 * HD, msb, lsb, n, 0, scale_out=sc, dtype=S.BF16)
+            planes.append((msb, lsb, sc))
+        a = S.attn_args()
+        a.B, a.H, a.n_q, a.n_kv, a.d_h, a.H_kept = B, H, n, n, d, H
+        a.q, a.q_dtype, a.q_ld_tok = x.data_ptr(), S.BF16, 3 * HD
+        a.quantized, a.kv_cap = 1, n
+        a.k_msb, a.k_lsb, a.k_scale = (t.data_ptr() for t in planes[0])
+        a.v_msb, a.v_lsb, a.v_scale = (t.data_ptr() for t in planes[1])
+        o = torch.zeros((B, n, HD), dtype=BF, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        a.o, a.o_ld_tok, a.dev_status, a.refetch_threshold = o.data_ptr(), HD, st.data_ptr(), 0.1
+        a.kernel = S.ATTN_TENSOR_CORE
+        w = ws(S.attention_workspace_size(a))
+        S.attention_layer(a, w, w.numel())
+        torch.cuda.synchronize()
+        assert int(st.item()) == want
