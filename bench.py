@@ -51,6 +51,45 @@ METRIC = {
 DATA = "synthetic (seeded N(0,1) activations, random-init weights)"
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the prefill attention kernels of
+# one BERT-base-shaped layer (32 sequences, 12 heads of 64, 512 keys, refetch below 0.1), summed
+# over attn_main, attn_full and attn_reduce from one ncu capture of
+#   python -m cascade_token_head_b200.cases attention --B 32 --H 12 --n 512 --d 64 --theta 0.1 --reps 1
+# with --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum -k regex:attn_ -c 3.
+# The capture belongs to the sources whose hash it carries: once any of them changes the line
+# reports traffic null until the kernels are captured again.
+TRAFFIC_SOURCES = ("attn_tc.cu", "attention.cu", "attn_reduce.cu", "attention.cuh", "tc_ptx.cuh",
+                   "exp2_poly.cuh", "common.cuh")
+CAPTURED_TRAFFIC = {
+    "prefill_attention_layer": {"sources_sha256": "3854332367032eee", "bytes": 50446592 + 772096 + 39170048 + 4048384,
+                                "kept_key_heads": 512 * 12},
+}
+
+
+def sources_hash(files=TRAFFIC_SOURCES) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "cascade_token_head_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def prefill_traffic(w):
+    """DRAM bytes of one step's attention launches: the captured layer scaled by the step's
+    sum over layers of kept keys x kept heads (null when the kernels changed since the capture)."""
+    c = CAPTURED_TRAFFIC["prefill_attention_layer"]
+    if w.name != "bert_base_prefill_bf16":
+        return None, "null: no DRAM capture of this workload's layer shape"
+    if sources_hash() != c["sources_sha256"]:
+        return None, "null: the attention kernels changed since their DRAM capture"
+    units = sum(w.token_keep[l] * w.head_keep[l] for l in range(w.L))
+    per_seq = c["bytes"] / 32.0
+    return per_seq * w.B * units / c["kept_key_heads"], (
+        "ncu capture of one 32x12x512 layer (attn_main + attn_full + attn_reduce), scaled by the step's "
+        "sum over layers of kept keys x kept heads and by the batch")
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -532,6 +571,7 @@ def prefill_arm(ctx, args, name):
     attn_s = statistics.mean(attn_ms) / 1e3
     achieved = flops / attn_s / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    traffic, traffic_src = prefill_traffic(w)
     result = {
         "metric": METRIC[name],
         "value": whole_job_rate(ctx.world, tokens_per_step, K, total_ms), "unit": "tokens/s", "n_gpus": ctx.world,
@@ -544,7 +584,7 @@ def prefill_arm(ctx, args, name):
         "roofline": {"kernel": "attention (spatten_attention_layer kernels, all layers)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} bf16 sustained (the MMAs take fp16 operands: same nominal "
-                                  f"dense rate, ratio 1)", "traffic": None,
+                                  f"dense rate, ratio 1)", "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_flops_per_step": flops, "attn_ms_per_step": attn_s * 1e3},
         "e2e": {"value": whole_job_rate(ctx.world, tokens_per_step, n_e2e, e2e_total), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -31,6 +31,9 @@ namespace spt {
 namespace {
 
 constexpr int kDWarps = 4;        // warps (items) per CTA of the items kernel
+#ifndef SPT_DECODE_BATCH
+#define SPT_DECODE_BATCH 8
+#endif
 constexpr int kCThreads = 256;    // threads per CTA of the combine kernel
 
 template <int DH>
@@ -39,7 +42,7 @@ struct DGeom {
   static constexpr int KPW = 32 / LPK;       // keys per warp step
   static constexpr int ITEM = 8192 / DH;     // keys per item: 128 (d_h 64), 64 (d_h 128)
   static constexpr int STEPS = ITEM / KPW;   // warp steps per item
-  static constexpr int BATCH = 8;            // steps whose row loads are in flight together
+  static constexpr int BATCH = SPT_DECODE_BATCH;   // steps whose row loads are in flight together
 };
 
 // Paired fp32 arithmetic: the sm_100 float2 intrinsics (two lanes per instruction).
