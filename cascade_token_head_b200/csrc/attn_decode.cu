@@ -8,9 +8,11 @@
 // The work of one row (b, kept head) is cut into items of decode_item_rows(d_h) consecutive
 // entries of its key list, one warp per item, and finished by a per-sequence combine step:
 //
-// items kernel (memory-bound, no block-level barrier): a warp streams the K and V code rows of
-//   its item once -- lane groups of d_h/16 lanes read 16-byte MSB and 8-byte packed LSB slices,
-//   batches of rows in flight together -- and evaluates both precisions the refetch rule can pick:
+// items kernel (memory-bound, no block-level barrier): a warp loads its item's cache rows, then
+//   copies every K and V code slice of the item into shared memory at once (cp.async, lane groups
+//   of d_h/16 lanes taking 16-byte MSB and 8-byte packed LSB slices of a row; the K copies form
+//   one group, the V copies a second, so the scores start while V is still in flight), and
+//   evaluates both precisions the refetch rule can pick:
 //   s1 = s_k * sm_scale * 16 (q . MSB_j)            (MSB pass)
 //   s2 = s_k * sm_scale (q . (16 MSB_j + LSB_j))     (full 12-bit codes)
 //   It writes, per variant, the item's max m, sum ell of exp(s - m), the exponentials
@@ -30,10 +32,7 @@
 namespace spt {
 namespace {
 
-constexpr int kDWarps = 4;        // warps (items) per CTA of the items kernel
-#ifndef SPT_DECODE_BATCH
-#define SPT_DECODE_BATCH 8
-#endif
+constexpr int kDWarps = 2;        // warps (items) per CTA of the items kernel
 constexpr int kCThreads = 256;    // threads per CTA of the combine kernel
 
 template <int DH>
@@ -42,7 +41,6 @@ struct DGeom {
   static constexpr int KPW = 32 / LPK;       // keys per warp step
   static constexpr int ITEM = 8192 / DH;     // keys per item: 128 (d_h 64), 64 (d_h 128)
   static constexpr int STEPS = ITEM / KPW;   // warp steps per item
-  static constexpr int BATCH = SPT_DECODE_BATCH;   // steps whose row loads are in flight together
 };
 
 // Paired fp32 arithmetic: the sm_100 float2 intrinsics (two lanes per instruction).
@@ -78,20 +76,52 @@ __device__ __forceinline__ void lsb16(uint2 v, float2* f) {
   }
 }
 
+// cp.async copies into shared memory (LDGSTS: no registers held while in flight)
+__device__ __forceinline__ uint32_t dsmem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dsmem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dsmem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Shared memory of one warp of the items kernel: the item's K and V code slices, lane l's slices
+// of warp step s at [s][l] (each lane reads back only the slices it copied itself), then the
+// scores / exponentials [NV][ITEM]; the lane groups' e * V sums reuse the K MSB area.
+template <int DH, bool LSB>
+struct DSmem {
+  static constexpr int STEPS = DGeom<DH>::STEPS, ITEM = DGeom<DH>::ITEM, KPW = DGeom<DH>::KPW;
+  static constexpr int NV = LSB ? 2 : 1;
+  static constexpr int kMsb = 0;
+  static constexpr int vMsb = kMsb + STEPS * 32 * 16;
+  static constexpr int kLsb = vMsb + STEPS * 32 * 16;
+  static constexpr int vLsb = kLsb + (LSB ? STEPS * 32 * 8 : 0);
+  static constexpr int sc = vLsb + (LSB ? STEPS * 32 * 8 : 0);
+  static constexpr int bytes = sc + NV * ITEM * 4;
+  static_assert(KPW * NV * DH * 4 <= STEPS * 32 * 16, "the e*V sums fit the K MSB area");
+};
+
 template <int DH, typename QT, bool LSB>
 __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnProblem p) {
   using G = DGeom<DH>;
-  constexpr int LPK = G::LPK, KPW = G::KPW, ITEM = G::ITEM, STEPS = G::STEPS, BATCH = G::BATCH;
-  constexpr int NV = LSB ? 2 : 1;   // variants: MSB pass [, full precision]
+  using SM = DSmem<DH, LSB>;
+  constexpr int LPK = G::LPK, KPW = G::KPW, ITEM = G::ITEM, STEPS = G::STEPS;
+  constexpr int NV = SM::NV;
   const spatten_attn_args& a = p.a;
-  __shared__ float s_sc[kDWarps][NV][ITEM];         // scores, then exponentials
-  __shared__ float s_o[kDWarps][KPW][NV * DH];      // per lane group sums of e * V
+  extern __shared__ __align__(16) unsigned char d_smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the (kept head, item) pairs of sequence b, numbered head-major, one per warp
   const int w_id = blockIdx.x * kDWarps + warp;
   const int slot = w_id / p.dec_items, item = w_id % p.dec_items;
   if (slot >= a.H_kept) return;   // warps are independent: no block-level barrier follows
+  unsigned char* wsm = d_smem + warp * SM::bytes;
+  float* s_sc = reinterpret_cast<float*>(wsm + SM::sc);
   const int b = blockIdx.y;
   const int h = head_of_slot(a, b, slot);
   const int sub = lane % LPK, grp = lane / LPK;
@@ -102,6 +132,16 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
   const int64_t bs = static_cast<int64_t>(b) * a.H_kept + slot;
   const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
 
+  // ---- the item's cache rows (one round trip), then every code slice of the item in flight at
+  // once: the K group, then the V group
+  int rid[STEPS];   // cache row of the key of step s and this lane group, -1 past the key list
+  uint32_t valid = 0;   // bit s: step s has a key
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int j = j0 + s * KPW + grp;
+    rid[s] = j < n ? (kv_idx ? __ldg(kv_idx + j) : j) : -1;
+    if (j < n) valid |= 1u << s;
+  }
   float2 qf[8];
   {
     const QT* q = static_cast<const QT*>(a.q) + static_cast<int64_t>(b) * a.n_q * a.q_ld_tok +
@@ -110,54 +150,56 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
     for (int i = 0; i < 8; ++i) qf[i] = make_float2(ld_as_float(q + 2 * i), ld_as_float(q + 2 * i + 1));
   }
   const float ks = a.k_scale[bh];
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    if (rid[s] < 0) continue;
+    const int64_t r = plane0 + rid[s];
+    cp_async16(wsm + SM::kMsb + (s * 32 + lane) * 16, a.k_msb + r * DH + sub * 16);
+    if (LSB) cp_async8(wsm + SM::kLsb + (s * 32 + lane) * 8, a.k_lsb + r * (DH / 2) + sub * 8);
+  }
+  cp_async_commit();
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    if (rid[s] < 0) continue;
+    const int64_t r = plane0 + rid[s];
+    cp_async16(wsm + SM::vMsb + (s * 32 + lane) * 16, a.v_msb + r * DH + sub * 16);
+    if (LSB) cp_async8(wsm + SM::vLsb + (s * 32 + lane) * 8, a.v_lsb + r * (DH / 2) + sub * 8);
+  }
+  cp_async_commit();
   const float c1 = 16.0f * ks * a.sm_scale, c2 = ks * a.sm_scale;
-  auto row_of = [&](int j) -> int64_t { return j < n ? plane0 + (kv_idx ? __ldg(kv_idx + j) : j) : -1; };
 
   // ---- scores of both variants -----------------------------------------------------------------
+  cp_async_wait<1>();
   float m1 = -INFINITY, m2 = -INFINITY;
-#pragma unroll 1
-  for (int s0 = 0; s0 < STEPS; s0 += BATCH) {
-    int64_t row[BATCH];
+#pragma unroll 4
+  for (int s = 0; s < STEPS; ++s) {
+    // d1 = q . MSB_j; d2 = q . LSB_j; the full-precision dot product is 16 d1 + d2
+    const uint4 km = *reinterpret_cast<const uint4*>(wsm + SM::kMsb + (s * 32 + lane) * 16);
+    float2 f[8];
+    msb16(km, f);
+    float2 a1 = make_float2(0.0f, 0.0f), a2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) row[u] = row_of(j0 + (s0 + u) * KPW + grp);
-    uint4 km[BATCH];
-    uint2 kl[BATCH];
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u)
-      km[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.k_msb + row[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 8; ++i) a1 = ffma2(qf[i], f[i], a1);
     if (LSB) {
+      const uint2 kl = *reinterpret_cast<const uint2*>(wsm + SM::kLsb + (s * 32 + lane) * 8);
+      float2 g[8];
+      lsb16(kl, g);
 #pragma unroll
-      for (int u = 0; u < BATCH; ++u)
-        kl[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint2*>(a.k_lsb + row[u] * (DH / 2)) + sub) : make_uint2(0, 0);
+      for (int i = 0; i < 8; ++i) a2 = ffma2(qf[i], g[i], a2);
     }
+    float d1 = a1.x + a1.y, d2 = a2.x + a2.y;
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      // d1 = q . MSB_j; d2 = q . LSB_j; the full-precision dot product is 16 d1 + d2
-      float2 f[8];
-      msb16(km[u], f);
-      float2 a1 = make_float2(0.0f, 0.0f), a2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a1 = ffma2(qf[i], f[i], a1);
-      if (LSB) {
-        float2 g[8];
-        lsb16(kl[u], g);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a2 = ffma2(qf[i], g[i], a2);
-      }
-      float d1 = a1.x + a1.y, d2 = a2.x + a2.y;
-#pragma unroll
-      for (int o2 = 1; o2 < LPK; o2 <<= 1) {
-        d1 += __shfl_xor_sync(0xffffffffu, d1, o2);
-        if (LSB) d2 += __shfl_xor_sync(0xffffffffu, d2, o2);
-      }
-      if (row[u] >= 0) {
-        const float s1 = d1 * c1, s2 = fmaf(16.0f, d1, d2) * c2;
-        m1 = fmaxf(m1, s1);
-        if (LSB) m2 = fmaxf(m2, s2);
-        if (sub == 0) {
-          s_sc[warp][0][(s0 + u) * KPW + grp] = s1;
-          if (LSB) s_sc[warp][NV - 1][(s0 + u) * KPW + grp] = s2;
-        }
+    for (int o2 = 1; o2 < LPK; o2 <<= 1) {
+      d1 += __shfl_xor_sync(0xffffffffu, d1, o2);
+      if (LSB) d2 += __shfl_xor_sync(0xffffffffu, d2, o2);
+    }
+    if ((valid >> s) & 1u) {   // a slice past the key list was not copied: its value is not used
+      const float s1 = d1 * c1, s2 = fmaf(16.0f, d1, d2) * c2;
+      m1 = fmaxf(m1, s1);
+      if (LSB) m2 = fmaxf(m2, s2);
+      if (sub == 0) {
+        s_sc[s * KPW + grp] = s1;
+        if (LSB) s_sc[(NV - 1) * ITEM + s * KPW + grp] = s2;
       }
     }
   }
@@ -172,13 +214,13 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
   for (int k = lane; k < ITEM; k += 32) {
     const int j = j0 + k;
     if (j < n) {
-      const float e1 = expf(s_sc[warp][0][k] - m1);
-      s_sc[warp][0][k] = e1;
+      const float e1 = expf(s_sc[k] - m1);
+      s_sc[k] = e1;
       e_out[j] = e1;
       l1 += e1;
       if (LSB) {
-        const float e2 = expf(s_sc[warp][NV - 1][k] - m2);
-        s_sc[warp][NV - 1][k] = e2;
+        const float e2 = expf(s_sc[(NV - 1) * ITEM + k] - m2);
+        s_sc[(NV - 1) * ITEM + k] = e2;
         e_out[vstride + j] = e2;
         l2 += e2;
       }
@@ -189,52 +231,41 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
   __syncwarp();
 
   // ---- sums of e * V codes ----------------------------------------------------------------------
+  cp_async_wait<0>();
   float2 o1[8], o2[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o1[i] = o2[i] = make_float2(0.0f, 0.0f);
-#pragma unroll 1
-  for (int s0 = 0; s0 < STEPS; s0 += BATCH) {
-    int64_t row[BATCH];
+#pragma unroll 4
+  for (int s = 0; s < STEPS; ++s) {
+    if (!((valid >> s) & 1u)) continue;
+    const int k = s * KPW + grp;
+    const uint4 vm = *reinterpret_cast<const uint4*>(wsm + SM::vMsb + (s * 32 + lane) * 16);
+    float2 f[8];
+    msb16(vm, f);
+    const float e1 = s_sc[k];
+    const float2 e1v = make_float2(e1, e1);
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) row[u] = row_of(j0 + (s0 + u) * KPW + grp);
-    uint4 vm[BATCH];
-    uint2 vl[BATCH];
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u)
-      vm[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.v_msb + row[u] * DH) + sub) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 8; ++i) o1[i] = ffma2(e1v, f[i], o1[i]);
     if (LSB) {
+      const uint2 vl = *reinterpret_cast<const uint2*>(wsm + SM::vLsb + (s * 32 + lane) * 8);
+      float2 g[8];
+      lsb16(vl, g);
+      const float e2 = s_sc[(NV - 1) * ITEM + k];
+      const float2 e2v = make_float2(e2, e2), sixteen = make_float2(16.0f, 16.0f);
 #pragma unroll
-      for (int u = 0; u < BATCH; ++u)
-        vl[u] = row[u] >= 0 ? __ldg(reinterpret_cast<const uint2*>(a.v_lsb + row[u] * (DH / 2)) + sub) : make_uint2(0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      if (row[u] < 0) continue;
-      const int k = (s0 + u) * KPW + grp;
-      float2 f[8];
-      msb16(vm[u], f);
-      const float e1 = s_sc[warp][0][k];
-      const float2 e1v = make_float2(e1, e1);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o1[i] = ffma2(e1v, f[i], o1[i]);
-      if (LSB) {
-        float2 g[8];
-        lsb16(vl[u], g);
-        const float e2 = s_sc[warp][NV - 1][k];
-        const float2 e2v = make_float2(e2, e2), sixteen = make_float2(16.0f, 16.0f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o2[i] = ffma2(e2v, ffma2(sixteen, f[i], g[i]), o2[i]);
-      }
+      for (int i = 0; i < 8; ++i) o2[i] = ffma2(e2v, ffma2(sixteen, f[i], g[i]), o2[i]);
     }
   }
-  // add the lane groups' sums through shared memory, in group order
+  // add the lane groups' sums through shared memory (the K MSB area, read by every lane before
+  // the last warp barrier), in group order
+  float* s_o = reinterpret_cast<float*>(wsm + SM::kMsb);   // [KPW][NV * DH]
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    s_o[warp][grp][sub * 16 + 2 * i] = o1[i].x;
-    s_o[warp][grp][sub * 16 + 2 * i + 1] = o1[i].y;
+    s_o[grp * NV * DH + sub * 16 + 2 * i] = o1[i].x;
+    s_o[grp * NV * DH + sub * 16 + 2 * i + 1] = o1[i].y;
     if (LSB) {
-      s_o[warp][grp][DH + sub * 16 + 2 * i] = o2[i].x;
-      s_o[warp][grp][DH + sub * 16 + 2 * i + 1] = o2[i].y;
+      s_o[grp * NV * DH + DH + sub * 16 + 2 * i] = o2[i].x;
+      s_o[grp * NV * DH + DH + sub * 16 + 2 * i + 1] = o2[i].y;
     }
   }
   __syncwarp();
@@ -242,7 +273,7 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
   for (int t = lane; t < NV * DH; t += 32) {
     float v = 0.0f;
 #pragma unroll
-    for (int g = 0; g < KPW; ++g) v += s_o[warp][g][t];
+    for (int g = 0; g < KPW; ++g) v += s_o[g * NV * DH + t];
     o_out[t] = v;
   }
   if (lane == 0)
@@ -251,11 +282,19 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
 
 // Row statistics of one kept head folded by one warp in a fixed order (lane-strided item partials,
 // then a butterfly); returns whether the row refetches, and the chosen variant's (m, 1/ell).
-template <bool LSB>
-__device__ __forceinline__ bool fold_row(const float4* st, int NI, float theta, float* m_out, float* inv_l_out) {
+// v0: this lane's first item statistics, st[lane] (kNoItem past the row), loaded by the caller so
+// that the load can be in flight with others.
+__device__ __forceinline__ float4 no_item() { return make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f); }
+__device__ __forceinline__ float4 first_item(const float4* st, int NI) {
   const int lane = threadIdx.x & 31;
-  float M1 = -INFINITY, M2 = -INFINITY;
-  for (int i = lane; i < NI; i += 32) {
+  return lane < NI ? st[lane] : no_item();
+}
+template <bool LSB>
+__device__ __forceinline__ bool fold_row(float4 v0, const float4* st, int NI, float theta, float* m_out,
+                                         float* inv_l_out) {
+  const int lane = threadIdx.x & 31;
+  float M1 = v0.x, M2 = v0.z;
+  for (int i = lane + 32; i < NI; i += 32) {
     const float4 v = st[i];
     M1 = fmaxf(M1, v.x);
     M2 = fmaxf(M2, v.z);
@@ -263,7 +302,11 @@ __device__ __forceinline__ bool fold_row(const float4* st, int NI, float theta, 
   M1 = warp_max(M1);
   if (LSB) M2 = warp_max(M2);
   float L1 = 0.0f, L2 = 0.0f;
-  for (int i = lane; i < NI; i += 32) {
+  if (lane < NI) {
+    L1 = v0.y * expf(v0.x - M1);
+    if (LSB) L2 = v0.w * expf(v0.z - M2);
+  }
+  for (int i = lane + 32; i < NI; i += 32) {
     const float4 v = st[i];
     L1 += v.y * expf(v.x - M1);
     if (LSB) L2 += v.w * expf(v.z - M2);
@@ -275,8 +318,15 @@ __device__ __forceinline__ bool fold_row(const float4* st, int NI, float theta, 
   *inv_l_out = 1.0f / (full ? L2 : L1);
   return full;
 }
+template <bool LSB>
+__device__ __forceinline__ bool fold_row(const float4* st, int NI, float theta, float* m_out, float* inv_l_out) {
+  return fold_row<LSB>(first_item(st, NI), st, NI, theta, m_out, inv_l_out);
+}
 
 constexpr int kCWarps = kCThreads / 32;
+constexpr int kCSlots = 4;    // kept heads per warp whose statistics a token block loads up front
+constexpr int kCHeads = 16;   // kept heads whose exponentials a token-block thread loads up front
+constexpr int kCItems = 4;    // items per thread whose partial outputs an output block loads up front
 
 template <int DH, typename QT, bool LSB>
 __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProblem p) {
@@ -299,35 +349,72 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
     if (!a.tok_imp && !p.head_col) return;
     const int j0 = blockIdx.x * kCThreads;
     const int it0 = j0 / ITEM;
-    float* factor = sh;                                   // [HK][TI] factors of items it0 ..
-    int* use_full = reinterpret_cast<int*>(sh + HK * TI); // [HK]
-    for (int slot = warp; slot < HK; slot += kCWarps) {
-      float m, inv_l;
-      const bool full = fold_row<LSB>(stats + static_cast<int64_t>(slot) * NI, NI, a.refetch_threshold, &m, &inv_l);
-      if (lane < TI && it0 + lane < NI) {
-        const float4 v = stats[static_cast<int64_t>(slot) * NI + it0 + lane];
-        factor[slot * TI + lane] = expf((full ? v.z : v.x) - m) * inv_l;
-      }
-      if (lane == 0) use_full[slot] = full ? 1 : 0;
-    }
-    __syncthreads();
     const int j = j0 + threadIdx.x;
-    if (j >= n) return;
-    const int it = j / ITEM - it0;
+    const bool jv = j < n;
     const int64_t vstride = static_cast<int64_t>(a.B) * HK * n;
     const float* e = p.dec_e + static_cast<int64_t>(b) * HK * n + j;
+    // independent of the row statistics, so in flight with their loads: the key's importance
+    // entry and the exponentials of both variants for the first kCHeads kept heads
+    int64_t dst = 0;
+    float cur = 0.0f;
+    if (jv && a.tok_imp) {
+      const int64_t col = a.tok_imp_map ? a.tok_imp_map[static_cast<int64_t>(b) * a.tok_imp_map_ld + j] : j;
+      dst = static_cast<int64_t>(b) * a.tok_imp_ld + col;
+      cur = a.tok_imp[dst];
+    }
+    float e1[kCHeads], e2[kCHeads];
+#pragma unroll
+    for (int u = 0; u < kCHeads; ++u) {
+      e1[u] = jv && u < HK ? e[static_cast<int64_t>(u) * n] : 0.0f;
+      e2[u] = LSB && jv && u < HK ? e[vstride + static_cast<int64_t>(u) * n] : 0.0f;
+    }
+    float* factor = sh;                                   // [HK][TI] factors of items it0 ..
+    int* use_full = reinterpret_cast<int*>(sh + HK * TI); // [HK]
+    float4 pre[kCSlots];
+#pragma unroll
+    for (int u = 0; u < kCSlots; ++u) {
+      const int slot = warp + u * kCWarps;
+      pre[u] = slot < HK ? first_item(stats + static_cast<int64_t>(slot) * NI, NI) : no_item();
+    }
+    auto fold_slot = [&](int slot, float4 v0) {
+      const float4* st = stats + static_cast<int64_t>(slot) * NI;
+      float m, inv_l;
+      const bool full = fold_row<LSB>(v0, st, NI, a.refetch_threshold, &m, &inv_l);
+      // the factors of items it0 .. it0 + TI - 1: from the first-item registers when they hold them
+      float4 v;
+      if (it0 + TI <= 32) {
+        v.x = __shfl_sync(0xffffffffu, v0.x, (it0 + lane) & 31);
+        v.z = __shfl_sync(0xffffffffu, v0.z, (it0 + lane) & 31);
+      } else if (lane < TI && it0 + lane < NI) {
+        v = st[it0 + lane];
+      }
+      if (lane < TI && it0 + lane < NI) factor[slot * TI + lane] = expf((full ? v.z : v.x) - m) * inv_l;
+      if (lane == 0) use_full[slot] = full ? 1 : 0;
+    };
+#pragma unroll
+    for (int u = 0; u < kCSlots; ++u)
+      if (warp + u * kCWarps < HK) fold_slot(warp + u * kCWarps, pre[u]);
+    for (int slot = warp + kCSlots * kCWarps; slot < HK; slot += kCWarps)
+      fold_slot(slot, first_item(stats + static_cast<int64_t>(slot) * NI, NI));
+    __syncthreads();
+    if (!jv) return;
+    const int it = j / ITEM - it0;
     float t = 0.0f;
     float* hc = p.head_col ? p.head_col + static_cast<int64_t>(b) * HK * n + j : nullptr;
-#pragma unroll 4
-    for (int slot = 0; slot < HK; ++slot) {
+#pragma unroll
+    for (int u = 0; u < kCHeads; ++u) {
+      if (u < HK) {
+        const float pj = (use_full[u] ? e2[u] : e1[u]) * factor[u * TI + it];
+        t += pj;
+        if (hc) hc[static_cast<int64_t>(u) * n] = pj;
+      }
+    }
+    for (int slot = kCHeads; slot < HK; ++slot) {
       const float pj = e[(use_full[slot] ? vstride : 0) + static_cast<int64_t>(slot) * n] * factor[slot * TI + it];
       t += pj;
       if (hc) hc[static_cast<int64_t>(slot) * n] = pj;
     }
-    if (a.tok_imp) {
-      const int64_t col = a.tok_imp_map ? a.tok_imp_map[static_cast<int64_t>(b) * a.tok_imp_map_ld + j] : j;
-      a.tok_imp[static_cast<int64_t>(b) * a.tok_imp_ld + col] += t;
-    }
+    if (a.tok_imp) a.tok_imp[dst] = cur + t;
     return;
   }
   if (p.v_sel) return;   // local value pruning: the pruned-output kernel writes the outputs
@@ -340,25 +427,37 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
     if (h >= 0 && threadIdx.x < DH) st_from_float(o + threadIdx.x, 0.0f);
     return;
   }
-  float* factor = sh;   // [NI]
-  __shared__ int s_full;
-  if (warp == 0) {
-    float m, inv_l;
-    const bool full = fold_row<LSB>(stats + static_cast<int64_t>(slot) * NI, NI, a.refetch_threshold, &m, &inv_l);
-    for (int i = lane; i < NI; i += 32) {
-      const float4 v = stats[static_cast<int64_t>(slot) * NI + i];
-      factor[i] = expf((full ? v.z : v.x) - m) * inv_l;
-    }
-    if (lane == 0) s_full = full ? 1 : 0;
-  }
-  __syncthreads();
-  const bool full = s_full != 0;
+  const int64_t bhh = static_cast<int64_t>(b) * a.H + h;
+  const float4* st = stats + static_cast<int64_t>(slot) * NI;
   const int dim = threadIdx.x % DH, g = threadIdx.x / DH;
+  // everything this thread reads, issued before the fold: the row's first item statistics, this
+  // thread's items' statistics and partial outputs of both variants, the value scale
+  const float4 v0 = first_item(st, NI);
+  const float* op = p.dec_o + (static_cast<int64_t>(b) * HK + slot) * NI * 2 * DH + dim;
+  float2 sx[kCItems];
+  float o1[kCItems], o2[kCItems];
+#pragma unroll
+  for (int u = 0; u < kCItems; ++u) {
+    const int i = g + u * IG;
+    const bool iv = i < NI;
+    const float4 si = iv ? st[i] : no_item();
+    sx[u] = make_float2(si.x, si.z);
+    o1[u] = iv ? op[static_cast<int64_t>(i) * 2 * DH] : 0.0f;
+    o2[u] = LSB && iv ? op[static_cast<int64_t>(i) * 2 * DH + DH] : 0.0f;
+  }
+  const float vs = a.v_scale[bhh];
+  // every warp folds the row (the same loads and order, so the same decision in every warp)
+  float m, inv_l;
+  const bool full = fold_row<LSB>(v0, st, NI, a.refetch_threshold, &m, &inv_l);
   {
-    const float* op = p.dec_o + (static_cast<int64_t>(b) * HK + slot) * NI * 2 * DH + (full ? DH : 0) + dim;
     float v = 0.0f;
-#pragma unroll 4
-    for (int i = g; i < NI; i += IG) v += op[static_cast<int64_t>(i) * 2 * DH] * factor[i];
+#pragma unroll
+    for (int u = 0; u < kCItems; ++u)
+      if (g + u * IG < NI) v += (full ? o2[u] : o1[u]) * (expf((full ? sx[u].y : sx[u].x) - m) * inv_l);
+    for (int i = g + kCItems * IG; i < NI; i += IG) {
+      const float4 si = st[i];
+      v += op[static_cast<int64_t>(i) * 2 * DH + (full ? DH : 0)] * (expf((full ? si.z : si.x) - m) * inv_l);
+    }
     part[g][dim] = v;
   }
   __syncthreads();
@@ -368,7 +467,7 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
 #pragma unroll
     for (int gg = 0; gg < IG; ++gg) v += part[gg][threadIdx.x];
     // the MSB-pass sums hold e * MSB_j; its dequantized value is s_v * 16 * MSB_j
-    v *= a.v_scale[static_cast<int64_t>(b) * a.H + h] * (full ? 1.0f : 16.0f);
+    v *= vs * (full ? 1.0f : 16.0f);
     st_from_float(o + threadIdx.x, v);
     absv = fabsf(v);
   }
@@ -378,7 +477,6 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_combine_kernel(AttnProb
   if (threadIdx.x == 0) {
     float hs = 0.0f;
     for (int w = 0; w < DH / 32; ++w) hs += red[w];
-    const int64_t bhh = static_cast<int64_t>(b) * a.H + h;
     if (a.head_imp) a.head_imp[bhh] += hs;
     if (a.refetch_flags) a.refetch_flags[bhh * a.refetch_flags_ld] = full ? 1 : 0;
     if (full && a.refetch_count) atomicAdd(a.refetch_count, 1);
@@ -455,27 +553,32 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_pruned_out_kernel(AttnP
   }
 }
 
-// dynamic shared memory of the combine kernel: the larger of a token block's factor table and
-// flags and an output block's factor row
-size_t combine_smem(int d_h, int H_kept, int items) {
+// dynamic shared memory of the combine kernel: a token block's factor table and flags
+size_t combine_smem(int d_h, int H_kept) {
   const int item_rows = d_h == 64 ? DGeom<64>::ITEM : DGeom<128>::ITEM;
   const int ti = (kCThreads + item_rows - 1) / item_rows + 1;
-  const size_t tok = static_cast<size_t>(H_kept) * (ti + 1) * 4;
-  const size_t out = static_cast<size_t>(items) * 4;
-  return tok > out ? tok : out;
+  return static_cast<size_t>(H_kept) * (ti + 1) * 4;
 }
 
 template <int DH, typename QT, bool LSB>
 int32_t launch(const AttnProblem& p, cudaStream_t st) {
   const int items = p.dec_items;
   const int64_t per_seq = static_cast<int64_t>(items) * p.a.H_kept;
+  constexpr int smem = kDWarps * DSmem<DH, LSB>::bytes;
+  static DeviceOnce once;
+  int dev = 0;
+  SPT_TRY(once_per_device(once, &dev, [](int) -> int32_t {
+    SPT_CUDA(cudaFuncSetAttribute(attn_decode_items_kernel<DH, QT, LSB>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    return SPATTEN_OK;
+  }));
   attn_decode_items_kernel<DH, QT, LSB>
-      <<<dim3(static_cast<unsigned>(ceil_div(per_seq, kDWarps)), p.a.B), kDWarps * 32, 0, st>>>(p);
+      <<<dim3(static_cast<unsigned>(ceil_div(per_seq, kDWarps)), p.a.B), kDWarps * 32, smem, st>>>(p);
   SPT_TRY(launch_status());
   const int nblk = static_cast<int>(ceil_div(p.a.n_kv, kCThreads));
   const int slots = p.a.H_kept + (p.a.zero_pruned_heads ? p.a.H - p.a.H_kept : 0);
   attn_decode_combine_kernel<DH, QT, LSB>
-      <<<dim3(nblk + slots, p.a.B), kCThreads, combine_smem(DH, p.a.H_kept, items), st>>>(p);
+      <<<dim3(nblk + slots, p.a.B), kCThreads, combine_smem(DH, p.a.H_kept), st>>>(p);
   return launch_status();
 }
 
@@ -501,9 +604,10 @@ int decode_item_rows(int d_h) { return d_h == 64 ? DGeom<64>::ITEM : DGeom<128>:
 
 bool attn_decode_supported(const spatten_attn_args& a) {
   if (!a.quantized || a.n_q != 1 || (a.d_h != 64 && a.d_h != 128)) return false;
-  // the combine step keeps item factors in shared memory (48 KB without opting in)
+  // up to 12 K items per row; a token block of the combine step keeps every kept head's factors
+  // in shared memory (48 KB without opting in)
   const int64_t items = ceil_div(a.n_kv, decode_item_rows(a.d_h));
-  return items <= 12 * 1024 && combine_smem(a.d_h, a.H_kept, static_cast<int>(items)) <= 48 * 1024;
+  return items <= 12 * 1024 && combine_smem(a.d_h, a.H_kept) <= 48 * 1024;
 }
 
 int32_t attn_decode_launch(const AttnProblem& p, cudaStream_t st) {
