@@ -525,6 +525,45 @@ __device__ __forceinline__ bool softmax_all(bool ok) {
 // stride of gridDim.x; TMEM, barriers and every ring counter live across items, so the producers
 // load the next item's query tile and first key tiles, and the MMA warp issues its first score
 // MMAs, while the softmax warps finish the previous item.
+// Zero-filled outputs of the pruned heads (slots H_kept .. H-1), shared out over the softmax warps
+// of all CTAs before their first scores arrive (the stores overlap the first tiles' loads): warp w
+// of the grid takes the units (sequence, pruned slot, 64 query rows) w, w + 8 * gridDim.x, ...
+template <int DH>
+__device__ __forceinline__ void zero_pruned_share(const spatten_attn_args& a, __nv_bfloat16* o, int warp, int lane) {
+  constexpr int kRows = 64, C8 = DH / 8;
+  const int np = a.H - a.H_kept;
+  const int rblk = (a.n_q + kRows - 1) / kRows;
+  const int64_t units = static_cast<int64_t>(a.B) * np * rblk;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * 8 + warp; u < units; u += static_cast<int64_t>(gridDim.x) * 8) {
+    const int rb = static_cast<int>(u % rblk);
+    const int ps = static_cast<int>((u / rblk) % np);
+    const int b = static_cast<int>(u / (static_cast<int64_t>(rblk) * np));
+    int h = ps;
+    if (a.head_idx) {
+      if (a.H <= 32) {
+        // the ps-th head (in index order) that no kept slot lists
+        const int32_t* hi = a.head_idx + static_cast<int64_t>(b) * a.head_idx_ld;
+        bool kept = lane >= a.H;
+        for (int s = 0; s < a.H_kept; ++s) kept |= hi[s] == lane;
+        uint32_t free_mask = __ballot_sync(0xffffffffu, !kept);
+        for (int k = 0; k < ps; ++k) free_mask &= free_mask - 1;
+        h = free_mask ? __ffs(free_mask) - 1 : -1;
+      } else {
+        h = head_of_slot(a, b, a.H_kept + ps);
+      }
+    } else {
+      h = a.H_kept + ps;
+    }
+    if (h < 0) continue;
+    const int i0 = rb * kRows, rows = min(kRows, a.n_q - i0);
+    for (int e = lane; e < rows * C8; e += 32) {
+      const int i = i0 + e / C8, c8 = e % C8;
+      *reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH +
+                                c8 * 8) = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
 template <int DH>
 __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   using C = MainCfg<DH>;
@@ -777,6 +816,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     }
   } else {
     // ------------------------------------------------------------------------- softmax
+    if (a.zero_pruned_heads && a.H_kept < a.H) zero_pruned_share<DH>(a, o, warp, lane);
     const int g = warp >> 2;                        // warpgroup
     const int r = tid & 127;                        // row within the warpgroup's tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -1019,21 +1059,6 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   if (warp == 11) {
     tc_after_sync();
     tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-// zero-filled outputs of the pruned heads (slots H_kept .. H-1): one CTA per (slot, sequence)
-template <int DH>
-__global__ void __launch_bounds__(256) attn_zero_heads_kernel(AttnProblem p) {
-  const spatten_attn_args& a = p.a;
-  const int slot = a.H_kept + blockIdx.x, b = blockIdx.y;
-  const int h = head_of_slot(a, b, slot);
-  if (h < 0) return;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
-  for (int e = threadIdx.x; e < a.n_q * (DH / 8); e += blockDim.x) {
-    const int i = e / (DH / 8), c8 = e % (DH / 8);
-    *reinterpret_cast<uint4*>(o + (static_cast<int64_t>(b) * a.n_q + i) * a.o_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8) =
-        make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -1387,10 +1412,6 @@ int32_t launch(const AttnProblem& p, cudaStream_t st) {
   const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
   attn_main_kernel<DH><<<grid, 384, MainCfg<DH>::kSmem, st>>>(p);
   SPT_TRY(launch_status());
-  if (p.a.zero_pruned_heads && p.a.H_kept < p.a.H) {
-    attn_zero_heads_kernel<DH><<<dim3(p.a.H - p.a.H_kept, p.a.B), 256, 0, st>>>(p);
-    SPT_TRY(launch_status());
-  }
   if (p.a.refetch_threshold > 0.0f) {
     attn_full_kernel<DH><<<dim3(p.n_qt, p.a.H_kept, p.a.B), 256, FullCfg<DH>::kSmem, st>>>(p);
     SPT_TRY(launch_status());
