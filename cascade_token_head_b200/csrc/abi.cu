@@ -3,6 +3,7 @@
 #include <cstdio>
 #include <cstring>
 
+#include "attention.cuh"
 #include "common.cuh"
 
 namespace spt {
@@ -64,3 +65,15 @@ extern "C" const char* spatten_status_string(int32_t s) {
 extern "C" const char* spatten_last_cuda_error(void) { return spt::g_last_cuda_error; }
 
 extern "C" uint64_t spatten_kernel_launch_count(void) { return spt::launches(); }
+
+namespace spt {
+namespace {
+std::atomic<uint32_t> g_wait_limit{0};
+}
+uint32_t wait_limit_setting() {
+  const uint32_t v = g_wait_limit.load(std::memory_order_relaxed);
+  return v ? v : kDefaultWaitLimit;
+}
+}  // namespace spt
+
+extern "C" void spatten_set_wait_limit(uint32_t polls) { spt::g_wait_limit.store(polls, std::memory_order_relaxed); }

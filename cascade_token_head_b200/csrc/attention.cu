@@ -151,6 +151,7 @@ int32_t attention_layer_timed(const spatten_attn_args* args, void* ws, size_t ws
   SPT_TRY(validate(*args));
   AttnProblem p;
   std::memcpy(&p.a, args, sizeof(spatten_attn_args));
+  p.wait_limit = wait_limit_setting();
   if (!(p.a.sm_scale > 0.0f)) p.a.sm_scale = 1.0f / std::sqrt(static_cast<float>(p.a.d_h));
   if (p.a.head_idx_ld == 0) p.a.head_idx_ld = p.a.H_kept;
   if (p.a.refetch_flags_ld == 0) p.a.refetch_flags_ld = p.a.n_q;

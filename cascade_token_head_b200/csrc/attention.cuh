@@ -6,6 +6,10 @@
 namespace spt {
 
 // Resolved attention problem (validated by the dispatcher).
+constexpr uint32_t kDefaultWaitLimit = 1u << 26;   // about a second of polling on one mbarrier phase
+// the limit given to the kernels of the next calls (spatten_set_wait_limit; 0 = the default)
+uint32_t wait_limit_setting();
+
 struct AttnProblem {
   spatten_attn_args a;       // copy of the caller's arguments, sm_scale resolved
   int qt_rows;               // query rows per CTA of the chosen kernel
@@ -31,6 +35,8 @@ struct AttnProblem {
   int32_t* v_sel = nullptr;         // ws [B][H_kept][v_keep] kept keys, ascending; decode: set when
                                     // the combine step leaves the outputs to the pruned-output kernel
   const uint8_t* v_mask = nullptr;  // ws [B][H_kept][n_kv] 1 = V vector kept (prefill second run)
+  // tensor-core kernels: polls of one pipeline wait before the kernel gives up (SPATTEN_E_TIMEOUT)
+  uint32_t wait_limit = kDefaultWaitLimit;
 };
 
 // Kernels (each returns a status after launching on `st`).

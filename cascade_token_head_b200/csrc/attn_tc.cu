@@ -56,7 +56,6 @@ namespace {
 using namespace tc;
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kWaitLimit = 1u << 26;   // polls of one mbarrier phase before giving up
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kProducerThreads = 96;
 // Of every four pairs of softmax exponentials in the main kernel, this many are computed by the
@@ -140,9 +139,11 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// bounded wait that also gives up once another role has aborted
+// bounded wait that also gives up once another role has aborted; abort_flag[1] is the number of
+// polls of one phase before giving up (AttnProblem::wait_limit)
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+  const uint32_t limit = static_cast<uint32_t>(abort_flag[1]);
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
   }
@@ -578,7 +579,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   __shared__ __align__(16) float nmb_s[2][128];   // transposed pass: -(m + log2 ell) of each query row
   __shared__ float hred[2][4];
   __shared__ uint32_t wcnt[8];
-  __shared__ int abort_s;
+  __shared__ int abort_s[2];   // [0] set when a role gave up waiting, [1] polls of one wait
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_items = p.n_pair * a.H_kept * a.B;
@@ -590,7 +591,8 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     tmem_relinquish();
   }
   if (tid == 0) {
-    abort_s = 0;
+    abort_s[0] = 0;
+    abort_s[1] = static_cast<int>(p.wait_limit);
     for (int qb = 0; qb < C::NQ; ++qb) {
       mbar_init(&bars[M_QF + qb], kProducerThreads);
       mbar_init(&bars[M_QE + qb], 1);
@@ -620,7 +622,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tmem = tmem_base_s;
-  volatile int* abort_flag = &abort_s;
+  volatile int* abort_flag = abort_s;
   bool aborted = false;
 
   // item -> (sequence, kept head slot, pair)
@@ -1050,6 +1052,12 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   }
   const bool any_abort = __syncthreads_or(aborted);
   if (any_abort && tid == 0) report(a.dev_status, SPATTEN_E_TIMEOUT);
+  // after an abort no flagged-row list of this CTA's items is valid: their counts become 0, so
+  // that the refetch and reduce kernels read none of them (item it's list is entry it)
+  if (any_abort && p.flag_cnt)
+    for (int64_t it = blockIdx.x + static_cast<int64_t>(tid) * gridDim.x; it < n_items;
+         it += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      p.flag_cnt[it] = 0;
   if (any_abort && warp == 11 && lane == 0) {   // every MMA already issued completes before TMEM is freed
     mma_commit(&bars[M_DR]);
     drain_wait(&bars[M_DR], 0u);
@@ -1084,7 +1092,7 @@ struct FullCfg {
 };
 
 enum : int { F_Q = 0, F_KF = 1, F_KE = 3, F_VF = 5, F_VE = 7, F_SF = 9, F_SR = 11, F_PF = 13, F_PE = 15, F_OD = 17,
-             F_RF = 18, F_RE = 21, F_N = 24 };
+             F_RF = 18, F_RE = 21, F_DR = 24, F_N = 25 };
 constexpr int kMaxPairs = 256;   // query rows per head up to 256 * 256
 
 template <int DH>
@@ -1098,7 +1106,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   __shared__ uint32_t tmem_base_s;
   __shared__ float colred[2][4][KT];
   __shared__ float hred[4];
-  __shared__ int abort_s;
+  __shared__ int abort_s[2];   // [0] set when a role gave up waiting, [1] polls of one wait
   __shared__ int pref[kMaxPairs + 1];
   __shared__ int rows[128];
 
@@ -1133,7 +1141,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     tmem_relinquish();
   }
   if (tid == 0) {
-    abort_s = 0;
+    abort_s[0] = 0;
+    abort_s[1] = static_cast<int>(p.wait_limit);
     mbar_init(&bars[F_Q], 224);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[F_KF + s], kProducerThreads);
@@ -1146,6 +1155,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       mbar_init(&bars[F_PE + s], 1);
     }
     mbar_init(&bars[F_OD], 1);
+    mbar_init(&bars[F_DR], 1);
     for (int s = 0; s < C::RS; ++s) {
       mbar_init(&bars[F_RF + s], 1);
       mbar_init(&bars[F_RE + s], kProducerThreads);
@@ -1156,7 +1166,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tmem = tmem_base_s;
-  volatile int* abort_flag = &abort_s;
+  volatile int* abort_flag = abort_s;
 
   const int64_t bh = static_cast<int64_t>(b) * a.H + h;
   const int64_t plane0 = bh * a.kv_cap;
@@ -1221,6 +1231,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       }
     };
     run_jobs(0, 3 * n_tiles);   // pass A keys, then pass B keys and values, without a block barrier
+    if (ptid == 0)   // after an abort: bulk copies already armed complete before shared memory is released
+      for (uint32_t gj = js.consumed; gj < js.issued; ++gj) drain_wait(&bars[F_RF + gj % C::RS], (gj / C::RS) & 1u);
   } else if (warp == 7) {
     // ------------------------------------------------------------------------- MMA issue
     uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0};
@@ -1385,6 +1397,10 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     if (lane == 0) hred[warp] = habs;
   }
   if (__syncthreads_or(aborted)) aborted = true;
+  if (aborted && warp == 7 && lane == 0) {   // every MMA already issued completes before TMEM is freed
+    mma_commit(&bars[F_DR]);
+    drain_wait(&bars[F_DR], 0u);
+  }
   if (tid == 0) {
     p.full_head[(static_cast<int64_t>(b) * a.H_kept + slot) * 2 * p.n_pair + u] = ((hred[0] + hred[1]) + hred[2]) + hred[3];
     if (aborted) report(a.dev_status, SPATTEN_E_TIMEOUT);

@@ -206,10 +206,58 @@ constexpr int kQBThreads = 512;
 template <typename T>
 constexpr int block_chunks() { return sizeof(T) == 2 ? 8 : 4; }   // chunks per thread (registers)
 
+// Amax of one bf16 chunk times |gain|: the sign-cleared bit patterns of finite bf16 values order
+// like their magnitudes, two patterns per 32-bit unsigned max; multiplying the largest magnitude by
+// |gain| rounds like the largest of the rounded products (rounding is monotone).  *nf is set when
+// the chunk holds an infinity or a NaN.
+__device__ __forceinline__ float chunk_amax_bf16(const uint4 w, float gabs, bool* nf) {
+  const uint32_t m2 = __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu), __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+  const uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  *nf = *nf || m >= 0x7F80u;
+  return __uint_as_float(m << 16) * gabs;
+}
+
+// quant8 for a finite amax-mode block (|v| <= amax, so every code is within +-2047 and none
+// saturates), on value pairs: t = v * (1/s) and the 1.5 * 2^23 rounding add as paired float
+// operations, the near-tie recheck (the IEEE division) only for the rare pair that needs it.  The
+// rounded float's bit pattern is 0x4B400000 + q: its bits 4..11 are the MSB byte q >> 4, its
+// bits 0..3 the LSB q & 15.
+__device__ __forceinline__ void quant8_bf16_finite(const uint4 w, float g, float s, float rcp, int8_t* msb_dst,
+                                                   uint8_t* lsb_dst) {
+  constexpr float kMagic = 12582912.0f;
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  uint32_t bits[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 v = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xFFFF0000u));
+    v = __fmul2_rn(v, make_float2(g, g));
+    const float2 t = __fmul2_rn(v, make_float2(rcp, rcp));
+    float2 tm = __fadd2_rn(t, make_float2(kMagic, kMagic));
+    const float2 r = __fadd2_rn(tm, make_float2(-kMagic, -kMagic));
+    const float2 d = __ffma2_rn(r, make_float2(-1.0f, -1.0f), t);   // t - rint(t), exact
+    if (fabsf(d.x) > 0.5f - 0.001953125f) tm.x = __fdiv_rn(v.x, s) + kMagic;
+    if (fabsf(d.y) > 0.5f - 0.001953125f) tm.y = __fdiv_rn(v.y, s) + kMagic;
+    bits[2 * i] = __float_as_uint(tm.x);
+    bits[2 * i + 1] = __float_as_uint(tm.y);
+  }
+  uint32_t m[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t* b = bits + 4 * h;
+    m[h] = __byte_perm(__byte_perm(b[0] >> 4, b[1] >> 4, 0x0040), __byte_perm(b[2] >> 4, b[3] >> 4, 0x0040), 0x5410);
+  }
+  uint32_t l = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) l |= (bits[i] & 15u) << (4 * i);
+  *reinterpret_cast<uint2*>(msb_dst) = make_uint2(m[0], m[1]);
+  *reinterpret_cast<uint32_t*>(lsb_dst) = l;
+}
+
 // C: chunks per head row (d_h / 8)
 template <typename T, int C>
 __global__ void __launch_bounds__(kQBThreads) quantize_amax_block_kernel(QArgs a) {
   constexpr int CH = block_chunks<T>();
+  constexpr bool kBf = sizeof(T) == 2;
   const QTensor& q = a.t[blockIdx.z];
   const int bh = blockIdx.x;
   const int b = bh / a.H, h = bh % a.H;
@@ -221,16 +269,39 @@ __global__ void __launch_bounds__(kQBThreads) quantize_amax_block_kernel(QArgs a
     const int e = threadIdx.x + u * kQBThreads;
     if (e < total) ch[u].load(chunk_ptr<T>(a, q, b, h, e / C, e % C));
   }
+  auto gain_of = [&](int e) -> float {
+    return q.gain ? q.gain[static_cast<int64_t>(b) * a.ld_gain + e / C] : 1.0f;
+  };
   float amax = 0.0f;
+  bool nonfinite = false;
 #pragma unroll
   for (int u = 0; u < CH; ++u) {
     const int e = threadIdx.x + u * kQBThreads;
     if (e < total) {
-      float v[8];
-      ch[u].get(v);
-      apply_gain(a, q, b, e / C, v);
+      if constexpr (kBf) {
+        amax = fmaxf(amax, chunk_amax_bf16(ch[u].w, fabsf(gain_of(e)), &nonfinite));
+      } else {
+        float v[8];
+        ch[u].get(v);
+        apply_gain(a, q, b, e / C, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
+    }
+  }
+  if (kBf && __syncthreads_or(nonfinite ? 1 : 0)) {
+    // an infinity or NaN in the block: the element-wise amax (fmaxf passes over NaNs)
+    amax = 0.0f;
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      const int e = threadIdx.x + u * kQBThreads;
+      if (e < total) {
+        float v[8];
+        ch[u].get(v);
+        apply_gain(a, q, b, e / C, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
     }
   }
   amax = warp_max(amax);
@@ -242,15 +313,22 @@ __global__ void __launch_bounds__(kQBThreads) quantize_amax_block_kernel(QArgs a
   const float s = block_amax == 0.0f ? 1.0f : __fdiv_rn(block_amax, kQMax);
   const float rcp = __frcp_rn(s);
   if (threadIdx.x == 0) q.scale_out[bh] = s;
+  const bool fast = kBf && block_amax <= 3.0e38f;   // finite (and not NaN): no code saturates
 #pragma unroll
   for (int u = 0; u < CH; ++u) {
     const int e = threadIdx.x + u * kQBThreads;
     if (e < total) {
       const int t = e / C, c = e % C;
+      const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
+      if constexpr (kBf) {
+        if (fast) {
+          quant8_bf16_finite(ch[u].w, gain_of(e), s, rcp, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
+          continue;
+        }
+      }
       float v[8];
       ch[u].get(v);
       apply_gain(a, q, b, t, v);
-      const int64_t row = static_cast<int64_t>(bh) * a.cap + a.row0 + t;
       quant8(v, s, rcp, q.msb + row * a.d_h + c * 8, q.lsb + row * (a.d_h / 2) + c * 4);
     }
   }

@@ -70,6 +70,8 @@ lib.spatten_status_string.restype = C.c_char_p
 lib.spatten_status_string.argtypes = [i32]
 lib.spatten_last_cuda_error.restype = C.c_char_p
 lib.spatten_kernel_launch_count.restype = C.c_uint64
+lib.spatten_set_wait_limit.restype = None
+lib.spatten_set_wait_limit.argtypes = [C.c_uint32]
 lib.spatten_quantize_kv.restype = i32
 lib.spatten_quantize_kv.argtypes = [vp, i32, i32, i32, i32, i32, i64, vp, i64, vp, vp, vp, i32, i32, vp, vp, vp]
 lib.spatten_attention_workspace_size.restype = sz
@@ -97,7 +99,7 @@ EXPORTS = ["spatten_abi_version", "spatten_status_string", "spatten_last_cuda_er
            "spatten_attention_workspace_size", "spatten_attention_layer", "spatten_attention_layer_noalloc",
            "spatten_topk_workspace_size",
            "spatten_topk_select", "spatten_gather_kept", "spatten_cascade_workspace_size",
-           "spatten_cascade_forward", "spatten_selftest_exp2_poly"]
+           "spatten_cascade_forward", "spatten_selftest_exp2_poly", "spatten_set_wait_limit"]
 
 
 class SpattenError(RuntimeError):
@@ -188,6 +190,11 @@ def selftest_exp2_poly(x, y, n, stream=None):
 
 def kernel_launch_count() -> int:
     return int(lib.spatten_kernel_launch_count())
+
+
+def set_wait_limit(polls: int) -> None:
+    """Polls of one pipeline wait of the tensor-core kernels before they give up (0: default)."""
+    lib.spatten_set_wait_limit(polls)
 
 
 def cascade_workspace_size(cfg: cascade_cfg) -> int:

@@ -71,6 +71,14 @@ const char* spatten_last_cuda_error(void);
 /* Number of kernels this library has launched in this process (its own kernels only; the cuBLASLt
  * projections are not counted).  A diagnostic for benchmarks and tests. */
 uint64_t spatten_kernel_launch_count(void);
+/* Polls of one pipeline wait (an mbarrier phase) after which the tensor-core attention kernels of
+ * the calls that follow give up: the kernel stops its work, waits (with a bound of its own) for the
+ * copies and MMAs it already started, releases its tensor memory, returns, and the call reports
+ * SPATTEN_E_TIMEOUT in its dev_status word.  0 restores the default (2^26 polls, about a second).
+ * Process-wide; read when a call is launched (a CUDA graph keeps the value it was captured with).
+ * A diagnostic: a small value makes the waits run out on purpose, so that the timeout path can be
+ * checked without a fault. */
+void spatten_set_wait_limit(uint32_t polls);
 
 /* =============================================================================================
  * spatten_quantize_kv -- progressive 12-bit quantization of K or V into an MSB and an LSB plane

@@ -84,11 +84,13 @@ def run_layer(S, raw, gain, B, H, n, d, theta, heads=None, kernel=0, dtype=BF, k
         a.tok_imp_map, a.tok_imp_map_ld = kvi.data_ptr(), kv_idx.shape[1]
     a.head_imp, a.refetch_flags, a.refetch_count = hed.data_ptr(), flags.data_ptr(), cnt.data_ptr()
     a.refetch_threshold, a.kernel, a.v_keep = theta, kernel, v_keep
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    a.dev_status = st.data_ptr()
     w = ws(S.attention_workspace_size(a))
     S.attention_layer(a, w, w.numel())
     torch.cuda.synchronize()
     out = dict(o=o.float().cpu().numpy(), tok=tok.cpu().numpy(), head=hed.cpu().numpy(),
-               flags=flags.cpu().numpy(), count=int(cnt.item()))
+               flags=flags.cpu().numpy(), count=int(cnt.item()), status=int(st.item()))
     if quantized:
         out.update(msbk=msbk.cpu().numpy(), lsbk=lsbk.cpu().numpy(), sk=sk.cpu().numpy().reshape(B, H),
                    msbv=msbv.cpu().numpy(), lsbv=lsbv.cpu().numpy(), sv=sv.cpu().numpy().reshape(B, H))
@@ -263,3 +265,26 @@ def test_attention_query_out_of_fp16_range_reports_status(cuda):
         S.attention_layer(a, w, w.numel())
         torch.cuda.synchronize()
         assert int(st.item()) == want
+
+
+def test_forced_timeout_reports_status_and_context_survives(cuda):
+    """The tensor-core kernels' bounded waits run out on purpose (spatten_set_wait_limit(1): one
+    poll per pipeline wait): the call reports SPATTEN_E_TIMEOUT in its status word and its kernels
+    return (the synchronize inside run_layer ends); the context stays usable: with the default
+    limit restored the same call reports 0 and repeats, bit for bit, the results of a run made
+    before the forced timeout."""
+    S = lib()
+    B, H, n, d = 1, 2, 130, 64
+    raw, gain = make_layer(B, H, n, d, seed=31, boost=5)
+    before = run_layer(S, raw, gain, B, H, n, d, 0.1, kernel=S.ATTN_TENSOR_CORE)
+    assert before["status"] == S.OK
+    try:
+        S.set_wait_limit(1)
+        timed_out = run_layer(S, raw, gain, B, H, n, d, 0.1, kernel=S.ATTN_TENSOR_CORE)
+    finally:
+        S.set_wait_limit(0)
+    assert timed_out["status"] == S.E_TIMEOUT
+    after = run_layer(S, raw, gain, B, H, n, d, 0.1, kernel=S.ATTN_TENSOR_CORE)
+    assert after["status"] == S.OK
+    for key in ("o", "tok", "head", "flags", "count"):
+        np.testing.assert_array_equal(after[key], before[key])

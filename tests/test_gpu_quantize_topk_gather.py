@@ -109,6 +109,45 @@ def test_quantize_half_integer_boundaries_amax_scale(cuda):
     np.testing.assert_array_equal(lsb.cpu().numpy(), l_ref)
 
 
+@pytest.mark.parametrize("gain", [False, True])
+def test_quantize_half_integer_boundaries_amax_scale_bf16(cuda, gain):
+    """bf16 blocks (the paired-arithmetic path of the amax kernel): values rounded to bf16 at and
+    one or two bf16 steps around (k + 1/2) s for small |k| (where bf16 steps are finer than one
+    code), with and without a row gain; bit-exact against the oracle."""
+    S = lib()
+    rng = synth.rng_for(4343 + gain)
+    B, H, n, d = 2, 3, 256, 64
+    vals = np.empty((B, n, H * d), np.float32)
+    for b in range(B):
+        for h in range(H):
+            amax = np.float32(torch.tensor(rng.uniform(0.5, 9.0)).to(BF).float().item())
+            s = np.float32(amax / np.float32(2047.0))
+            k = rng.integers(-120, 120, size=n * d)
+            centre = torch.from_numpy(((k + 0.5) * np.float64(s)).astype(np.float32)).to(BF)
+            bits = centre.view(torch.int16).to(torch.int32) + torch.from_numpy(rng.integers(-2, 3, size=n * d)).to(torch.int32)
+            blk = bits.to(torch.int16).view(BF).float().numpy().reshape(n, d)
+            blk = np.clip(blk, -amax, amax)
+            blk[0, 0] = amax
+            vals[b, :, h * d:(h + 1) * d] = blk
+    gains = None
+    if gain:
+        gains = np.ones((B, n), np.float32)
+        gains[:, rng.choice(n, size=12, replace=False)] = 4.0
+    x = to_dev(vals, BF)
+    assert np.array_equal(x.float().cpu().numpy(), vals)   # every value is a bf16
+    msb = torch.zeros((B, H, n, d), dtype=torch.int8, device="cuda")
+    lsb = torch.zeros((B, H, n, d // 2), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(B * H, dtype=torch.float32, device="cuda")
+    S.quantize_kv(x, B, H, n, d, H * d, msb, lsb, n, 0, scale_out=sc, row_gain=to_dev(gains) if gain else None,
+                  ld_gain=n, dtype=S.BF16)
+    torch.cuda.synchronize()
+    m_ref, l_ref, s_ref = oracle_quantize_blocks(np.ascontiguousarray(vals.reshape(B, n, H, d).transpose(0, 2, 1, 3)),
+                                                 gains)
+    np.testing.assert_array_equal(sc.cpu().numpy().reshape(B, H), s_ref)
+    np.testing.assert_array_equal(msb.cpu().numpy(), m_ref)
+    np.testing.assert_array_equal(lsb.cpu().numpy(), l_ref)
+
+
 def test_quantize_full_size_bert_layer0(cuda):
     """K of the BERT-base layer-0 projection shape [32, 12, 512, 64], bf16, with boosted rows."""
     S = lib()
