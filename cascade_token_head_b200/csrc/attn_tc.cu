@@ -139,10 +139,9 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// bounded wait that also gives up once another role has aborted; abort_flag[1] is the number of
-// polls of one phase before giving up (AttnProblem::wait_limit)
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const uint32_t limit = static_cast<uint32_t>(abort_flag[1]);
+// bounded wait that also gives up once another role has aborted; `limit` polls of one phase
+// before giving up (AttnProblem::wait_limit)
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t limit) {
   for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
@@ -293,7 +292,7 @@ __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int
 // packed LSB rows (DH/2 bytes) at raw + KT*DH; rows >= valid are zero-filled
 // keep (V tiles under local value pruning): row r of the tile is kept iff keep[r] != 0; dropped
 // rows are zero-filled like the rows past the end
-template <int DH, int KT>
+template <int DH, int KT, bool KEEP>
 __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw, bool with_lsb, int valid,
                                                uint32_t off_hi, int ptid, const uint8_t* keep) {
   constexpr int L16 = DH / 16;
@@ -308,7 +307,7 @@ __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw
     const int r = e / L16, c16 = e % L16;
     m[i] = make_uint4(0u, 0u, 0u, 0u);
     lb[i] = make_uint2(0u, 0u);
-    if (e < TOTAL && r < valid && (!keep || keep[r])) {
+    if (e < TOTAL && r < valid && (!KEEP || keep[r])) {
       m[i] = *reinterpret_cast<const uint4*>(raw + r * DH + c16 * 16);
       if (with_lsb) lb[i] = *reinterpret_cast<const uint2*>(raw + KT * DH + r * (DH / 2) + c16 * 8);
     }
@@ -319,7 +318,7 @@ __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw
     if (e >= TOTAL) break;
     const int r = e / L16, c16 = e % L16;
     uint32_t hi[8], lo[8];
-    if (r < valid && (!keep || keep[r])) {
+    if (r < valid && (!KEEP || keep[r])) {
       cvt16_s8x16(m[i], hi);
       if (with_lsb) {
         cvt_u4x16(lb[i], lo);
@@ -358,6 +357,7 @@ struct JobStream {
   uint32_t issued = 0;   // jobs of this stream issued so far (loader)
   uint32_t consumed = 0; // jobs of this stream converted so far
   const uint8_t* vmask = nullptr;   // [n_kv] V vectors kept (local value pruning) or NULL
+  uint32_t wlim = kDefaultWaitLimit;  // polls of one wait before giving up
 
   __device__ __forceinline__ int jobs() const { return 3 * n_tiles; }
   __device__ __forceinline__ void job(int j, bool& is_v, int& t) const {
@@ -376,7 +376,7 @@ struct JobStream {
       const uint32_t jn = issued;
       const uint32_t gj = g0 + jn;
       const uint32_t st = gj % RS;
-      if (!wait_bar(&raw_empty[st], ((gj / RS) & 1u) ^ 1u, abort_flag)) return false;
+      if (!wait_bar(&raw_empty[st], ((gj / RS) & 1u) ^ 1u, abort_flag, wlim)) return false;
       bool is_v;
       int t;
       job(static_cast<int>(jn), is_v, t);
@@ -405,9 +405,13 @@ struct JobStream {
     }
     const uint32_t gj = g0 + static_cast<uint32_t>(j);
     const uint32_t st = gj % RS;
-    if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag)) return false;
-    convert_staged<DH, KT>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
-                           keep ? keep + t * KT : nullptr);
+    if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag, wlim)) return false;
+    if (keep)
+      convert_staged<DH, KT, true>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
+                                   keep + t * KT);
+    else
+      convert_staged<DH, KT, false>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
+                                    nullptr);
     mbar_arrive(&raw_empty[st]);
     ++consumed;
     return true;
@@ -542,11 +546,11 @@ __device__ __forceinline__ void zero_pruned_share(const spatten_attn_args& a, __
     int h = ps;
     if (a.head_idx) {
       if (a.H <= 32) {
-        // the ps-th head (in index order) that no kept slot lists
+        // the ps-th head (in index order) that no kept slot lists: lane s loads slot s's head
         const int32_t* hi = a.head_idx + static_cast<int64_t>(b) * a.head_idx_ld;
-        bool kept = lane >= a.H;
-        for (int s = 0; s < a.H_kept; ++s) kept |= hi[s] == lane;
-        uint32_t free_mask = __ballot_sync(0xffffffffu, !kept);
+        const int hs = lane < a.H_kept ? hi[lane] : -1;
+        const uint32_t kept = __reduce_or_sync(0xffffffffu, hs >= 0 && hs < 32 ? 1u << hs : 0u);
+        uint32_t free_mask = ~kept & (a.H == 32 ? 0xffffffffu : (1u << a.H) - 1u);
         for (int k = 0; k < ps; ++k) free_mask &= free_mask - 1;
         h = free_mask ? __ffs(free_mask) - 1 : -1;
       } else {
@@ -579,7 +583,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   __shared__ __align__(16) float nmb_s[2][128];   // transposed pass: -(m + log2 ell) of each query row
   __shared__ float hred[2][4];
   __shared__ uint32_t wcnt[8];
-  __shared__ int abort_s[2];   // [0] set when a role gave up waiting, [1] polls of one wait
+  __shared__ int abort_s;   // set when a role gave up waiting
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_items = p.n_pair * a.H_kept * a.B;
@@ -591,8 +595,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     tmem_relinquish();
   }
   if (tid == 0) {
-    abort_s[0] = 0;
-    abort_s[1] = static_cast<int>(p.wait_limit);
+    abort_s = 0;
     for (int qb = 0; qb < C::NQ; ++qb) {
       mbar_init(&bars[M_QF + qb], kProducerThreads);
       mbar_init(&bars[M_QE + qb], 1);
@@ -622,7 +625,8 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tmem = tmem_base_s;
-  volatile int* abort_flag = abort_s;
+  volatile int* abort_flag = &abort_s;
+  const uint32_t wlim = p.wait_limit;   // polls of one pipeline wait
   bool aborted = false;
 
   // item -> (sequence, kept head slot, pair)
@@ -673,6 +677,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
       JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
                                   abort_flag, gjob};
+      js.wlim = wlim;
       if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
       struct Track {   // records the stream's progress however the item's loop is left
         JobStream<DH, KT, C::RS>& js;
@@ -686,7 +691,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         // this item's query tile was copied (bf16) into buffer qb during the previous item, or just
         // below for the first item: convert it in place to fp16 (each thread its own chunks)
         if (qc == 0) {
-          if (!wait_bar(&bars[M_QE + qb], 1u, abort_flag)) { aborted = true; break; }
+          if (!wait_bar(&bars[M_QE + qb], 1u, abort_flag, wlim)) { aborted = true; break; }
           copy_q_async(it, qb);
         }
         cp_async_wait_all();
@@ -695,7 +700,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         mbar_arrive(&bars[M_QF + qb]);
       } else {
         // query tile of the item once the previous item's score MMAs have read the buffer
-        if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
         constexpr int NCH = 256 * (DH / 8);
         constexpr int BATCH = 8;
         const int i0 = pair * 256;
@@ -732,7 +737,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
           // the next item's query rows into it
           if (j == n_tiles && it + static_cast<int>(gridDim.x) < n_items) {
             const uint32_t nb = (qc + 1) % C::NQ;
-            if (!wait_bar(&bars[M_QE + nb], (((qc + 1) / C::NQ) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+            if (!wait_bar(&bars[M_QE + nb], (((qc + 1) / C::NQ) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
             copy_q_async(it + static_cast<int>(gridDim.x), nb);
           }
         }
@@ -742,7 +747,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         js.job(j, is_v, t);
         uint32_t& cnt = is_v ? vc : kc;
         const uint32_t st = cnt % NST;
-        if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
         if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, kv_idx)) { aborted = true; break; }
         mbar_arrive(&bars[(is_v ? M_VF : M_KF) + st]);
         ++cnt;
@@ -761,15 +766,15 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       // orientation) or S^T = K Q^T (pass B, transposed)
       auto qk_both = [&](bool trans) -> bool {
         const uint32_t ks = kc % NST;
-        if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag)) return false;
+        if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag, wlim)) return false;
         const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
-        if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag)) return false;
+        if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag, wlim)) return false;
         tc_after_sync();
         if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS, sK, sQ0);
         else mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
         mma_commit(&bars[M_SF + 0]);
         ++sc[0];
-        if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag)) return false;
+        if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag, wlim)) return false;
         tc_after_sync();
         if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS + KT, sK, sQ1);
         else mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
@@ -783,24 +788,24 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         const uint32_t qb = ic % C::NQ;
         sQ0 = smem_u32(smem + C::oQ + qb * 2 * C::QB);
         sQ1 = sQ0 + C::QB;
-        if (!wait_bar(&bars[M_QF + qb], (ic / C::NQ) & 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[M_QF + qb], (ic / C::NQ) & 1u, abort_flag, wlim)) { aborted = true; break; }
         for (int t = 0; t < n_tiles && !aborted; ++t)   // pass A
           if (!qk_both(false)) aborted = true;
         if (aborted) break;
         if (!qk_both(true)) { aborted = true; break; }   // pass B, tile 0
         if (n_tiles == 1) mma_commit(&bars[M_QE + qb]);  // the item's last read of Q is issued
         // the previous item's O must have been read before this item's first P V overwrites it
-        if (!wait_bar(&bars[M_OE], (ic & 1u) ^ 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[M_OE], (ic & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
         for (int t = 0; t < n_tiles && !aborted; ++t) {
           if (t + 1 < n_tiles) {
             if (!qk_both(true)) { aborted = true; break; }
             if (t + 2 == n_tiles) mma_commit(&bars[M_QE + qb]);
           }
           const uint32_t vs = vc % NST;
-          if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag)) { aborted = true; break; }
+          if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag, wlim)) { aborted = true; break; }
           const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
           for (int gg = 0; gg < 2 && !aborted; ++gg) {
-            if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag)) { aborted = true; break; }
+            if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag, wlim)) { aborted = true; break; }
             tc_after_sync();
             if constexpr (C::kT)
               mma_pv_mn<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
@@ -837,7 +842,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
 
       // ---- pass A: MSB statistics
       for (int t = 0; t < n_tiles; ++t) {
-        if (!__all_sync(0xffffffffu, wait_bar(&bars[M_SF + g], sc & 1u, abort_flag))) { aborted = true; break; }
+        if (!__all_sync(0xffffffffu, wait_bar(&bars[M_SF + g], sc & 1u, abort_flag, wlim))) { aborted = true; break; }
         tc_after_sync();
 #pragma unroll 1
         for (int hh = 0; hh < KT / 64; ++hh) {
@@ -891,7 +896,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         const float2 c2x2 = make_float2(c2, c2);
         const uint32_t kcol = (static_cast<uint32_t>(r) >> 3) * 1024u + (static_cast<uint32_t>(r) & 7u) * 128u;
         for (int t = 0; t < n_tiles; ++t) {
-          if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag), 1 + g)) { aborted = true; break; }
+          if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag, wlim), 1 + g)) { aborted = true; break; }
           tc_after_sync();
           const int key = t * KT + r;
           const bool key_ok = key < a.n_kv;
@@ -909,7 +914,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
               tc_before_sync();
               mbar_arrive(&bars[M_SR + g]);
               ++sc;
-            } else if (!wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag), 1 + g)) {
+            } else if (!wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag, wlim), 1 + g)) {
               // the previous tile's P V must be done before this tile's P overwrites the buffer
               aborted = true;
               break;
@@ -955,7 +960,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         const int qt128 = pair * 2 + g;
         const int64_t part_row = ((static_cast<int64_t>(b) * a.H_kept + slot) * p.n_qt + qt128) * a.n_kv;
         for (int t = 0; t < n_tiles; ++t) {
-          if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag), 1 + g)) { aborted = true; break; }
+          if (!wg_all(wait_bar(&bars[M_SF + g], sc & 1u, abort_flag, wlim), 1 + g)) { aborted = true; break; }
           tc_after_sync();
 #pragma unroll 1
           for (int hh = 0; hh < KT / 64; ++hh) {
@@ -970,7 +975,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
             }
             // the previous tile's P V must be done before this tile's P overwrites the buffer; the
             // score load and the exponentials below overlap it
-            if (hh == 0 && !wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag), 1 + g)) {
+            if (hh == 0 && !wg_all(wait_bar(&bars[M_PE + g], (pc & 1u) ^ 1u, abort_flag, wlim), 1 + g)) {
               aborted = true;
               break;
             }
@@ -1020,7 +1025,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
       // ---- epilogue: O of the unflagged rows, head importance partial, refetch flags
       float habs = 0.0f;
       if (!aborted) {
-        if (!wg_all(wait_bar(&bars[M_OD], oc & 1u, abort_flag), 1 + g)) aborted = true;
+        if (!wg_all(wait_bar(&bars[M_OD], oc & 1u, abort_flag, wlim), 1 + g)) aborted = true;
       }
       if (!aborted) {
         tc_after_sync();
@@ -1106,7 +1111,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   __shared__ uint32_t tmem_base_s;
   __shared__ float colred[2][4][KT];
   __shared__ float hred[4];
-  __shared__ int abort_s[2];   // [0] set when a role gave up waiting, [1] polls of one wait
+  __shared__ int abort_s;   // set when a role gave up waiting
   __shared__ int pref[kMaxPairs + 1];
   __shared__ int rows[128];
 
@@ -1141,8 +1146,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     tmem_relinquish();
   }
   if (tid == 0) {
-    abort_s[0] = 0;
-    abort_s[1] = static_cast<int>(p.wait_limit);
+    abort_s = 0;
     mbar_init(&bars[F_Q], 224);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[F_KF + s], kProducerThreads);
@@ -1166,7 +1170,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   __syncthreads();
   tc_after_sync();
   const uint32_t tmem = tmem_base_s;
-  volatile int* abort_flag = abort_s;
+  volatile int* abort_flag = &abort_s;
+  const uint32_t wlim = p.wait_limit;   // polls of one pipeline wait
 
   const int64_t bh = static_cast<int64_t>(b) * a.H + h;
   const int64_t plane0 = bh * a.kv_cap;
@@ -1214,6 +1219,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     const int ptid = tid - 128;
     JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[F_RF], &bars[F_RE], &a, plane0, n_tiles, true, ptid,
                                 abort_flag};
+    js.wlim = wlim;
     if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
     uint32_t kc = 0, vc = 0;
     auto run_jobs = [&](int j0, int j1) {
@@ -1224,7 +1230,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
         js.job(j, is_v, t);
         uint32_t& cnt = is_v ? vc : kc;
         const uint32_t st = cnt & 1u;
-        if (!wait_bar(&bars[(is_v ? F_VE : F_KE) + st], ((cnt >> 1) & 1u) ^ 1u, abort_flag)) { aborted = true; return; }
+        if (!wait_bar(&bars[(is_v ? F_VE : F_KE) + st], ((cnt >> 1) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; return; }
         if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, kv_idx)) { aborted = true; return; }
         mbar_arrive(&bars[(is_v ? F_VF : F_KF) + st]);
         ++cnt;
@@ -1239,9 +1245,9 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     const uint32_t sQ = smem_u32(smem + C::oQ);
     auto qk = [&](int t) -> bool {
       const uint32_t ks = kc & 1u;
-      if (!wait_bar(&bars[F_KF + ks], (kc >> 1) & 1u, abort_flag)) return false;
+      if (!wait_bar(&bars[F_KF + ks], (kc >> 1) & 1u, abort_flag, wlim)) return false;
       const int sb = t & 1;
-      if (!wait_bar(&bars[F_SR + sb], (sc[sb] & 1u) ^ 1u, abort_flag)) return false;
+      if (!wait_bar(&bars[F_SR + sb], (sc[sb] & 1u) ^ 1u, abort_flag, wlim)) return false;
       tc_after_sync();
       const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
       mma_qk<DH, KT>(tmem + C::tS + sb * KT, sQ, sK, 0);   // the combined (16·MSB + LSB) tile
@@ -1252,7 +1258,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       return true;
     };
     if (lane == 0) {
-      if (!wait_bar(&bars[F_Q], 0, abort_flag)) aborted = true;
+      if (!wait_bar(&bars[F_Q], 0, abort_flag, wlim)) aborted = true;
       for (int t = 0; t < n_tiles && !aborted; ++t)
         if (!qk(t)) aborted = true;
     }
@@ -1261,9 +1267,9 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       for (int t = 0; t < n_tiles && !aborted; ++t) {
         if (t + 1 < n_tiles && !qk(t + 1)) { aborted = true; break; }
         const int pb = 0;   // single P buffer
-        if (!wait_bar(&bars[F_PF + pb], pc[pb] & 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[F_PF + pb], pc[pb] & 1u, abort_flag, wlim)) { aborted = true; break; }
         const uint32_t vs = vc & 1u;
-        if (!wait_bar(&bars[F_VF + vs], (vc >> 1) & 1u, abort_flag)) { aborted = true; break; }
+        if (!wait_bar(&bars[F_VF + vs], (vc >> 1) & 1u, abort_flag, wlim)) { aborted = true; break; }
         tc_after_sync();
         const uint32_t sP = smem_u32(smem + C::oP + pb * C::PB);
         const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
@@ -1280,7 +1286,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
     uint32_t sc[2] = {0, 0};
     for (int t = 0; t < n_tiles; ++t) {
       const int sb = t & 1;
-      if (!__all_sync(0xffffffffu, wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag))) { aborted = true; break; }
+      if (!__all_sync(0xffffffffu, wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag, wlim))) { aborted = true; break; }
       tc_after_sync();
       if (warp_live) {
 #pragma unroll 1
@@ -1312,8 +1318,8 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
       for (int t = 0; t < n_tiles; ++t) {
         const int sb = t & 1;
         const int pb = 0;   // single P buffer
-        if (!wg_all(wait_bar(&bars[F_PE + pb], (pc[pb] & 1u) ^ 1u, abort_flag), 1)) { aborted = true; break; }
-        if (!wg_all(wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag), 1)) { aborted = true; break; }
+        if (!wg_all(wait_bar(&bars[F_PE + pb], (pc[pb] & 1u) ^ 1u, abort_flag, wlim), 1)) { aborted = true; break; }
+        if (!wg_all(wait_bar(&bars[F_SF + sb], sc[sb] & 1u, abort_flag, wlim), 1)) { aborted = true; break; }
         tc_after_sync();
         uint8_t* Pt = smem + C::oP + pb * C::PB;
 #pragma unroll 1
@@ -1375,7 +1381,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   // ------------------------------------------------------------------------- epilogue
   float habs = 0.0f;
   if (warp < 4 && !aborted) {
-    if (!wait_bar(&bars[F_OD], 0, abort_flag)) aborted = true;
+    if (!wait_bar(&bars[F_OD], 0, abort_flag, wlim)) aborted = true;
     aborted = __any_sync(0xffffffffu, aborted);   // warp-uniform before the TMEM loads
     tc_after_sync();
     if (!aborted && warp_live) {
