@@ -106,14 +106,16 @@ __device__ __forceinline__ void cvt_u4x16(uint2 raw, uint32_t* out8) {
     }
   }
 }
-// true when one of eight bf16 values is out of fp16 range: magnitude 65536 or more (the bf16
-// patterns from 0x4780 up; bf16 has no value in (65504, 65536)), infinity or NaN
-__device__ __forceinline__ bool bf16x8_out_of_f16(uint4 u) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  bool out = false;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) out |= ((w[i] & 0x7FFFu) >= 0x4780u) || (((w[i] >> 16) & 0x7FFFu) >= 0x4780u);
-  return out;
+// Range check of bf16 values against fp16: the running maximum `mx` of the sign-cleared bit
+// patterns (two 16-bit maxima per word; patterns order like magnitudes, NaNs above infinity) is
+// out of range from 0x4780 up: magnitude 65536 or more (bf16 has no value in (65504, 65536)),
+// infinity or NaN.
+__device__ __forceinline__ uint32_t bf16x8_absmax(uint4 u, uint32_t mx) {
+  constexpr uint32_t M = 0x7FFF7FFFu;
+  return __vmaxu2(mx, __vmaxu2(__vmaxu2(u.x & M, u.y & M), __vmaxu2(u.z & M, u.w & M)));
+}
+__device__ __forceinline__ bool bf16_absmax_out_of_f16(uint32_t mx) {
+  return (mx & 0xFFFFu) >= 0x4780u || (mx >> 16) >= 0x4780u;
 }
 // eight bf16 values -> four fp16 pairs (the query tile); exact for magnitudes in [2^-14, 65504]
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
@@ -660,13 +662,15 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     };
     // bf16 -> fp16 in place, each thread the chunks it copied
     auto convert_q_in_place = [&](uint32_t qbuf) {
+      uint32_t mx = 0u;
       for (int e = ptid; e < QCH; e += kProducerThreads) {
         const int rr = e / (DH / 8), c8 = e % (DH / 8);
         uint4* p = reinterpret_cast<uint4*>(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128));
         const uint4 v = *p;
-        if (bf16x8_out_of_f16(v)) report(a.dev_status, SPATTEN_E_RANGE);
+        mx = bf16x8_absmax(v, mx);
         *p = bf16x8_to_f16x8(v);
       }
+      if (bf16_absmax_out_of_f16(mx)) report(a.dev_status, SPATTEN_E_RANGE);
     };
     uint32_t g_issued = 0, g_consumed = 0;   // staging-ring jobs issued / converted, whole kernel
     for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++qc) {
@@ -705,6 +709,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
         constexpr int BATCH = 8;
         const int i0 = pair * 256;
         const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+        uint32_t qmx = 0u;
         for (int e0 = ptid; e0 < NCH; e0 += BATCH * kProducerThreads) {
           uint4 qv[BATCH];
 #pragma unroll
@@ -721,12 +726,13 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
             const int e = e0 + k * kProducerThreads;
             const int rr = e / (DH / 8), c8 = e % (DH / 8);
             if (e < NCH) {
-              if (bf16x8_out_of_f16(qv[k])) report(a.dev_status, SPATTEN_E_RANGE);
+              qmx = bf16x8_absmax(qv[k], qmx);
               *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) =
                   bf16x8_to_f16x8(qv[k]);
             }
           }
         }
+        if (bf16_absmax_out_of_f16(qmx)) report(a.dev_status, SPATTEN_E_RANGE);
         fence_async_smem();
         mbar_arrive(&bars[M_QF]);
       }
@@ -1202,15 +1208,17 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
         qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + rows[rr]) * a.q_ld_tok +
                                                      static_cast<int64_t>(h) * DH) + c8);
     }
+    uint32_t qmx = 0u;
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int e = tid + k * 224;
       const int rr = e / (DH / 8), c8 = e % (DH / 8);
       if (e < NCH) {
-        if (bf16x8_out_of_f16(qv[k])) report(a.dev_status, SPATTEN_E_RANGE);
+        qmx = bf16x8_absmax(qv[k], qmx);
         *reinterpret_cast<uint4*>(smem + C::oQ + tile_off(rr, c8, 128)) = bf16x8_to_f16x8(qv[k]);
       }
     }
+    if (bf16_absmax_out_of_f16(qmx)) report(a.dev_status, SPATTEN_E_RANGE);
     fence_async_smem();
     mbar_arrive(&bars[F_Q]);
   }
