@@ -1086,7 +1086,10 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
 // =================================================================================================
 template <int DH>
 struct FullCfg {
-  static constexpr int KT = DH == 64 ? 128 : 64;
+  // 64-key tiles: two CTAs of d_h 64 fit one SM (shared memory and tensor memory), so that two
+  // heads' producers and softmax warps overlap
+  static constexpr int KT = 64;
+  static constexpr uint32_t kTmem = 256;         // S (2 x KT columns) and O (DH columns)
   static constexpr uint32_t QB = 128u * DH * 2u;
   static constexpr uint32_t TB = static_cast<uint32_t>(KT) * DH * 2u;
   static constexpr uint32_t PB = 128u * KT * 2u;
@@ -1107,7 +1110,7 @@ enum : int { F_Q = 0, F_KF = 1, F_KE = 3, F_VF = 5, F_VE = 7, F_SF = 9, F_SR = 1
 constexpr int kMaxPairs = 256;   // query rows per head up to 256 * 256
 
 template <int DH>
-__global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
+__global__ void __launch_bounds__(256, DH == 64 ? 2 : 1) attn_full_kernel(AttnProblem p) {
   using C = FullCfg<DH>;
   constexpr int KT = C::KT;
   const spatten_attn_args& a = p.a;
@@ -1148,7 +1151,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
 
   if (warp == 7) {
-    tmem_alloc(&tmem_base_s, kTmemCols);
+    tmem_alloc(&tmem_base_s, C::kTmem);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -1423,7 +1426,7 @@ __global__ void __launch_bounds__(256, 1) attn_full_kernel(AttnProblem p) {
   __syncthreads();
   if (warp == 7) {
     tc_after_sync();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::kTmem);
   }
 }
 
