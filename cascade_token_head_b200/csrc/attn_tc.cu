@@ -17,12 +17,14 @@
 //  MAIN  persistent: one CTA per SM walks the work items (sequence, kept head, 256 query rows) with
 //        a stride of the grid; TMEM, barriers and all ring counters live across items, so the
 //        producers load the next item's query tile and first key tiles, and the MMA warp issues its
-//        first score MMAs, while the softmax warps finish the current item.  384 threads:
+//        first score MMAs, while the softmax warps finish the current item.  d_h 64: 512 threads:
 //          warps 0-7   two softmax warpgroups; warpgroup g owns query rows 128g..128g+127 of the
 //                      CTA, thread r of a warpgroup is TMEM lane r of that warpgroup's S and O
-//          warps 8-10  producers: the item's query tile, then K/V MSB tiles converted into
+//          warps 8-14  producers: the item's query tile, then K/V MSB tiles converted into
 //                      2-stage rings
-//          warp 11     MMA issue (lane 0) and TMEM allocation
+//          warp 15     MMA issue (lane 0) and TMEM allocation
+//        The softmax warpgroups run with more registers than the launch gives (setmaxnreg),
+//        warpgroups 2-3 with fewer.  d_h 128: 384 threads, producer warps 8-10, MMA warp 11.
 //        pass A computes S_msb tile by tile (the two warpgroups' tiles alternate on the tensor
 //        core while the other warpgroup runs its softmax) -> row max / exp-sum -> refetch flags;
 //        the flagged rows of the CTA are written, ascending, to a packed list.  Pass B computes
@@ -57,7 +59,17 @@ using namespace tc;
 
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kProducerThreads = 96;
+constexpr int kProducerThreads = 96;    // refetch kernel: warps 4-6
+// main kernel, d_h 64: 16 warps = softmax warpgroups 0 and 1, producer warps 8-14, MMA warp 15.
+// The two softmax warpgroups raise their register limit and the other two lower theirs
+// (setmaxnreg), so that seven producer warps fit beside softmax threads that need 160 registers:
+// 256 x 168 + 256 x 88 = 65536 = 512 threads x 128 registers at launch.  d_h 128: 12 warps,
+// producer warps 8-10, MMA warp 11, no split (168 registers per thread at launch).
+template <int DH> constexpr int kMainThreads = DH == 64 ? 512 : 384;
+template <int DH> constexpr int kMainProducers = kMainThreads<DH> - 256 - 32;
+template <int DH> constexpr int kMainMmaWarp = kMainThreads<DH> / 32 - 1;
+constexpr uint32_t kSoftmaxRegs = 168, kOtherRegs = 88;
+static_assert(256 * kSoftmaxRegs + 256 * kOtherRegs <= 65536, "register split");
 // Of every four pairs of softmax exponentials in the main kernel, this many are computed by the
 // FMA-pipe polynomial (exp2_poly2) and the rest by the ex2 instruction: the two units then share
 // the work.
@@ -264,12 +276,12 @@ __device__ __forceinline__ void add_f16x8(uint32_t* hi, const uint32_t* lo) {
   }
 }
 
-template <int DH, int KT>
+template <int DH, int KT, int NP>
 __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int64_t plane0, const int32_t* kv_idx,
                                              const int8_t* msb, const uint8_t* lsb, uint32_t off_hi, int ptid,
                                              const uint8_t* keep) {
   constexpr int L16 = DH / 16;
-  for (int e = ptid; e < KT * L16; e += kProducerThreads) {
+  for (int e = ptid; e < KT * L16; e += NP) {
     const int r = e / L16, c16 = e % L16;
     const int key = t * KT + r;
     uint32_t hi[8], lo[8];
@@ -294,18 +306,18 @@ __device__ __forceinline__ void produce_tile(uint8_t* smem, int t, int n_kv, int
 // packed LSB rows (DH/2 bytes) at raw + KT*DH; rows >= valid are zero-filled
 // keep (V tiles under local value pruning): row r of the tile is kept iff keep[r] != 0; dropped
 // rows are zero-filled like the rows past the end
-template <int DH, int KT, bool KEEP>
+template <int DH, int KT, bool KEEP, int NP>
 __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw, bool with_lsb, int valid,
                                                uint32_t off_hi, int ptid, const uint8_t* keep) {
   constexpr int L16 = DH / 16;
   constexpr int TOTAL = KT * L16;
-  constexpr int NIT = (TOTAL + kProducerThreads - 1) / kProducerThreads;
+  constexpr int NIT = (TOTAL + NP - 1) / NP;
   // every staged read of this thread first (all in flight together), then the conversions
   uint4 m[NIT];
   uint2 lb[NIT];
 #pragma unroll
   for (int i = 0; i < NIT; ++i) {
-    const int e = ptid + i * kProducerThreads;
+    const int e = ptid + i * NP;
     const int r = e / L16, c16 = e % L16;
     m[i] = make_uint4(0u, 0u, 0u, 0u);
     lb[i] = make_uint2(0u, 0u);
@@ -316,7 +328,7 @@ __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw
   }
 #pragma unroll
   for (int i = 0; i < NIT; ++i) {
-    const int e = ptid + i * kProducerThreads;
+    const int e = ptid + i * NP;
     if (e >= TOTAL) break;
     const int r = e / L16, c16 = e % L16;
     uint32_t hi[8], lo[8];
@@ -342,13 +354,13 @@ __device__ __forceinline__ void convert_staged(uint8_t* smem, const uint8_t* raw
 // all producer threads convert staged tiles shared -> shared; with an index list they load rows
 // directly.  `emit(is_v, t, stage_dst_hi, stage_dst_lo)` gives the destination of the converted
 // tile and performs the ring handshake around `fill`.
-template <int DH, int KT, int RS>
+template <int DH, int KT, int RS, int NP>   // NP producer threads
 struct JobStream {
   static constexpr uint32_t kMsb = KT * DH;
   uint8_t* smem;
   uint32_t o_raw, raw_bytes;   // staging ring: RS slots of raw_bytes
   uint64_t* raw_full;          // [RS]
-  uint64_t* raw_empty;         // [RS], count kProducerThreads
+  uint64_t* raw_empty;         // [RS], count NP
   const spatten_attn_args* a;
   int64_t plane0;
   int n_tiles;
@@ -401,7 +413,7 @@ struct JobStream {
     job(j, is_v, t);
     const uint8_t* keep = (is_v && vmask) ? vmask : nullptr;
     if (kv_idx) {
-      produce_tile<DH, KT>(smem, t, a->n_kv, plane0, kv_idx, is_v ? a->v_msb : a->k_msb,
+      produce_tile<DH, KT, NP>(smem, t, a->n_kv, plane0, kv_idx, is_v ? a->v_msb : a->k_msb,
                            with_lsb ? (is_v ? a->v_lsb : a->k_lsb) : nullptr, off_hi, ptid, keep);
       return true;
     }
@@ -409,10 +421,10 @@ struct JobStream {
     const uint32_t st = gj % RS;
     if (!wait_bar(&raw_full[st], (gj / RS) & 1u, abort_flag, wlim)) return false;
     if (keep)
-      convert_staged<DH, KT, true>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
+      convert_staged<DH, KT, true, NP>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
                                    keep + t * KT);
     else
-      convert_staged<DH, KT, false>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
+      convert_staged<DH, KT, false, NP>(smem, smem + o_raw + st * raw_bytes, with_lsb, valid_rows(t), off_hi, ptid,
                                     nullptr);
     mbar_arrive(&raw_empty[st]);
     ++consumed;
@@ -572,7 +584,7 @@ __device__ __forceinline__ void zero_pruned_share(const spatten_attn_args& a, __
 }
 
 template <int DH>
-__global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
+__global__ void __launch_bounds__(kMainThreads<DH>, 1) attn_main_kernel(AttnProblem p) {
   using C = MainCfg<DH>;
   constexpr int KT = C::KT;
   constexpr int NST = C::NST;
@@ -592,20 +604,20 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
   const int n_tiles = (a.n_kv + KT - 1) / KT;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
 
-  if (warp == 11) {
+  if (warp == kMainMmaWarp<DH>) {
     tmem_alloc(&tmem_base_s, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
     abort_s = 0;
     for (int qb = 0; qb < C::NQ; ++qb) {
-      mbar_init(&bars[M_QF + qb], kProducerThreads);
+      mbar_init(&bars[M_QF + qb], kMainProducers<DH>);
       mbar_init(&bars[M_QE + qb], 1);
     }
     mbar_init(&bars[M_OE], 256);
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&bars[M_KF + s], kProducerThreads);
-      mbar_init(&bars[M_VF + s], kProducerThreads);
+      mbar_init(&bars[M_KF + s], kMainProducers<DH>);
+      mbar_init(&bars[M_VF + s], kMainProducers<DH>);
       mbar_init(&bars[M_KE + s], 1);
       mbar_init(&bars[M_VE + s], 1);
     }
@@ -619,7 +631,7 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     mbar_init(&bars[M_DR], 1);
     for (int s = 0; s < C::RS; ++s) {
       mbar_init(&bars[M_RF + s], 1);
-      mbar_init(&bars[M_RE + s], kProducerThreads);
+      mbar_init(&bars[M_RE + s], kMainProducers<DH>);
     }
     fence_mbar_init();
   }
@@ -639,195 +651,201 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     b = bs / a.H_kept;
   };
 
-  if (warp >= 8 && warp < 11) {
-    // ------------------------------------------------------------------------- producers
-    const int ptid = tid - 256;
-    uint32_t kc = 0, vc = 0, gjob = 0, qc = 0;
-    constexpr int QCH = 256 * (DH / 8);   // 16-byte chunks of one item's query rows
-    // the item's 256 query rows of its head, bf16, into query buffer qb at their swizzled fp16
-    // positions (rows past n_q zero-filled); one commit group
-    auto copy_q_async = [&](int item, uint32_t qbuf) {
-      int b, slot, pair;
-      item_coords(item, b, slot, pair);
-      const int h = head_of_slot(a, b, slot);
-      const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-      for (int e = ptid; e < QCH; e += kProducerThreads) {
-        const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = pair * 256 + rr;
-        const bool ok = qi < a.n_q;
-        const __nv_bfloat16* src =
-            ok ? q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8 : q;
-        cp_async16(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128), src, ok ? 16u : 0u);
-      }
-      cp_async_commit();
-    };
-    // bf16 -> fp16 in place, each thread the chunks it copied
-    auto convert_q_in_place = [&](uint32_t qbuf) {
-      uint32_t mx = 0u;
-      for (int e = ptid; e < QCH; e += kProducerThreads) {
-        const int rr = e / (DH / 8), c8 = e % (DH / 8);
-        uint4* p = reinterpret_cast<uint4*>(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128));
-        const uint4 v = *p;
-        mx = bf16x8_absmax(v, mx);
-        *p = bf16x8_to_f16x8(v);
-      }
-      if (bf16_absmax_out_of_f16(mx)) report(a.dev_status, SPATTEN_E_RANGE);
-    };
-    uint32_t g_issued = 0, g_consumed = 0;   // staging-ring jobs issued / converted, whole kernel
-    for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++qc) {
-      int b, slot, pair;
-      item_coords(it, b, slot, pair);
-      const int h = head_of_slot(a, b, slot);
-      const int64_t plane0 = (static_cast<int64_t>(b) * a.H + h) * a.kv_cap;
-      const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
-      JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
-                                  abort_flag, gjob};
-      js.wlim = wlim;
-      if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
-      struct Track {   // records the stream's progress however the item's loop is left
-        JobStream<DH, KT, C::RS>& js;
-        uint32_t &gi, &gc;
-        __device__ ~Track() { gi = js.g0 + js.issued; gc = js.g0 + js.consumed; }
-      } track{js, g_issued, g_consumed};
-      // the first raw key tiles start before the query tile (both in flight together)
-      if (!kv_idx && ptid == 0 && !js.issue_ahead(0)) { aborted = true; break; }
-      const uint32_t qb = qc % C::NQ;
-      if constexpr (C::NQ == 2) {
-        // this item's query tile was copied (bf16) into buffer qb during the previous item, or just
-        // below for the first item: convert it in place to fp16 (each thread its own chunks)
-        if (qc == 0) {
-          if (!wait_bar(&bars[M_QE + qb], 1u, abort_flag, wlim)) { aborted = true; break; }
-          copy_q_async(it, qb);
-        }
-        cp_async_wait_all();
-        convert_q_in_place(qb);
-        fence_async_smem();
-        mbar_arrive(&bars[M_QF + qb]);
-      } else {
-        // query tile of the item once the previous item's score MMAs have read the buffer
-        if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
-        constexpr int NCH = 256 * (DH / 8);
-        constexpr int BATCH = 8;
-        const int i0 = pair * 256;
+  if (warp >= 8) {
+    // warpgroups 2 and 3 (producers, MMA warp) give registers up to the softmax warpgroups; every
+    // warp of a warpgroup executes this one instruction
+    if constexpr (DH == 64) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    if (warp < kMainMmaWarp<DH>) {
+      // ------------------------------------------------------------------------- producers
+      const int ptid = tid - 256;
+      uint32_t kc = 0, vc = 0, gjob = 0, qc = 0;
+      constexpr int QCH = 256 * (DH / 8);   // 16-byte chunks of one item's query rows
+      // the item's 256 query rows of its head, bf16, into query buffer qb at their swizzled fp16
+      // positions (rows past n_q zero-filled); one commit group
+      auto copy_q_async = [&](int item, uint32_t qbuf) {
+        int b, slot, pair;
+        item_coords(item, b, slot, pair);
+        const int h = head_of_slot(a, b, slot);
         const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-        uint32_t qmx = 0u;
-        for (int e0 = ptid; e0 < NCH; e0 += BATCH * kProducerThreads) {
-          uint4 qv[BATCH];
-#pragma unroll
-          for (int k = 0; k < BATCH; ++k) {
-            const int e = e0 + k * kProducerThreads;
-            const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + rr;
-            qv[k] = make_uint4(0, 0, 0, 0);
-            if (e < NCH && qi < a.n_q)
-              qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
-                                                           static_cast<int64_t>(h) * DH) + c8);
+        for (int e = ptid; e < QCH; e += kMainProducers<DH>) {
+          const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = pair * 256 + rr;
+          const bool ok = qi < a.n_q;
+          const __nv_bfloat16* src =
+              ok ? q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok + static_cast<int64_t>(h) * DH + c8 * 8 : q;
+          cp_async16(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128), src, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+      };
+      // bf16 -> fp16 in place, each thread the chunks it copied
+      auto convert_q_in_place = [&](uint32_t qbuf) {
+        uint32_t mx = 0u;
+        for (int e = ptid; e < QCH; e += kMainProducers<DH>) {
+          const int rr = e / (DH / 8), c8 = e % (DH / 8);
+          uint4* p = reinterpret_cast<uint4*>(smem + C::oQ + qbuf * 2 * C::QB + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128));
+          const uint4 v = *p;
+          mx = bf16x8_absmax(v, mx);
+          *p = bf16x8_to_f16x8(v);
+        }
+        if (bf16_absmax_out_of_f16(mx)) report(a.dev_status, SPATTEN_E_RANGE);
+      };
+      uint32_t g_issued = 0, g_consumed = 0;   // staging-ring jobs issued / converted, whole kernel
+      for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++qc) {
+        int b, slot, pair;
+        item_coords(it, b, slot, pair);
+        const int h = head_of_slot(a, b, slot);
+        const int64_t plane0 = (static_cast<int64_t>(b) * a.H + h) * a.kv_cap;
+        const int32_t* kv_idx = a.kv_idx ? a.kv_idx + static_cast<int64_t>(b) * a.kv_idx_ld : nullptr;
+        JobStream<DH, KT, C::RS, kMainProducers<DH>> js{smem, C::oRaw, C::RAWB, &bars[M_RF], &bars[M_RE], &a, plane0, n_tiles, false, ptid,
+                                    abort_flag, gjob};
+        js.wlim = wlim;
+        if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
+        struct Track {   // records the stream's progress however the item's loop is left
+          JobStream<DH, KT, C::RS, kMainProducers<DH>>& js;
+          uint32_t &gi, &gc;
+          __device__ ~Track() { gi = js.g0 + js.issued; gc = js.g0 + js.consumed; }
+        } track{js, g_issued, g_consumed};
+        // the first raw key tiles start before the query tile (both in flight together)
+        if (!kv_idx && ptid == 0 && !js.issue_ahead(0)) { aborted = true; break; }
+        const uint32_t qb = qc % C::NQ;
+        if constexpr (C::NQ == 2) {
+          // this item's query tile was copied (bf16) into buffer qb during the previous item, or just
+          // below for the first item: convert it in place to fp16 (each thread its own chunks)
+          if (qc == 0) {
+            if (!wait_bar(&bars[M_QE + qb], 1u, abort_flag, wlim)) { aborted = true; break; }
+            copy_q_async(it, qb);
           }
-#pragma unroll
-          for (int k = 0; k < BATCH; ++k) {
-            const int e = e0 + k * kProducerThreads;
-            const int rr = e / (DH / 8), c8 = e % (DH / 8);
-            if (e < NCH) {
-              qmx = bf16x8_absmax(qv[k], qmx);
-              *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) =
-                  bf16x8_to_f16x8(qv[k]);
+          cp_async_wait_all();
+          convert_q_in_place(qb);
+          fence_async_smem();
+          mbar_arrive(&bars[M_QF + qb]);
+        } else {
+          // query tile of the item once the previous item's score MMAs have read the buffer
+          if (!wait_bar(&bars[M_QE], (qc & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
+          constexpr int NCH = 256 * (DH / 8);
+          constexpr int BATCH = 8;
+          const int i0 = pair * 256;
+          const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+          uint32_t qmx = 0u;
+          for (int e0 = ptid; e0 < NCH; e0 += BATCH * kMainProducers<DH>) {
+            uint4 qv[BATCH];
+  #pragma unroll
+            for (int k = 0; k < BATCH; ++k) {
+              const int e = e0 + k * kMainProducers<DH>;
+              const int rr = e / (DH / 8), c8 = e % (DH / 8), qi = i0 + rr;
+              qv[k] = make_uint4(0, 0, 0, 0);
+              if (e < NCH && qi < a.n_q)
+                qv[k] = __ldg(reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * a.n_q + qi) * a.q_ld_tok +
+                                                             static_cast<int64_t>(h) * DH) + c8);
+            }
+  #pragma unroll
+            for (int k = 0; k < BATCH; ++k) {
+              const int e = e0 + k * kMainProducers<DH>;
+              const int rr = e / (DH / 8), c8 = e % (DH / 8);
+              if (e < NCH) {
+                qmx = bf16x8_absmax(qv[k], qmx);
+                *reinterpret_cast<uint4*>(smem + C::oQ + (rr >> 7) * C::QB + tile_off(rr & 127, c8, 128)) =
+                    bf16x8_to_f16x8(qv[k]);
+              }
             }
           }
+          if (bf16_absmax_out_of_f16(qmx)) report(a.dev_status, SPATTEN_E_RANGE);
+          fence_async_smem();
+          mbar_arrive(&bars[M_QF]);
         }
-        if (bf16_absmax_out_of_f16(qmx)) report(a.dev_status, SPATTEN_E_RANGE);
-        fence_async_smem();
-        mbar_arrive(&bars[M_QF]);
-      }
-      // pass A keys, then pass B keys and values
-      for (int j = 0; j < 3 * n_tiles; ++j) {
-        if constexpr (C::NQ == 2) {
-          // at the first pass-B job the previous item is done with the other query buffer: copy
-          // the next item's query rows into it
-          if (j == n_tiles && it + static_cast<int>(gridDim.x) < n_items) {
-            const uint32_t nb = (qc + 1) % C::NQ;
-            if (!wait_bar(&bars[M_QE + nb], (((qc + 1) / C::NQ) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
-            copy_q_async(it + static_cast<int>(gridDim.x), nb);
+        // pass A keys, then pass B keys and values
+        for (int j = 0; j < 3 * n_tiles; ++j) {
+          if constexpr (C::NQ == 2) {
+            // at the first pass-B job the previous item is done with the other query buffer: copy
+            // the next item's query rows into it
+            if (j == n_tiles && it + static_cast<int>(gridDim.x) < n_items) {
+              const uint32_t nb = (qc + 1) % C::NQ;
+              if (!wait_bar(&bars[M_QE + nb], (((qc + 1) / C::NQ) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
+              copy_q_async(it + static_cast<int>(gridDim.x), nb);
+            }
           }
+          if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; break; }
+          bool is_v;
+          int t;
+          js.job(j, is_v, t);
+          uint32_t& cnt = is_v ? vc : kc;
+          const uint32_t st = cnt % NST;
+          if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
+          if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, kv_idx)) { aborted = true; break; }
+          mbar_arrive(&bars[(is_v ? M_VF : M_KF) + st]);
+          ++cnt;
         }
-        if (!kv_idx && ptid == 0 && !js.issue_ahead(j)) { aborted = true; break; }
-        bool is_v;
-        int t;
-        js.job(j, is_v, t);
-        uint32_t& cnt = is_v ? vc : kc;
-        const uint32_t st = cnt % NST;
-        if (!wait_bar(&bars[(is_v ? M_VE : M_KE) + st], ((cnt / NST) & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
-        if (!js.convert(j, (is_v ? C::oV : C::oK) + st * C::TB, kv_idx)) { aborted = true; break; }
-        mbar_arrive(&bars[(is_v ? M_VF : M_KF) + st]);
-        ++cnt;
+        gjob += 3 * n_tiles;
       }
-      gjob += 3 * n_tiles;
-    }
-    cp_async_wait_all();   // no query copy may land after the CTA has left
-    if (aborted && ptid == 0)   // bulk copies already armed complete before shared memory is released
-      for (uint32_t gj = g_consumed; gj < g_issued; ++gj) drain_wait(&bars[M_RF + gj % C::RS], (gj / C::RS) & 1u);
-  } else if (warp == 11) {
-    // ------------------------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0}, ic = 0;
-      uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
-      // scores of one key tile for both warpgroups: S = Q K^T (pass A, and pass B in row
-      // orientation) or S^T = K Q^T (pass B, transposed)
-      auto qk_both = [&](bool trans) -> bool {
-        const uint32_t ks = kc % NST;
-        if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag, wlim)) return false;
-        const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
-        if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag, wlim)) return false;
-        tc_after_sync();
-        if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS, sK, sQ0);
-        else mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
-        mma_commit(&bars[M_SF + 0]);
-        ++sc[0];
-        if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag, wlim)) return false;
-        tc_after_sync();
-        if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS + KT, sK, sQ1);
-        else mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
-        mma_commit(&bars[M_SF + 1]);
-        ++sc[1];
-        mma_commit(&bars[M_KE + ks]);
-        ++kc;
-        return true;
-      };
-      for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++ic) {
-        const uint32_t qb = ic % C::NQ;
-        sQ0 = smem_u32(smem + C::oQ + qb * 2 * C::QB);
-        sQ1 = sQ0 + C::QB;
-        if (!wait_bar(&bars[M_QF + qb], (ic / C::NQ) & 1u, abort_flag, wlim)) { aborted = true; break; }
-        for (int t = 0; t < n_tiles && !aborted; ++t)   // pass A
-          if (!qk_both(false)) aborted = true;
-        if (aborted) break;
-        if (!qk_both(true)) { aborted = true; break; }   // pass B, tile 0
-        if (n_tiles == 1) mma_commit(&bars[M_QE + qb]);  // the item's last read of Q is issued
-        // the previous item's O must have been read before this item's first P V overwrites it
-        if (!wait_bar(&bars[M_OE], (ic & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
-        for (int t = 0; t < n_tiles && !aborted; ++t) {
-          if (t + 1 < n_tiles) {
-            if (!qk_both(true)) { aborted = true; break; }
-            if (t + 2 == n_tiles) mma_commit(&bars[M_QE + qb]);
-          }
-          const uint32_t vs = vc % NST;
-          if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag, wlim)) { aborted = true; break; }
-          const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
-          for (int gg = 0; gg < 2 && !aborted; ++gg) {
-            if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag, wlim)) { aborted = true; break; }
-            tc_after_sync();
-            if constexpr (C::kT)
-              mma_pv_mn<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
-            else
-              mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
-            mma_commit(&bars[M_PE + gg]);
-            ++pc[gg];
-          }
+      cp_async_wait_all();   // no query copy may land after the CTA has left
+      if (aborted && ptid == 0)   // bulk copies already armed complete before shared memory is released
+        for (uint32_t gj = g_consumed; gj < g_issued; ++gj) drain_wait(&bars[M_RF + gj % C::RS], (gj / C::RS) & 1u);
+    } else {
+      // ------------------------------------------------------------------------- MMA issue
+      if (lane == 0) {
+        uint32_t kc = 0, vc = 0, sc[2] = {0, 0}, pc[2] = {0, 0}, ic = 0;
+        uint32_t sQ0 = smem_u32(smem + C::oQ), sQ1 = smem_u32(smem + C::oQ + C::QB);
+        // scores of one key tile for both warpgroups: S = Q K^T (pass A, and pass B in row
+        // orientation) or S^T = K Q^T (pass B, transposed)
+        auto qk_both = [&](bool trans) -> bool {
+          const uint32_t ks = kc % NST;
+          if (!wait_bar(&bars[M_KF + ks], (kc / NST) & 1u, abort_flag, wlim)) return false;
+          const uint32_t sK = smem_u32(smem + C::oK + ks * C::TB);
+          if (!wait_bar(&bars[M_SR + 0], (sc[0] & 1u) ^ 1u, abort_flag, wlim)) return false;
+          tc_after_sync();
+          if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS, sK, sQ0);
+          else mma_qk<DH, KT>(tmem + C::tS, sQ0, sK, 0);
+          mma_commit(&bars[M_SF + 0]);
+          ++sc[0];
+          if (!wait_bar(&bars[M_SR + 1], (sc[1] & 1u) ^ 1u, abort_flag, wlim)) return false;
+          tc_after_sync();
+          if (C::kT && trans) mma_kq<DH, KT>(tmem + C::tS + KT, sK, sQ1);
+          else mma_qk<DH, KT>(tmem + C::tS + KT, sQ1, sK, 0);
+          mma_commit(&bars[M_SF + 1]);
+          ++sc[1];
+          mma_commit(&bars[M_KE + ks]);
+          ++kc;
+          return true;
+        };
+        for (int it = blockIdx.x; it < n_items && !aborted; it += gridDim.x, ++ic) {
+          const uint32_t qb = ic % C::NQ;
+          sQ0 = smem_u32(smem + C::oQ + qb * 2 * C::QB);
+          sQ1 = sQ0 + C::QB;
+          if (!wait_bar(&bars[M_QF + qb], (ic / C::NQ) & 1u, abort_flag, wlim)) { aborted = true; break; }
+          for (int t = 0; t < n_tiles && !aborted; ++t)   // pass A
+            if (!qk_both(false)) aborted = true;
           if (aborted) break;
-          mma_commit(&bars[M_VE + vs]);
-          ++vc;
+          if (!qk_both(true)) { aborted = true; break; }   // pass B, tile 0
+          if (n_tiles == 1) mma_commit(&bars[M_QE + qb]);  // the item's last read of Q is issued
+          // the previous item's O must have been read before this item's first P V overwrites it
+          if (!wait_bar(&bars[M_OE], (ic & 1u) ^ 1u, abort_flag, wlim)) { aborted = true; break; }
+          for (int t = 0; t < n_tiles && !aborted; ++t) {
+            if (t + 1 < n_tiles) {
+              if (!qk_both(true)) { aborted = true; break; }
+              if (t + 2 == n_tiles) mma_commit(&bars[M_QE + qb]);
+            }
+            const uint32_t vs = vc % NST;
+            if (!wait_bar(&bars[M_VF + vs], (vc / NST) & 1u, abort_flag, wlim)) { aborted = true; break; }
+            const uint32_t sV = smem_u32(smem + C::oV + vs * C::TB);
+            for (int gg = 0; gg < 2 && !aborted; ++gg) {
+              if (!wait_bar(&bars[M_PF + gg], pc[gg] & 1u, abort_flag, wlim)) { aborted = true; break; }
+              tc_after_sync();
+              if constexpr (C::kT)
+                mma_pv_mn<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
+              else
+                mma_pv<DH, KT>(tmem + C::tO + gg * DH, smem_u32(smem + C::oP + gg * C::PB), sV, t > 0 ? 1u : 0u);
+              mma_commit(&bars[M_PE + gg]);
+              ++pc[gg];
+            }
+            if (aborted) break;
+            mma_commit(&bars[M_VE + vs]);
+            ++vc;
+          }
+          if (!aborted) mma_commit(&bars[M_OD]);
         }
-        if (!aborted) mma_commit(&bars[M_OD]);
       }
     }
   } else {
+    if constexpr (DH == 64) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ------------------------------------------------------------------------- softmax
     if (a.zero_pruned_heads && a.H_kept < a.H) zero_pruned_share<DH>(a, o, warp, lane);
     const int g = warp >> 2;                        // warpgroup
@@ -1069,13 +1087,13 @@ __global__ void __launch_bounds__(384, 1) attn_main_kernel(AttnProblem p) {
     for (int64_t it = blockIdx.x + static_cast<int64_t>(tid) * gridDim.x; it < n_items;
          it += static_cast<int64_t>(gridDim.x) * blockDim.x)
       p.flag_cnt[it] = 0;
-  if (any_abort && warp == 11 && lane == 0) {   // every MMA already issued completes before TMEM is freed
+  if (any_abort && warp == kMainMmaWarp<DH> && lane == 0) {   // every MMA already issued completes before TMEM is freed
     mma_commit(&bars[M_DR]);
     drain_wait(&bars[M_DR], 0u);
   }
   tc_before_sync();
   __syncthreads();
-  if (warp == 11) {
+  if (warp == kMainMmaWarp<DH>) {
     tc_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -1228,7 +1246,7 @@ __global__ void __launch_bounds__(256, DH == 64 ? 2 : 1) attn_full_kernel(AttnPr
   if (warp >= 4 && warp < 7) {
     // ------------------------------------------------------------------------- producers
     const int ptid = tid - 128;
-    JobStream<DH, KT, C::RS> js{smem, C::oRaw, C::RAWB, &bars[F_RF], &bars[F_RE], &a, plane0, n_tiles, true, ptid,
+    JobStream<DH, KT, C::RS, kProducerThreads> js{smem, C::oRaw, C::RAWB, &bars[F_RF], &bars[F_RE], &a, plane0, n_tiles, true, ptid,
                                 abort_flag};
     js.wlim = wlim;
     if (p.v_mask) js.vmask = p.v_mask + (static_cast<int64_t>(b) * a.H_kept + slot) * a.n_kv;
@@ -1435,6 +1453,12 @@ int32_t launch(const AttnProblem& p, cudaStream_t st) {
   static DeviceOnce once;
   int dev = 0;
   SPT_TRY(once_per_device(once, &dev, [](int) -> int32_t {
+    // the register split waits, without a bound, for registers the block holds: launch only when
+    // the block's registers at launch cover it
+    cudaFuncAttributes fa{};
+    SPT_CUDA(cudaFuncGetAttributes(&fa, attn_main_kernel<DH>));
+    if (DH == 64 && static_cast<int64_t>(fa.numRegs) * kMainThreads<DH> < 256LL * kSoftmaxRegs + 256LL * kOtherRegs)
+      return SPATTEN_E_UNSUPPORTED;
     SPT_CUDA(cudaFuncSetAttribute(attn_main_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(MainCfg<DH>::kSmem)));
     SPT_CUDA(cudaFuncSetAttribute(attn_full_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1443,7 +1467,7 @@ int32_t launch(const AttnProblem& p, cudaStream_t st) {
   }));
   const int64_t items = static_cast<int64_t>(p.n_pair) * p.a.H_kept * p.a.B;
   const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
-  attn_main_kernel<DH><<<grid, 384, MainCfg<DH>::kSmem, st>>>(p);
+  attn_main_kernel<DH><<<grid, kMainThreads<DH>, MainCfg<DH>::kSmem, st>>>(p);
   SPT_TRY(launch_status());
   if (p.a.refetch_threshold > 0.0f) {
     attn_full_kernel<DH><<<dim3(p.n_qt, p.a.H_kept, p.a.B), 256, FullCfg<DH>::kSmem, st>>>(p);
