@@ -81,7 +81,11 @@ def prefill_traffic(w):
     c = CAPTURED_TRAFFIC["prefill_attention_layer"]
     if w.name != "bert_base_prefill_bf16":
         return None, "null: no DRAM capture of this workload's layer shape"
-    if sources_hash() != c["sources_sha256"]:
+    try:
+        current = sources_hash()
+    except OSError:
+        return None, "null: the kernel sources are not beside this package"
+    if current != c["sources_sha256"]:
         return None, "null: the attention kernels changed since their DRAM capture"
     units = sum(w.token_keep[l] * w.head_keep[l] for l in range(w.L))
     per_seq = c["bytes"] / 32.0
