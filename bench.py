@@ -61,7 +61,7 @@ DATA = "synthetic (seeded N(0,1) activations, random-init weights)"
 TRAFFIC_SOURCES = ("attn_tc.cu", "attention.cu", "attn_reduce.cu", "attention.cuh", "tc_ptx.cuh",
                    "exp2_poly.cuh", "common.cuh")
 CAPTURED_TRAFFIC = {
-    "prefill_attention_layer": {"sources_sha256": "3854332367032eee", "bytes": 50446592 + 772096 + 39170048 + 4048384,
+    "prefill_attention_layer": {"sources_sha256": "362aa693a0bf0658", "bytes": 50435328 + 1255168 + 39167232 + 4048640,
                                 "kept_key_heads": 512 * 12},
 }
 

@@ -7,6 +7,9 @@
 // fully-connected layers run off the attention engine -- here on the library GEMM (cuBLASLt),
 // everything else in this library's kernels.  The host never reads device memory inside the loop
 // (all sizes come from the schedule), so a whole forward can be captured in a CUDA graph.
+// The next layer's selections (top-k of the importance vectors) depend on the attention step but
+// not on the output projection, so they run on a second stream of the library's own, forked from
+// and joined back to the caller's stream by events, overlapping the projection GEMMs.
 #include <cublasLt.h>
 
 #include <algorithm>
@@ -199,6 +202,58 @@ spatten_attn_args base_attn(const spatten_cascade_cfg& c) {
 }
 
 // ------------------------------------------------------------------------------------------------
+// side stream: one per device and host thread, created on the first call outside a stream capture
+// (creating a stream inside one is not allowed; such a call runs its selections on the caller's
+// stream instead)
+// ------------------------------------------------------------------------------------------------
+struct Side {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t origin = nullptr;   // the stream forked from; null when running on it
+  cudaStream_t use(cudaStream_t st) const { return origin ? s : st; }
+};
+
+int32_t side_fork(cudaStream_t st, Side** out) {
+  thread_local Side sides[64];
+  *out = nullptr;
+  int dev = 0;
+  SPT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return SPATTEN_OK;
+  Side& sd = sides[dev];
+  sd.origin = nullptr;
+  *out = &sd;
+  if (!sd.s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    SPT_CUDA(cudaStreamIsCapturing(st, &cs));
+    if (cs != cudaStreamCaptureStatusNone) return SPATTEN_OK;
+    SPT_CUDA(cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking));
+    SPT_CUDA(cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming));
+    SPT_CUDA(cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming));
+  }
+  SPT_CUDA(cudaEventRecord(sd.fork, st));
+  SPT_CUDA(cudaStreamWaitEvent(sd.s, sd.fork, 0));
+  sd.origin = st;
+  return SPATTEN_OK;
+}
+
+int32_t side_join(Side* sd) {
+  if (!sd || !sd->origin) return SPATTEN_OK;
+  SPT_CUDA(cudaEventRecord(sd->join, sd->s));
+  SPT_CUDA(cudaStreamWaitEvent(sd->origin, sd->join, 0));
+  sd->origin = nullptr;
+  return SPATTEN_OK;
+}
+
+// joins an open fork when the forward leaves early (an error), so that no stream capture is left
+// with an unjoined stream
+struct SideGuard {
+  Side*& sd;
+  ~SideGuard() {
+    if (sd) side_join(sd);
+  }
+};
+
+// ------------------------------------------------------------------------------------------------
 // prefill
 // ------------------------------------------------------------------------------------------------
 int32_t run_prefill(const spatten_cascade_cfg& c, const spatten_layer_weights* w, spatten_cascade_io& io,
@@ -219,6 +274,8 @@ int32_t run_prefill(const spatten_cascade_cfg& c, const spatten_layer_weights* w
   char* nxt = ws.xb;
   float* g_cur = ws.gain_a;
   float* g_nxt = ws.gain_b;
+  Side* side = nullptr;
+  SideGuard guard{side};
   for (int l = 0; l < L; ++l) {
     const int k = c.token_keep[l], Hl = c.head_keep[l];
     int32_t* kept_l = io.kept_tok + static_cast<int64_t>(l) * B * T;
@@ -271,32 +328,42 @@ int32_t run_prefill(const spatten_cascade_cfg& c, const spatten_layer_weights* w
     if (io.trace_o)
       SPT_TRY(copy2d(static_cast<char*>(io.trace_o) + static_cast<size_t>(l) * B * T * HD * es, T * HD * es, ws.o,
                      k * HD * es, k * HD * es, B, st));
-    // residual: X[B*k, D] += O[B*k, HD] @ W_o   (pruned heads' O are zero)
-    SPT_TRY(gemm_rm(ws.o, w[l].w_o, cur, B * k, D, static_cast<int>(HD), c.dtype, true, ws.gemm_ws, st));
     if (io.trace_tok_imp)
       SPT_CUDA(cudaMemcpyAsync(io.trace_tok_imp + static_cast<size_t>(l) * B * T, io.tok_imp, sizeof(float) * B * T,
                                cudaMemcpyDeviceToDevice, st));
     if (io.trace_head_imp)
       SPT_CUDA(cudaMemcpyAsync(io.trace_head_imp + static_cast<size_t>(l) * B * H, io.head_imp, sizeof(float) * B * H,
                                cudaMemcpyDeviceToDevice, st));
+    const int k2 = l + 1 < L ? c.token_keep[l + 1] : 0;
+    if (l + 1 < L) {
+      // the next layer's selections, beside the projection: token top-k_{l+1} of the cumulative
+      // importance over S_l (read through kept_l), the kept rows' gains, the head selection
+      SPT_TRY(side_fork(st, &side));
+      const cudaStream_t ss = side ? side->use(st) : st;
+      auto select = [&]() -> int32_t {
+        int32_t* kept_n = io.kept_tok + static_cast<int64_t>(l + 1) * B * T;
+        SPT_TRY(spatten_topk_select(io.tok_imp, B, k, T, k2, kept_l, T, ws.sel, T, kept_n, nullptr, 0, io.dev_status,
+                                    ss));
+        if (gain)
+          SPT_TRY(spatten_gather_kept(g_cur, static_cast<int64_t>(k) * 4, 4, k, 4, B, ws.sel, T, k2, g_nxt,
+                                      static_cast<int64_t>(k2) * 4, 4, nullptr, 0, nullptr, 0, nullptr, ss));
+        const int H2 = c.head_keep[l + 1];
+        int32_t* khead_n = io.kept_head + static_cast<int64_t>(l + 1) * B * H;
+        if (H2 < Hl)
+          return spatten_topk_select(io.head_imp, B, Hl, H, H2, khead_l, H, ws.head_sel, H, khead_n, nullptr, 0,
+                                     io.dev_status, ss);
+        SPT_CUDA(cudaMemcpyAsync(khead_n, khead_l, sizeof(int32_t) * B * H, cudaMemcpyDeviceToDevice, ss));
+        return SPATTEN_OK;
+      };
+      SPT_TRY(select());
+    }
+    // residual: X[B*k, D] += O[B*k, HD] @ W_o   (pruned heads' O are zero)
+    SPT_TRY(gemm_rm(ws.o, w[l].w_o, cur, B * k, D, static_cast<int>(HD), c.dtype, true, ws.gemm_ws, st));
     if (l == L - 1) break;
-    // token selection: top-k_{l+1} of the cumulative importance over S_l (read through kept_l)
-    const int k2 = c.token_keep[l + 1];
-    int32_t* kept_n = io.kept_tok + static_cast<int64_t>(l + 1) * B * T;
-    SPT_TRY(spatten_topk_select(io.tok_imp, B, k, T, k2, kept_l, T, ws.sel, T, kept_n, nullptr, 0, io.dev_status, st));
+    SPT_TRY(side_join(side));
+    side = nullptr;
     SPT_TRY(spatten_gather_kept(cur, static_cast<int64_t>(k) * D * es, D * es, k, D * es, B, ws.sel, T, k2, nxt,
                                 static_cast<int64_t>(k2) * D * es, D * es, nullptr, 0, nullptr, 0, nullptr, st));
-    if (gain)
-      SPT_TRY(spatten_gather_kept(g_cur, static_cast<int64_t>(k) * 4, 4, k, 4, B, ws.sel, T, k2, g_nxt,
-                                  static_cast<int64_t>(k2) * 4, 4, nullptr, 0, nullptr, 0, nullptr, st));
-    // head selection
-    const int H2 = c.head_keep[l + 1];
-    int32_t* khead_n = io.kept_head + static_cast<int64_t>(l + 1) * B * H;
-    if (H2 < Hl)
-      SPT_TRY(spatten_topk_select(io.head_imp, B, Hl, H, H2, khead_l, H, ws.head_sel, H, khead_n, nullptr, 0,
-                                  io.dev_status, st));
-    else
-      SPT_CUDA(cudaMemcpyAsync(khead_n, khead_l, sizeof(int32_t) * B * H, cudaMemcpyDeviceToDevice, st));
     std::swap(cur, nxt);
     std::swap(g_cur, g_nxt);
   }
@@ -317,6 +384,8 @@ int32_t run_decode(const spatten_cascade_cfg& c, const spatten_layer_weights* w,
   SPT_TRY(iota_rows(io.kept_tok, cap, n, B, st));
   SPT_CUDA(cudaMemcpyAsync(ws.xa, io.x, static_cast<size_t>(B) * D * es, cudaMemcpyDeviceToDevice, st));
   char* x = ws.xa;
+  Side* side = nullptr;   // the previous layer's cache-row selection, beside this layer's projections
+  SideGuard guard{side};
   for (int l = 0; l < L; ++l) {
     const int k = c.token_keep[l];
     const spatten_decode_cache& cc = io.caches[l];
@@ -355,18 +424,24 @@ int32_t run_decode(const spatten_cascade_cfg& c, const spatten_layer_weights* w,
     a.refetch_flags_ld = 1;
     a.refetch_count = io.refetch_count ? io.refetch_count + l : nullptr;
     a.dev_status = io.dev_status;
+    SPT_TRY(side_join(side));   // this layer's kept cache rows
+    side = nullptr;
     SPT_TRY(attention_layer_timed(&a, ws.attn_ws, ws.attn_ws_bytes, st, ev(io, 2 * l), ev(io, 2 * l + 1)));
     if (io.trace_o)
       SPT_CUDA(cudaMemcpyAsync(static_cast<char*>(io.trace_o) + static_cast<size_t>(l) * B * HD * es, ws.o,
                                static_cast<size_t>(B) * HD * es, cudaMemcpyDeviceToDevice, st));
-    SPT_TRY(gemm_rm(ws.o, w[l].w_o, x, B, D, static_cast<int>(HD), c.dtype, true, ws.gemm_ws, st));
     if (io.trace_tok_imp)
       SPT_CUDA(cudaMemcpyAsync(io.trace_tok_imp + static_cast<size_t>(l) * B * cap, io.dec_tok_imp,
                                sizeof(float) * B * cap, cudaMemcpyDeviceToDevice, st));
-    if (l == L - 1) break;
-    int32_t* kept_n = io.kept_tok + static_cast<int64_t>(l + 1) * B * cap;
-    SPT_TRY(spatten_topk_select(io.dec_tok_imp, B, k, cap, c.token_keep[l + 1], kept_l, cap, nullptr, cap, kept_n,
-                                nullptr, 0, io.dev_status, st));
+    if (l + 1 < L) {
+      // the next layer's kept cache rows, beside this layer's output projection and the next
+      // layer's input projection and cache append (joined before the next attention step)
+      SPT_TRY(side_fork(st, &side));
+      int32_t* kept_n = io.kept_tok + static_cast<int64_t>(l + 1) * B * cap;
+      SPT_TRY(spatten_topk_select(io.dec_tok_imp, B, k, cap, c.token_keep[l + 1], kept_l, cap, nullptr, cap, kept_n,
+                                  nullptr, 0, io.dev_status, side ? side->use(st) : st));
+    }
+    SPT_TRY(gemm_rm(ws.o, w[l].w_o, x, B, D, static_cast<int>(HD), c.dtype, true, ws.gemm_ws, st));
   }
   SPT_CUDA(cudaMemcpyAsync(io.x_out, x, static_cast<size_t>(B) * D * es, cudaMemcpyDeviceToDevice, st));
   return SPATTEN_OK;

@@ -279,6 +279,12 @@ int32_t spatten_gather_kept(const void* src, int64_t src_batch, int64_t src_row,
  * layer: project x_l; append its K/V to the layer's cache planes at row n (prompt-time scale,
  * saturating); attend over S_l (S_0 = rows 0..n); I += P; x_{l+1} = x_l + O @ W_o;
  * S_{l+1} = top-k_{l+1}(I restricted to S_l) with k_l = token_keep[l] (all heads kept).
+ *
+ * STREAMS: all work is ordered on `stream`.  The next layer's selections run on a second stream
+ * of the library's own (one per device and host thread, created on the first call made outside a
+ * stream capture), forked from `stream` after the attention step and joined back by events before
+ * their results are read, so that they overlap the projections; a stream capture of the call
+ * captures both.  A call made inside a capture before that stream exists runs them on `stream`.
  * ============================================================================================= */
 enum spatten_mode { SPATTEN_PREFILL = 0, SPATTEN_DECODE_STEP = 1 };
 
