@@ -113,7 +113,7 @@ def quantize_case(B, H, n, d, reps):
     return dict(case="quantize", B=B, H=H, n=n, d=d, ms=ms, bytes=byts, gbs=byts / ms / 1e6)
 
 
-def decode_case(B, H, n, d, keep, theta, reps):
+def decode_case(B, H, n, d, keep, theta, reps, kernel=0):
     g = synth.rng_for(11)
     HD = H * d
     kv = torch.from_numpy(g.standard_normal((B, n, 3 * HD))).to(torch.bfloat16).cuda()
@@ -139,12 +139,12 @@ def decode_case(B, H, n, d, keep, theta, reps):
     cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
     a.o, a.o_ld_tok, a.tok_imp, a.tok_imp_ld = o.data_ptr(), HD, tok.data_ptr(), n
     a.tok_imp_map, a.tok_imp_map_ld, a.refetch_count = idx.data_ptr(), keep, cnt.data_ptr()
-    a.refetch_threshold = theta
+    a.refetch_threshold, a.kernel = theta, kernel
     ws = torch.empty(S.attention_workspace_size(a), dtype=torch.uint8, device="cuda")
     ms = _time(lambda: S.attention_layer(a, ws, ws.numel()), reps)
     refetched = int(cnt.item()) / (2 * reps + 1)
     byts = B * H * keep * d * 2.0 + refetched * keep * d + B * keep * 4.0
-    return dict(case="decode", B=B, H=H, n=n, keep=keep, d=d, ms=ms, bytes=byts, gbs=byts / ms / 1e6,
+    return dict(case="decode", B=B, H=H, n=n, keep=keep, d=d, kernel=kernel, theta=theta, ms=ms, bytes=byts, gbs=byts / ms / 1e6,
                 refetch_frac=refetched / (B * H))
 
 
@@ -197,7 +197,7 @@ def main(argv=None):
     elif a.case == "quantize":
         r = quantize_case(a.B, a.H, a.n, a.d, a.reps)
     elif a.case == "decode":
-        r = decode_case(a.B, a.H, a.n, a.d, a.keep, a.theta, a.reps)
+        r = decode_case(a.B, a.H, a.n, a.d, a.keep, a.theta, a.reps, a.kernel)
     else:
         r = decode_step_case(a.reps)
     print(json.dumps(r), flush=True)

@@ -20,7 +20,8 @@ bool choose_path(const spatten_attn_args& a, Path* out) {
   switch (a.kernel) {
     case SPATTEN_ATTN_CUDA_CORE: *out = Path::kSimt; return true;
     case SPATTEN_ATTN_TENSOR_CORE: *out = Path::kTc; return attn_tc_supported(a);
-    case SPATTEN_ATTN_DECODE: *out = Path::kDecode; return attn_decode_supported(a);
+    case SPATTEN_ATTN_DECODE:
+    case SPATTEN_ATTN_DECODE_PREDICATED: *out = Path::kDecode; return attn_decode_supported(a);
     default: break;
   }
   if (attn_decode_supported(a)) *out = Path::kDecode;
@@ -40,7 +41,7 @@ int rows_per_cta(Path p) {
 int32_t validate(const spatten_attn_args& a) {
   if (a.B < 1 || a.H < 1 || a.n_q < 1 || a.n_kv < 1) return SPATTEN_E_ARG;
   if (a.B > 65535 || a.H > 1024) return SPATTEN_E_ARG;
-  if (a.kernel < SPATTEN_ATTN_AUTO || a.kernel > SPATTEN_ATTN_DECODE) return SPATTEN_E_ARG;
+  if (a.kernel < SPATTEN_ATTN_AUTO || a.kernel > SPATTEN_ATTN_DECODE_PREDICATED) return SPATTEN_E_ARG;
   if (a.v_keep < 0) return SPATTEN_E_ARG;
   if (a.d_h != 64 && a.d_h != 128) return SPATTEN_E_UNSUPPORTED;
   if (a.H_kept < 1 || a.H_kept > a.H) return SPATTEN_E_ARG;
@@ -90,6 +91,7 @@ size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
   float* de = nullptr;
   float* ds = nullptr;
   float* dob = nullptr;
+  int32_t* dfl = nullptr;
   if (path == Path::kDecode) {
     const int ir = decode_item_rows(a.d_h);
     items = static_cast<int>(ceil_div(a.n_kv, ir));
@@ -97,6 +99,7 @@ size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
     de = c.take<float>(2 * bh * a.n_kv);
     ds = c.take<float>(bh * items * 4);
     dob = c.take<float>(bh * items * 2 * a.d_h);
+    if (a.kernel == SPATTEN_ATTN_DECODE_PREDICATED && a.refetch_threshold > 0.0f) dfl = c.take<int32_t>(bh);
   }
   if (path == Path::kTc) {
     fl = c.take<int32_t>(static_cast<size_t>(a.B) * a.H_kept * n_pair * 256);
@@ -130,6 +133,7 @@ size_t layout(const spatten_attn_args& a, Path path, AttnProblem* p) {
     p->dec_e = de;
     p->dec_stat = ds;
     p->dec_o = dob;
+    p->dec_flag = dfl;
   }
   return c.used;
 }

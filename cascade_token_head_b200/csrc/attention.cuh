@@ -29,6 +29,7 @@ struct AttnProblem {
   float* dec_e;              // ws [2][B][H_kept][n_kv] exp(s - item max): MSB-only, full precision
   float* dec_stat;           // ws [B][H_kept][dec_items][4] item max and sum, both variants
   float* dec_o;              // ws [B][H_kept][dec_items][2][d_h] item sum of exp * V, both variants
+  int32_t* dec_flag = nullptr;  // ws [B][H_kept] predicated form only: rows whose LSBs are read
   // local value pruning (a.v_keep in [1, n_kv)): each kept head's column sums of P, its kept keys
   // and (prefill) the V mask of the second run
   float* head_col = nullptr;        // ws [B][H_kept][n_kv] (decode: written by the combine step)

@@ -106,7 +106,10 @@ struct DSmem {
   static_assert(KPW * NV * DH * 4 <= STEPS * 32 * 16, "the e*V sums fit the K MSB area");
 };
 
-template <int DH, typename QT, bool LSB>
+// FLAGGED: the full-precision pass of the predicated form, run only for the rows the MSB pass
+// flagged (p.dec_flag); it recomputes the MSB variant with the same arithmetic, so the values it
+// rewrites are the ones already there
+template <int DH, typename QT, bool LSB, bool FLAGGED = false>
 __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnProblem p) {
   using G = DGeom<DH>;
   using SM = DSmem<DH, LSB>;
@@ -120,6 +123,7 @@ __global__ void __launch_bounds__(kDWarps * 32) attn_decode_items_kernel(AttnPro
   const int w_id = blockIdx.x * kDWarps + warp;
   const int slot = w_id / p.dec_items, item = w_id % p.dec_items;
   if (slot >= a.H_kept) return;   // warps are independent: no block-level barrier follows
+  if (FLAGGED && !p.dec_flag[static_cast<int64_t>(blockIdx.y) * a.H_kept + slot]) return;
   unsigned char* wsm = d_smem + warp * SM::bytes;
   float* s_sc = reinterpret_cast<float*>(wsm + SM::sc);
   const int b = blockIdx.y;
@@ -553,6 +557,18 @@ __global__ void __launch_bounds__(kCThreads) attn_decode_pruned_out_kernel(AttnP
   }
 }
 
+// Predicated form: the refetch decision of every (sequence, kept head) row from its MSB-pass item
+// statistics, folded exactly as the combine step folds them (one warp per row).
+__global__ void __launch_bounds__(32) attn_decode_flag_kernel(AttnProblem p) {
+  const int slot = blockIdx.x, b = blockIdx.y;
+  const int64_t row = static_cast<int64_t>(b) * p.a.H_kept + slot;
+  float m, inv_l;
+  // the MSB pass wrote (m1, l1, m1, l1): the full-precision fold sees the MSB statistics
+  const bool full = fold_row<true>(reinterpret_cast<const float4*>(p.dec_stat) + row * p.dec_items, p.dec_items,
+                                   p.a.refetch_threshold, &m, &inv_l);
+  if (threadIdx.x == 0) p.dec_flag[row] = full ? 1 : 0;
+}
+
 // dynamic shared memory of the combine kernel: a token block's factor table and flags
 size_t combine_smem(int d_h, int H_kept) {
   const int item_rows = d_h == 64 ? DGeom<64>::ITEM : DGeom<128>::ITEM;
@@ -560,21 +576,33 @@ size_t combine_smem(int d_h, int H_kept) {
   return static_cast<size_t>(H_kept) * (ti + 1) * 4;
 }
 
-template <int DH, typename QT, bool LSB>
-int32_t launch(const AttnProblem& p, cudaStream_t st) {
-  const int items = p.dec_items;
-  const int64_t per_seq = static_cast<int64_t>(items) * p.a.H_kept;
+template <int DH, typename QT, bool LSB, bool FLAGGED>
+int32_t launch_items(const AttnProblem& p, cudaStream_t st) {
   constexpr int smem = kDWarps * DSmem<DH, LSB>::bytes;
   static DeviceOnce once;
   int dev = 0;
   SPT_TRY(once_per_device(once, &dev, [](int) -> int32_t {
-    SPT_CUDA(cudaFuncSetAttribute(attn_decode_items_kernel<DH, QT, LSB>,
+    SPT_CUDA(cudaFuncSetAttribute(attn_decode_items_kernel<DH, QT, LSB, FLAGGED>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     return SPATTEN_OK;
   }));
-  attn_decode_items_kernel<DH, QT, LSB>
+  const int64_t per_seq = static_cast<int64_t>(p.dec_items) * p.a.H_kept;
+  attn_decode_items_kernel<DH, QT, LSB, FLAGGED>
       <<<dim3(static_cast<unsigned>(ceil_div(per_seq, kDWarps)), p.a.B), kDWarps * 32, smem, st>>>(p);
-  SPT_TRY(launch_status());
+  return launch_status();
+}
+
+template <int DH, typename QT, bool LSB>
+int32_t launch(const AttnProblem& p, cudaStream_t st) {
+  if (LSB && p.dec_flag) {
+    // predicated: the MSB planes for every row, the decision, the LSB planes for the flagged rows
+    SPT_TRY((launch_items<DH, QT, false, false>(p, st)));
+    attn_decode_flag_kernel<<<dim3(p.a.H_kept, p.a.B), 32, 0, st>>>(p);
+    SPT_TRY(launch_status());
+    SPT_TRY((launch_items<DH, QT, true, true>(p, st)));
+  } else {
+    SPT_TRY((launch_items<DH, QT, LSB, false>(p, st)));
+  }
   const int nblk = static_cast<int>(ceil_div(p.a.n_kv, kCThreads));
   const int slots = p.a.H_kept + (p.a.zero_pruned_heads ? p.a.H - p.a.H_kept : 0);
   attn_decode_combine_kernel<DH, QT, LSB>

@@ -21,7 +21,7 @@ lib = C.CDLL(LIB_PATH)
 OK, E_ARG, E_SHAPE, E_ALIGN, E_WORKSPACE, E_NONFINITE, E_CUDA, E_TIMEOUT, E_UNSUPPORTED, E_INDEX, E_RANGE = range(11)
 F32, BF16 = 0, 1
 PREFILL, DECODE_STEP = 0, 1
-ATTN_AUTO, ATTN_CUDA_CORE, ATTN_TENSOR_CORE, ATTN_DECODE = 0, 1, 2, 3
+ATTN_AUTO, ATTN_CUDA_CORE, ATTN_TENSOR_CORE, ATTN_DECODE, ATTN_DECODE_PREDICATED = 0, 1, 2, 3, 4
 MAX_LAYERS = 64
 
 vp, i32, i64, f32, sz = C.c_void_p, C.c_int32, C.c_int64, C.c_float, C.c_size_t

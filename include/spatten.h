@@ -185,7 +185,13 @@ enum spatten_attn_kernel {
   SPATTEN_ATTN_AUTO = 0,
   SPATTEN_ATTN_CUDA_CORE = 1,
   SPATTEN_ATTN_TENSOR_CORE = 2,
-  SPATTEN_ATTN_DECODE = 3
+  SPATTEN_ATTN_DECODE = 3,
+  /* the decode kernel with a predicated LSB fetch (theta > 0): a first pass over the MSB planes of
+   * every row, the refetch decision per row, then a full-precision pass that reads the LSB planes
+   * of the flagged rows only (their MSB planes again, usually from L2).  The results are the
+   * same, bit for bit, as SPATTEN_ATTN_DECODE's; it reads fewer bytes when few rows refetch and
+   * costs a second pass when most do. */
+  SPATTEN_ATTN_DECODE_PREDICATED = 4
 };
 
 size_t spatten_attention_workspace_size(const spatten_attn_args* a);

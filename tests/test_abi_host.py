@@ -144,7 +144,7 @@ def test_attention_argument_errors_and_workspace(S):
     assert L.spatten_attention_workspace_size(C.byref(_attn(S))) > 0
     for over, want in [(dict(d_h=96), S.E_UNSUPPORTED), (dict(H_kept=5), S.E_ARG), (dict(H_kept=3), S.E_ARG),
                        (dict(q=0), S.E_ARG), (dict(q_ld_tok=100), S.E_SHAPE), (dict(kv_cap=50), S.E_SHAPE),
-                       (dict(q=(1 << 20) + 8), S.E_ALIGN), (dict(kernel=9), S.E_ARG), (dict(v_keep=-1), S.E_ARG)]:
+                       (dict(q=(1 << 20) + 8), S.E_ALIGN), (dict(kernel=9), S.E_ARG), (dict(kernel=5), S.E_ARG), (dict(v_keep=-1), S.E_ARG)]:
         assert L.spatten_attention_layer(C.byref(_attn(S, **over)), 1 << 24, 1 << 30, None) == want, over
     # workspace too small
     assert L.spatten_attention_layer(C.byref(_attn(S)), 1 << 24, 16, None) == S.E_WORKSPACE
@@ -155,6 +155,13 @@ def test_attention_argument_errors_and_workspace(S):
     assert L.spatten_attention_workspace_size(C.byref(_attn(S, v_keep=100))) == base
     # a forced kernel that cannot run the problem
     assert L.spatten_attention_layer(C.byref(_attn(S, kernel=S.ATTN_DECODE)), 1 << 24, 1 << 30, None) == S.E_UNSUPPORTED
+    assert (L.spatten_attention_layer(C.byref(_attn(S, kernel=S.ATTN_DECODE_PREDICATED)), 1 << 24, 1 << 30, None)
+            == S.E_UNSUPPORTED)
+    # the predicated decode form keeps one refetch flag per (sequence, kept head) when theta > 0
+    size = lambda **o: L.spatten_attention_workspace_size(C.byref(_attn(S, n_q=1, **o)))
+    single = size(kernel=S.ATTN_DECODE, refetch_threshold=0.1)
+    assert size(kernel=S.ATTN_DECODE_PREDICATED, refetch_threshold=0.1) >= single + 2 * 4 * 4
+    assert size(kernel=S.ATTN_DECODE_PREDICATED, refetch_threshold=0.0) == size(kernel=S.ATTN_DECODE, refetch_threshold=0.0)
 
 
 def test_cascade_cfg_checks_and_workspace(S):

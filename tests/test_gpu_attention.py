@@ -223,6 +223,41 @@ def test_attention_decode_index_listed(cuda, kernel, d, theta, cap, n_kv, keep):
         assert np.all(got["tok"][b, mask] == 0)
 
 
+@pytest.mark.parametrize("d,cap,n_kv,keep", [(64, 1300, 1153, None), (128, 700, 611, [0, 2, 3]), (64, 300, 7, None)])
+def test_decode_predicated_lsb_fetch(cuda, d, cap, n_kv, keep):
+    """SPATTEN_ATTN_DECODE_PREDICATED: the MSB planes of every row, the refetch decision, then the
+    LSB planes of the flagged rows only.  With a threshold at which some rows refetch and others
+    do not, its outputs, importances, flags and count are bit-identical to the single-pass decode
+    kernel's (SPATTEN_ATTN_DECODE), and they match the oracle; at theta 0 it is the MSB pass."""
+    S = lib()
+    B, H = 4, 4
+    g = synth.rng_for(7 * d + n_kv)
+    raw, gain = make_layer(B, H, cap, d, seed=41 + d, boost=max(1, cap // 12))
+    kv_idx = np.stack([np.sort(g.choice(cap, n_kv, replace=False)) for _ in range(B)]).astype(np.int32)
+    heads = None if keep is None else np.array([keep] * B, np.int32)
+    rows = B * (H if keep is None else len(keep))
+    # a threshold between the rows' MSB-pass maximum probabilities: some rows refetch, some not
+    theta, single = None, None
+    for t in (0.5, 0.3, 0.2, 0.1, 0.05, 0.02, 0.01, 0.005, 0.002):
+        single = run_layer(S, raw, gain, B, H, cap, d, t, heads=heads, kernel=S.ATTN_DECODE, kv_idx=kv_idx, n_q=1)
+        if 0 < single["count"] < rows:
+            theta = t
+            break
+    assert theta is not None, "no threshold splits the rows"
+    pred = run_layer(S, raw, gain, B, H, cap, d, theta, heads=heads, kernel=S.ATTN_DECODE_PREDICATED,
+                     kv_idx=kv_idx, n_q=1)
+    print(f"theta {theta}: {single['count']} of {rows} rows refetch")
+    for key in ("o", "tok", "head", "flags", "count", "status"):
+        np.testing.assert_array_equal(pred[key], single[key])
+    ref = oracle_layer(raw, gain, B, H, cap, d, theta, heads, BF, pred, kv_idx=kv_idx, n_q=1)
+    check(pred, ref, heads, H, d, 2e-2, 1e-2, "decode (predicated)")
+    zero = run_layer(S, raw, gain, B, H, cap, d, 0.0, heads=heads, kernel=S.ATTN_DECODE_PREDICATED, kv_idx=kv_idx,
+                     n_q=1)
+    zero_single = run_layer(S, raw, gain, B, H, cap, d, 0.0, heads=heads, kernel=S.ATTN_DECODE, kv_idx=kv_idx, n_q=1)
+    for key in ("o", "tok", "head", "count"):
+        np.testing.assert_array_equal(zero[key], zero_single[key])
+
+
 def test_attention_deterministic(cuda):
     S = lib()
     B, H, n, d = 2, 6, 300, 64
