@@ -206,3 +206,23 @@ def test_cascade_deterministic(cuda):
     hb = host(a)
     for key in ("x_out", "kept_tok", "kept_head", "tok_imp", "head_imp", "refetch"):
         np.testing.assert_array_equal(ha[key], hb[key])
+
+
+def test_cascade_untraced_equals_traced(cuda):
+    """Without traces the importance reduction and the next layer's selections run on the
+    library's second stream, beside the output projection; with traces they stay on the caller's
+    stream.  Both orders give bit-identical results (the same kernels in the same data order)."""
+    S = lib()
+    from fractions import Fraction
+    w = synth.PrefillWorkload("side", B=4, T=256, D=768, H=12, d_h=64, L=5, dtype="bf16",
+                              token_keep=synth.geometric_keep(256, Fraction(9, 10), 5), head_keep=[12, 12, 11, 11, 10],
+                              quant=True, theta=0.1, boost=("uniform", 13, 4.0))
+    d = synth.draw_prefill(w)
+    a = upload_prefill(S, w, d, trace=False)
+    run_prefill(S, a)
+    plain = host(a)
+    t = upload_prefill(S, w, d, trace=True)
+    run_prefill(S, t)
+    traced = host(t)
+    for key in ("x_out", "kept_tok", "kept_head", "tok_imp", "head_imp", "refetch"):
+        np.testing.assert_array_equal(plain[key], traced[key])
