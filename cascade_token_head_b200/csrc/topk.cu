@@ -12,9 +12,9 @@
 //                  through distributed shared memory.  Each CTA keeps up to kResident keys of its
 //                  chunk in shared memory; the rest is streamed again from L2 in every pass.
 //   n >= 65536 with the caller's workspace (sample / filter / resolve / output kernels): a
-//                  sampled rank window around the k-th key, one streaming pass that counts the keys
-//                  above the window and collects the window's keys, an exact select among those
-//                  candidates, one streaming pass that writes the output (see the section below).
+//                  sampled rank window around the k-th key, one streaming pass that marks the keys
+//                  above the window in a bit mask and collects the window's keys, an exact select among those
+//                  candidates, an output pass over that pass's bit mask (see the section below).
 // In every form a key is kept if it is above the threshold T, or equal to T and among the first
 // (k - #above) equal keys in index order (ties go to the lower index), and warp ballots / block
 // scans give each kept key its output slot in ascending index order.
@@ -504,8 +504,9 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 }
 
 // ------------------------------------------------------------------------------------------------
-// Long rows (n >= kStreamMin, scores read directly, caller workspace given): two streaming passes
-// over the scores, with two one-CTA-per-row steps on small data between them.
+// Long rows (n >= kStreamMin, scores read directly, caller workspace given): one streaming pass
+// over the scores between a sample and an exact select on small data (one CTA per row each), then
+// an output pass over the pass's bit mask and candidates.
 //  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256) and finds by a digit
 //           search the sample keys e0 >= e64 at the two ends of a rank window around the sample
 //           rank of the k-th key (+-4 sigma of the sampling error + 16; an end past the sample is
@@ -518,15 +519,17 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 //  resolve  one CTA per row: the sub-bin holding the k-th key, the exact threshold among that
 //           sub-bin's candidates as the (need)-th largest (key, ~index) composite (ties to the lower
 //           index), whether the keys equal to T are split by index, and every chunk's output offset
-//  output   per chunk: key > T, or key = T and index <= T_index (key >= T when the keys equal to T
-//           are all taken), written in index order
+//  output   per chunk: the filter's bit mask of the keys above the window, plus the chunk's
+//           candidates with key > T, or key = T and index <= T_index, written in index order (the
+//           scores are not read again)
 // A row whose k-th key fell outside the window, or whose buffers overflowed, is marked and done
 // again by the cluster kernel (only_rows).
 // The filter reads a warp's 512 keys as four coalesced 16-byte loads per lane (load q of lane t
-// holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span); the output step reads them as 16
-// columns of 32 (see there).  Both compare floats against the window ends and the threshold turned
-// back into floats (the key map is monotone, and -0.0 equals +0.0 on both sides); a NaN fails every
-// ordered comparison, lands in the candidate list and is reported by the resolve step.
+// holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span) and compares floats against the
+// window ends turned back into floats (the key map is monotone, and -0.0 equals +0.0 on both
+// sides); a NaN fails every ordered comparison, lands in the candidate list and is reported by the
+// resolve step.  Its above-window bits go out in index order, one 32-bit word per 32 keys, so the
+// output step only adds the selected candidates' bits and turns each word into indices.
 // ------------------------------------------------------------------------------------------------
 constexpr int kStreamMin = 65536;
 constexpr int kSRuns = 64, kSRun = 256, kSamples = kSRuns * kSRun;   // 16 K sample keys per row
@@ -550,7 +553,10 @@ struct StreamWs {
   uint32_t* hist;       // [R][nchunk][kBins]   candidates of each chunk per sub-bin
   uint2* cand;          // [R][cap]  (score bits, index)
   uint32_t* chunk_off;  // [R][nchunk]
-  uint32_t* res;        // [R][4]   valid, T key, T index, keys equal to T split by index
+  uint32_t* gtmask;     // [R][nchunk][kChunk / 32]  bit j % 32 of word j / 32: chunk key j is above
+                        //            the window
+  uint2* chunk_cand;    // [R][nchunk]  (first slot, count) of the chunk's candidates in cand
+  uint32_t* res;        // [R][4]   valid, T key, T index, unused
   int32_t* fallback;    // [R]
   int cap, nchunk;
 };
@@ -792,18 +798,19 @@ __device__ __forceinline__ void load_span(const float* row, int jw, int n, float
 
 __device__ __forceinline__ int span_off(int u) { return 128 * (u >> 2) + (u & 3); }
 
-// count above fe0 and the candidate mask (bit u: f[u] in [fe64, fe0], or NaN)
+// the above-window mask (bit u: f[u] > fe0) and the candidate mask (bit u: f[u] in [fe64, fe0],
+// or NaN) of one lane's kFKeys keys
 template <bool FULL>
-__device__ __forceinline__ void filter_span(const float* row, int jw, int n, float fe0, float fe64, uint32_t& gt,
+__device__ __forceinline__ void filter_span(const float* row, int jw, int n, float fe0, float fe64, uint32_t& gm,
                                             uint32_t& cm) {
   float f[kFKeys];
   load_span<FULL>(row, jw, n, f);
-  gt = 0u;
+  gm = 0u;
   cm = 0u;
 #pragma unroll
   for (int u = 0; u < kFKeys; ++u) {
     if (FULL || span_off(u) < n - jw) {
-      gt += f[u] > fe0 ? 1u : 0u;
+      if (f[u] > fe0) gm |= 1u << u;
       if (!(f[u] < fe64 || f[u] > fe0)) cm |= 1u << u;
     }
   }
@@ -819,9 +826,24 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, Stre
   const BinMap bm{en.z, en.w};
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   const int jw = c * kChunk + warp * (32 * kFKeys) + 4 * lane;
-  uint32_t gt, cm;
-  if ((c + 1) * kChunk <= a.n) filter_span<true>(row, jw, a.n, fe0, fe64, gt, cm);
-  else filter_span<false>(row, jw, a.n, fe0, fe64, gt, cm);
+  const int64_t rc = static_cast<int64_t>(r) * w.nchunk + c;
+  uint32_t gm, cm;
+  if ((c + 1) * kChunk <= a.n) filter_span<true>(row, jw, a.n, fe0, fe64, gm, cm);
+  else filter_span<false>(row, jw, a.n, fe0, fe64, gm, cm);
+  {
+    // load q of lanes 8 g .. 8 g + 7 covers word 4 q + g of the warp's 16 (32 keys each), lane
+    // 8 g + i at bits 4 i .. 4 i + 3
+    uint32_t* dst = w.gtmask + rc * (kChunk / 32) + warp * kFKeys;
+#pragma unroll
+    for (int q = 0; q < kFKeys / 4; ++q) {
+      uint32_t v = ((gm >> (4 * q)) & 0xFu) << (4 * (lane & 7));
+      v |= __shfl_xor_sync(0xffffffffu, v, 1);
+      v |= __shfl_xor_sync(0xffffffffu, v, 2);
+      v |= __shfl_xor_sync(0xffffffffu, v, 4);
+      if ((lane & 7) == 0) dst[4 * q + (lane >> 3)] = v;
+    }
+  }
+  uint32_t gt = __popc(gm);
   const uint32_t nc = __popc(cm);
   uint32_t inc = nc;
 #pragma unroll
@@ -845,12 +867,14 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, Stre
     const uint32_t g = __reduce_add_sync(0xffffffffu, lane < kFWarps ? wg[lane] : 0u);
     uint32_t base = 0u;
     if (lane == 0) {
-      w.chunk_gt[static_cast<int64_t>(r) * w.nchunk + c] = g;
+      w.chunk_gt[rc] = g;
       if (tot) base = atomicAdd(&w.ccount[r], tot);
     }
     base = __shfl_sync(0xffffffffu, base, 0);
     // a chunk whose candidates would pass the list's end writes none (the row falls back)
-    if (lane < kFWarps) wb[lane] = base + tot <= static_cast<uint32_t>(w.cap) ? base + xi - x : 0xFFFFFFFFu;
+    const bool fits = base + tot <= static_cast<uint32_t>(w.cap);
+    if (lane == 0) w.chunk_cand[rc] = make_uint2(fits ? base : 0u, fits ? tot : 0u);
+    if (lane < kFWarps) wb[lane] = fits ? base + xi - x : 0xFFFFFFFFu;
   }
   __syncthreads();
   const uint32_t wbase = wb[warp];
@@ -867,7 +891,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, Stre
     }
   }
   __syncthreads();
-  if (tid < kBins) w.hist[(static_cast<int64_t>(r) * w.nchunk + c) * kBins + tid] = hist[tid];
+  if (tid < kBins) w.hist[rc * kBins + tid] = hist[tid];
 }
 
 // exclusive prefix sum over a 1024-thread block (part: [32] scratch, free again after return)
@@ -1005,7 +1029,6 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
   const uint32_t need = k - above_s;   // 1 <= need <= m
   // T = the need-th largest composite; the selected ones of the sub-bin are counted per chunk
   uint64_t T;
-  bool split = true;   // without the count below the output takes the exact test
   if (m <= static_cast<uint32_t>(kRThreads)) {   // uniform: sort the sub-bin
     uint64_t x = tid < static_cast<int>(m) ? bc[tid] : 0ull;   // 0: below every composite
     x = bitonic_desc_1024(x, bc);
@@ -1016,10 +1039,6 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     if (s && lane == __ffs(grp) - 1) atomicAdd(&cnt[chunk], __popc(grp));
     __syncthreads();
     T = t_s;
-    // are the keys equal to T's split by index (some above T, some below)?
-    const bool eq = tid < static_cast<int>(m) && static_cast<uint32_t>(x >> 32) == static_cast<uint32_t>(T >> 32);
-    const int n_eq = __syncthreads_count(eq), n_eq_sel = __syncthreads_count(eq && tid < static_cast<int>(need));
-    split = n_eq_sel < n_eq;
   } else {
     // two bits per round (the largest T with count(>= T) >= need)
     uint64_t v[kBinCap / kRThreads];
@@ -1087,71 +1106,83 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     rr[0] = 1u;
     rr[1] = t_key;
     rr[2] = t_idx;
-    rr[3] = split ? 1u : 0u;
+    rr[3] = 0u;
     w.fallback[r] = 0;
   }
 }
 
-// The output step reads a warp's 512 keys as 16 columns of 32 consecutive keys (lane t of column
-// c: key 32 c + t of the warp's span), so each column's selection is one ballot and its selected
-// indices go out as one coalesced store in index order.  Selection: f >= T when no key equal to T
-// lies past T_index (EXACT false), else f > T, or f == T and index <= T_index.
-template <bool FULL, bool EXACT>
-__device__ __forceinline__ void select_cols(const float* row, int span, int n, float tf, uint32_t t_idx, uint32_t* m) {
-  const int lane = threadIdx.x & 31;
-  float f[kFKeys];
-#pragma unroll
-  for (int col = 0; col < kFKeys; ++col) {
-    const int j = span + 32 * col + lane;
-    f[col] = (FULL || j < n) ? __ldg(row + j) : __int_as_float(0x7FFFFFFF);   // NaN: never selected
-  }
-#pragma unroll
-  for (int col = 0; col < kFKeys; ++col) {
-    const uint32_t j = static_cast<uint32_t>(span + 32 * col + lane);
-    const bool sel = EXACT ? (f[col] > tf || (f[col] == tf && j <= t_idx)) : f[col] >= tf;
-    m[col] = __ballot_sync(0xffffffffu, sel);
-  }
-}
-
+// The output step: the chunk's above-window words (from the filter) in shared memory, the bits of
+// its selected candidates (key > T, or key = T and index <= T_index) added; warp w turns words
+// 16 w .. 16 w + 15 (keys 512 w .. 512 w + 511 of the chunk) into indices, staged in shared memory
+// in index order at the output's 16-byte phase; the block then writes the chunk's run of indices
+// with aligned 16-byte stores (scalar stores only at the run's two ragged ends).
 __global__ void __launch_bounds__(kFThreads, 4) topk_output_kernel(TArgs a, StreamWs w) {
+  __shared__ __align__(16) uint32_t sel[kChunk / 32];
+  __shared__ __align__(16) int32_t stage[kChunk + 4];
   __shared__ uint32_t wc[kFWarps];
   const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t* rr = w.res + static_cast<int64_t>(r) * 4;
   if (!rr[0]) return;   // uniform: the row is redone by the fallback
-  const float tf = key_float(rr[1]);
-  const uint32_t t_idx = rr[2];
-  const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
-  const int span = c * kChunk + warp * (32 * kFKeys);
-  const bool full = (c + 1) * kChunk <= a.n;
-  uint32_t m[kFKeys];
-  if (rr[3]) {
-    if (full) select_cols<true, true>(row, span, a.n, tf, t_idx, m);
-    else select_cols<false, true>(row, span, a.n, tf, t_idx, m);
-  } else {
-    if (full) select_cols<true, false>(row, span, a.n, tf, t_idx, m);
-    else select_cols<false, false>(row, span, a.n, tf, t_idx, m);
+  const uint32_t t_key = rr[1], t_idx = rr[2];
+  const int64_t rc = static_cast<int64_t>(r) * w.nchunk + c;
+  if (tid < kChunk / 32) sel[tid] = w.gtmask[rc * (kChunk / 32) + tid];
+  __syncthreads();
+  const uint2 cc = w.chunk_cand[rc];
+  const uint2* cand = w.cand + static_cast<int64_t>(r) * w.cap + cc.x;
+  const uint32_t j0 = static_cast<uint32_t>(c) * kChunk;
+  for (uint32_t i = tid; i < cc.y; i += kFThreads) {
+    const uint2 e = cand[i];
+    const uint32_t key = float_key(__uint_as_float(e.x));
+    if (key > t_key || (key == t_key && e.y <= t_idx)) {
+      const uint32_t p = e.y - j0;   // < kChunk: the filter listed the chunk's own keys
+      atomicOr(&sel[p >> 5], 1u << (p & 31));
+    }
   }
+  __syncthreads();
+  const uint4* words = reinterpret_cast<const uint4*>(&sel[warp * kFKeys]);   // four words per load
   uint32_t cw = 0u;
 #pragma unroll
-  for (int col = 0; col < kFKeys; ++col) cw += __popc(m[col]);
+  for (int g = 0; g < kFKeys / 4; ++g) {
+    const uint4 v = words[g];
+    cw += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+  }
   if (lane == 0) wc[warp] = cw;
   __syncthreads();
-  uint32_t pos = w.chunk_off[static_cast<int64_t>(r) * w.nchunk + c] +
-                 __reduce_add_sync(0xffffffffu, lane < warp ? wc[lane] : 0u);
+  const uint32_t total = __reduce_add_sync(0xffffffffu, lane < kFWarps ? wc[lane] : 0u);
+  const uint32_t off = w.chunk_off[rc];
   int32_t* out = a.idx_out + static_cast<int64_t>(r) * a.ld_out;
-  const uint32_t kk = static_cast<uint32_t>(a.k), bit = 1u << lane, lt = bit - 1u;
-  if (pos + cw <= kk) {   // warp-uniform; always, when the counts agree
+  // the output position off + i goes to stage[ph + i], ph = (off + i) - i mod 4 in words of the
+  // destination address, so 16-byte groups of the output are 16-byte groups of the stage
+  const uint32_t ph = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(out + off) >> 2) & 3u;
+  {
+    uint32_t pos = ph + __reduce_add_sync(0xffffffffu, lane < warp ? wc[lane] : 0u);
+    const int span = c * kChunk + warp * (32 * kFKeys);
+    const uint32_t bit = 1u << lane, lt = bit - 1u;
 #pragma unroll
-    for (int col = 0; col < kFKeys; ++col) {
-      if (m[col] & bit) out[pos + __popc(m[col] & lt)] = span + 32 * col + lane;
-      pos += __popc(m[col]);
+    for (int g = 0; g < kFKeys / 4; ++g) {
+      const uint4 v = words[g];
+      const uint32_t m4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (m4[u] & bit) stage[pos + __popc(m4[u] & lt)] = span + 32 * (4 * g + u) + lane;
+        pos += __popc(m4[u]);
+      }
     }
-  } else {
+  }
+  __syncthreads();
+  // never past k (always within, when the counts agree)
+  const uint32_t kk = static_cast<uint32_t>(a.k);
+  const uint32_t cnt = off >= kk ? 0u : min(total, kk - off);
+  const uint32_t end = ph + cnt;
+  int32_t* base = out + off - ph;   // 16-byte aligned; written only at [ph, end)
+  for (uint32_t v = tid; 4 * v < end; v += kFThreads) {
+    const uint32_t p = 4 * v;
+    if (p >= ph && p + 4 <= end) {
+      reinterpret_cast<int4*>(base)[v] = *reinterpret_cast<const int4*>(&stage[p]);
+    } else {
 #pragma unroll
-    for (int col = 0; col < kFKeys; ++col) {
-      const uint32_t p = pos + __popc(m[col] & lt);
-      if ((m[col] & bit) && p < kk) out[p] = span + 32 * col + lane;
-      pos += __popc(m[col]);
+      for (uint32_t u = 0; u < 4; ++u)
+        if (p + u >= ph && p + u < end) base[p + u] = stage[p + u];
     }
   }
 }
@@ -1172,6 +1203,8 @@ size_t stream_ws_bytes(int R, int n) {
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_gt
   take(static_cast<size_t>(R) * nchunk * kBins * 4);   // hist
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_off
+  take(static_cast<size_t>(R) * nchunk * (kChunk / 8)); // gtmask
+  take(static_cast<size_t>(R) * nchunk * 8);           // chunk_cand
   take(static_cast<size_t>(R) * 16);                   // res
   take(static_cast<size_t>(R) * 4);                    // fallback
   take(static_cast<size_t>(R) * stream_cap(n) * 8);    // cand
@@ -1211,6 +1244,8 @@ int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaSt
   v.chunk_gt += static_cast<int64_t>(r0) * w.nchunk;
   v.hist += static_cast<int64_t>(r0) * w.nchunk * kBins;
   v.chunk_off += static_cast<int64_t>(r0) * w.nchunk;
+  v.gtmask += static_cast<int64_t>(r0) * w.nchunk * (kChunk / 32);
+  v.chunk_cand += static_cast<int64_t>(r0) * w.nchunk;
   v.res += static_cast<int64_t>(r0) * 4;
   v.fallback += r0;
   v.cand += static_cast<int64_t>(r0) * w.cap;
@@ -1247,6 +1282,8 @@ int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
   w.chunk_gt = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
   w.hist = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * kBins * 4));
   w.chunk_off = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
+  w.gtmask = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * (kChunk / 8)));
+  w.chunk_cand = reinterpret_cast<uint2*>(take(static_cast<size_t>(R) * w.nchunk * 8));
   w.res = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * 16));
   w.fallback = reinterpret_cast<int32_t*>(take(static_cast<size_t>(R) * 4));
   w.cand = reinterpret_cast<uint2*>(take(static_cast<size_t>(R) * w.cap * 8));

@@ -322,8 +322,8 @@ def test_topk_long_rows_bracket_misses_fall_back(cuda, with_ws):
 
 def test_topk_long_rows_tie_group_at_threshold(cuda):
     """Long rows on the streaming path whose k-th value is shared by eight keys: the selection takes
-    one, three, four or all eight of them, always the lowest indices of the group (the tie rule),
-    so the output step meets both its split-tie and its whole-group test.  Bit-exact."""
+    one, three, four or all eight of them, always the lowest indices of the group (the tie rule):
+    the threshold either splits the group by index or takes it whole.  Bit-exact."""
     S = lib()
     g = synth.rng_for(78)
     R_, n, k = 4, 131072, 40000
