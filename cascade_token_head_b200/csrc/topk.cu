@@ -519,17 +519,19 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 //  resolve  one CTA per row: the sub-bin holding the k-th key, the exact threshold among that
 //           sub-bin's candidates as the (need)-th largest (key, ~index) composite (ties to the lower
 //           index), whether the keys equal to T are split by index, and every chunk's output offset
-//  output   per chunk: the filter's bit mask of the keys above the window, plus the chunk's
-//           candidates with key > T, or key = T and index <= T_index, written in index order (the
-//           scores are not read again)
+//           It also sets the mask bits of the selected candidates: every candidate of the sub-bins
+//           above T's, and T's own selected part.
+//  output   per chunk: the indices of the mask's set bits, written in index order (the scores are
+//           not read again)
 // A row whose k-th key fell outside the window, or whose buffers overflowed, is marked and done
 // again by the cluster kernel (only_rows).
 // The filter reads a warp's 512 keys as four coalesced 16-byte loads per lane (load q of lane t
 // holds keys 128 q + 4 t .. 128 q + 4 t + 3 of the warp's span) and compares floats against the
 // window ends turned back into floats (the key map is monotone, and -0.0 equals +0.0 on both
 // sides); a NaN fails every ordered comparison, lands in the candidate list and is reported by the
-// resolve step.  Its above-window bits go out in index order, one 32-bit word per 32 keys, so the
-// output step only adds the selected candidates' bits and turns each word into indices.
+// resolve step.  Its above-window bits go out in index order, one 32-bit word per 32 keys; the
+// resolve step adds the selected candidates' bits, and the output step turns each word into
+// indices.
 // ------------------------------------------------------------------------------------------------
 constexpr int kStreamMin = 65536;
 constexpr int kSRuns = 64, kSRun = 256, kSamples = kSRuns * kSRun;   // 16 K sample keys per row
@@ -553,9 +555,8 @@ struct StreamWs {
   uint32_t* hist;       // [R][nchunk][kBins]   candidates of each chunk per sub-bin
   uint2* cand;          // [R][cap]  (score bits, index)
   uint32_t* chunk_off;  // [R][nchunk]
-  uint32_t* gtmask;     // [R][nchunk][kChunk / 32]  bit j % 32 of word j / 32: chunk key j is above
-                        //            the window
-  uint2* chunk_cand;    // [R][nchunk]  (first slot, count) of the chunk's candidates in cand
+  uint32_t* gtmask;     // [R][nchunk][kChunk / 32]  bit j % 32 of word j / 32 (row key j): above the
+                        //            window (filter), or a selected candidate (resolve)
   uint32_t* res;        // [R][4]   valid, T key, T index, unused
   int32_t* fallback;    // [R]
   int cap, nchunk;
@@ -872,9 +873,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, Stre
     }
     base = __shfl_sync(0xffffffffu, base, 0);
     // a chunk whose candidates would pass the list's end writes none (the row falls back)
-    const bool fits = base + tot <= static_cast<uint32_t>(w.cap);
-    if (lane == 0) w.chunk_cand[rc] = make_uint2(fits ? base : 0u, fits ? tot : 0u);
-    if (lane < kFWarps) wb[lane] = fits ? base + xi - x : 0xFFFFFFFFu;
+    if (lane < kFWarps) wb[lane] = base + tot <= static_cast<uint32_t>(w.cap) ? base + xi - x : 0xFFFFFFFFu;
   }
   __syncthreads();
   const uint32_t wbase = wb[warp];
@@ -994,10 +993,12 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     stream_fail(w, r);
     return;
   }
-  // the sub-bin's candidates as (key, ~index) composites; the one pass over the candidate list,
-  // which also looks for NaNs (they pass the filter)
+  // the one pass over the candidate list: the sub-bins above js are selected whole (their mask
+  // bits set), sub-bin js is collected as (key, ~index) composites; NaNs (they pass the filter) are
+  // looked for on the way
   const BinMap bm{w.ends[4 * r + 2], w.ends[4 * r + 3]};
   const uint2* cand = w.cand + static_cast<int64_t>(r) * w.cap;
+  uint32_t* mrow = w.gtmask + static_cast<int64_t>(r) * nchunk * (kChunk / 32);
   const uint32_t lt_mask = (1u << lane) - 1u;
   bool nan_seen = false;
   for (uint32_t i0 = 0; i0 < ncand; i0 += BP * kRThreads) {
@@ -1011,7 +1012,10 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     for (int u = 0; u < BP; ++u) {
       const float f = __uint_as_float(cd[u].x);
       nan_seen |= f != f;
-      const bool hit = i0 + tid + u * kRThreads < ncand && bin_of(f, bm) == js;
+      const bool live = i0 + tid + u * kRThreads < ncand;
+      const int b = bin_of(f, bm);
+      if (live && b < js) atomicOr(&mrow[cd[u].y >> 5], 1u << (cd[u].y & 31u));
+      const bool hit = live && b == js;
       const uint32_t m = __ballot_sync(0xffffffffu, hit);
       if (m) {
         const int leader = __ffs(m) - 1;
@@ -1034,7 +1038,9 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     x = bitonic_desc_1024(x, bc);
     if (tid == static_cast<int>(need) - 1) t_s = x;
     const bool s = tid < static_cast<int>(min(need, m));
-    const uint32_t chunk = s ? (~static_cast<uint32_t>(x)) / kChunk : 0xFFFFFFFFu;
+    const uint32_t j = ~static_cast<uint32_t>(x);
+    if (s) atomicOr(&mrow[j >> 5], 1u << (j & 31u));
+    const uint32_t chunk = s ? j / kChunk : 0xFFFFFFFFu;
     const uint32_t grp = __match_any_sync(0xffffffffu, chunk);
     if (s && lane == __ffs(grp) - 1) atomicAdd(&cnt[chunk], __popc(grp));
     __syncthreads();
@@ -1075,7 +1081,9 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
 #pragma unroll
     for (int u = 0; u < kBinCap / kRThreads; ++u) {
       const bool s = u < nv && v[u] >= T && v[u] != 0ull;
-      const uint32_t chunk = s ? (~static_cast<uint32_t>(v[u])) / kChunk : 0xFFFFFFFFu;
+      const uint32_t j = ~static_cast<uint32_t>(v[u]);
+      if (s) atomicOr(&mrow[j >> 5], 1u << (j & 31u));
+      const uint32_t chunk = s ? j / kChunk : 0xFFFFFFFFu;
       const uint32_t grp = __match_any_sync(0xffffffffu, chunk);
       if (s && lane == __ffs(grp) - 1) atomicAdd(&cnt[chunk], __popc(grp));
     }
@@ -1111,45 +1119,28 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
   }
 }
 
-// The output step: the chunk's above-window words (from the filter) in shared memory, the bits of
-// its selected candidates (key > T, or key = T and index <= T_index) added; warp w turns words
-// 16 w .. 16 w + 15 (keys 512 w .. 512 w + 511 of the chunk) into indices, staged in shared memory
-// in index order at the output's 16-byte phase; the block then writes the chunk's run of indices
-// with aligned 16-byte stores (scalar stores only at the run's two ragged ends).
+// The output step: warp w turns the chunk's selection words 16 w .. 16 w + 15 (keys 512 w ..
+// 512 w + 511 of the chunk) into indices, staged in shared memory in index order at the output's
+// 16-byte phase; the block then writes the chunk's run of indices with aligned 16-byte stores
+// (scalar stores only at the run's two ragged ends).  Its global reads (the threshold record, the
+// words, the chunk's output offset) are independent of one another.
 __global__ void __launch_bounds__(kFThreads, 4) topk_output_kernel(TArgs a, StreamWs w) {
   __shared__ __align__(16) uint32_t sel[kChunk / 32];
   __shared__ __align__(16) int32_t stage[kChunk + 4];
   __shared__ uint32_t wc[kFWarps];
   const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t* rr = w.res + static_cast<int64_t>(r) * 4;
-  if (!rr[0]) return;   // uniform: the row is redone by the fallback
-  const uint32_t t_key = rr[1], t_idx = rr[2];
   const int64_t rc = static_cast<int64_t>(r) * w.nchunk + c;
-  if (tid < kChunk / 32) sel[tid] = w.gtmask[rc * (kChunk / 32) + tid];
-  __syncthreads();
-  const uint2 cc = w.chunk_cand[rc];
-  const uint2* cand = w.cand + static_cast<int64_t>(r) * w.cap + cc.x;
-  const uint32_t j0 = static_cast<uint32_t>(c) * kChunk;
-  for (uint32_t i = tid; i < cc.y; i += kFThreads) {
-    const uint2 e = cand[i];
-    const uint32_t key = float_key(__uint_as_float(e.x));
-    if (key > t_key || (key == t_key && e.y <= t_idx)) {
-      const uint32_t p = e.y - j0;   // < kChunk: the filter listed the chunk's own keys
-      atomicOr(&sel[p >> 5], 1u << (p & 31));
-    }
-  }
-  __syncthreads();
+  const uint32_t valid = w.res[static_cast<int64_t>(r) * 4];
+  const uint32_t word = lane < kFKeys ? w.gtmask[rc * (kChunk / 32) + warp * kFKeys + lane] : 0u;
+  const uint32_t off = w.chunk_off[rc];
+  if (!valid) return;   // uniform: the row is redone by the fallback
+  if (lane < kFKeys) sel[warp * kFKeys + lane] = word;
+  __syncwarp();
   const uint4* words = reinterpret_cast<const uint4*>(&sel[warp * kFKeys]);   // four words per load
-  uint32_t cw = 0u;
-#pragma unroll
-  for (int g = 0; g < kFKeys / 4; ++g) {
-    const uint4 v = words[g];
-    cw += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
-  }
+  const uint32_t cw = __reduce_add_sync(0xffffffffu, __popc(word));
   if (lane == 0) wc[warp] = cw;
   __syncthreads();
   const uint32_t total = __reduce_add_sync(0xffffffffu, lane < kFWarps ? wc[lane] : 0u);
-  const uint32_t off = w.chunk_off[rc];
   int32_t* out = a.idx_out + static_cast<int64_t>(r) * a.ld_out;
   // the output position off + i goes to stage[ph + i], ph = (off + i) - i mod 4 in words of the
   // destination address, so 16-byte groups of the output are 16-byte groups of the stage
@@ -1204,7 +1195,6 @@ size_t stream_ws_bytes(int R, int n) {
   take(static_cast<size_t>(R) * nchunk * kBins * 4);   // hist
   take(static_cast<size_t>(R) * nchunk * 4);           // chunk_off
   take(static_cast<size_t>(R) * nchunk * (kChunk / 8)); // gtmask
-  take(static_cast<size_t>(R) * nchunk * 8);           // chunk_cand
   take(static_cast<size_t>(R) * 16);                   // res
   take(static_cast<size_t>(R) * 4);                    // fallback
   take(static_cast<size_t>(R) * stream_cap(n) * 8);    // cand
@@ -1245,7 +1235,6 @@ int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaSt
   v.hist += static_cast<int64_t>(r0) * w.nchunk * kBins;
   v.chunk_off += static_cast<int64_t>(r0) * w.nchunk;
   v.gtmask += static_cast<int64_t>(r0) * w.nchunk * (kChunk / 32);
-  v.chunk_cand += static_cast<int64_t>(r0) * w.nchunk;
   v.res += static_cast<int64_t>(r0) * 4;
   v.fallback += r0;
   v.cand += static_cast<int64_t>(r0) * w.cap;
@@ -1283,7 +1272,6 @@ int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
   w.hist = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * kBins * 4));
   w.chunk_off = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * 4));
   w.gtmask = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * w.nchunk * (kChunk / 8)));
-  w.chunk_cand = reinterpret_cast<uint2*>(take(static_cast<size_t>(R) * w.nchunk * 8));
   w.res = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(R) * 16));
   w.fallback = reinterpret_cast<int32_t*>(take(static_cast<size_t>(R) * 4));
   w.cand = reinterpret_cast<uint2*>(take(static_cast<size_t>(R) * w.cap * 8));

@@ -88,7 +88,7 @@ def test_topk_argument_errors(S):
 def test_topk_workspace_size_rules(S):
     """The optional top-k workspace: none below 64 K keys per row; from there, at least the
     candidate lists (8 bytes per candidate, max(4096, n/16) candidates per row) plus the per-chunk
-    counters and candidate spans (8 K-key chunks) and the above-window bit mask (one bit per key);
+    counters (8 K-key chunks) and the selection bit mask (one bit per key);
     linear in the row count; k does not matter; rows longer than 8192 chunks (64 M keys) take the
     cluster kernel and need none."""
     f = S.topk_workspace_size
@@ -96,7 +96,7 @@ def test_topk_workspace_size_rules(S):
         assert f(64, n, max(1, n // 2)) == 0
     for n in (65536, 262144, 1048576, 1 << 22):
         nchunk = -(-n // 8192)
-        need = 64 * (max(4096, n // 16) * 8 + nchunk * (4 + 4 + 64 * 4 + 8 + 8192 // 8))
+        need = 64 * (max(4096, n // 16) * 8 + nchunk * (4 + 4 + 64 * 4 + 8192 // 8))
         b = f(64, n, n // 2)
         assert b >= need
         assert b == f(64, n, 1) == f(64, n, n - 1)
