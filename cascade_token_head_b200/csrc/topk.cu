@@ -589,6 +589,15 @@ __device__ __forceinline__ int bin_of(float f, const BinMap& m) {
   return min(max(b, 0), kBins - 1);
 }
 
+// Programmatic dependent launch between the streaming steps: the filter, resolve and output
+// kernels are launched with programmatic stream serialisation, so their CTAs may start while the
+// previous step still runs (every CTA of that step is resident by then: each one triggers at its
+// start).  grid_dep_wait() returns once the previous step's grid has completed and its writes are
+// visible; nothing that step writes is read before it.  The filter issues its score loads (input
+// only) before the wait, beside the sample step.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // bitonic sort of one value per thread over a 1024-thread block, descending (thread t ends with
 // sorted position t); partners closer than a warp exchange by shuffles, the others through
 // `scratch` [1024]; every thread must call it, and scratch is free again after a block barrier
@@ -709,6 +718,7 @@ __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamW
   constexpr int KPT = kSamples / kRThreads;   // 16 sample keys per thread
   static_assert(kL1 == kRThreads, "one first-level key per thread");
   __shared__ SampleSmem sm;
+  grid_dep_trigger();
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   // thread t reads 16 consecutive keys of run t / 16 (runs start on a 16-byte boundary)
@@ -802,10 +812,8 @@ __device__ __forceinline__ int span_off(int u) { return 128 * (u >> 2) + (u & 3)
 // the above-window mask (bit u: f[u] > fe0) and the candidate mask (bit u: f[u] in [fe64, fe0],
 // or NaN) of one lane's kFKeys keys
 template <bool FULL>
-__device__ __forceinline__ void filter_span(const float* row, int jw, int n, float fe0, float fe64, uint32_t& gm,
+__device__ __forceinline__ void filter_span(const float* f, int jw, int n, float fe0, float fe64, uint32_t& gm,
                                             uint32_t& cm) {
-  float f[kFKeys];
-  load_span<FULL>(row, jw, n, f);
   gm = 0u;
   cm = 0u;
 #pragma unroll
@@ -822,15 +830,21 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_filter_kernel(TArgs a, Stre
   __shared__ uint32_t hist[kBins];
   const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < kBins) hist[tid] = 0u;
-  const float4 en = reinterpret_cast<const float4*>(w.ends)[r];
-  const float fe0 = en.x, fe64 = en.y;
-  const BinMap bm{en.z, en.w};
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
   const int jw = c * kChunk + warp * (32 * kFKeys) + 4 * lane;
   const int64_t rc = static_cast<int64_t>(r) * w.nchunk + c;
+  const bool full = (c + 1) * kChunk <= a.n;
+  float f[kFKeys];
+  if (full) load_span<true>(row, jw, a.n, f);
+  else load_span<false>(row, jw, a.n, f);
+  grid_dep_trigger();
+  grid_dep_wait();   // the window ends and the zeroed candidate count come from the sample step
+  const float4 en = reinterpret_cast<const float4*>(w.ends)[r];
+  const float fe0 = en.x, fe64 = en.y;
+  const BinMap bm{en.z, en.w};
   uint32_t gm, cm;
-  if ((c + 1) * kChunk <= a.n) filter_span<true>(row, jw, a.n, fe0, fe64, gm, cm);
-  else filter_span<false>(row, jw, a.n, fe0, fe64, gm, cm);
+  if (full) filter_span<true>(f, jw, a.n, fe0, fe64, gm, cm);
+  else filter_span<false>(f, jw, a.n, fe0, fe64, gm, cm);
   {
     // load q of lanes 8 g .. 8 g + 7 covers word 4 q + g of the warp's 16 (32 keys each), lane
     // 8 g + i at bits 4 i .. 4 i + 3
@@ -940,6 +954,8 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     n_bc = 0u;
     js_s = kBins;   // no sub-bin found: the row falls back
   }
+  grid_dep_trigger();
+  grid_dep_wait();   // everything below reads the filter step's results
   const int nchunk = w.nchunk;
   uint32_t g = 0u;
   for (int c = tid; c < nchunk; c += kRThreads) {
@@ -1130,6 +1146,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_output_kernel(TArgs a, Stre
   __shared__ uint32_t wc[kFWarps];
   const int c = blockIdx.x, r = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t rc = static_cast<int64_t>(r) * w.nchunk + c;
+  grid_dep_wait();   // everything below reads the resolve step's results
   const uint32_t valid = w.res[static_cast<int64_t>(r) * 4];
   const uint32_t word = lane < kFKeys ? w.gtmask[rc * (kChunk / 32) + warp * kFKeys + lane] : 0u;
   const uint32_t off = w.chunk_off[rc];
@@ -1222,6 +1239,23 @@ size_t topk_workspace_bytes(int R, int n, int k) {
 
 int32_t cluster_launch(const TArgs& a, cudaStream_t st);
 
+// a streaming step launched with programmatic stream serialisation (see grid_dep_wait)
+int32_t launch_after_previous(void (*kernel)(TArgs, StreamWs), dim3 grid, int threads, size_t smem, cudaStream_t st,
+                              const TArgs& g, const StreamWs& v) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SPT_CUDA(cudaLaunchKernelEx(&cfg, kernel, g, v));
+  return launch_status();
+}
+
 // the four steps for rows [r0, r0 + rows)
 int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaStream_t st) {
   TArgs g = a;
@@ -1240,12 +1274,10 @@ int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaSt
   v.cand += static_cast<int64_t>(r0) * w.cap;
   topk_sample_kernel<<<rows, kRThreads, 0, st>>>(g, v);
   SPT_TRY(launch_status());
-  topk_filter_kernel<<<dim3(w.nchunk, rows), kFThreads, 0, st>>>(g, v);
-  SPT_TRY(launch_status());
-  topk_resolve_kernel<<<rows, kRThreads, static_cast<size_t>(kBinCap) * 8 + static_cast<size_t>(w.nchunk) * 4, st>>>(g, v);
-  SPT_TRY(launch_status());
-  topk_output_kernel<<<dim3(w.nchunk, rows), kFThreads, 0, st>>>(g, v);
-  return launch_status();
+  SPT_TRY(launch_after_previous(topk_filter_kernel, dim3(w.nchunk, rows), kFThreads, 0, st, g, v));
+  SPT_TRY(launch_after_previous(topk_resolve_kernel, dim3(rows), kRThreads,
+                                static_cast<size_t>(kBinCap) * 8 + static_cast<size_t>(w.nchunk) * 4, st, g, v));
+  return launch_after_previous(topk_output_kernel, dim3(w.nchunk, rows), kFThreads, 0, st, g, v);
 }
 
 int32_t topk_stream_launch(const TArgs& a, void* ws, cudaStream_t st) {
