@@ -338,6 +338,32 @@ def test_topk_long_rows_tie_group_at_threshold(cuda):
         np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
 
 
+def test_topk_long_rows_crowded_threshold_sub_bin(cuda):
+    """Long rows on the streaming path whose threshold sub-bin holds between 1024 and 8192
+    candidates, so the resolve step takes its 64-bit digit search (and marks the selected ones
+    there): 3000 keys sharing the k-th value (rows 0-1, the group split at different offsets), or
+    3000 distinct values 1e-7 apart (about 1.7 float32 ulps at 0.6), a span of 3e-4 against a
+    sub-bin width near 1e-3, around the k-th value (rows 2-3).  The window (about 3.3 % of 262144 keys) plus the group stays inside the candidate
+    list (16384).  Bit-exact against the oracle."""
+    S = lib()
+    g = synth.rng_for(80)
+    R_, n, k = 4, 262144, 100000
+    x = g.random((R_, n)).astype(np.float32)
+    for r in range(R_):
+        order = np.argsort(-x[r].astype(np.float64), kind="stable")
+        v = x[r, order[k - 1]]
+        lo = max(0, k - 1 - (500 if r % 2 == 0 else 2500))
+        grp = order[lo:lo + 3000]                        # 3000 keys ranked around the k-th
+        if r < 2:
+            x[r, grp] = v                                 # one tie group holding the threshold
+        else:
+            x[r, grp] = (v.astype(np.float64) + (np.arange(3000) - 1500) * 1e-7).astype(np.float32)
+    got, _, st = _topk_gpu(S, x, k)
+    assert st == 0
+    for r in range(R_):
+        np.testing.assert_array_equal(got[r], R.topk_select(x[r].astype(np.float64), k))
+
+
 def test_topk_long_rows_special_values_and_strides(cuda):
     """Long rows (n = 100003: a ragged last chunk) with special values, bit-exact against the
     oracle for k from 1 to n - 7:
