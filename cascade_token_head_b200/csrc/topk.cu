@@ -507,10 +507,11 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 // Long rows (n >= kStreamMin, scores read directly, caller workspace given): one streaming pass
 // over the scores between a sample and an exact select on small data (one CTA per row each), then
 // an output pass over the pass's bit mask and candidates.
-//  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256) and finds by a digit
-//           search the sample keys e0 >= e64 at the two ends of a rank window around the sample
-//           rank of the k-th key (+-4 sigma of the sampling error + 16; an end past the sample is
-//           left open).  The search runs first on one key in 16, whose own window, widened by its
+//  sample   one CTA per row draws 16 K keys (64 evenly spaced runs of 256; 8 K keys in runs of 128
+//           for rows under 512 K keys) and finds by a digit search the sample keys e0 >= e64 at
+//           the two ends of a rank window around the sample rank of the k-th key (+-4 sigma of the
+//           sampling error + 16; an end past the sample is left open).  The search runs first on
+//           each thread's first key (one in 16, or in 8), whose own window, widened by its
 //           sampling error, bounds the few thousand sample keys the exact search then needs.  It
 //           also fixes the sub-bin scale: 64 steps of equal width in value between the window's
 //           ends (the sample's extreme key in place of an open end).
@@ -534,7 +535,7 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 // indices.
 // ------------------------------------------------------------------------------------------------
 constexpr int kStreamMin = 65536;
-constexpr int kSRuns = 64, kSRun = 256, kSamples = kSRuns * kSRun;   // 16 K sample keys per row
+constexpr int kSRuns = 64;                                              // sample runs per row
 constexpr int kBins = 64;
 constexpr int kRThreads = 1024;                                         // sample and resolve CTAs
 constexpr int kFThreads = 512;                                          // filter and output CTAs
@@ -543,7 +544,16 @@ constexpr int kFKeys = 16;                                              // keys 
 constexpr int kChunk = kFThreads * kFKeys;                              // 8 K keys per filter/output CTA
 constexpr int kBinCap = 8192;                                           // candidates of one sub-bin
 constexpr int kL1 = 1024;                                               // first-level sample keys
-constexpr int kSList = 4096;                                            // second-level sample keys
+// the sample of one row: KPT keys per thread of a 1024-thread CTA, in 64 runs of 16 threads'
+// keys; the second-level list holds a quarter of the sample.  16 K keys (KPT 16) for rows of
+// 512 K keys and more, 8 K (KPT 8) below: a smaller sample costs a wider window (more candidates
+// for the filter and resolve steps), which pays off only where the sample step is a large share
+template <int KPT>
+struct SampleCfg {
+  static constexpr int kSRun = 16 * KPT;                 // keys per run
+  static constexpr int kSamples = kSRuns * kSRun;        // sample keys per row
+  static constexpr int kSList = kSamples / 4;            // second-level sample keys
+};
 constexpr int kMaxChunks = 8192;
 
 struct StreamWs {
@@ -623,10 +633,11 @@ __device__ __forceinline__ V bitonic_desc_1024(V x, V* scratch) {
   return x;
 }
 
+template <int KPT>
 struct SampleSmem {
   uint32_t red[2][3][32];
   uint32_t cnt[32];
-  uint32_t list[kSList];
+  uint32_t list[SampleCfg<KPT>::kSList];
   int rank[2];        // sample ranks of the window's ends
   int open[2];        // the window's top / bottom end lies past the sample
   int l1[2];          // first-level ranks of the outer bounds (< 0 / >= kL1: no bound)
@@ -637,8 +648,8 @@ struct SampleSmem {
 // are 0 and never counted): the largest T with count(>= T) >= need, two bits per round; counts fit
 // 16 bits (at most 16 K), two per word.  While the two share their high bits one set of three
 // counts serves both.
-template <int NK>
-__device__ __forceinline__ void search2(const uint32_t* key, uint32_t need_a, uint32_t need_b, SampleSmem& sm,
+template <int NK, class SM>
+__device__ __forceinline__ void search2(const uint32_t* key, uint32_t need_a, uint32_t need_b, SM& sm,
                                         uint32_t& ta, uint32_t& tb) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   ta = 0u;
@@ -699,8 +710,8 @@ __device__ __forceinline__ void append_keys(bool in, uint32_t key, uint32_t* lis
 
 // the window's ends from the NK keys per thread, which hold every sample key ranked in the window;
 // `base` more sample keys lie above all of them
-template <int NK>
-__device__ __forceinline__ void window_ends(const uint32_t* key, uint32_t base, SampleSmem& sm, int r, StreamWs& w) {
+template <int NK, class SM>
+__device__ __forceinline__ void window_ends(const uint32_t* key, uint32_t base, SM& sm, int r, StreamWs& w) {
   const uint32_t need_a = static_cast<uint32_t>(sm.rank[0]) + 1u - base;
   const uint32_t need_b = static_cast<uint32_t>(sm.rank[1]) + 1u - base;
   uint32_t ta, tb;
@@ -714,10 +725,12 @@ __device__ __forceinline__ void window_ends(const uint32_t* key, uint32_t base, 
   }
 }
 
+template <int KPT>
 __global__ void __launch_bounds__(kRThreads) topk_sample_kernel(TArgs a, StreamWs w) {
-  constexpr int KPT = kSamples / kRThreads;   // 16 sample keys per thread
+  constexpr int kSRun = SampleCfg<KPT>::kSRun, kSamples = SampleCfg<KPT>::kSamples, kSList = SampleCfg<KPT>::kSList;
+  static_assert(kSamples == KPT * kRThreads, "KPT sample keys per thread");
   static_assert(kL1 == kRThreads, "one first-level key per thread");
-  __shared__ SampleSmem sm;
+  __shared__ SampleSmem<KPT> sm;
   grid_dep_trigger();
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* row = a.scores + static_cast<int64_t>(r) * a.ld;
@@ -1272,7 +1285,8 @@ int32_t stream_chain(const TArgs& a, const StreamWs& w, int r0, int rows, cudaSt
   v.res += static_cast<int64_t>(r0) * 4;
   v.fallback += r0;
   v.cand += static_cast<int64_t>(r0) * w.cap;
-  topk_sample_kernel<<<rows, kRThreads, 0, st>>>(g, v);
+  if (g.n >= 512 * 1024) topk_sample_kernel<16><<<rows, kRThreads, 0, st>>>(g, v);
+  else topk_sample_kernel<8><<<rows, kRThreads, 0, st>>>(g, v);
   SPT_TRY(launch_status());
   SPT_TRY(launch_after_previous(topk_filter_kernel, dim3(w.nchunk, rows), kFThreads, 0, st, g, v));
   SPT_TRY(launch_after_previous(topk_resolve_kernel, dim3(rows), kRThreads,

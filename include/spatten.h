@@ -239,10 +239,10 @@ int32_t spatten_attention_layer_noalloc(const spatten_attn_args* a, void* stream
  *  Workspace (ws, ws_bytes): optional, device memory of spatten_topk_workspace_size(R, n, k)
  *  bytes (0 for rows shorter than 65,536 keys).  Given it, rows of at least 65,536 keys read
  *  directly (map NULL, scores 16-byte aligned, ld a multiple of 4) take a one-read streaming path:
- *  a 16 K-key sample brackets the k-th key, one pass over the scores marks the keys above the
- *  bracket in a bit mask and collects the bracket's keys, the exact threshold is chosen among
- *  them, and the output is written from the mask and the selected bracket keys; rows whose bracket
- *  misses fall back to the cluster radix select.  Without it (or with fewer bytes)
+ *  a 16 K-key sample (8 K below 512 K keys) brackets the k-th key, one pass over the scores marks
+ *  the keys above the bracket in a bit mask and collects the bracket's keys, the exact threshold is
+ *  chosen among them, and the output is written from the mask and the selected bracket keys; rows
+ *  whose bracket misses fall back to the cluster radix select.  Without it (or with fewer bytes)
  *  every row takes the cluster radix select.  Results are identical either way.  The workspace
  *  holds only this call's intermediates (nothing to clear): later calls on the same stream may
  *  reuse it, calls that overlap on the GPU need one each.
