@@ -515,13 +515,13 @@ __global__ void __launch_bounds__(G == 1 ? 128 : 32 * G) topk_small_kernel(TArgs
 //           sampling error, bounds the few thousand sample keys the exact search then needs.  It
 //           also fixes the sub-bin scale: 64 steps of equal width in value between the window's
 //           ends (the sample's extreme key in place of an open end).
-//  filter   per chunk of 8 K keys: the count above e0, the keys in [e64, e0] appended as (score
-//           bits, index) to the row's candidate list, and their histogram over the 64 sub-bins
+//  filter   per chunk of 8 K keys: the keys above e0 (a count and a bit mask), the keys in
+//           [e64, e0] appended as (score bits, index) to the row's candidate list, and their
+//           histogram over the 64 sub-bins
 //  resolve  one CTA per row: the sub-bin holding the k-th key, the exact threshold among that
 //           sub-bin's candidates as the (need)-th largest (key, ~index) composite (ties to the lower
-//           index), whether the keys equal to T are split by index, and every chunk's output offset
-//           It also sets the mask bits of the selected candidates: every candidate of the sub-bins
-//           above T's, and T's own selected part.
+//           index), and every chunk's output offset.  It also sets the mask bits of the selected
+//           candidates: every candidate of the sub-bins above T's, and T's own selected part.
 //  output   per chunk: the indices of the mask's set bits, written in index order (the scores are
 //           not read again)
 // A row whose k-th key fell outside the window, or whose buffers overflowed, is marked and done
@@ -567,7 +567,7 @@ struct StreamWs {
   uint32_t* chunk_off;  // [R][nchunk]
   uint32_t* gtmask;     // [R][nchunk][kChunk / 32]  bit j % 32 of word j / 32 (row key j): above the
                         //            window (filter), or a selected candidate (resolve)
-  uint32_t* res;        // [R][4]   valid, T key, T index, unused
+  uint32_t* res;        // [R][4]   valid, T key, T index, spare
   int32_t* fallback;    // [R]
   int cap, nchunk;
 };
@@ -1143,7 +1143,7 @@ __global__ void __launch_bounds__(kRThreads) topk_resolve_kernel(TArgs a, Stream
     rr[0] = 1u;
     rr[1] = t_key;
     rr[2] = t_idx;
-    rr[3] = 0u;
+    rr[3] = 0u;   // spare
     w.fallback[r] = 0;
   }
 }
